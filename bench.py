@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the workload:
+pa_reshape_and_cache of this step's new tokens, then pa_decode (split-K decode
+kernel + log-sum-exp merge) — and, for the mixed prefill workload,
+pa_chunked_prefill as well.  Inputs are seeded synthetic tensors already
+resident in HBM when the timed region starts; every workload except the tiny
+one reads more KV than the 126 MB L2 holds per step, and the tiny one flushes
+L2 between steps.  Times are CUDA-event times on the launching stream,
+bracketed by barrier + synchronize, max over ranks.  Rank 0 prints one JSON
+line.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the workload (the sequences of a decode batch are
+independent; the path has no exchange step), so the value is the whole-job
+throughput of N replicas (weak scaling).
+
+--impl reference times the fp64 CPU oracle (the plain restatement of what the
+path computes) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- helpers
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+def decode_algorithmic_bytes(b: workloads.PagedBatch) -> int:
+    """KV of every token at its exact length, q and out, table rows, seq_lens."""
+    e = b.q.element_size()
+    lens = b.seq_lens.cpu().numpy().astype(np.int64)
+    B = len(lens)
+    kv = int(lens.sum()) * 2 * b.num_kv_heads * b.head_dim * e
+    qo = 2 * B * b.num_q_heads * b.head_dim * e
+    tables = B * int(math.ceil(int(lens.max()) / b.block_size)) * 4
+    return kv + qo + tables + 4 * B
+
+
+def prefill_flops(b: workloads.PagedBatch) -> int:
+    """4*D*Hq per (query, visible key) pair (QK^T and PV, 2 flops per MAC)."""
+    lens = b.seq_lens.cpu().numpy().astype(np.int64)
+    qsl = b.query_start_loc.cpu().numpy().astype(np.int64)
+    pairs = 0
+    for s in range(len(lens)):
+        n = int(qsl[s + 1] - qsl[s])
+        L = int(lens[s])
+        pairs += sum(L - n + i + 1 for i in range(n))
+    return 4 * b.head_dim * b.num_q_heads * pairs
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def aggregate_max(value: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- the step
+
+class Step:
+    """All device buffers of one workload and the hot-path calls of one step."""
+
+    def __init__(self, batches, pa, stream):
+        self.pa = pa
+        self.stream = stream
+        self.batches = batches
+        self.decode = [b for b in batches if b.query_start_loc is None]
+        self.prefill = [b for b in batches if b.query_start_loc is not None]
+        self.ws = {}
+        self.out = {}
+        for b in batches:
+            self.out[id(b)] = torch.empty_like(b.q)
+            if b.query_start_loc is None:
+                n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
+                self.ws[id(b)] = torch.empty(max(n, 16), dtype=torch.uint8, device=b.q.device) if n else None
+        self.max_len = {id(b): b.max_seq_len for b in batches}
+        self.max_q = {id(b): b.max_query_len for b in batches}
+        self.launches = 0
+        self.ev_dec = []
+
+    def run(self, record=None):
+        pa = self.pa
+        n = 0
+        for b in self.batches:
+            pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping,
+                                    stream=self.stream)
+            n += pa.pa_last_launch_count()
+        for b in self.prefill:
+            pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
+                                  b.seq_lens, b.query_start_loc, b.scale, self.max_q[id(b)],
+                                  self.max_len[id(b)], None, stream=self.stream)
+            n += pa.pa_last_launch_count()
+        for b in self.decode:
+            if record is not None:
+                record[0].record(self.stream)
+            pa.pa_decode(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
+                         b.scale, self.max_len[id(b)], 0, self.ws[id(b)], stream=self.stream)
+            n += pa.pa_last_launch_count()
+            if record is not None:
+                record[1].record(self.stream)
+        self.launches += n
+        return n
+
+
+def host_inputs(b: workloads.PagedBatch):
+    """Pinned host copies of a step's per-step inputs (everything but the cache)."""
+    names = ["q", "k_new", "v_new", "slot_mapping", "seq_lens", "block_tables"]
+    if b.query_start_loc is not None:
+        names.append("query_start_loc")
+    return {n: getattr(b, n).cpu().pin_memory() for n in names}
+
+
+# ---------------------------------------------------------------- arms
+
+def run_ours(args, rank, world, device):
+    import paged_kv_cache_332_b200 as pa
+    pa.lib()  # fails loudly if the library is missing
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device=device)
+    batches = workloads.WORKLOADS[args.workload](device=device)
+    step = Step(batches, pa, stream)
+    dec = step.decode[0] if step.decode else None
+    pre = step.prefill[0] if step.prefill else None
+    kv_bytes = sum(b.k_cache.numel() * b.k_cache.element_size() * 2 for b in batches)
+    flush = None
+    if kv_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    def one(record=None):
+        if flush is not None:
+            flush.fill_(1.0)
+        return step.run(record)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one()
+    torch.cuda.synchronize(device)
+
+    # ---- timed region (device-resident inputs)
+    step.launches = 0
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(device) as clocks:
+        barrier()
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                if flush is not None:
+                    flush.fill_(float(i))
+                ev[i][0].record(stream)
+                step.run(evd[i] if dec is not None else None)
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    local_ms = sum(step_ms)
+    launches = step.launches
+    dec_ms = [a.elapsed_time(b) for a, b in evd] if dec is not None else []
+    total_ms = aggregate_max(local_ms, device)
+
+    # ---- end to end: per-step H2D of the step's inputs from pinned host
+    # memory, the C-ABI calls, D2H of the outputs
+    hosts = [host_inputs(b) for b in batches]
+    outs_h = [torch.empty(step.out[id(b)].shape, dtype=b.q.dtype).pin_memory() for b in batches]
+    h2d = sum(t.numel() * t.element_size() for h in hosts for t in h.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            for b, h in zip(batches, hosts):
+                for n, t in h.items():
+                    getattr(b, n).copy_(t, non_blocking=True)
+            step.run()
+            for b, o in zip(batches, outs_h):
+                o.copy_(step.out[id(b)], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    e2e_ms = aggregate_max(e0.elapsed_time(e1), device)
+
+    # ---- metric
+    tokens = sum(b.num_seqs for b in step.decode) + sum(int(b.q.shape[0]) for b in step.prefill)
+    value = world * tokens * args.steps / (total_ms / 1e3)
+    peaks = measured_peaks()
+    line = {
+        "metric": "paged decode tokens/s (one layer) and achieved HBM GB/s of pa_decode",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if batches[0].dtype == torch.bfloat16 else "fp16",
+        "data": "synthetic (seeded N(0,1) q/K/V, FIFO free-list block tables)",
+        "impl": "ours",
+        "gpu_launches": launches,
+    }
+    cfg = {"workload": "+".join(b.name for b in batches), "parallelism": "replicas%d" % world,
+           "l2": "flushed between steps" if flush is not None else
+           "inputs larger than L2 (%.0f MB of KV cache per replica)" % (kv_bytes / 1e6)}
+    if dec is not None:
+        cfg.update(num_seqs=dec.num_seqs, q_heads=dec.num_q_heads, kv_heads=dec.num_kv_heads,
+                   head_dim=dec.head_dim, block_size=dec.block_size,
+                   context_tokens=int(dec.seq_lens.sum().item()))
+    line["config"] = cfg
+    if dec is not None:
+        ab = decode_algorithmic_bytes(dec)
+        dmean = statistics.mean(dec_ms)
+        ach = ab / (dmean / 1e3) / 1e9
+        line["roofline"] = {"kernel": "pa_decode (paged_decode_kernel + lse_reduce_kernel)",
+                            "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                            "peak_source": peaks["source"], "unit": "GB/s",
+                            "frac": round(ach / peaks["hbm_gbs"], 4),
+                            "frac_of_8TBs_spec": round(ach / 8000.0, 4),
+                            "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
+                            "traffic": None}
+        line["context_tokens_per_s"] = round(world * int(dec.seq_lens.sum().item()) * args.steps
+                                             / (total_ms / 1e3), 1)
+    if pre is not None:
+        line["prefill_tflop_per_step"] = prefill_flops(pre) / 1e12
+    line["e2e"] = {"value": round(world * tokens * e2e_steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    line["clocks"] = clocks.summary()
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(batches, args)
+    return line
+
+
+def cpu_baseline(batches, args, budget_s=None):
+    """Time the oracle, as it stands, on a bounded sample of the workload and
+    scale to the metric (decoded tokens per second of a full step)."""
+    import oracle.paged_attention as opa
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    budget_s = budget_s if budget_s is not None else args.cpu_budget
+    dec = [b for b in batches if b.query_start_loc is None]
+    b = dec[0] if dec else batches[0]
+    lens = b.seq_lens.cpu().numpy()
+    order = np.random.Generator(np.random.PCG64(0)).permutation(len(lens))
+    t_used, ctx_done, seqs_done = 0.0, 0, 0
+    for s in order:
+        s = int(s)
+        sub_t0 = time.perf_counter()
+        bt = b.block_tables[s:s + 1].cpu()
+        L = int(lens[s])
+        nblk = -(-L // b.block_size)
+        ids = bt[0, :nblk].long().to(b.k_cache.device)
+        kc = opa.to_f64(b.k_cache.index_select(0, ids))
+        vc = opa.to_f64(b.v_cache.index_select(0, ids))
+        tbl = np.arange(nblk, dtype=np.int32)[None, :]
+        q = opa.to_f64(b.q[s:s + 1])
+        t0 = time.perf_counter()
+        opa.paged_decode(q, kc, vc, tbl, np.array([L]), b.scale)
+        t_used += time.perf_counter() - t0
+        ctx_done += L
+        seqs_done += 1
+        if t_used >= budget_s:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    total_ctx = int(lens.sum())
+    est_step_s = t_used * total_ctx / max(ctx_done, 1)
+    value = b.num_seqs / est_step_s
+    return {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d sequences of %s (%d of %d context tokens), oracle time %.1f s "
+                      "scaled by context tokens to one full step" % (seqs_done, len(lens), b.name,
+                                                                     ctx_done, total_ctx, t_used)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    batches = workloads.WORKLOADS[args.workload](device="cpu")
+    for _ in range(args.warmup):
+        cpu_baseline(batches, args, budget_s=1.0)
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(batches, args, budget_s=args.ref_step_budget)
+        vals.append(last["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    dec = [b for b in batches if b.query_start_loc is None]
+    b = dec[0] if dec else batches[0]
+    line = {
+        "metric": "paged decode tokens/s (one layer) and achieved HBM GB/s of pa_decode",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(b.num_seqs / value * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1) q/K/V, FIFO free-list block tables)",
+        "impl": "reference",
+        "config": {"workload": "+".join(x.name for x in batches), "parallelism": "replicas%d" % world},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": last["sample"] + "; each step a bounded sample, %.1f s wall" % wall},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixed", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--ref-step-budget", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1 and args.impl == "ours":
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

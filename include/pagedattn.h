@@ -1,0 +1,170 @@
+/*
+ * libpagedattn — PagedAttention hot path for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on KV-cache paging, cited by title and section):
+ *   [P1] "大模型推理内存优化从 KV Cache 分页到连续批处理的工程实践" (seekfood.cn):
+ *        "KV Cache 的内存开销与分页机制" (fixed-size physical blocks, per-sequence
+ *        block table, on-demand allocation, shared prefix blocks),
+ *        "PagedAttention 的 CUDA Kernel 实现" (attention reads K/V indirectly through
+ *        the block table), "工程边界与架构取舍" (decode is memory-bound and reads
+ *        the whole cache; long prompts are prefilled in chunks).
+ *   [P2] "KV Cache管理优化：大模型推理显存瓶颈突破" (intelliparadigm), 2.1 (one
+ *        pre-allocated pool, no per-request allocation), 2.2 (blocks of 16-32 tokens).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller, contiguous in the
+ *    stated row-major layout; the library keeps no reference after the call returns.
+ *  - KV caches: k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim] of
+ *    fp16 or bf16 (PA_F16 / PA_BF16); the two caches share one layout.
+ *  - Block tables: int32 [num_seqs, max_blocks_per_seq]; entry j of row s is the
+ *    physical block that holds tokens j*block_size .. j*block_size+block_size-1 of
+ *    sequence s.  Entries past a sequence's last block are never read.
+ *  - A slot is physical_block * block_size + offset_in_block.
+ *  - GQA: q-heads [g*G, (g+1)*G) use kv-head g, with G = num_q_heads / num_kv_heads.
+ *  - Supported: head_dim 128, block_size 16 or 32, G in {1, 2, 4, 8}, fp16 / bf16.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and never synchronise the host.  The library allocates no device memory
+ *    on any call; scratch space comes from the caller (`workspace`).
+ *  - Return value: PA_OK once the kernels are launched, or an error found on the host
+ *    before any launch (nothing is launched then).
+ *  - Errors that depend on device data (a slot or block id outside the cache, a
+ *    sequence longer than its table or than max_seq_len, an inconsistent
+ *    query_start_loc) never fault or trap: the kernel skips the offending rows (their
+ *    outputs are unspecified), ORs a PA_DEVERR_* bit into a per-device flag and goes
+ *    on.  Read and clear the flag with pa_get_device_error().
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, inconsistent shape */
+  PA_ERR_UNSUPPORTED = 2,          /* head_dim, block_size, GQA group or dtype not built */
+  PA_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes below the matching *_workspace_size */
+  PA_ERR_CUDA = 4,                 /* a CUDA runtime/driver call failed (launch, tensor map) */
+  PA_ERR_DEVICE_DATA = 5           /* pa_get_device_error found a device-side data error */
+} pa_status;
+
+/* Device-side error bits (pa_get_device_error). */
+#define PA_DEVERR_SLOT_RANGE   0x1  /* reshape_and_cache: slot >= num_blocks*block_size   */
+#define PA_DEVERR_BLOCK_RANGE  0x2  /* a needed block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_SEQ_TOO_LONG 0x4  /* seq_len > max_blocks_per_seq*block_size or > max_seq_len */
+#define PA_DEVERR_QUERY_LAYOUT 0x8  /* prefill: query_start_loc not monotone, q_len > seq_len
+                                       or q_len > max_query_len */
+#define PA_DEVERR_TIMEOUT      0x10 /* an in-kernel pipeline wait gave up (never expected) */
+
+/* Human-readable name of a status code (static string, never NULL). */
+PA_API const char* pa_status_string(int status);
+
+/*
+ * reshape_and_cache — write this step's K/V rows into their cache slots.
+ * [P1] "KV Cache 的内存开销与分页机制": a generated token's K and V go to the next
+ * free place of the sequence's current block (a new block is taken when it is full).
+ *
+ *   k, v          [T, num_kv_heads, head_dim]  rows to store (same dtype as the caches)
+ *   k_cache,
+ *   v_cache       [num_blocks, block_size, num_kv_heads, head_dim]  updated in place
+ *   slot_mapping  int32 [T]: destination slot of token t; a negative slot skips the
+ *                 token (padding).  Two tokens with one slot in a call: undefined.
+ * The copy is bitwise.  A slot >= num_blocks*block_size is skipped and sets
+ * PA_DEVERR_SLOT_RANGE.  T == 0 launches nothing.
+ */
+PA_API pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                               const int32_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int num_blocks, int block_size, pa_dtype dtype,
+                               void* stream);
+
+/*
+ * Bytes of scratch `pa_decode` needs for the split-K partials: for sequences longer
+ * than one partition it keeps, per (sequence, q-head, partition), the normalised
+ * partial output (head_dim fp32) and its running max and sum (2 fp32).
+ * partition_size 0 means the library's choice (the same one pa_decode makes).
+ * Returns 0 when a single partition covers max_seq_len (no reduction pass).
+ */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
+                                int partition_size);
+
+/*
+ * pa_decode — single-query attention of each sequence over its paged KV cache.
+ * [P1] "PagedAttention 的 CUDA Kernel 实现" and "工程边界与架构取舍": each sequence's
+ * query attends to every cached token of the sequence (the token appended this step
+ * included: call pa_reshape_and_cache first), K/V reached through the block table.
+ *
+ *   out           [num_seqs, num_q_heads, head_dim]   softmax(scale * q K^T) V, rounded
+ *                                                     to nearest even in `dtype`
+ *   q             [num_seqs, num_q_heads, head_dim]
+ *   block_tables  int32 [num_seqs, max_blocks_per_seq]
+ *   seq_lens      int32 [num_seqs] (device): tokens of each sequence, 0 gives zeros
+ *   max_seq_len   host-side upper bound of seq_lens; sizes the grid and the
+ *                 partition count.  A longer sequence sets PA_DEVERR_SEQ_TOO_LONG.
+ *   partition_size  split-K partition in tokens (multiple of 16), 0 = library choice.
+ *                 Each (sequence, kv-head, partition) is one work item; sequences
+ *                 longer than one partition are merged by a log-sum-exp pass.
+ *   workspace     device scratch of at least pa_decode_workspace_size(...) bytes
+ *                 (may be NULL when that size is 0); contents need no initialisation.
+ */
+PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* seq_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                    int head_dim, float scale, int block_size, int num_blocks,
+                    int max_seq_len, int partition_size, void* workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+/* Bytes of scratch pa_chunked_prefill needs (0 in this version: no split-K). */
+PA_API size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len, int num_q_heads,
+                                         int head_dim, int max_seq_len);
+
+/*
+ * pa_chunked_prefill — causal attention of a chunk of new queries over the paged
+ * context.  [P1] "工程边界与架构取舍": a long prompt is processed in chunks; prefill is
+ * a dense matrix product (tensor cores).  The chunk's own K/V must already be in the
+ * cache (pa_reshape_and_cache first).
+ *
+ *   out, q            [total_q, num_q_heads, head_dim], total_q = query_start_loc[num_seqs]
+ *   query_start_loc   int32 [num_seqs+1] (device): exclusive prefix sum of chunk lengths
+ *   seq_lens          int32 [num_seqs] (device): context length including the chunk.
+ *                     Query i of sequence s sits at position seq_lens[s]-q_len_s+i and
+ *                     attends to keys 0 .. that position, inclusive.
+ *   max_query_len     host-side upper bound of the chunk lengths
+ *   max_seq_len       host-side upper bound of seq_lens
+ */
+PA_API pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* seq_lens, const int32_t* query_start_loc,
+                             int num_seqs, int max_query_len, int num_q_heads,
+                             int num_kv_heads, int head_dim, float scale, int block_size,
+                             int num_blocks, int max_seq_len, void* workspace,
+                             size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the calling device's PA_DEVERR_* flag into
+ * *code.  Returns PA_OK when the flag was 0, PA_ERR_DEVICE_DATA when it was not, or
+ * PA_ERR_CUDA if the synchronisation or the copy failed.
+ */
+PA_API pa_status pa_get_device_error(void* stream, int32_t* code);
+
+/* Number of kernel launches the most recent call on this host thread issued (0 when it
+ * returned an error before launching).  For launch accounting in benchmarks. */
+PA_API int pa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

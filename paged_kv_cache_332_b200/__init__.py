@@ -1,0 +1,180 @@
+"""Python binding for libpagedattn (PagedAttention hot path on B200).
+
+A thin ctypes layer over the C ABI declared in ``include/pagedattn.h``: each
+function here has the name of the C entry point it calls, takes torch tensors
+(device memory, contiguous, the layouts of the header), passes their pointers
+and sizes, and raises :class:`PagedAttnError` on a non-OK status.  All
+computation happens in the CUDA kernels of ``libpagedattn.so``; there is no
+fallback, and importing this package fails loudly when the library is missing.
+
+Build the library with ``python -m paged_kv_cache_332_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
+    "pa_decode_workspace_size", "pa_decode", "pa_chunked_prefill_workspace_size",
+    "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
+    "PA_DEVERR",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libpagedattn.so")
+
+PA_OK = 0
+PA_F16, PA_BF16 = 0, 1
+PA_DEVERR = {"SLOT_RANGE": 0x1, "BLOCK_RANGE": 0x2, "SEQ_TOO_LONG": 0x4, "QUERY_LAYOUT": 0x8,
+             "TIMEOUT": 0x10}
+
+# (name, restype, argtypes) of every entry point declared in include/pagedattn.h
+_vp, _i32, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+_SIGS = [
+    ("pa_status_string", ctypes.c_char_p, [_i32]),
+    ("pa_reshape_and_cache", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    ("pa_decode_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
+    ("pa_decode", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f, _i32, _i32,
+                         _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_chunked_prefill_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
+    ("pa_chunked_prefill", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
+                                  _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_get_device_error", _i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
+    ("pa_last_launch_count", _i32, []),
+]
+EXPORTED_SYMBOLS = [n for n, _, _ in _SIGS]
+
+_lib = None
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__("%s: %s" % (what, pa_status_string(status)))
+
+
+def lib():
+    """The loaded ``libpagedattn.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ImportError("libpagedattn.so not built: run `python -m paged_kv_cache_332_b200.build`"
+                              " (no CPU fallback exists)")
+        L = ctypes.CDLL(library_path)
+        for name, res, args in _SIGS:
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def pa_status_string(status: int) -> str:
+    return lib().pa_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError("libpagedattn takes float16 or bfloat16 tensors, got %s" % t.dtype)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libpagedattn takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libpagedattn takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _i32tensor(t, what):
+    if t.dtype != torch.int32:
+        raise TypeError("%s must be int32" % what)
+    return _ptr(t)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status, what):
+    if status != PA_OK:
+        raise PagedAttnError(status, what)
+
+
+def pa_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, stream=None):
+    """Scatter ``k``/``v`` [T, Hkv, D] into ``k_cache``/``v_cache``
+    [N, bs, Hkv, D] at ``slot_mapping`` (int32 [T], negative = skip)."""
+    N, bs, Hkv, D = k_cache.shape
+    T = k.shape[0]
+    _check(lib().pa_reshape_and_cache(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                      _i32tensor(slot_mapping, "slot_mapping"), T, Hkv, D, N, bs,
+                                      _dtype_code(k_cache), _stream(stream)),
+           "pa_reshape_and_cache")
+
+
+def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, partition_size=0):
+    return int(lib().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len,
+                                              partition_size))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,
+              partition_size=0, workspace=None, stream=None):
+    """Paged single-query attention.  ``q``/``out`` [B, Hq, D]; ``block_tables``
+    int32 [B, max_blocks]; ``seq_lens`` int32 [B]; ``workspace`` a device
+    tensor of at least :func:`pa_decode_workspace_size` bytes (or None when
+    that is 0)."""
+    N, bs, Hkv, D = k_cache.shape
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                           _i32tensor(block_tables, "block_tables"), block_tables.shape[1],
+                           _i32tensor(seq_lens, "seq_lens"), B, Hq, Hkv, D, float(scale), bs, N,
+                           int(max_seq_len), int(partition_size), _ptr(workspace), ws_bytes,
+                           _dtype_code(k_cache), _stream(stream)),
+           "pa_decode")
+
+
+def pa_chunked_prefill_workspace_size(num_seqs, max_query_len, num_q_heads, head_dim, max_seq_len):
+    return int(lib().pa_chunked_prefill_workspace_size(num_seqs, max_query_len, num_q_heads,
+                                                       head_dim, max_seq_len))
+
+
+def pa_chunked_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, scale,
+                       max_query_len, max_seq_len, workspace=None, stream=None):
+    """Causal chunk attention over the paged context.  ``q``/``out``
+    [total_q, Hq, D]; ``query_start_loc`` int32 [B+1]."""
+    N, bs, Hkv, D = k_cache.shape
+    _, Hq, _ = q.shape
+    B = seq_lens.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_chunked_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _i32tensor(block_tables, "block_tables"), block_tables.shape[1],
+                                    _i32tensor(seq_lens, "seq_lens"),
+                                    _i32tensor(query_start_loc, "query_start_loc"), B,
+                                    int(max_query_len), Hq, Hkv, D, float(scale), bs, N,
+                                    int(max_seq_len), _ptr(workspace), ws_bytes,
+                                    _dtype_code(k_cache), _stream(stream)),
+           "pa_chunked_prefill")
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error bits."""
+    code = ctypes.c_int32(0)
+    st = lib().pa_get_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (PA_OK, 5):
+        raise PagedAttnError(st, "pa_get_device_error")
+    return int(code.value)
+
+
+def pa_last_launch_count() -> int:
+    return int(lib().pa_last_launch_count())

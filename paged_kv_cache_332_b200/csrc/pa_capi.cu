@@ -1,0 +1,119 @@
+// Status strings, the per-device error flag, SM-count cache and TMA
+// descriptor encoding for libpagedattn.
+#include <mutex>
+
+#include "pa_host.h"
+
+// One int per device that loads the library; kernels OR PA_DEVERR_* bits into it.
+static __device__ int g_pa_device_error = 0;
+
+namespace pa {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+thread_local int g_last_launches = 0;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int current_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+  return d;
+}
+}  // namespace
+
+int* device_error_flag() {
+  const int d = current_device();
+  if (d < 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pa_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[d] = static_cast<int*>(p);
+  }
+  return g_err_ptr[d];
+}
+
+int num_sms() {
+  const int d = current_device();
+  if (d < 0) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[d]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return 0;
+    g_sms[d] = n;
+  }
+  return g_sms[d];
+}
+
+bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,
+                       int num_kv_heads, int head_dim, int box_rows) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  }
+  // innermost first: head_dim, kv-head, token-in-block, block
+  const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
+                              (cuuint64_t)block_size, (cuuint64_t)num_blocks};
+  const cuuint64_t row = (cuuint64_t)head_dim * 2;
+  const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const cuuint32_t box[4] = {(cuuint32_t)head_dim, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(cache), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+void set_launch_count(int n) { g_last_launches = n; }
+
+}  // namespace pa
+
+extern "C" {
+
+const char* pa_status_string(int s) {
+  switch (s) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE_TOO_SMALL: return "PA_ERR_WORKSPACE_TOO_SMALL";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_DEVICE_DATA: return "PA_ERR_DEVICE_DATA";
+    default: return "PA_ERR_UNKNOWN";
+  }
+}
+
+pa_status pa_get_device_error(void* stream, int32_t* code) {
+  if (!code) return PA_ERR_INVALID_ARG;
+  *code = 0;
+  int* flag = pa::device_error_flag();
+  if (!flag) return PA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, flag, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemsetAsync(flag, 0, sizeof(int), s) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  *code = v;
+  return v ? PA_ERR_DEVICE_DATA : PA_OK;
+}
+
+int pa_last_launch_count(void) { return pa::g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// reshape_and_cache: scatter this step's K/V rows into their cache slots.
+//
+// Page "大模型推理内存优化从 KV Cache 分页到连续批处理的工程实践", section
+// "KV Cache 的内存开销与分页机制": a new token's K and V are stored at the next
+// free place of the sequence's current physical block.  The caller passes the
+// destination slot (block * block_size + offset) of every token.
+//
+// In the cache layout [num_blocks, block_size, num_kv_heads, head_dim] all kv-heads
+// of one slot form one contiguous row of num_kv_heads*head_dim elements, exactly
+// like a token's row of k / v [T, num_kv_heads, head_dim].  So the scatter is one
+// contiguous row copy per token: one warp per token moves the K row and the V row
+// with 16-byte vector loads and stores.  The work is pure HBM traffic:
+// 2 * T * num_kv_heads * head_dim * 2 bytes read and the same written.
+#include "pa_device.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+__global__ void __launch_bounds__(256) reshape_and_cache_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int32_t* __restrict__ slot_mapping, int num_tokens,
+    int row_vecs, long long num_slots, int* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= num_tokens) return;
+  const long long slot = slot_mapping[warp];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (lane == 0) flag_error(err, PA_DEVERR_SLOT_RANGE);
+    return;
+  }
+  const uint4* ks = k + (long long)warp * row_vecs;
+  const uint4* vs = v + (long long)warp * row_vecs;
+  uint4* kd = k_cache + slot * row_vecs;
+  uint4* vd = v_cache + slot * row_vecs;
+  for (int i = lane; i < row_vecs; i += 32) {
+    const uint4 a = __ldg(ks + i);
+    const uint4 b = __ldg(vs + i);
+    kd[i] = a;
+    vd[i] = b;
+  }
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cache,
+                                          void* v_cache, const int32_t* slot_mapping,
+                                          int num_tokens, int num_kv_heads, int head_dim,
+                                          int num_blocks, int block_size, pa_dtype dtype,
+                                          void* stream) {
+  pa::set_launch_count(0);
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+      block_size <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 128 || (block_size != 16 && block_size != 32)) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  const uintptr_t al = (uintptr_t)k | (uintptr_t)v | (uintptr_t)k_cache | (uintptr_t)v_cache;
+  if (al & 15) return PA_ERR_INVALID_ARG;  // 16-byte vector access
+  int* err = pa::device_error_flag();
+  if (!err) return PA_ERR_CUDA;
+  const int row_vecs = num_kv_heads * head_dim * 2 / 16;
+  const int threads = 256;
+  const int blocks = (int)(((long long)num_tokens * 32 + threads - 1) / threads);
+  pa::reshape_and_cache_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, num_tokens, row_vecs,
+      (long long)num_blocks * block_size, err);
+  const pa_status st = pa::check_launch();
+  if (st == PA_OK) pa::set_launch_count(1);
+  return st;
+}

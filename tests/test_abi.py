@@ -1,0 +1,113 @@
+"""C-ABI checks that need no GPU: the library builds and loads, it exports every
+entry point ``include/pagedattn.h`` declares, and host-side validation returns
+the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def palib():
+    from paged_kv_cache_332_b200 import build
+    build.build()
+    import paged_kv_cache_332_b200 as pa
+    return pa
+
+
+def test_header_declares_the_hot_path():
+    syms = declared_symbols()
+    for s in ("pa_reshape_and_cache", "pa_decode", "pa_chunked_prefill", "pa_decode_workspace_size",
+              "pa_get_device_error", "pa_status_string"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(palib):
+    L = ctypes.CDLL(palib.library_path)
+    missing = [s for s in declared_symbols() if not hasattr(L, s)]
+    assert not missing, missing
+    assert sorted(palib.EXPORTED_SYMBOLS) == declared_symbols()
+
+
+def test_only_pa_symbols_exported(palib):
+    # hidden visibility: nothing but the C ABI leaks out of the library
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", palib.library_path], capture_output=True,
+                         text=True).stdout
+    names = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert names and all(n.startswith("pa_") for n in names), names
+
+
+def test_status_strings(palib):
+    assert palib.pa_status_string(0) == "PA_OK"
+    assert palib.pa_status_string(3) == "PA_ERR_WORKSPACE_TOO_SMALL"
+    assert palib.pa_status_string(99) == "PA_ERR_UNKNOWN"
+
+
+def test_workspace_size_arithmetic(palib):
+    # one partition covers the sequence -> no scratch
+    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 0) == 0
+    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 512) == 0
+    # 8000 tokens at 512 per partition -> 16 partitions of (128 + 2) fp32 per (seq, q-head)
+    assert palib.pa_decode_workspace_size(64, 32, 128, 8000, 512) == 64 * 32 * 16 * 130 * 4
+    assert palib.pa_decode_workspace_size(32, 64, 128, 32768, 512) == 32 * 64 * 64 * 130 * 4
+    assert palib.pa_decode_workspace_size(2, 8, 128, 100, 16) == 2 * 8 * 7 * 130 * 4
+    assert palib.pa_chunked_prefill_workspace_size(4, 512, 64, 128, 8000) == 0
+
+
+def _raw(palib):
+    return palib.lib()
+
+
+def test_invalid_arguments_rejected_on_host(palib):
+    L = _raw(palib)
+    nul = None
+    # reshape_and_cache: unsupported head_dim / block_size / dtype, negative count
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 4, 8, 64, 16, 16, 0, nul) == 2
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 4, 8, 128, 16, 24, 0, nul) == 2
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 4, 8, 128, 16, 16, 7, nul) == 2
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, -1, 8, 128, 16, 16, 0, nul) == 1
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 4, 8, 128, 16, 16, 0, nul) == 1
+    assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 0, 8, 128, 16, 16, 0, nul) == 0
+    p = ctypes.c_void_p(4096)
+    args = dict(out=p, q=p, kc=p, vc=p, bt=p, mb=8, sl=p, B=2, Hq=8, Hkv=8, D=128, scale=0.1,
+                bs=16, N=16, maxlen=100, P=0, ws=None, wsb=0, dt=0, st=None)
+
+    def dec(**kw):
+        a = dict(args); a.update(kw)
+        return L.pa_decode(a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["mb"], a["sl"], a["B"],
+                           a["Hq"], a["Hkv"], a["D"], a["scale"], a["bs"], a["N"], a["maxlen"],
+                           a["P"], a["ws"], a["wsb"], a["dt"], a["st"])
+    assert dec(D=64) == 2                    # head_dim must be 128
+    assert dec(bs=8) == 2                    # block size 16 or 32
+    assert dec(Hq=12, Hkv=8) == 1            # Hq not a multiple of Hkv
+    assert dec(Hq=24, Hkv=8) == 2            # GQA group 3 not built
+    assert dec(Hq=128, Hkv=8) == 2           # GQA group 16 not built
+    assert dec(P=24) == 1                    # partition not a multiple of 16
+    assert dec(q=None) == 1                  # null pointer
+    assert dec(q=ctypes.c_void_p(4100)) == 1  # misaligned
+    assert dec(dt=3) == 2
+    assert dec(B=0) == 0                     # nothing to do
+    assert dec(maxlen=8000, P=512) == 3      # needs a workspace
+    assert dec(maxlen=8000, P=512, ws=p, wsb=100) == 3
+
+
+def test_product_package_does_not_touch_oracle():
+    # the product path never imports the oracle
+    pkg = os.path.join(ROOT, "paged_kv_cache_332_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "dense_attention" not in text, f

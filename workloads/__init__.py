@@ -183,7 +183,8 @@ def make_batch(name: str, *, seq_lens: List[int], q_lens: Optional[List[int]] = 
                num_q_heads: int, num_kv_heads: int, block_size: int, num_blocks: int,
                dtype: torch.dtype, seed: int, device="cpu",
                shared_groups: Optional[List[List[int]]] = None,
-               shared_prefix_tokens: int = 0, head_dim: int = HEAD_DIM) -> PagedBatch:
+               shared_prefix_tokens: int = 0, head_dim: int = HEAD_DIM,
+               prefill: Optional[bool] = None) -> PagedBatch:
     """Build a batch.  ``seq_lens`` are final context lengths (after this
     step's append); ``q_lens`` are the tokens appended this step per
     sequence (1 for decode, the chunk length for chunked prefill).
@@ -192,6 +193,10 @@ def make_batch(name: str, *, seq_lens: List[int], q_lens: Optional[List[int]] = 
     q -> new K -> new V (torch generator seeded with ``seed``).  Every cache
     slot, used or not, holds an N(0,1) value; this step's tokens are then
     written by ``reshape_and_cache`` from ``k_new``/``v_new``.
+
+    A decode batch (every q_len <= 1, unless ``prefill`` says otherwise) has one
+    query row per sequence, also for empty sequences; a prefill batch has one
+    row per chunk token and a ``query_start_loc``.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     B = len(seq_lens)
@@ -208,17 +213,17 @@ def make_batch(name: str, *, seq_lens: List[int], q_lens: Optional[List[int]] = 
     T = len(slots)
     qsl = np.zeros(B + 1, dtype=np.int32)
     qsl[1:] = np.cumsum(q_lens)
+    is_prefill = any(ql > 1 for ql in q_lens) if prefill is None else prefill
 
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     cshape = (num_blocks, block_size, num_kv_heads, head_dim)
     k_cache = _randn(cshape, dtype, gen, device)
     v_cache = _randn(cshape, dtype, gen, device)
-    nq = int(qsl[-1])
+    nq = int(qsl[-1]) if is_prefill else B
     q = _randn((nq, num_q_heads, head_dim), dtype, gen, device)
     k_new = _randn((T, num_kv_heads, head_dim), dtype, gen, device)
     v_new = _randn((T, num_kv_heads, head_dim), dtype, gen, device)
-    is_prefill = any(ql != 1 for ql in q_lens)
     return PagedBatch(
         name=name, dtype=dtype, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
         head_dim=head_dim, block_size=block_size, num_blocks=num_blocks,
