@@ -22,7 +22,8 @@
  *    sequence s.  Entries past a sequence's last block are never read.
  *  - A slot is physical_block * block_size + offset_in_block.
  *  - GQA: q-heads [g*G, (g+1)*G) use kv-head g, with G = num_q_heads / num_kv_heads.
- *  - Supported: head_dim 128, block_size 16 or 32, G in {1, 2, 4, 8}, fp16 / bf16.
+ *  - Supported: head_dim 128, block_size 16 or 32, G in {1, 2, 4, 8}, fp16 / bf16,
+ *    up to 4096 sequences per decode call.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and never synchronise the host.  The library allocates no device memory
  *    on any call; scratch space comes from the caller (`workspace`).
@@ -113,7 +114,8 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   seq_lens      int32 [num_seqs] (device): tokens of each sequence, 0 gives zeros
  *   max_seq_len   host-side upper bound of seq_lens; sizes the grid and the
  *                 partition count.  A longer sequence sets PA_DEVERR_SEQ_TOO_LONG.
- *   partition_size  split-K partition in tokens (multiple of 16), 0 = library choice.
+ *   partition_size  split-K partition in tokens (multiple of 16, at most 2048),
+ *                 0 = library choice (512).
  *                 Each (sequence, kv-head, partition) is one work item; sequences
  *                 longer than one partition are merged by a log-sum-exp pass.
  *   workspace     device scratch of at least pa_decode_workspace_size(...) bytes

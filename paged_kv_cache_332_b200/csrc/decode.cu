@@ -9,30 +9,31 @@
 // For sequence s and q-head qh (kv-head h = qh / G):
 //   out[s, qh] = sum_j softmax_j(scale * q[s, qh] . K[s, h, j]) V[s, h, j],  j < seq_len[s].
 //
-// Design on B200 (the page's own kernel tricks — block-table entries in shared
-// memory, coalesced in-block reads, prefetch of the next block — kept where they
-// still pay):
-//  * Work item = (sequence, kv-head, partition of `P` tokens).  A persistent grid of
-//    one CTA per SM walks the items round-robin, so the KV stream never drains
-//    between items.
-//  * One producer warp stages each item's block-table entries in shared memory
-//    (one coalesced load per 32 tiles) and issues one 4-D TMA copy per 16-token tile
-//    of K and of V (a tile = 16 rows x 256 B of one kv-head inside one physical
-//    block) into an NSTAGE-deep ring of shared-memory stages guarded by mbarriers.
-//  * Consumer warps share each K/V tile across the G q-heads of the kv-head (GQA).
-//    For q.k, 8 lanes split one token's 128 dims (16 each, two 16-byte shared-memory
-//    reads); a warp-shuffle halving exchange sums up to 4 heads at once, leaving every
-//    lane with one (token, head) logit.  Each warp keeps its own online softmax
-//    (running max m, sum l, fp32 accumulator) over its slice of every stage;
-//    p.V uses lanes over head_dim (4 dims per lane).
-//  * At the end of an item the warps' states are merged in shared memory.  A
-//    sequence that fits one partition writes `out` directly; longer ones write the
-//    normalised partial (o, m, l) to the caller's workspace and a log-sum-exp pass
-//    (lse_reduce_kernel) merges the partitions.
-//  * Logits are kept in the log2 domain (q pre-scaled by scale*log2 e) so the
-//    exponentials are single ex2 instructions.
-// Every wait is bounded; bad table entries or lengths never fault (they are
-// skipped and flagged).
+// Design on B200.  The page's kernel tricks (block-table entries in shared memory,
+// coalesced in-block reads, prefetching the next block) are kept where they pay:
+//  * Work item = (sequence, partition of P tokens, pair of kv-heads).  A persistent grid
+//    of one CTA per SM walks a fixed item order round-robin: every full-size partition
+//    first, then each sequence's last (partial) partition, largest first, so the tail of
+//    the launch is made of the smallest items.
+//  * Tile = 16 consecutive tokens of the item's kv-heads inside one physical block: one
+//    4-D TMA copy of K and one of V (16 rows of HB*256 contiguous bytes each).  A staging
+//    warp runs up to four items ahead: it copies each item's block-table entries into
+//    shared memory (one coalesced read per 32 entries) and starts the TMA copy of the
+//    item's q rows.  A producer warp gives every ring of tile slots its own lane; each
+//    lane polls its ring without blocking and issues the next tile's copies as soon as a
+//    slot frees, so several tiles are requested at once and the copies of the next tiles
+//    are in flight while the current ones are computed.
+//  * Consumer warps share each tile across the G q-heads of a kv-head (GQA; up to four
+//    heads per warp).  q.k: 8 lanes split a token's 128 dims (16 each, two 16-byte
+//    shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving exchange sums
+//    four heads at once.  Each warp keeps its own online softmax (running max m, sum l,
+//    fp32 accumulator over 4 dims per lane).
+//  * When a warp finishes its share of an item it parks (m, l, acc) in shared memory;
+//    the last warp to finish merges the item (no CTA-wide barrier).  A sequence that fits
+//    one partition writes `out`; longer ones write the normalised partial (o, m, l) to the
+//    caller's workspace, merged by a log-sum-exp pass (lse_reduce_kernel).
+//  * Logits live in the log2 domain (q pre-scaled by scale*log2 e): one ex2 each.
+// Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
 #include <algorithm>
 
 #include "pa_device.cuh"
@@ -42,65 +43,76 @@ namespace pa {
 
 struct DecodeArgs {
   void* out;
-  const void* q;
   const int32_t* block_tables;
   const int32_t* seq_lens;
   float* part_o;   // [B, Hq, max_parts, 128]
-  float* part_ml;  // [B, Hq, max_parts, 2]   (running max in log2 units, sum)
+  float* part_ml;  // [B, Hq, max_parts, 2]   (max in log2 units, sum)
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
-  int part_size, max_parts, seq_cap, flag_cta;
+  int part_size, max_parts, seq_cap, slots_per_ring;
   float qscale;  // scale * log2(e)
 };
 
 constexpr int kD = 128;
 constexpr int kTileTok = 16;
-constexpr int kTileBytes = kTileTok * kD * 2;  // one TMA box: 16 rows x 256 B
+constexpr int kRowBytes = kD * 2;   // one token of one kv-head
+constexpr int kQSlots = 4;          // items staged ahead
+constexpr int kMergeSlots = 2;      // items being merged
+constexpr int kMaxSlots = 32;
+constexpr int kMaxTilesPerItem = 128;  // partition <= 2048 tokens
+constexpr int kSortBuckets = 128;
 
-template <int G_, int NCW_>
+template <int G_, int HB_, int NCW_>
 struct DecodeCfg {
   static constexpr int G = G_;
-  static constexpr int NCW = NCW_;                     // consumer warps
-  static constexpr int GW = G < 4 ? G : 4;             // heads per warp
-  static constexpr int HG = G / GW;                    // head groups
-  static constexpr int TGS = NCW / HG;                 // token groups
-  static constexpr int TPW = 8;                        // tokens per warp per stage
-  static constexpr int TOK_STAGE = TPW * TGS;
-  static constexpr int TPS = TOK_STAGE / kTileTok;     // tiles per stage
-  static constexpr int NPASS = TPW / 4;
-  static constexpr int STAGE_BYTES = TPS * kTileBytes;  // K part; V part follows
-  static constexpr int NSTAGE = (128 * 1024) / (2 * STAGE_BYTES);
-  static constexpr int THREADS = (NCW + 1) * 32;
+  static constexpr int HB = HB_;                   // kv-heads per item (and per TMA box)
+  static constexpr int NCW = NCW_;                 // consumer warps
+  static constexpr int GW = G < 4 ? G : 4;         // q-heads per warp
+  static constexpr int HG = G / GW;                // warps per kv-head per token group
+  static constexpr int WPT = HB * HG;              // warps reading one tile
+  static constexpr int TGS = NCW / WPT;            // rings (token groups)
+  static constexpr int THREADS = (NCW + 2) * 32;   // + producer warp + staging warp
+  static constexpr int WARP_PROD = NCW;
+  static constexpr int WARP_STAGE = NCW + 1;
   static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);
-  // shared-memory carve-up (bytes)
-  static constexpr int OFF_BAR = NSTAGE * 2 * STAGE_BYTES;
-  static constexpr int OFF_TBL = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int OFF_MISC = OFF_TBL + 32 * 4;  // abort flag (+pad)
-  static constexpr int OFF_P = OFF_MISC + 16;
-  static constexpr int OFF_A = OFF_P + NCW * TPW * GW * 4;
-  static constexpr int OFF_RACC = OFF_A + NCW * GW * 4;
-  static constexpr int OFF_RM = OFF_RACC + NCW * GW * kD * 4;
-  static constexpr int OFF_RL = OFF_RM + NCW * GW * 4;
-  static constexpr int OFF_SEQ = OFF_RL + NCW * GW * 4;  // int seq_start[B+1], int len[B]
-  static_assert(TOK_STAGE % kTileTok == 0, "stage must hold whole tiles");
-  static_assert(32 % TPS == 0, "table chunk must hold whole stages");
-  static_assert(NSTAGE >= 2, "need a pipeline");
-  static_assert(OFF_RACC % 16 == 0, "float4 alignment");
+  static constexpr int TILE_BYTES = kTileTok * HB * kRowBytes;  // K (or V) of a tile
+  static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
+  static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of an item
+  // shared-memory carve-up (bytes); the tile ring comes last (runtime size)
+  static constexpr int OFF_FULL = 0;
+  static constexpr int OFF_EMPTY = OFF_FULL + kMaxSlots * 8;
+  static constexpr int OFF_QFULL = OFF_EMPTY + kMaxSlots * 8;
+  static constexpr int OFF_QEMPTY = OFF_QFULL + kQSlots * 8;
+  static constexpr int OFF_TFULL = OFF_QEMPTY + kQSlots * 8;
+  static constexpr int OFF_TEMPTY = OFF_TFULL + kQSlots * 8;
+  static constexpr int OFF_MFREE = OFF_TEMPTY + kQSlots * 8;
+  static constexpr int OFF_MCNT = OFF_MFREE + kMergeSlots * 8;
+  static constexpr int OFF_ABORT = OFF_MCNT + kMergeSlots * 4;
+  static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
+  static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerItem * 4;
+  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;           // p pairs per warp
+  static constexpr int OFF_A = OFF_P + NCW * kTileTok * GW * 8;    // alpha per warp
+  static constexpr int OFF_RACC = ((OFF_A + NCW * GW * 4 + 15) / 16) * 16;
+  static constexpr int OFF_RM = OFF_RACC + kMergeSlots * NCW * GW * kD * 4;
+  static constexpr int OFF_RL = OFF_RM + kMergeSlots * NCW * GW * 4;
+  static constexpr int OFF_SORT = OFF_RL + kMergeSlots * NCW * GW * 4;
+  static constexpr int OFF_SEQ = OFF_SORT + kSortBuckets * 4;      // 3 int arrays
+  static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0 && OFF_RACC % 16 == 0, "alignment");
+  static_assert(TGS >= 1 && NCW % WPT == 0 && TGS <= 32, "warp split");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
-
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
 // Bounded wait that turns into a no-op once any warp of the CTA gave up.
-__device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int* err) {
+__device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err) {
   if (*abort_flag) return;
   if (!mbar_wait(bar, parity, err)) *abort_flag = 1;
 }
 
-// Sum a warp's per-lane partial dot products over each 8-lane token group for
-// GW heads at once.  Returns the full sum of head hh(lane):
+// Sum per-lane partial dot products over each 8-lane token group for GW heads at
+// once (halving exchange).  Returns the sum for head hh(lane):
 //   GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;  GW=1: hh = 0.
 template <int GW>
 __device__ __forceinline__ float reduce_heads(const float (&d)[GW], int lane);
@@ -145,66 +157,82 @@ __device__ __forceinline__ int head_of_lane(int lane) {
   return GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)) : (GW == 2 ? ((lane >> 2) & 1) : 0);
 }
 
-// Unpack 8 packed 16-bit values into fp32.
-template <typename T>
-__device__ __forceinline__ void unpack8(const uint4& w, float* f) {
-  float2 a = Elem<T>::unpack2(w.x), b = Elem<T>::unpack2(w.y);
-  float2 c = Elem<T>::unpack2(w.z), d = Elem<T>::unpack2(w.w);
-  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-  f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
-}
-
-// Item index -> (sequence, partition, kv-head).  Items are ordered
-// (sequence, partition, kv-head); seq_start holds each sequence's first
-// (sequence, partition) pair.
-__device__ __forceinline__ void decode_item(int item, int Hkv, const int* seq_start, int B, int& s,
-                                            int& p, int& h) {
-  const int sp = item / Hkv;
-  h = item - sp * Hkv;
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (seq_start[mid] <= sp) lo = mid; else hi = mid - 1;
+// The launch's item order: item i -> (sequence s, partition p, kv-head group hp).
+struct Schedule {
+  const int* fstart;  // [B+1] prefix of full partitions per sequence
+  const int* slen;    // [B]   clamped lengths
+  const int* order;   // [B]   sequences by size of their last partition, largest first
+  int B, NHP, P, nfull;
+  __device__ __forceinline__ void item(int i, int& s, int& p, int& hp) const {
+    const int sp = i / NHP;
+    hp = i - sp * NHP;
+    if (sp < nfull) {
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (fstart[mid] <= sp) lo = mid; else hi = mid - 1;
+      }
+      s = lo;
+      p = sp - fstart[lo];
+    } else {
+      s = order[sp - nfull];
+      p = fstart[s + 1] - fstart[s];  // the last partition
+    }
   }
-  s = lo;
-  p = sp - seq_start[lo];
-}
+  __device__ __forceinline__ int ntiles(int s, int p) const {
+    const int tok0 = p * P;
+    return cdiv(max(min(slen[s], tok0 + P) - tok0, 0), kTileTok);
+  }
+};
 
-template <typename T, int G, int NCW>
-__global__ void __launch_bounds__(DecodeCfg<G, NCW>::THREADS, 1)
+template <typename T, int G, int HB, int NCW>
+__global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
-  using C = DecodeCfg<G, NCW>;
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
+  using C = DecodeCfg<G, HB, NCW>;
+  constexpr int GW = C::GW;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* empty = full + C::NSTAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + C::OFF_QFULL);
+  uint64_t* qempty = reinterpret_cast<uint64_t*>(smem + C::OFF_QEMPTY);
+  uint64_t* tfull = reinterpret_cast<uint64_t*>(smem + C::OFF_TFULL);
+  uint64_t* tempty = reinterpret_cast<uint64_t*>(smem + C::OFF_TEMPTY);
+  uint64_t* mfree = reinterpret_cast<uint64_t*>(smem + C::OFF_MFREE);
+  int* mcnt = reinterpret_cast<int*>(smem + C::OFF_MCNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
   int* tbl = reinterpret_cast<int*>(smem + C::OFF_TBL);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
-  float* pbuf = reinterpret_cast<float*>(smem + C::OFF_P);
+  uint8_t* qbuf = smem + C::OFF_Q;
+  float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
   float* abuf = reinterpret_cast<float*>(smem + C::OFF_A);
   float* racc = reinterpret_cast<float*>(smem + C::OFF_RACC);
   float* rm = reinterpret_cast<float*>(smem + C::OFF_RM);
   float* rl = reinterpret_cast<float*>(smem + C::OFF_RL);
-  int* seq_start = reinterpret_cast<int*>(smem + C::OFF_SEQ);
-  int* seq_len = seq_start + a.num_seqs + 1;
+  int* cursor = reinterpret_cast<int*>(smem + C::OFF_SORT);
+  const int B = a.num_seqs;
+  int* fstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);
+  int* slen = fstart + B + 1;
+  int* order = slen + B;
+  uint8_t* ring = smem + ((C::OFF_SEQ + (3 * B + 1) * 4 + 1023) / 1024) * 1024;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int B = a.num_seqs;
-  const int Hkv = a.num_kv_heads;
   const int P = a.part_size;
+  const int nsw = a.slots_per_ring;
 
-  // ---- per-sequence partition counts and their prefix sum (warp 0)
+  // ---- schedule: clamped lengths, full-partition prefix, last partitions by size
   if (warp == 0) {
+    for (int b = lane; b < kSortBuckets; b += 32) cursor[b] = 0;
     const int per = (B + 31) / 32;
     const int lo = min(B, lane * per), hi = min(B, lo + per);
     int sum = 0;
     for (int s = lo; s < hi; ++s) {
       const int raw = a.seq_lens[s];
       const int L = clamp_len(raw, a.seq_cap);
-      if (raw != L && blockIdx.x == a.flag_cta) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
-      seq_len[s] = L;
-      sum += max(1, cdiv(L, P));
+      if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
+      slen[s] = L;
+      sum += max(1, cdiv(L, P)) - 1;
     }
     int incl = sum;
 #pragma unroll
@@ -214,232 +242,356 @@ __global__ void __launch_bounds__(DecodeCfg<G, NCW>::THREADS, 1)
     }
     int run = incl - sum;
     for (int s = lo; s < hi; ++s) {
-      seq_start[s] = run;
-      run += max(1, cdiv(seq_len[s], P));
+      fstart[s] = run;
+      run += max(1, cdiv(slen[s], P)) - 1;
     }
-    if (lane == 31) seq_start[B] = incl;
+    if (lane == 31) fstart[B] = incl;
+    __syncwarp();
+    // stable counting sort of the sequences by their last partition, largest first
+    auto bucket = [&](int s) {
+      const int L = slen[s];
+      const int r = L - (max(1, cdiv(L, P)) - 1) * P;  // 0..P
+      return (int)(((long long)(P - r) * kSortBuckets) / (P + 1));
+    };
+    for (int base = 0; base < B; base += 32) {
+      const int s = base + lane;
+      if (s < B) atomicAdd(&cursor[bucket(s)], 1);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int run2 = 0;
+      for (int b = 0; b < kSortBuckets; ++b) {
+        const int c = cursor[b];
+        cursor[b] = run2;
+        run2 += c;
+      }
+    }
+    __syncwarp();
+    for (int base = 0; base < B; base += 32) {
+      const int s = base + lane;
+      const int bk = s < B ? bucket(s) : kSortBuckets + lane;
+      const unsigned same = __match_any_sync(0xffffffffu, bk);
+      const int rank = __popc(same & ((1u << lane) - 1));
+      if (s < B) order[cursor[bk] + rank] = s;
+      __syncwarp();
+      if (s < B && rank == 0) cursor[bk] += __popc(same);
+      __syncwarp();
+    }
   }
   if (threadIdx.x == 32) {
-    for (int i = 0; i < C::NSTAGE; ++i) {
+    for (int i = 0; i < C::TGS * nsw; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], C::NCW);
+      mbar_init(&empty[i], C::WPT);
+    }
+    for (int i = 0; i < kQSlots; ++i) {
+      mbar_init(&qfull[i], 1);
+      mbar_init(&qempty[i], C::NCW);
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], C::TGS);
+    }
+    for (int i = 0; i < kMergeSlots; ++i) {
+      mbar_init(&mfree[i], 1);
+      mcnt[i] = 0;
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  const int total = seq_start[B] * Hkv;
+  const int NHP = a.num_kv_heads / HB;
+  Schedule sch{fstart, slen, order, B, NHP, P, fstart[B]};
+  const int total = (sch.nfull + B) * NHP;
 
-  if (warp == C::NCW) {
-    // ================= producer warp: block-table staging + TMA =================
-    if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-    }
-    int st = 0;
-    uint32_t ph = 0;
-    const int bs_mask = (1 << a.log2_bs) - 1;
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      int s, p, h;
-      decode_item(item, Hkv, seq_start, B, s, p, h);
-      const int tok0 = p * P;
-      const int tok1 = min(seq_len[s], tok0 + P);
-      const int ntile = cdiv(max(tok1 - tok0, 0), kTileTok);
+  if (warp == C::WARP_STAGE) {
+    // ============ staging warp: block-table entries + q rows, items ahead ============
+    if (lane == 0) prefetch_tmap(&tmQ);
+    int k = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+      const int qs = k % kQSlots;
+      const uint32_t par = ((k / kQSlots) & 1) ^ 1;
+      wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read item k-4's q
+      wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // producer issued its tiles
+      int s, p, hp;
+      sch.item(item, s, p, hp);
+      const int ntile = sch.ntiles(s, p);
       const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
-      for (int c = 0; c < ntile; c += 32) {
-        int id = -1;
-        if (c + lane < ntile) {
-          const int pos = tok0 + (c + lane) * kTileTok;
-          id = __ldg(trow + (pos >> a.log2_bs));
+      const int tok0 = p * P;
+      int ids[kMaxTilesPerItem / 32];
+#pragma unroll
+      for (int j = 0; j < kMaxTilesPerItem / 32; ++j) {
+        const int t = j * 32 + lane;
+        ids[j] = t < ntile ? __ldg(trow + ((tok0 + t * kTileTok) >> a.log2_bs)) : -1;
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxTilesPerItem / 32; ++j) {
+        const int t = j * 32 + lane;
+        if (t < ntile) {
+          int id = ids[j];
           if ((unsigned)id >= (unsigned)a.num_blocks) {
             flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
             id = -1;
           }
+          tbl[qs * kMaxTilesPerItem + t] = id;
         }
-        __syncwarp();
-        tbl[lane] = id;
-        __syncwarp();
-        if (lane == 0) {
-          const int nchunk = min(32, ntile - c);
-          for (int j = 0; j < nchunk; j += C::TPS) {
-            wait_or_abort(&empty[st], ph ^ 1, abort_flag, a.err);
-            const int nv = min(C::TPS, nchunk - j);
-            uint32_t bytes = 0;
-            if (!*abort_flag)
-              for (int t = 0; t < nv; ++t) bytes += tbl[j + t] >= 0 ? 2 * kTileBytes : 0;
-            mbar_arrive_expect_tx(&full[st], bytes);
-            if (bytes) {
-              uint8_t* kd = smem + st * 2 * C::STAGE_BYTES;
-              for (int t = 0; t < nv; ++t) {
-                const int bid = tbl[j + t];
-                if (bid < 0) continue;
-                const int row = (tok0 + (c + j + t) * kTileTok) & bs_mask;
-                tma_load_4d(kd + t * kTileBytes, &tmK, 0, h, row, bid, &full[st]);
-                tma_load_4d(kd + C::STAGE_BYTES + t * kTileBytes, &tmV, 0, h, row, bid, &full[st]);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const bool ok = !*abort_flag;
+        mbar_arrive_expect_tx(&qfull[qs], ok ? C::QBYTES : 0);
+        if (ok) tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HB * G, s, &qfull[qs]);
+        mbar_arrive(&tfull[qs]);
+      }
+    }
+    return;
+  }
+
+  if (warp == C::WARP_PROD) {
+    // ============ producer warp: lane r feeds ring r ============
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    const int r = lane;
+    int k = 0, item = blockIdx.x, s = 0, p = 0, hp = 0, ntile = 0, t = r, pos = 0;
+    bool done = (r >= C::TGS) || item >= total;
+    bool entered = false;
+    if (!done) {
+      sch.item(item, s, p, hp);
+      ntile = sch.ntiles(s, p);
+    }
+    const int bs_mask = (1 << a.log2_bs) - 1;
+    unsigned long long t_idle = 0;
+    while (!__all_sync(0xffffffffu, done)) {
+      bool progressed = false;
+      if (!done) {
+        if (*abort_flag) {
+          done = true;
+        } else {
+          if (!entered && mbar_test_wait(&tfull[k % kQSlots], (k / kQSlots) & 1)) entered = true;
+          if (entered && t < ntile) {
+            const int slot = r * nsw + pos % nsw;
+            if (mbar_test_wait(&empty[slot], ((pos / nsw) & 1) ^ 1)) {
+              const int bid = tbl[(k % kQSlots) * kMaxTilesPerItem + t];
+              mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
+              if (bid >= 0) {
+                const int row = (p * P + t * kTileTok) & bs_mask;
+                uint8_t* dst = ring + slot * C::SLOT_BYTES;
+                tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
+                tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
               }
+              ++pos;
+              t += C::TGS;
+              progressed = true;
             }
-            if (++st == C::NSTAGE) { st = 0; ph ^= 1; }
           }
+          if (entered && t >= ntile) {  // this ring's share of the item is issued
+            mbar_arrive(&tempty[k % kQSlots]);
+            ++k;
+            item += gridDim.x;
+            entered = false;
+            t = r;
+            progressed = true;
+            if (item >= total) {
+              done = true;
+            } else {
+              sch.item(item, s, p, hp);
+              ntile = sch.ntiles(s, p);
+            }
+          }
+        }
+      }
+      if (__any_sync(0xffffffffu, progressed)) {
+        t_idle = 0;
+      } else {
+        const unsigned long long now = globaltimer_ns();
+        if (t_idle == 0) {
+          t_idle = now;
+        } else if (now - t_idle > kWaitLimitNs) {
+          if (lane == 0) {
+            flag_error(a.err, PA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          done = true;
         }
       }
     }
     return;
   }
 
-  // ======================= consumer warps =======================
-  constexpr int GW = C::GW;
-  const int hg = warp % C::HG;
-  const int tg = warp / C::HG;
+  // ===================== consumer warps =====================
+  const int kvsub = warp % HB;
+  const int hg = (warp / HB) % C::HG;
+  const int tg = warp / C::WPT;
   const int sub = lane & 7;
   const int tp = lane >> 3;
   const int hh = head_of_lane<GW>(lane);
   const bool writer = (lane & C::DUPMASK) == 0;
-  const int wt0 = tg * C::TPW;
-  float* pw = pbuf + warp * C::TPW * GW;
-  int st = 0;
-  uint32_t ph = 0;
+  float2* pw = pbuf + warp * kTileTok * GW;
+  int mypos = 0;
+  int k = 0;
 
-  for (int item = blockIdx.x; item < total; item += gridDim.x) {
-    int s, p, h;
-    decode_item(item, Hkv, seq_start, B, s, p, h);
+  for (int item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+    int s, p, hp;
+    sch.item(item, s, p, hp);
     const int tok0 = p * P;
-    const int tok1 = min(seq_len[s], tok0 + P);
+    const int tok1 = min(slen[s], tok0 + P);
     const int ntile = cdiv(max(tok1 - tok0, 0), kTileTok);
-    const int qh0 = h * G + hg * GW;
+    const int qs = k % kQSlots;
 
-    // q for this warp's GW heads: dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8)
-    float qf[GW][16];
+    // q of this warp's GW heads, dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8),
+    // as (even, odd) pairs, pre-scaled into the log2 domain
+    float2 q2[GW][8];
+    wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
     {
-      const T* qb = static_cast<const T*>(a.q) + ((long long)s * a.num_q_heads + qh0) * kD;
+      const uint8_t* qb = qbuf + qs * C::QBYTES + (kvsub * G + hg * GW) * kRowBytes;
 #pragma unroll
       for (int j = 0; j < GW; ++j) {
-        const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(qb + j * kD + 8 * sub));
-        const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(qb + j * kD + 64 + 8 * sub));
-        unpack8<T>(w0, qf[j]);
-        unpack8<T>(w1, qf[j] + 8);
+        const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + 128 + sub * 16);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) qf[j][i] *= a.qscale;
+        for (int i = 0; i < 8; ++i) {
+          const float2 f = Elem<T>::unpack2(w[i]);
+          q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
+        }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qempty[qs]);
     float m = -INFINITY, l = 0.f;
-    float acc[GW][4];
+    float2 acc[GW][2];
 #pragma unroll
-    for (int j = 0; j < GW; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+    for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
 
-    for (int j0 = 0; j0 < ntile; j0 += C::TPS) {
-      wait_or_abort(&full[st], ph, abort_flag, a.err);
-      const int valid = min(C::TOK_STAGE, tok1 - (tok0 + j0 * kTileTok));
-      const int nv = min(max(valid - wt0, 0), C::TPW);
-      if (nv > 0) {
-        const uint8_t* Ks = smem + st * 2 * C::STAGE_BYTES;
-        const uint8_t* Vs = Ks + C::STAGE_BYTES;
-        float x[C::NPASS];
+    for (int t = tg; t < ntile; t += C::TGS) {
+      const int slot = tg * nsw + mypos % nsw;
+      const uint32_t par = (mypos / nsw) & 1;
+      ++mypos;
+      wait_or_abort(&full[slot], par, abort_flag, a.err);
+      const int nvalid = min(kTileTok, tok1 - (tok0 + t * kTileTok));
+      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + kvsub * kRowBytes;
+      const uint8_t* Vs = Ks + C::TILE_BYTES;
+
+      // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
+      float x[4];
 #pragma unroll
-        for (int ps = 0; ps < C::NPASS; ++ps) {
-          const int r = wt0 + ps * 4 + tp;
-          const uint4 w0 = *reinterpret_cast<const uint4*>(Ks + r * 256 + sub * 16);
-          const uint4 w1 = *reinterpret_cast<const uint4*>(Ks + r * 256 + 128 + sub * 16);
-          float kf[16];
-          unpack8<T>(w0, kf);
-          unpack8<T>(w1, kf + 8);
-          float d[GW];
+      for (int ps = 0; ps < 4; ++ps) {
+        const int rr = ps * 4 + tp;
+        const uint8_t* kr = Ks + rr * (HB * kRowBytes);
+        const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        float2 kf[8];
 #pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            float e0 = 0.f, e1 = 0.f;
+        for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(w[i]);
+        float d[GW];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              e0 = fmaf(qf[jj][i], kf[i], e0);
-              e1 = fmaf(qf[jj][i + 1], kf[i + 1], e1);
-            }
-            d[jj] = e0 + e1;
-          }
-          const float xv = reduce_heads<GW>(d, lane);
-          x[ps] = (ps * 4 + tp < nv) ? xv : -INFINITY;
+        for (int jj = 0; jj < GW; ++jj) {
+          float2 e = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
+          d[jj] = e.x + e.y;
         }
-        // online softmax over the warp's tokens of this stage, per head hh
-        float mx = x[0];
+        const float xv = reduce_heads<GW>(d, lane);
+        x[ps] = rr < nvalid ? xv : -INFINITY;
+      }
+      // ---- online softmax over the tile, per head hh
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m, mx);
+      const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
+      m = m_new;
+      float psum = 0.f;
 #pragma unroll
-        for (int ps = 1; ps < C::NPASS; ++ps) mx = fmaxf(mx, x[ps]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m, mx);
-        const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
-        m = m_new;
-        float psum = 0.f;
+      for (int ps = 0; ps < 4; ++ps) {
+        const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
+        psum += pv;
+        if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
+      }
+      l = l * alpha + psum;
+      if (writer && tp == 0) abuf[warp * GW + hh] = alpha;
+      __syncwarp();
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-        for (int ps = 0; ps < C::NPASS; ++ps) {
-          const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
-          psum += pv;
-          if (writer) pw[(ps * 4 + tp) * GW + hh] = pv;
+        for (int jj = 0; jj < GW; ++jj) {
+          const float al = abuf[warp * GW + jj];
+          const float2 a2 = make_float2(al, al);
+          acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
+          acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
         }
-        l = l * alpha + psum;
-        if (writer && tp == 0) abuf[warp * GW + hh] = alpha;
-        __syncwarp();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      }
+      // ---- p.V: lane owns dims [4*lane, 4*lane+4)
+      auto pv_row = [&](int tt) {
+        const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
+        const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
 #pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            const float al = abuf[warp * GW + jj];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[jj][i] *= al;
-          }
+        for (int jj = 0; jj < GW; ++jj) {
+          const float2 pp = pw[tt * GW + jj];
+          acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
+          acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
         }
-        for (int t = 0; t < nv; ++t) {
-          const uint2 vw = *reinterpret_cast<const uint2*>(Vs + (wt0 + t) * 256 + lane * 8);
-          const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
-          float pj[GW];
+      };
+      if (nvalid == kTileTok) {
 #pragma unroll
-          for (int jj = 0; jj < GW; ++jj) pj[jj] = pw[t * GW + jj];
-#pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            acc[jj][0] = fmaf(pj[jj], v01.x, acc[jj][0]);
-            acc[jj][1] = fmaf(pj[jj], v01.y, acc[jj][1]);
-            acc[jj][2] = fmaf(pj[jj], v23.x, acc[jj][2]);
-            acc[jj][3] = fmaf(pj[jj], v23.y, acc[jj][3]);
-          }
-        }
+        for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
+      } else {
+        for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      if (++st == C::NSTAGE) { st = 0; ph ^= 1; }
+      if (lane == 0) mbar_arrive(&empty[slot]);
     }
 
-    // ---- merge the warps' (m, l, acc) and write
+    // ---- park (m, l, acc); the last warp of the item merges and writes
     l += __shfl_xor_sync(0xffffffffu, l, 8);
     l += __shfl_xor_sync(0xffffffffu, l, 16);
+    const int ms = k % kMergeSlots;
+    wait_or_abort(&mfree[ms], ((k / kMergeSlots) & 1) ^ 1, abort_flag, a.err);
+    float* racc_s = racc + ms * (C::NCW * GW * kD);
+    float* rm_s = rm + ms * (C::NCW * GW);
+    float* rl_s = rl + ms * (C::NCW * GW);
 #pragma unroll
     for (int jj = 0; jj < GW; ++jj)
-      *reinterpret_cast<float4*>(racc + (warp * GW + jj) * kD + lane * 4) =
-          make_float4(acc[jj][0], acc[jj][1], acc[jj][2], acc[jj][3]);
+      *reinterpret_cast<float4*>(racc_s + (warp * GW + jj) * kD + lane * 4) =
+          make_float4(acc[jj][0].x, acc[jj][0].y, acc[jj][1].x, acc[jj][1].y);
     if (writer && tp == 0) {
-      rm[warp * GW + hh] = m;
-      rl[warp * GW + hh] = l;
+      rm_s[warp * GW + hh] = m;
+      rl_s[warp * GW + hh] = l;
     }
-    named_bar_sync(1, C::NCW * 32);
-    const int nparts = seq_start[s + 1] - seq_start[s];
-    for (int o = threadIdx.x; o < G * 32; o += C::NCW * 32) {
-      const int r = o >> 5;   // head within the kv group
-      const int c4 = o & 31;  // 4-dim chunk
-      const int g2 = r / GW, jj = r % GW;
+    __threadfence_block();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&mcnt[ms], 1) == C::NCW - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) continue;
+    __threadfence_block();
+    const int nparts = fstart[s + 1] - fstart[s] + 1;
+    // outputs: HB kv-heads x G q-heads x 32 chunks of 4 dims
+    for (int o = lane; o < HB * G * 32; o += 32) {
+      const int c4 = o & 31;
+      const int r = o >> 5;                // q-head within the item
+      const int kv = r / G, rg = r % G;    // kv-head within the pair, head in its group
+      const int g2 = rg / GW, jj = rg % GW;
       float M = -INFINITY;
 #pragma unroll
-      for (int t2 = 0; t2 < C::TGS; ++t2) M = fmaxf(M, rm[(t2 * C::HG + g2) * GW + jj]);
+      for (int t2 = 0; t2 < C::TGS; ++t2) {
+        const int w2 = (t2 * C::HG + g2) * HB + kv;
+        M = fmaxf(M, rm_s[w2 * GW + jj]);
+      }
       float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
       float den = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int t2 = 0; t2 < C::TGS; ++t2) {
-          const int w2 = t2 * C::HG + g2;
-          const float mw = rm[w2 * GW + jj];
+          const int w2 = (t2 * C::HG + g2) * HB + kv;
+          const float mw = rm_s[w2 * GW + jj];
           const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - M);
-          den += f * rl[w2 * GW + jj];
-          const float4 v = *reinterpret_cast<const float4*>(racc + (w2 * GW + jj) * kD + c4 * 4);
+          den += f * rl_s[w2 * GW + jj];
+          const float4 v = *reinterpret_cast<const float4*>(racc_s + (w2 * GW + jj) * kD + c4 * 4);
           num.x += f * v.x; num.y += f * v.y; num.z += f * v.z; num.w += f * v.w;
         }
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
-      const int qh = h * G + r;
+      const int qh = (hp * HB + kv) * G + rg;
       if (nparts == 1) {
         const uint32_t lo = Elem<T>::pack2(num.x * inv, num.y * inv);
         const uint32_t hi = Elem<T>::pack2(num.z * inv, num.w * inv);
@@ -452,7 +604,12 @@ __global__ void __launch_bounds__(DecodeCfg<G, NCW>::THREADS, 1)
         if (c4 == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(M, den);
       }
     }
-    named_bar_sync(1, C::NCW * 32);
+    __syncwarp();
+    if (lane == 0) {
+      mcnt[ms] = 0;
+      __threadfence_block();
+      mbar_arrive(&mfree[ms]);
+    }
   }
 }
 
@@ -468,6 +625,7 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
   const int n = max(1, cdiv(L, a.part_size));
   if (n <= 1) return;  // written by the decode kernel
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (long long)gw * a.max_parts;
+  // lane i holds partition i's (m, l) for the first 32 partitions
   float M = -INFINITY;
   for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
 #pragma unroll
@@ -475,7 +633,23 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
   float den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* po = a.part_o + (long long)gw * a.max_parts * kD + lane * 4;
-  for (int i = 0; i < n; ++i) {
+  int i = 0;
+  for (; i + 4 <= n; i += 4) {
+    float f[4];
+    float4 o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 v = ml[i + u];
+      f[u] = v.x == -INFINITY ? 0.f : fast_exp2(v.x - M) * v.y;
+      o[u] = *reinterpret_cast<const float4*>(po + (long long)(i + u) * kD);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      den += f[u];
+      num.x += f[u] * o[u].x; num.y += f[u] * o[u].y; num.z += f[u] * o[u].z; num.w += f[u] * o[u].w;
+    }
+  }
+  for (; i < n; ++i) {
     const float2 v = ml[i];
     const float f = v.x == -INFINITY ? 0.f : fast_exp2(v.x - M) * v.y;
     den += f;
@@ -489,32 +663,37 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
 }
 
 constexpr int kDefaultPartition = 512;
+constexpr int kMaxPartition = kMaxTilesPerItem * kTileTok;
 constexpr int kConsumerWarps = 8;
-constexpr int kMaxSeqs = 8192;
+constexpr int kMaxSeqs = 4096;
+constexpr int kMaxSmem = 227 * 1024;
 
 inline int choose_partition(int partition_size) {
   return partition_size > 0 ? partition_size : kDefaultPartition;
 }
 
-inline int num_parts_host(int max_seq_len, int P) {
-  return std::max(1, (max_seq_len + P - 1) / P);
-}
+inline int num_parts_host(int max_seq_len, int P) { return std::max(1, (max_seq_len + P - 1) / P); }
 
-template <typename T, int G>
-pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeArgs& a,
-                        cudaStream_t stream) {
-  using C = DecodeCfg<G, kConsumerWarps>;
-  const size_t smem = C::OFF_SEQ + (size_t)(2 * a.num_seqs + 1) * 4;
-  if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
-  auto kern = paged_decode_kernel<T, G, kConsumerWarps>;
+template <typename T, int G, int HB>
+pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
+                        DecodeArgs a, cudaStream_t stream) {
+  using C = DecodeCfg<G, HB, kConsumerWarps>;
+  const size_t ring_off = ((C::OFF_SEQ + (size_t)(3 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
+  if (ring_off + (size_t)2 * C::TGS * C::SLOT_BYTES > kMaxSmem) return PA_ERR_UNSUPPORTED;
+  int nsw = (int)((kMaxSmem - ring_off) / ((size_t)C::TGS * C::SLOT_BYTES));
+  nsw = std::min(nsw, kMaxSlots / C::TGS);
+  if (nsw < 2) return PA_ERR_UNSUPPORTED;
+  a.slots_per_ring = nsw;
+  const size_t smem = ring_off + (size_t)C::TGS * nsw * C::SLOT_BYTES;
+  auto kern = paged_decode_kernel<T, G, HB, kConsumerWarps>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
-  const long long items_max = (long long)a.num_seqs * a.num_kv_heads * a.max_parts;
+  const long long items_max = (long long)a.num_seqs * (a.num_kv_heads / HB) * a.max_parts;
   const int sms = num_sms();
   if (sms <= 0) return PA_ERR_CUDA;
   const int grid = (int)std::min<long long>(items_max, sms);
-  kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, a);
+  kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
   if (a.max_parts > 1) {
@@ -527,14 +706,14 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const De
   return PA_OK;
 }
 
-template <typename T>
+template <typename T, int HB>
 pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                         const DecodeArgs& a, cudaStream_t stream) {
+                         const CUtensorMap& tmQ, const DecodeArgs& a, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_decode<T, 1>(tmK, tmV, a, stream);
-    case 2: return launch_decode<T, 2>(tmK, tmV, a, stream);
-    case 4: return launch_decode<T, 4>(tmK, tmV, a, stream);
-    case 8: return launch_decode<T, 8>(tmK, tmV, a, stream);
+    case 1: return launch_decode<T, 1, HB>(tmK, tmV, tmQ, a, stream);
+    case 2: return launch_decode<T, 2, HB>(tmK, tmV, tmQ, a, stream);
+    case 4: return launch_decode<T, 4, HB>(tmK, tmV, tmQ, a, stream);
+    case 8: return launch_decode<T, 8, HB>(tmK, tmV, tmQ, a, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -568,6 +747,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   const int G = num_q_heads / num_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
   if (partition_size % 16) return PA_ERR_INVALID_ARG;
+  if (partition_size > pa::kMaxPartition) return PA_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PA_OK;
   if (num_seqs > pa::kMaxSeqs) return PA_ERR_UNSUPPORTED;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
@@ -582,14 +762,24 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   int* err = pa::device_error_flag();
   if (!err) return PA_ERR_CUDA;
 
-  CUtensorMap tmK, tmV;
-  if (!pa::encode_cache_tmap(&tmK, k_cache, num_blocks, block_size, num_kv_heads, head_dim, 16) ||
-      !pa::encode_cache_tmap(&tmV, v_cache, num_blocks, block_size, num_kv_heads, head_dim, 16))
+  // two kv-heads per item and TMA box when the head count allows (512-byte rows)
+  const int HB = (num_kv_heads % 2 == 0) ? 2 : 1;
+  CUtensorMap tmK, tmV, tmQ;
+  const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
+                             (uint64_t)num_blocks};
+  const uint64_t row = (uint64_t)head_dim * 2;
+  const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
+  const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads, (uint64_t)num_seqs};
+  const uint64_t qstr[2] = {row, row * num_q_heads};
+  const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)(HB * G), 1};
+  if (!pa::encode_tmap_16bit(&tmK, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !pa::encode_tmap_16bit(&tmV, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !pa::encode_tmap_16bit(&tmQ, q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))
     return PA_ERR_CUDA;
 
   pa::DecodeArgs a;
   a.out = out;
-  a.q = q;
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
   a.part_o = need ? static_cast<float*>(workspace) : nullptr;
@@ -605,11 +795,13 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   a.part_size = P;
   a.max_parts = parts;
   const long long cap_tbl = (long long)max_blocks_per_seq * block_size;
-  const long long cap_grid = (long long)parts * P;
-  a.seq_cap = (int)std::min<long long>(std::min<long long>(cap_tbl, cap_grid), max_seq_len);
-  a.flag_cta = 0;
+  a.seq_cap = (int)std::min<long long>(cap_tbl, max_seq_len);
+  a.slots_per_ring = 0;
   a.qscale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dtype == PA_F16 ? pa::dispatch_group<__half>(G, tmK, tmV, a, st)
-                         : pa::dispatch_group<__nv_bfloat16>(G, tmK, tmV, a, st);
+  if (dtype == PA_F16)
+    return HB == 2 ? pa::dispatch_group<__half, 2>(G, tmK, tmV, tmQ, a, st)
+                   : pa::dispatch_group<__half, 1>(G, tmK, tmV, tmQ, a, st);
+  return HB == 2 ? pa::dispatch_group<__nv_bfloat16, 2>(G, tmK, tmV, tmQ, a, st)
+                 : pa::dispatch_group<__nv_bfloat16, 1>(G, tmK, tmV, tmQ, a, st);
 }

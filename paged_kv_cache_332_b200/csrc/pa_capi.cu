@@ -53,32 +53,47 @@ int num_sms() {
   return g_sms[d];
 }
 
+static bool load_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return true;
+}
+
+bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle) {
+  if (!load_encoder() || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, rank, const_cast<void*>(base), d,
+                        st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,
                        int num_kv_heads, int head_dim, int box_rows) {
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_encode) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-              cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || !fn)
-        return false;
-      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-    }
-  }
   // innermost first: head_dim, kv-head, token-in-block, block
-  const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
-                              (cuuint64_t)block_size, (cuuint64_t)num_blocks};
-  const cuuint64_t row = (cuuint64_t)head_dim * 2;
-  const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
-  const cuuint32_t box[4] = {(cuuint32_t)head_dim, 1, (cuuint32_t)box_rows, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(cache), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
+                            (uint64_t)num_blocks};
+  const uint64_t row = (uint64_t)head_dim * 2;
+  const uint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const uint32_t box[4] = {(uint32_t)head_dim, 1, (uint32_t)box_rows, 1};
+  return encode_tmap_16bit(out, cache, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 void set_launch_count(int n) { g_last_launches = n; }

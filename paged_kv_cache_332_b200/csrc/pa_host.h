@@ -21,6 +21,12 @@ int num_sms();
 bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,
                        int num_kv_heads, int head_dim, int box_rows);
 
+// Encode a tiled TMA descriptor over a row-major tensor of 16-bit elements.
+// dims/box innermost first; strides_bytes[i] is the stride of dimension i+1.
+bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle);
+
 // Launch accounting for pa_last_launch_count().
 void set_launch_count(int n);
 

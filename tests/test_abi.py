@@ -94,6 +94,7 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(Hq=24, Hkv=8) == 2            # GQA group 3 not built
     assert dec(Hq=128, Hkv=8) == 2           # GQA group 16 not built
     assert dec(P=24) == 1                    # partition not a multiple of 16
+    assert dec(P=4096) == 2                  # partition above 2048 tokens
     assert dec(q=None) == 1                  # null pointer
     assert dec(q=ctypes.c_void_p(4100)) == 1  # misaligned
     assert dec(dt=3) == 2
