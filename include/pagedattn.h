@@ -128,6 +128,35 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     int max_seq_len, int partition_size, void* workspace,
                     size_t workspace_bytes, pa_dtype dtype, void* stream);
 
+/*
+ * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
+ * The paper has no counterpart to this call; it exists for callers whose device memory
+ * is owned by someone else (an engine's pre-allocated KV pool, a host framework that
+ * forbids raw cudaMalloc) or who must not risk the device-wide synchronisation an
+ * allocation can cause.  Arguments and results are those of pa_decode without the
+ * workspace: the split-K partials go to a fixed array inside the library,
+ * pa_decode_noalloc_scratch_bytes() long (32 MiB), which every GPU that loads the
+ * library holds until the process exits.
+ *  - Sizes whose partials need more than that (pa_decode_workspace_size(...) >
+ *    pa_decode_noalloc_scratch_bytes()) return PA_ERR_WORKSPACE_TOO_SMALL and launch
+ *    nothing.
+ *  - The first call on a device looks up that device's array address (with the device
+ *    current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its last contents there;
+ *    nothing in it needs to start at zero.  Calls that overlap on the GPU (different
+ *    streams, no ordering between them) race on the array: order them.
+ *  - The call itself allocates no memory.
+ */
+PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, float scale,
+                                   int block_size, int num_blocks, int max_seq_len,
+                                   int partition_size, pa_dtype dtype, void* stream);
+
+/* Size in bytes of the fixed scratch array pa_decode_noalloc uses (per device). */
+PA_API size_t pa_decode_noalloc_scratch_bytes(void);
+
 /* Bytes of scratch pa_chunked_prefill needs (0 in this version: no split-K). */
 PA_API size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len, int num_q_heads,
                                          int head_dim, int max_seq_len);

@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
-    "pa_decode_workspace_size", "pa_decode", "pa_chunked_prefill_workspace_size",
+    "pa_decode_workspace_size", "pa_decode", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
+    "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
     "PA_DEVERR",
 ]
@@ -39,6 +40,9 @@ _SIGS = [
     ("pa_decode_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_decode", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f, _i32, _i32,
                          _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_decode_noalloc", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f,
+                                 _i32, _i32, _i32, _i32, _i32, _vp]),
+    ("pa_decode_noalloc_scratch_bytes", _sz, []),
     ("pa_chunked_prefill_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_chunked_prefill", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
                                   _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
@@ -142,6 +146,27 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
                            int(max_seq_len), int(partition_size), _ptr(workspace), ws_bytes,
                            _dtype_code(k_cache), _stream(stream)),
            "pa_decode")
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,
+                      partition_size=0, stream=None):
+    """pa_decode for callers that cannot allocate device memory: the split-K
+    partials live in a fixed array inside the library
+    (:func:`pa_decode_noalloc_scratch_bytes` per device, held until exit).
+    Calls on one device share that array, so calls that overlap on the GPU
+    race; make the first call on a device before any stream capture."""
+    N, bs, Hkv, D = k_cache.shape
+    B, Hq, _ = q.shape
+    _check(lib().pa_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                   _i32tensor(block_tables, "block_tables"), block_tables.shape[1],
+                                   _i32tensor(seq_lens, "seq_lens"), B, Hq, Hkv, D, float(scale),
+                                   bs, N, int(max_seq_len), int(partition_size),
+                                   _dtype_code(k_cache), _stream(stream)),
+           "pa_decode_noalloc")
+
+
+def pa_decode_noalloc_scratch_bytes() -> int:
+    return int(lib().pa_decode_noalloc_scratch_bytes())
 
 
 def pa_chunked_prefill_workspace_size(num_seqs, max_query_len, num_q_heads, head_dim, max_seq_len):

@@ -35,6 +35,7 @@
 //  * Logits live in the log2 domain (q pre-scaled by scale*log2 e): one ex2 each.
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
 #include <algorithm>
+#include <mutex>
 
 #include "pa_device.cuh"
 #include "pa_host.h"
@@ -805,3 +806,60 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   return HB == 2 ? pa::dispatch_group<__nv_bfloat16, 2>(G, tmK, tmV, tmQ, a, st)
                  : pa::dispatch_group<__nv_bfloat16, 1>(G, tmK, tmV, tmQ, a, st);
 }
+
+// ---------------------------------------------------------------------------
+// Decode without any caller-provided scratch.
+//
+// Some callers cannot allocate device memory on their own: code that runs inside a
+// serving loop whose memory is entirely owned by an engine's pre-allocated pool (the
+// pool hands out KV blocks, not scratch buffers), plugins whose host framework forbids
+// raw cudaMalloc, and latency-critical paths where an allocation could synchronise the
+// device.  For them this entry point keeps the split-K partials in a fixed array that
+// lives in this file (kNoAllocScratchBytes on every GPU that loads the library, held
+// until the process exits) and otherwise runs exactly pa_decode.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {};
+
+// Device address of this device's scratch array (looked up once per device, with that
+// device current).  nullptr if the lookup failed.
+void* scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* seq_lens,
+                                       int num_seqs, int num_q_heads, int num_kv_heads,
+                                       int head_dim, float scale, int block_size, int num_blocks,
+                                       int max_seq_len, int partition_size, pa_dtype dtype,
+                                       void* stream) {
+  pa::set_launch_count(0);
+  const size_t need =
+      pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, partition_size);
+  if (need > kNoAllocScratchBytes) return PA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if (need) {
+    scratch = scratch_for_current_device();
+    if (!scratch) return PA_ERR_CUDA;
+  }
+  return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                   num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size, num_blocks,
+                   max_seq_len, partition_size, scratch, need ? kNoAllocScratchBytes : 0, dtype,
+                   stream);
+}
+
+extern "C" size_t pa_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
