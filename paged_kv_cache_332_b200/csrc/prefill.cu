@@ -1,13 +1,557 @@
-// Chunked prefill over the paged cache (tensor-core kernel follows).
+// Chunked prefill over the paged KV cache, on the sm_100a tensor cores (tcgen05).
+//
+// What it computes — page "大模型推理内存优化从 KV Cache 分页到连续批处理的工程实践",
+// section "工程边界与架构取舍": a long prompt is processed in chunks, and prefill is a
+// dense matrix product.  Sequence s has n = qsl[s+1]-qsl[s] new queries, the last n of
+// its L = seq_len[s] tokens (their K/V already cached).  Query i sits at position
+// L-n+i and attends causally to keys 0..L-n+i (inclusive), reached through the block
+// table:  out[qsl[s]+i, qh] = softmax_j(scale * q . K[j]) V[j].
+//
+// Design:
+//  * CTA = (sequence, kv-head, block of 2*MQ queries).  Rows of a 128-row M-tile are
+//    (query, q-head of the kv-head's GQA group): MQ = 128/G queries x G heads, so one
+//    K/V tile serves every head of the group.  Two M-tiles per CTA share each K/V tile
+//    and ping-pong: while the softmax of one runs, the tensor core works on the other.
+//  * TMEM (512 columns): S0, S1 (128 fp32 columns each, keys of the tile), O0, O1
+//    (128 columns, head_dim).  P (16-bit) is written back over the first 64 columns of
+//    S and fed to the P.V MMA straight from TMEM.
+//  * Q: each softmax thread copies its own row (bounds-checked 16-byte loads; rows past
+//    the chunk are zero) into shared memory in the 128-byte-swizzled K-major layout the
+//    MMA reads.  Warp 0 is the TMA producer: per 128-key tile, one box per 16-token run
+//    of a physical block for K and for V (block id from the block table), into a
+//    two-stage K ring and a two-stage V ring.
+//  * Warp 1: allocates TMEM and issues every tcgen05.mma from one thread:
+//    S_a = Q_a K^T (M=128, N=128, K=128 as 8 x K16), O_a += P_a V (A in TMEM,
+//    V as an MN-major B operand), tcgen05.commit to mbarriers.
+//  * Warps 4-7 / 8-11: softmax of M-tile 0 / 1, one thread per row: causal mask on
+//    the diagonal tiles, row max, ex2 in the log2 domain, row sum, P packed to 16 bits.
+//    The output row is rescaled only when the running max grows by more than 8 (a
+//    factor 256); every p stays <= 2^8, and the final normalisation uses the same
+//    reference, so the result is unchanged.
+//  * Keys at or past L in the last tile: K is masked in the softmax; V rows are
+//    zero-filled (TMA out-of-range fill for whole runs, a shared-memory clear for the
+//    tail of a partial block) so that 0 * (stale value) never reaches the sum.
+// Every wait is bounded; on a timeout the CTA flags PA_DEVERR_TIMEOUT, runs to its end
+// without further waits and frees its TMEM.
+#include <algorithm>
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_host.h"
 
+namespace pa {
+namespace prefill {
+
+constexpr int kD = 128;
+constexpr int kBN = 128;              // keys per tile
+constexpr int kM = 128;               // rows per M-tile
+constexpr int kHalfBytes = kM * 128;  // 128 rows x 64 elements x 2 B (one SW128 half)
+constexpr int kTileBytes = 2 * kHalfBytes;  // 32 KB: a 128 x 128 16-bit tile
+constexpr int kThreads = 12 * 32;
+
+struct Args {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const int32_t* qsl;
+  int* err;
+  int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
+  int max_query_len, seq_cap, qblocks;
+  float qscale;  // scale * log2(e)
+};
+
+// shared memory carve-up
+constexpr int OFF_Q = 0;                               // 2 M-tiles x 32 KB
+constexpr int OFF_K = OFF_Q + 2 * kTileBytes;          // 2 stages x 32 KB
+constexpr int OFF_V = OFF_K + 2 * kTileBytes;          // 2 stages x 32 KB
+constexpr int OFF_BAR = OFF_V + 2 * kTileBytes;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_full[2]
+constexpr int NBAR = 1 + 2 * 7;
+constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+constexpr int OFF_ABORT = OFF_TMEM + 8;
+constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;  // + alignment slack
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)(lbo_bytes >> 4) << 16) |
+         ((uint64_t)(sbo_bytes >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, M=128, N=128.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                       uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+      "r"(w[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Wait that stops waiting once the CTA has given up.
+__device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err) {
+  if (*abort_flag) return;
+  if (!mbar_wait(bar, parity, err)) *abort_flag = 1;
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  return Elem<T>::pack2(lo, hi);
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunked_prefill_kernel(const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const Args a) {
+  constexpr int MQ = kM / G;  // queries per M-tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bar;
+  uint64_t* k_full = bar + 1;
+  uint64_t* k_empty = bar + 3;
+  uint64_t* v_full = bar + 5;
+  uint64_t* v_empty = bar + 7;
+  uint64_t* s_full = bar + 9;
+  uint64_t* p_full = bar + 11;
+  uint64_t* o_full = bar + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- which (sequence, kv-head, query block)
+  const int qb = blockIdx.x % a.qblocks;
+  const int h = (blockIdx.x / a.qblocks) % a.num_kv_heads;
+  const int s = blockIdx.x / (a.qblocks * a.num_kv_heads);
+  const int q_begin = a.qsl[s];
+  const int n = a.qsl[s + 1] - q_begin;
+  const int Lraw = a.seq_lens[s];
+  const int L = Lraw < 0 ? 0 : (Lraw > a.seq_cap ? a.seq_cap : Lraw);
+  const int q0 = qb * 2 * MQ;
+  if (n < 0 || n > L || n > a.max_query_len || Lraw != L) {
+    if (threadIdx.x == 0 && qb == 0 && h == 0)
+      flag_error(a.err, (n < 0 || n > L || n > a.max_query_len) ? PA_DEVERR_QUERY_LAYOUT
+                                                               : PA_DEVERR_SEQ_TOO_LONG);
+    if (n < 0 || n > L || n > a.max_query_len) return;
+  }
+  if (q0 >= n) return;  // this query block is past the chunk (uniform for the CTA)
+  // keys any row of this CTA can see: [0, kv_end)
+  const int kv_end = min(L, L - n + min(n, q0 + 2 * MQ));
+  const int n_kt = (kv_end + kBN - 1) / kBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 8);  // one arrival per softmax warp once its Q rows are in place
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_full[i], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================== TMA producer ========================
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
+      const int bs_mask = (1 << a.log2_bs) - 1;
+      for (int kt = 0; kt < n_kt; ++kt) {
+        const int st = kt & 1;
+        const uint32_t ph = ((kt >> 1) & 1) ^ 1;
+        // block ids of the tile's eight 16-token runs (out of range -> zero fill)
+        int bid[8], row[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int pos = kt * kBN + r * 16;
+          bid[r] = a.num_blocks;  // past the tensor: TMA fills zeros
+          row[r] = pos & bs_mask;
+          if (pos < L) {
+            const int id = __ldg(trow + (pos >> a.log2_bs));
+            if ((unsigned)id < (unsigned)a.num_blocks) bid[r] = id;
+            else flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
+          }
+        }
+        wait_or_abort(&k_empty[st], ph, abort_flag, a.err);
+        mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int kh = 0; kh < 2; ++kh)
+            tma_load_4d(smem + OFF_K + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmK,
+                        kh * 64, h, row[r], bid[r], &k_full[st]);
+        wait_or_abort(&v_empty[st], ph, abort_flag, a.err);
+        mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int kh = 0; kh < 2; ++kh)
+            tma_load_4d(smem + OFF_V + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmV,
+                        kh * 64, h, row[r], bid[r], &v_full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================== MMA issuer ========================
+    if (lane == 0) {
+      constexpr bool BF = sizeof(T) == 2 && !std::is_same<T, __half>::value;
+      const uint32_t id_qk = idesc_f16(BF, false);
+      const uint32_t id_pv = idesc_f16(BF, true);
+      const uint32_t sQ = smem_u32(smem + OFF_Q);
+      const uint32_t sK = smem_u32(smem + OFF_K);
+      const uint32_t sV = smem_u32(smem + OFF_V);
+      auto issue_s = [&](int mt, int kt) {
+        const int st = kt & 1;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint64_t da = sw128_desc(sQ + mt * kTileBytes + off, 16, 1024);
+          const uint64_t db = sw128_desc(sK + st * kTileBytes + off, 16, 1024);
+          mma_ss(tmem + mt * 128, da, db, id_qk, kk > 0);
+        }
+        mma_commit(&s_full[mt]);
+      };
+      auto issue_pv = [&](int mt, int kt) {
+        const int st = kt & 1;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t db = sw128_desc(sV + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
+          mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (kt > 0 || kk > 0));
+        }
+      };
+      wait_or_abort(q_full, 0, abort_flag, a.err);
+      tc_fence_after();
+      if (n_kt > 0) {
+        wait_or_abort(&k_full[0], 0, abort_flag, a.err);
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&k_empty[0]);
+      }
+      for (int kt = 0; kt < n_kt; ++kt) {
+        const int st = kt & 1;
+        const bool more = kt + 1 < n_kt;
+        wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
+        if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
+        for (int mt = 0; mt < 2; ++mt) {
+          wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
+          tc_fence_after();
+          issue_pv(mt, kt);
+          if (more) issue_s(mt, kt + 1);
+        }
+        if (more) mma_commit(&k_empty[(kt + 1) & 1]);
+        mma_commit(&v_empty[st]);
+      }
+      mma_commit(&o_full[0]);
+      mma_commit(&o_full[1]);
+    }
+  } else if (warp >= 4) {
+    // ======================== softmax warpgroups ========================
+    const int mt = (warp - 4) >> 2;
+    const int wq = warp & 3;              // TMEM lane quarter
+    const int r = wq * 32 + lane;         // row of the M-tile
+    const int qi = q0 + mt * MQ + r / G;  // query index within the chunk
+    const bool row_valid = qi < n;
+    const int limit = L - n + min(qi, n - 1);  // last visible key (inclusive)
+    const uint32_t t_s = tmem + ((uint32_t)(wq * 32) << 16) + mt * 128;
+    const uint32_t t_o = tmem + ((uint32_t)(wq * 32) << 16) + 256 + mt * 128;
+    // lowest limit in the warp decides whether a tile needs the causal mask
+    int wlim = limit;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) wlim = min(wlim, __shfl_xor_sync(0xffffffffu, wlim, o));
+    {
+      // this thread's Q row -> shared memory, 128-byte swizzle: 16-byte chunk j of row r
+      // of a 64-element half sits at chunk position j ^ (r % 8)
+      const uint4* src = reinterpret_cast<const uint4*>(
+          static_cast<const T*>(a.q) +
+          ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD);
+      uint8_t* dst = smem + OFF_Q + mt * kTileBytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 w = row_valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(dst + (c >> 3) * kHalfBytes + (((c & 7) ^ (r & 7)) << 4)) = w;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full);
+    }
+    float m_ref = -INFINITY, l = 0.f;
+    for (int kt = 0; kt < n_kt; ++kt) {
+      wait_or_abort(&s_full[mt], kt & 1, abort_flag, a.err);
+      tc_fence_after();
+      const int key0 = kt * kBN;
+      const bool need_mask = key0 + kBN - 1 > wlim;
+      float v[32];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(t_s + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x = (need_mask && key0 + c * 32 + i > limit) ? -INFINITY : v[i];
+          mx = fmaxf(mx, x);
+        }
+      }
+      mx *= a.qscale;
+      // lazy reference max: move it only when this tile exceeds it by more than 8
+      float alpha = 1.f;
+      if (mx > m_ref + 8.f) {
+        alpha = fast_exp2(m_ref - mx);  // m_ref = -inf -> 0
+        m_ref = mx;
+      }
+      if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(t_o + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st32(t_o + c * 32, v);
+        }
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(t_s + c * 32, v);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const bool k0 = !(need_mask && key0 + c * 32 + i > limit);
+          const bool k1 = !(need_mask && key0 + c * 32 + i + 1 > limit);
+          const float p0 = k0 ? fast_exp2(fmaf(v[i], a.qscale, -m_ref)) : 0.f;
+          const float p1 = k1 ? fast_exp2(fmaf(v[i + 1], a.qscale, -m_ref)) : 0.f;
+          sum += p0 + p1;
+          w[i >> 1] = pack16<T>(p0, p1);
+        }
+        tmem_st16(t_s + c * 16, w);
+      }
+      l = l * alpha + sum;
+      // keys past the sequence end in the last tile: clear their V rows
+      if (mt == 0 && kt == n_kt - 1 && L < key0 + kBN) {
+        wait_or_abort(&v_full[kt & 1], (kt >> 1) & 1, abort_flag, a.err);
+        uint8_t* vt = smem + OFF_V + (kt & 1) * kTileBytes;
+        const int first = L - key0;  // first row to clear
+        for (int i = threadIdx.x - 128; i < (kBN - first) * 16; i += 128) {
+          const int rr = first + i / 16, chunk = i % 16;  // 16 x 16 B per row (two halves)
+          *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + rr * 128 + (chunk & 7) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[mt]);
+    }
+    // ---- epilogue: O / l -> out
+    wait_or_abort(&o_full[mt], 0, abort_flag, a.err);
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    T* orow = static_cast<T*>(a.out) +
+              ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      tmem_ld32(t_o + c * 32, v);
+      if (row_valid && n_kt > 0) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) w[i >> 1] = pack16<T>(v[i] * inv, v[i + 1] * inv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(orow + c * 32 + j * 8) =
+              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+template <typename T, int G>
+pa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
+                 cudaStream_t stream) {
+  auto kern = chunked_prefill_kernel<T, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  const long long grid = (long long)a.num_seqs * a.num_kv_heads * a.qblocks;
+  if (grid <= 0) return PA_OK;
+  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(tk, tv, a);
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
+  set_launch_count(1);
+  return PA_OK;
+}
+
+template <typename T>
+pa_status dispatch(int G, const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
+                   cudaStream_t stream) {
+  switch (G) {
+    case 1: return launch<T, 1>(tk, tv, a, stream);
+    case 2: return launch<T, 2>(tk, tv, a, stream);
+    case 4: return launch<T, 4>(tk, tv, a, stream);
+    case 8: return launch<T, 8>(tk, tv, a, stream);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace prefill
+}  // namespace pa
+
 extern "C" size_t pa_chunked_prefill_workspace_size(int, int, int, int, int) { return 0; }
 
-extern "C" pa_status pa_chunked_prefill(void*, const void*, const void*, const void*,
-                                        const int32_t*, int, const int32_t*, const int32_t*, int,
-                                        int, int, int, int, float, int, int, int, void*, size_t,
-                                        pa_dtype, void*) {
+extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* seq_lens,
+                                        const int32_t* query_start_loc, int num_seqs,
+                                        int max_query_len, int num_q_heads, int num_kv_heads,
+                                        int head_dim, float scale, int block_size, int num_blocks,
+                                        int max_seq_len, void* workspace, size_t workspace_bytes,
+                                        pa_dtype dtype, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
   pa::set_launch_count(0);
-  return PA_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
+      max_seq_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 128 || (block_size != 16 && block_size != 32)) return PA_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads) return PA_ERR_INVALID_ARG;
+  const int G = num_q_heads / num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !query_start_loc)
+    return PA_ERR_INVALID_ARG;
+  if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
+    return PA_ERR_INVALID_ARG;
+  int* err = pa::device_error_flag();
+  if (!err) return PA_ERR_CUDA;
+  const int MQ = 128 / G;
+  CUtensorMap tk, tv;
+  const uint64_t row = (uint64_t)head_dim * 2;
+  const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
+                             (uint64_t)num_blocks};
+  const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const uint32_t cbox[4] = {64, 1, 16, 1};
+  if (!pa::encode_tmap_16bit(&tk, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !pa::encode_tmap_16bit(&tv, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B))
+    return PA_ERR_CUDA;
+  pa::prefill::Args a;
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.qsl = query_start_loc;
+  a.err = err;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.log2_bs = block_size == 16 ? 4 : 5;
+  a.num_blocks = num_blocks;
+  a.max_query_len = max_query_len;
+  a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_seq_len);
+  a.qblocks = (max_query_len + 2 * MQ - 1) / (2 * MQ);
+  a.qscale = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dtype == PA_F16 ? pa::prefill::dispatch<__half>(G, tk, tv, a, st)
+                         : pa::prefill::dispatch<__nv_bfloat16>(G, tk, tv, a, st);
 }
