@@ -58,6 +58,23 @@ def measured_peaks():
                 source="fallback")
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    kernel source changed since the capture (or no capture matches)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(kernel)
+        if not rec or rec.get("workload") != workload:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+        return int(rec["dram_bytes_per_launch"]) if h.startswith(rec["source_sha256_prefix"]) else None
+    except Exception:
+        return None
+
+
 def decode_algorithmic_bytes(b: workloads.PagedBatch) -> int:
     """KV of every token at its exact length, q and out, table rows, seq_lens."""
     e = b.q.element_size()
@@ -173,7 +190,7 @@ class Step:
         self.launches = 0
         self.ev_dec = []
 
-    def run(self, record=None):
+    def run(self, record=None, record_pre=None):
         pa = self.pa
         n = 0
         for b in self.batches:
@@ -181,10 +198,14 @@ class Step:
                                     stream=self.stream)
             n += pa.pa_last_launch_count()
         for b in self.prefill:
+            if record_pre is not None:
+                record_pre[0].record(self.stream)
             pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
                                   b.seq_lens, b.query_start_loc, b.scale, self.max_q[id(b)],
                                   self.max_len[id(b)], None, stream=self.stream)
             n += pa.pa_last_launch_count()
+            if record_pre is not None:
+                record_pre[1].record(self.stream)
         for b in self.decode:
             if record is not None:
                 record[0].record(self.stream)
@@ -237,6 +258,8 @@ def run_ours(args, rank, world, device):
           for _ in range(args.steps)]
     evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     with ClockSampler(device) as clocks:
         barrier()
         torch.cuda.synchronize(device)
@@ -245,7 +268,7 @@ def run_ours(args, rank, world, device):
                 if flush is not None:
                     flush.fill_(float(i))
                 ev[i][0].record(stream)
-                step.run(evd[i] if dec is not None else None)
+                step.run(evd[i] if dec is not None else None, evp[i] if pre is not None else None)
                 ev[i][1].record(stream)
         torch.cuda.synchronize(device)
         barrier()
@@ -253,6 +276,7 @@ def run_ours(args, rank, world, device):
     local_ms = sum(step_ms)
     launches = step.launches
     dec_ms = [a.elapsed_time(b) for a, b in evd] if dec is not None else []
+    pre_ms = [a.elapsed_time(b) for a, b in evp] if pre is not None else []
     total_ms = aggregate_max(local_ms, device)
 
     # ---- end to end: per-step H2D of the step's inputs from pinned host
@@ -317,11 +341,20 @@ def run_ours(args, rank, world, device):
                             "frac": round(ach / peaks["hbm_gbs"], 4),
                             "frac_of_8TBs_spec": round(ach / 8000.0, 4),
                             "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
-                            "traffic": None}
+                            "traffic": recorded_traffic("paged_decode_kernel", dec.name)}
         line["context_tokens_per_s"] = round(world * int(dec.seq_lens.sum().item()) * args.steps
                                              / (total_ms / 1e3), 1)
     if pre is not None:
-        line["prefill_tflop_per_step"] = prefill_flops(pre) / 1e12
+        fl = prefill_flops(pre)
+        pmean = statistics.mean(pre_ms)
+        tf = fl / (pmean / 1e3) / 1e12
+        peak_tf = peaks["bf16_tflops"]
+        line["roofline_prefill"] = {"kernel": "pa_chunked_prefill (chunked_prefill_kernel, tcgen05)",
+                                    "bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
+                                    "peak_source": peaks["source"] + " bf16 dense burst",
+                                    "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4),
+                                    "flop_per_launch": fl, "ms_per_launch": round(pmean, 5),
+                                    "traffic": None}
     line["e2e"] = {"value": round(world * tokens * e2e_steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     line["clocks"] = clocks.summary()
