@@ -184,7 +184,7 @@ class Step:
             self.out[id(b)] = torch.empty_like(b.q)
             if b.query_start_loc is None:
                 n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
-                self.ws[id(b)] = torch.empty(max(n, 16), dtype=torch.uint8, device=b.q.device) if n else None
+                self.ws[id(b)] = torch.empty(n, dtype=torch.uint8, device=b.q.device)
         self.max_len = {id(b): b.max_seq_len for b in batches}
         self.max_q = {id(b): b.max_query_len for b in batches}
         self.launches = 0

@@ -135,8 +135,8 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
               partition_size=0, workspace=None, stream=None):
     """Paged single-query attention.  ``q``/``out`` [B, Hq, D]; ``block_tables``
     int32 [B, max_blocks]; ``seq_lens`` int32 [B]; ``workspace`` a device
-    tensor of at least :func:`pa_decode_workspace_size` bytes (or None when
-    that is 0)."""
+    tensor of at least :func:`pa_decode_workspace_size` bytes (256-byte
+    aligned, as torch's allocator returns)."""
     N, bs, Hkv, D = k_cache.shape
     B, Hq, _ = q.shape
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -152,7 +152,8 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, m
                       partition_size=0, stream=None):
     """pa_decode for callers that cannot allocate device memory: the split-K
     partials live in a fixed array inside the library
-    (:func:`pa_decode_noalloc_scratch_bytes` per device, held until exit).
+    (:func:`pa_decode_noalloc_scratch_bytes` per device, held until exit), as does
+    the kernel's work-item counter.
     Calls on one device share that array, so calls that overlap on the GPU
     race; make the first call on a device before any stream capture."""
     N, bs, Hkv, D = k_cache.shape

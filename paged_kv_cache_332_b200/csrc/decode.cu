@@ -11,28 +11,29 @@
 //
 // Design on B200.  The page's kernel tricks (block-table entries in shared memory,
 // coalesced in-block reads, prefetching the next block) are kept where they pay:
-//  * Work item = (sequence, partition of P tokens, pair of kv-heads).  A persistent grid
-//    of one CTA per SM walks a fixed item order round-robin: every full-size partition
-//    first, then each sequence's last (partial) partition, largest first, so the tail of
-//    the launch is made of the smallest items.
-//  * Tile = 16 consecutive tokens of the item's kv-heads inside one physical block: one
-//    4-D TMA copy of K and one of V (16 rows of HB*256 contiguous bytes each).  A staging
-//    warp runs up to four items ahead: it copies each item's block-table entries into
-//    shared memory (one coalesced read per 32 entries) and starts the TMA copy of the
-//    item's q rows.  A producer warp gives every ring of tile slots its own lane; each
-//    lane polls its ring without blocking and issues the next tile's copies as soon as a
-//    slot frees, so several tiles are requested at once and the copies of the next tiles
-//    are in flight while the current ones are computed.
-//  * Consumer warps share each tile across the G q-heads of a kv-head (GQA; up to four
-//    heads per warp).  q.k: 8 lanes split a token's 128 dims (16 each, two 16-byte
-//    shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving exchange sums
-//    four heads at once.  Each warp keeps its own online softmax (running max m, sum l,
-//    fp32 accumulator over 4 dims per lane).
-//  * When a warp finishes its share of an item it parks (m, l, acc) in shared memory;
-//    the last warp to finish merges the item (no CTA-wide barrier).  A sequence that fits
-//    one partition writes `out`; longer ones write the normalised partial (o, m, l) to the
-//    caller's workspace, merged by a log-sum-exp pass (lse_reduce_kernel).
-//  * Logits live in the log2 domain (q pre-scaled by scale*log2 e): one ex2 each.
+//  * Reads are whole physical blocks: one 4-D TMA box brings 16 tokens of K for HB
+//    kv-heads (HB = all eight of a LLaMA-70B-style layer: one contiguous 32 KB block), a
+//    second box the same of V.  Measured on B200, boxes of one or two kv-heads (256 or
+//    512-byte runs scattered over randomly placed blocks) stream at 2.4-4.4 TB/s while
+//    whole 2 KB rows stream at 7 TB/s.
+//  * Work item = (sequence, partition of P tokens, group of HB kv-heads).  Items are
+//    ordered every full partition first, then each sequence's last partition largest
+//    first; a persistent grid of one CTA per SM hands them out through an atomic counter
+//    (a largest-first dynamic schedule).
+//  * One consumer warp per kv-head of the item handles all G q-heads of that kv-head
+//    over every tile of the item, so no two warps share an output and no merge inside
+//    the CTA is needed.  q.k: 8 lanes split a token's 128 dims (16 each, two 16-byte
+//    shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving exchange that
+//    sums all G heads at once.  Online softmax (running max m, sum l) in the log2 domain
+//    (q pre-scaled by scale*log2 e: one ex2 per logit); p.V with lanes over head_dim.
+//  * A staging warp claims items and, up to two items ahead, copies their block-table
+//    entries into shared memory (one coalesced read per 32 entries) and starts the TMA
+//    copy of their q rows.  A producer thread walks the tiles in order and issues the
+//    two boxes of each as soon as a slot of the shared ring frees (blocking waits take
+//    no issue slots from the consumers).
+//  * A sequence that fits one partition writes `out` directly; longer ones write
+//    normalised partials (o, m, l) to the caller's workspace, merged by a log-sum-exp pass
+//    (lse_reduce_kernel).
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
 #include <algorithm>
 #include <mutex>
@@ -48,58 +49,51 @@ struct DecodeArgs {
   const int32_t* seq_lens;
   float* part_o;   // [B, Hq, max_parts, 128]
   float* part_ml;  // [B, Hq, max_parts, 2]   (max in log2 units, sum)
+  int* counter;    // dynamic item counter (zeroed before the launch)
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
-  int part_size, max_parts, seq_cap, slots_per_ring;
-  float qscale;  // scale * log2(e)
+  int part_size, max_parts, seq_cap;
+  int ring_off, nslots;  // shared-memory offset of the tile ring and its slot count
+  float qscale;          // scale * log2(e)
 };
 
 constexpr int kD = 128;
 constexpr int kTileTok = 16;
-constexpr int kRowBytes = kD * 2;   // one token of one kv-head
-constexpr int kQSlots = 4;          // items staged ahead
-constexpr int kMergeSlots = 2;      // items being merged
-constexpr int kMaxSlots = 32;
+constexpr int kRowBytes = kD * 2;      // one token of one kv-head
+constexpr int kQSlots = 2;             // items staged ahead
+constexpr int kMaxSlots = 8;
 constexpr int kMaxTilesPerItem = 128;  // partition <= 2048 tokens
-constexpr int kSortBuckets = 128;
+constexpr int kSortBuckets = 128;      // = 32 lanes x 4 in the bucket scan
+constexpr int kWorkspaceHeader = 256;  // bytes: the item counter
 
-template <int G_, int HB_, int NCW_>
+template <int G_, int HB_>
 struct DecodeCfg {
   static constexpr int G = G_;
-  static constexpr int HB = HB_;                   // kv-heads per item (and per TMA box)
-  static constexpr int NCW = NCW_;                 // consumer warps
-  static constexpr int GW = G < 4 ? G : 4;         // q-heads per warp
-  static constexpr int HG = G / GW;                // warps per kv-head per token group
-  static constexpr int WPT = HB * HG;              // warps reading one tile
-  static constexpr int TGS = NCW / WPT;            // rings (token groups)
-  static constexpr int THREADS = (NCW + 2) * 32;   // + producer warp + staging warp
-  static constexpr int WARP_PROD = NCW;
-  static constexpr int WARP_STAGE = NCW + 1;
-  static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);
+  static constexpr int HB = HB_;                  // kv-heads per item = consumer warps
+  static constexpr int GW = G;                    // q-heads per warp
+  static constexpr int THREADS = (HB + 2) * 32;   // + producer warp + staging warp
+  static constexpr int WARP_PROD = HB;
+  static constexpr int WARP_STAGE = HB + 1;
+  static constexpr int DUPMASK = GW == 8 ? 0 : (GW == 4 ? 1 : (GW == 2 ? 3 : 7));
   static constexpr int TILE_BYTES = kTileTok * HB * kRowBytes;  // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
   static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of an item
-  // shared-memory carve-up (bytes); the tile ring comes last (runtime size)
+  // shared-memory carve-up (bytes); the sequence arrays and then the ring follow
   static constexpr int OFF_FULL = 0;
   static constexpr int OFF_EMPTY = OFF_FULL + kMaxSlots * 8;
   static constexpr int OFF_QFULL = OFF_EMPTY + kMaxSlots * 8;
   static constexpr int OFF_QEMPTY = OFF_QFULL + kQSlots * 8;
   static constexpr int OFF_TFULL = OFF_QEMPTY + kQSlots * 8;
   static constexpr int OFF_TEMPTY = OFF_TFULL + kQSlots * 8;
-  static constexpr int OFF_MFREE = OFF_TEMPTY + kQSlots * 8;
-  static constexpr int OFF_MCNT = OFF_MFREE + kMergeSlots * 8;
-  static constexpr int OFF_ABORT = OFF_MCNT + kMergeSlots * 4;
+  static constexpr int OFF_ITEM = OFF_TEMPTY + kQSlots * 8;     // claimed item per slot
+  static constexpr int OFF_ABORT = OFF_ITEM + kQSlots * 4;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
   static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerItem * 4;
-  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;           // p pairs per warp
-  static constexpr int OFF_A = OFF_P + NCW * kTileTok * GW * 8;    // alpha per warp
-  static constexpr int OFF_RACC = ((OFF_A + NCW * GW * 4 + 15) / 16) * 16;
-  static constexpr int OFF_RM = OFF_RACC + kMergeSlots * NCW * GW * kD * 4;
-  static constexpr int OFF_RL = OFF_RM + kMergeSlots * NCW * GW * 4;
-  static constexpr int OFF_SORT = OFF_RL + kMergeSlots * NCW * GW * 4;
-  static constexpr int OFF_SEQ = OFF_SORT + kSortBuckets * 4;      // 3 int arrays
-  static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0 && OFF_RACC % 16 == 0, "alignment");
-  static_assert(TGS >= 1 && NCW % WPT == 0 && TGS <= 32, "warp split");
+  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;          // p pairs per warp
+  static constexpr int OFF_A = OFF_P + HB * kTileTok * GW * 8;     // alpha per warp
+  static constexpr int OFF_SORT = ((OFF_A + HB * GW * 4 + 15) / 16) * 16;
+  static constexpr int OFF_SEQ = OFF_SORT + kSortBuckets * 4;       // 3 int arrays
+  static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -114,9 +108,34 @@ __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
 
 // Sum per-lane partial dot products over each 8-lane token group for GW heads at
 // once (halving exchange).  Returns the sum for head hh(lane):
-//   GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;  GW=1: hh = 0.
+//   GW=8: hh = 4*bit2 + 2*bit1 + bit0;  GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;
+//   GW=1: hh = 0.
 template <int GW>
 __device__ __forceinline__ float reduce_heads(const float (&d)[GW], int lane);
+
+template <>
+__device__ __forceinline__ float reduce_heads<8>(const float (&d)[8], int lane) {
+  const bool b2 = lane & 4;
+  float k[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b2 ? d[i + 4] : d[i];
+    const float send = b2 ? d[i] : d[i + 4];
+    k[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  const bool b1 = lane & 2;
+  float k2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b1 ? k[i + 2] : k[i];
+    const float send = b1 ? k[i] : k[i + 2];
+    k2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  const bool b0 = lane & 1;
+  const float keep = b0 ? k2[1] : k2[0];
+  const float send = b0 ? k2[0] : k2[1];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
 
 template <>
 __device__ __forceinline__ float reduce_heads<4>(const float (&d)[4], int lane) {
@@ -155,7 +174,15 @@ __device__ __forceinline__ float reduce_heads<1>(const float (&d)[1], int lane) 
 
 template <int GW>
 __device__ __forceinline__ int head_of_lane(int lane) {
-  return GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)) : (GW == 2 ? ((lane >> 2) & 1) : 0);
+  return GW == 8 ? (lane & 7)
+                 : (GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1))
+                            : (GW == 2 ? ((lane >> 2) & 1) : 0));
+}
+
+// A lane that holds head jj's value after reduce_heads (with tp = 0).
+template <int GW>
+__device__ __forceinline__ int lane_of_head(int jj) {
+  return GW == 8 ? jj : (GW == 4 ? (((jj >> 1) << 2) | ((jj & 1) << 1)) : (GW == 2 ? jj * 4 : 0));
 }
 
 // The launch's item order: item i -> (sequence s, partition p, kv-head group hp).
@@ -186,12 +213,12 @@ struct Schedule {
   }
 };
 
-template <typename T, int G, int HB, int NCW>
-__global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
+template <typename T, int G, int HB>
+__global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
-  using C = DecodeCfg<G, HB, NCW>;
+  using C = DecodeCfg<G, HB>;
   constexpr int GW = C::GW;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
@@ -200,27 +227,23 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
   uint64_t* qempty = reinterpret_cast<uint64_t*>(smem + C::OFF_QEMPTY);
   uint64_t* tfull = reinterpret_cast<uint64_t*>(smem + C::OFF_TFULL);
   uint64_t* tempty = reinterpret_cast<uint64_t*>(smem + C::OFF_TEMPTY);
-  uint64_t* mfree = reinterpret_cast<uint64_t*>(smem + C::OFF_MFREE);
-  int* mcnt = reinterpret_cast<int*>(smem + C::OFF_MCNT);
+  volatile int* item_of = reinterpret_cast<volatile int*>(smem + C::OFF_ITEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
   int* tbl = reinterpret_cast<int*>(smem + C::OFF_TBL);
   uint8_t* qbuf = smem + C::OFF_Q;
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
   float* abuf = reinterpret_cast<float*>(smem + C::OFF_A);
-  float* racc = reinterpret_cast<float*>(smem + C::OFF_RACC);
-  float* rm = reinterpret_cast<float*>(smem + C::OFF_RM);
-  float* rl = reinterpret_cast<float*>(smem + C::OFF_RL);
   int* cursor = reinterpret_cast<int*>(smem + C::OFF_SORT);
   const int B = a.num_seqs;
   int* fstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);
   int* slen = fstart + B + 1;
   int* order = slen + B;
-  uint8_t* ring = smem + ((C::OFF_SEQ + (3 * B + 1) * 4 + 1023) / 1024) * 1024;
+  uint8_t* ring = smem + a.ring_off;
+  const int nslots = a.nslots;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int P = a.part_size;
-  const int nsw = a.slots_per_ring;
 
   // ---- schedule: clamped lengths, full-partition prefix, last partitions by size
   if (warp == 0) {
@@ -259,13 +282,19 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
       if (s < B) atomicAdd(&cursor[bucket(s)], 1);
     }
     __syncwarp();
-    if (lane == 0) {
-      int run2 = 0;
-      for (int b = 0; b < kSortBuckets; ++b) {
-        const int c = cursor[b];
-        cursor[b] = run2;
-        run2 += c;
+    {  // exclusive scan of the bucket counts, 4 buckets per lane
+      int c[4], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { c[j] = cursor[lane * 4 + j]; tot += c[j]; }
+      int inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
       }
+      int run2 = inc - tot;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { cursor[lane * 4 + j] = run2; run2 += c[j]; }
     }
     __syncwarp();
     for (int base = 0; base < B; base += 32) {
@@ -279,20 +308,16 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
       __syncwarp();
     }
   }
-  if (threadIdx.x == 32) {
-    for (int i = 0; i < C::TGS * nsw; ++i) {
+  if (threadIdx.x == C::WARP_STAGE * 32) {
+    for (int i = 0; i < nslots; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], C::WPT);
+      mbar_init(&empty[i], HB);
     }
     for (int i = 0; i < kQSlots; ++i) {
       mbar_init(&qfull[i], 1);
-      mbar_init(&qempty[i], C::NCW);
+      mbar_init(&qempty[i], HB);
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], C::TGS);
-    }
-    for (int i = 0; i < kMergeSlots; ++i) {
-      mbar_init(&mfree[i], 1);
-      mcnt[i] = 0;
+      mbar_init(&tempty[i], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -303,14 +328,24 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
   const int total = (sch.nfull + B) * NHP;
 
   if (warp == C::WARP_STAGE) {
-    // ============ staging warp: block-table entries + q rows, items ahead ============
+    // ===== staging warp: claims items; block-table entries + q rows, two items ahead =====
     if (lane == 0) prefetch_tmap(&tmQ);
-    int k = 0;
-    for (int item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+    for (int k = 0;; ++k) {
       const int qs = k % kQSlots;
       const uint32_t par = ((k / kQSlots) & 1) ^ 1;
-      wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read item k-4's q
-      wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // producer issued its tiles
+      wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read item k-2's q
+      wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // its tiles were issued
+      int item = 0;
+      if (lane == 0) item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(a.counter, 1);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (item >= total || *abort_flag) {  // tell the other warps there is no more work
+        if (lane == 0) {
+          item_of[qs] = -1;
+          mbar_arrive_expect_tx(&qfull[qs], 0);
+          mbar_arrive(&tfull[qs]);
+        }
+        break;
+      }
       int s, p, hp;
       sch.item(item, s, p, hp);
       const int ntile = sch.ntiles(s, p);
@@ -336,9 +371,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        const bool ok = !*abort_flag;
-        mbar_arrive_expect_tx(&qfull[qs], ok ? C::QBYTES : 0);
-        if (ok) tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HB * G, s, &qfull[qs]);
+        item_of[qs] = item;
+        mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
+        tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HB * G, s, &qfull[qs]);
         mbar_arrive(&tfull[qs]);
       }
     }
@@ -346,104 +381,62 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
   }
 
   if (warp == C::WARP_PROD) {
-    // ============ producer warp: lane r feeds ring r ============
+    // ===== producer: one thread walks every tile in order into the shared ring =====
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-    }
-    const int r = lane;
-    int k = 0, item = blockIdx.x, s = 0, p = 0, hp = 0, ntile = 0, t = r, pos = 0;
-    bool done = (r >= C::TGS) || item >= total;
-    bool entered = false;
-    if (!done) {
-      sch.item(item, s, p, hp);
-      ntile = sch.ntiles(s, p);
-    }
-    const int bs_mask = (1 << a.log2_bs) - 1;
-    unsigned long long t_idle = 0;
-    while (!__all_sync(0xffffffffu, done)) {
-      bool progressed = false;
-      if (!done) {
-        if (*abort_flag) {
-          done = true;
-        } else {
-          if (!entered && mbar_test_wait(&tfull[k % kQSlots], (k / kQSlots) & 1)) entered = true;
-          if (entered && t < ntile) {
-            const int slot = r * nsw + pos % nsw;
-            if (mbar_test_wait(&empty[slot], ((pos / nsw) & 1) ^ 1)) {
-              const int bid = tbl[(k % kQSlots) * kMaxTilesPerItem + t];
-              mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
-              if (bid >= 0) {
-                const int row = (p * P + t * kTileTok) & bs_mask;
-                uint8_t* dst = ring + slot * C::SLOT_BYTES;
-                tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
-                tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
-              }
-              ++pos;
-              t += C::TGS;
-              progressed = true;
-            }
-          }
-          if (entered && t >= ntile) {  // this ring's share of the item is issued
-            mbar_arrive(&tempty[k % kQSlots]);
-            ++k;
-            item += gridDim.x;
-            entered = false;
-            t = r;
-            progressed = true;
-            if (item >= total) {
-              done = true;
-            } else {
-              sch.item(item, s, p, hp);
-              ntile = sch.ntiles(s, p);
-            }
+      const int bs_mask = (1 << a.log2_bs) - 1;
+      int cnt = 0;
+      for (int k = 0;; ++k) {
+        const int qs = k % kQSlots;
+        wait_or_abort(&tfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
+        const int item = item_of[qs];
+        if (item < 0 || *abort_flag) break;
+        int s, p, hp;
+        sch.item(item, s, p, hp);
+        const int ntile = sch.ntiles(s, p);
+        for (int t = 0; t < ntile; ++t, ++cnt) {
+          const int slot = cnt % nslots;
+          wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err);
+          const int bid = *abort_flag ? -1 : tbl[qs * kMaxTilesPerItem + t];
+          mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
+          if (bid >= 0) {
+            const int row = (p * P + t * kTileTok) & bs_mask;
+            uint8_t* dst = ring + slot * C::SLOT_BYTES;
+            tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
+            tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
           }
         }
-      }
-      if (__any_sync(0xffffffffu, progressed)) {
-        t_idle = 0;
-      } else {
-        const unsigned long long now = globaltimer_ns();
-        if (t_idle == 0) {
-          t_idle = now;
-        } else if (now - t_idle > kWaitLimitNs) {
-          if (lane == 0) {
-            flag_error(a.err, PA_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          done = true;
-        }
+        mbar_arrive(&tempty[qs]);
       }
     }
     return;
   }
 
-  // ===================== consumer warps =====================
-  const int kvsub = warp % HB;
-  const int hg = (warp / HB) % C::HG;
-  const int tg = warp / C::WPT;
+  // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
   const int sub = lane & 7;
   const int tp = lane >> 3;
   const int hh = head_of_lane<GW>(lane);
   const bool writer = (lane & C::DUPMASK) == 0;
   float2* pw = pbuf + warp * kTileTok * GW;
-  int mypos = 0;
-  int k = 0;
+  int cnt = 0;
 
-  for (int item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+  for (int k = 0;; ++k) {
+    const int qs = k % kQSlots;
+    wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
+    const int item = item_of[qs];
+    if (item < 0 || *abort_flag) break;
     int s, p, hp;
     sch.item(item, s, p, hp);
     const int tok0 = p * P;
     const int tok1 = min(slen[s], tok0 + P);
     const int ntile = cdiv(max(tok1 - tok0, 0), kTileTok);
-    const int qs = k % kQSlots;
 
-    // q of this warp's GW heads, dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8),
+    // q of this warp's G heads, dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8),
     // as (even, odd) pairs, pre-scaled into the log2 domain
     float2 q2[GW][8];
-    wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
     {
-      const uint8_t* qb = qbuf + qs * C::QBYTES + (kvsub * G + hg * GW) * kRowBytes;
+      const uint8_t* qb = qbuf + qs * C::QBYTES + warp * G * kRowBytes;
 #pragma unroll
       for (int j = 0; j < GW; ++j) {
         const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
@@ -463,13 +456,12 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
 #pragma unroll
     for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
 
-    for (int t = tg; t < ntile; t += C::TGS) {
-      const int slot = tg * nsw + mypos % nsw;
-      const uint32_t par = (mypos / nsw) & 1;
-      ++mypos;
-      wait_or_abort(&full[slot], par, abort_flag, a.err);
+    for (int t = 0; t < ntile; ++t, ++cnt) {
+      const int slot = cnt % nslots;
+      wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
       const int nvalid = min(kTileTok, tok1 - (tok0 + t * kTileTok));
-      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + kvsub * kRowBytes;
+      // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
+      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + warp * kRowBytes;
       const uint8_t* Vs = Ks + C::TILE_BYTES;
 
       // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
@@ -542,74 +534,26 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, NCW>::THREADS, 1)
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
 
-    // ---- park (m, l, acc); the last warp of the item merges and writes
+    // ---- finish: l summed over the 4 token groups; m and l of every head to every lane
     l += __shfl_xor_sync(0xffffffffu, l, 8);
     l += __shfl_xor_sync(0xffffffffu, l, 16);
-    const int ms = k % kMergeSlots;
-    wait_or_abort(&mfree[ms], ((k / kMergeSlots) & 1) ^ 1, abort_flag, a.err);
-    float* racc_s = racc + ms * (C::NCW * GW * kD);
-    float* rm_s = rm + ms * (C::NCW * GW);
-    float* rl_s = rl + ms * (C::NCW * GW);
-#pragma unroll
-    for (int jj = 0; jj < GW; ++jj)
-      *reinterpret_cast<float4*>(racc_s + (warp * GW + jj) * kD + lane * 4) =
-          make_float4(acc[jj][0].x, acc[jj][0].y, acc[jj][1].x, acc[jj][1].y);
-    if (writer && tp == 0) {
-      rm_s[warp * GW + hh] = m;
-      rl_s[warp * GW + hh] = l;
-    }
-    __threadfence_block();
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(&mcnt[ms], 1) == C::NCW - 1;
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) continue;
-    __threadfence_block();
     const int nparts = fstart[s + 1] - fstart[s] + 1;
-    // outputs: HB kv-heads x G q-heads x 32 chunks of 4 dims
-    for (int o = lane; o < HB * G * 32; o += 32) {
-      const int c4 = o & 31;
-      const int r = o >> 5;                // q-head within the item
-      const int kv = r / G, rg = r % G;    // kv-head within the pair, head in its group
-      const int g2 = rg / GW, jj = rg % GW;
-      float M = -INFINITY;
 #pragma unroll
-      for (int t2 = 0; t2 < C::TGS; ++t2) {
-        const int w2 = (t2 * C::HG + g2) * HB + kv;
-        M = fmaxf(M, rm_s[w2 * GW + jj]);
-      }
-      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-      float den = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int t2 = 0; t2 < C::TGS; ++t2) {
-          const int w2 = (t2 * C::HG + g2) * HB + kv;
-          const float mw = rm_s[w2 * GW + jj];
-          const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - M);
-          den += f * rl_s[w2 * GW + jj];
-          const float4 v = *reinterpret_cast<const float4*>(racc_s + (w2 * GW + jj) * kD + c4 * 4);
-          num.x += f * v.x; num.y += f * v.y; num.z += f * v.z; num.w += f * v.w;
-        }
-      }
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      const int qh = (hp * HB + kv) * G + rg;
+    for (int jj = 0; jj < GW; ++jj) {
+      const float lj = __shfl_sync(0xffffffffu, l, lane_of_head<GW>(jj));
+      const float mj = __shfl_sync(0xffffffffu, m, lane_of_head<GW>(jj));
+      const float inv = lj > 0.f ? 1.f / lj : 0.f;
+      const int qh = (hp * HB + warp) * G + jj;
+      const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
+      const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
       if (nparts == 1) {
-        const uint32_t lo = Elem<T>::pack2(num.x * inv, num.y * inv);
-        const uint32_t hi = Elem<T>::pack2(num.z * inv, num.w * inv);
-        T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + qh) * kD + c4 * 4;
-        *reinterpret_cast<uint2*>(ob) = make_uint2(lo, hi);
+        T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + qh) * kD + lane * 4;
+        *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
       } else {
         const long long row = ((long long)s * a.num_q_heads + qh) * a.max_parts + p;
-        *reinterpret_cast<float4*>(a.part_o + row * kD + c4 * 4) =
-            make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
-        if (c4 == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(M, den);
+        *reinterpret_cast<float4*>(a.part_o + row * kD + lane * 4) = make_float4(o0, o1, o2, o3);
+        if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
       }
-    }
-    __syncwarp();
-    if (lane == 0) {
-      mcnt[ms] = 0;
-      __threadfence_block();
-      mbar_arrive(&mfree[ms]);
     }
   }
 }
@@ -626,7 +570,6 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
   const int n = max(1, cdiv(L, a.part_size));
   if (n <= 1) return;  // written by the decode kernel
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (long long)gw * a.max_parts;
-  // lane i holds partition i's (m, l) for the first 32 partitions
   float M = -INFINITY;
   for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
 #pragma unroll
@@ -634,28 +577,25 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
   float den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* po = a.part_o + (long long)gw * a.max_parts * kD + lane * 4;
-  int i = 0;
-  for (; i + 4 <= n; i += 4) {
-    float f[4];
-    float4 o[4];
+  // eight partitions per round: all loads of a round are in flight together
+  for (int i0 = 0; i0 < n; i0 += 8) {
+    float2 mlv[8];
+    float4 ov[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 v = ml[i + u];
-      f[u] = v.x == -INFINITY ? 0.f : fast_exp2(v.x - M) * v.y;
-      o[u] = *reinterpret_cast<const float4*>(po + (long long)(i + u) * kD);
+    for (int u = 0; u < 8; ++u) {
+      if (i0 + u < n) {
+        mlv[u] = ml[i0 + u];
+        ov[u] = *reinterpret_cast<const float4*>(po + (long long)(i0 + u) * kD);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      den += f[u];
-      num.x += f[u] * o[u].x; num.y += f[u] * o[u].y; num.z += f[u] * o[u].z; num.w += f[u] * o[u].w;
+    for (int u = 0; u < 8; ++u) {
+      if (i0 + u < n) {
+        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - M) * mlv[u].y;
+        den += f;
+        num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
+      }
     }
-  }
-  for (; i < n; ++i) {
-    const float2 v = ml[i];
-    const float f = v.x == -INFINITY ? 0.f : fast_exp2(v.x - M) * v.y;
-    den += f;
-    const float4 o = *reinterpret_cast<const float4*>(po + (long long)i * kD);
-    num.x += f * o.x; num.y += f * o.y; num.z += f * o.z; num.w += f * o.w;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* ob = static_cast<T*>(a.out) + (long long)gw * kD + lane * 4;
@@ -663,14 +603,29 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
       make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
 }
 
-constexpr int kDefaultPartition = 512;
+constexpr int kDefaultPartition = 256;
 constexpr int kMaxPartition = kMaxTilesPerItem * kTileTok;
-constexpr int kConsumerWarps = 8;
 constexpr int kMaxSeqs = 4096;
 constexpr int kMaxSmem = 227 * 1024;
 
-inline int choose_partition(int partition_size) {
-  return partition_size > 0 ? partition_size : kDefaultPartition;
+// kv-heads per item: all of them up to eight (whole 2 KB rows for 8 heads of 128)
+inline int heads_per_item(int num_kv_heads) {
+  for (int hb = 8; hb > 1; hb >>= 1)
+    if (num_kv_heads % hb == 0) return hb;
+  return 1;
+}
+
+// Library choice of the split-K partition: 256 tokens, halved (down to 64) while even
+// the upper bound on the work items (every sequence at max_seq_len) would leave fewer
+// than four items per SM for the dynamic schedule to balance.
+inline int choose_partition(int partition_size, int num_seqs, int num_kv_heads,
+                            int max_seq_len) {
+  if (partition_size > 0) return partition_size;
+  const long long groups = (long long)num_seqs * (num_kv_heads / heads_per_item(num_kv_heads));
+  const int sms = std::max(1, num_sms());
+  int P = kDefaultPartition;
+  while (P > 64 && groups * std::max(1, (max_seq_len + P - 1) / P) < 4LL * sms) P /= 2;
+  return P;
 }
 
 inline int num_parts_host(int max_seq_len, int P) { return std::max(1, (max_seq_len + P - 1) / P); }
@@ -678,15 +633,15 @@ inline int num_parts_host(int max_seq_len, int P) { return std::max(1, (max_seq_
 template <typename T, int G, int HB>
 pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                         DecodeArgs a, cudaStream_t stream) {
-  using C = DecodeCfg<G, HB, kConsumerWarps>;
+  using C = DecodeCfg<G, HB>;
   const size_t ring_off = ((C::OFF_SEQ + (size_t)(3 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
-  if (ring_off + (size_t)2 * C::TGS * C::SLOT_BYTES > kMaxSmem) return PA_ERR_UNSUPPORTED;
-  int nsw = (int)((kMaxSmem - ring_off) / ((size_t)C::TGS * C::SLOT_BYTES));
-  nsw = std::min(nsw, kMaxSlots / C::TGS);
-  if (nsw < 2) return PA_ERR_UNSUPPORTED;
-  a.slots_per_ring = nsw;
-  const size_t smem = ring_off + (size_t)C::TGS * nsw * C::SLOT_BYTES;
-  auto kern = paged_decode_kernel<T, G, HB, kConsumerWarps>;
+  const long long room = (long long)kMaxSmem - (long long)ring_off;
+  const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
+  if (nslots < 2) return PA_ERR_UNSUPPORTED;
+  a.ring_off = (int)ring_off;
+  a.nslots = nslots;
+  const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
+  auto kern = paged_decode_kernel<T, G, HB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
@@ -694,6 +649,7 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   const int sms = num_sms();
   if (sms <= 0) return PA_ERR_CUDA;
   const int grid = (int)std::min<long long>(items_max, sms);
+  if (cudaMemsetAsync(a.counter, 0, sizeof(int), stream) != cudaSuccess) return PA_ERR_CUDA;
   kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
@@ -707,14 +663,26 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   return PA_OK;
 }
 
-template <typename T, int HB>
-pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV,
+template <typename T, int G>
+pa_status dispatch_hb(int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                      const CUtensorMap& tmQ, const DecodeArgs& a, cudaStream_t stream) {
+  switch (HB) {
+    case 1: return launch_decode<T, G, 1>(tmK, tmV, tmQ, a, stream);
+    case 2: return launch_decode<T, G, 2>(tmK, tmV, tmQ, a, stream);
+    case 4: return launch_decode<T, G, 4>(tmK, tmV, tmQ, a, stream);
+    case 8: return launch_decode<T, G, 8>(tmK, tmV, tmQ, a, stream);
+    default: return PA_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T>
+pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const CUtensorMap& tmQ, const DecodeArgs& a, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_decode<T, 1, HB>(tmK, tmV, tmQ, a, stream);
-    case 2: return launch_decode<T, 2, HB>(tmK, tmV, tmQ, a, stream);
-    case 4: return launch_decode<T, 4, HB>(tmK, tmV, tmQ, a, stream);
-    case 8: return launch_decode<T, 8, HB>(tmK, tmV, tmQ, a, stream);
+    case 1: return dispatch_hb<T, 1>(HB, tmK, tmV, tmQ, a, stream);
+    case 2: return dispatch_hb<T, 2>(HB, tmK, tmV, tmQ, a, stream);
+    case 4: return dispatch_hb<T, 4>(HB, tmK, tmV, tmQ, a, stream);
+    case 8: return dispatch_hb<T, 8>(HB, tmK, tmV, tmQ, a, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -724,10 +692,12 @@ pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV,
 extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim,
                                            int max_seq_len, int partition_size) {
   if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
-  const int P = pa::choose_partition(partition_size);
+  // the automatic choice may pick down to 64 tokens; size for the most partitions
+  const int P = partition_size > 0 ? partition_size : 64;
   const int parts = pa::num_parts_host(max_seq_len, P);
-  if (parts <= 1) return 0;
-  return (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * sizeof(float);
+  const size_t partials =
+      parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * sizeof(float) : 0;
+  return pa::kWorkspaceHeader + partials;
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -754,21 +724,20 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
   if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
     return PA_ERR_INVALID_ARG;
-  const int P = pa::choose_partition(partition_size);
+  const int P = pa::choose_partition(partition_size, num_seqs, num_kv_heads, max_seq_len);
   const int parts = pa::num_parts_host(max_seq_len, P);
-  const size_t need =
-      pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, partition_size);
-  if (need && (!workspace || workspace_bytes < need)) return PA_ERR_WORKSPACE_TOO_SMALL;
-  if (need && ((uintptr_t)workspace & 15)) return PA_ERR_INVALID_ARG;
+  const size_t partials = parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * 4 : 0;
+  const size_t need = pa::kWorkspaceHeader + partials;
+  if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
+  if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
   int* err = pa::device_error_flag();
   if (!err) return PA_ERR_CUDA;
 
-  // two kv-heads per item and TMA box when the head count allows (512-byte rows)
-  const int HB = (num_kv_heads % 2 == 0) ? 2 : 1;
+  const int HB = pa::heads_per_item(num_kv_heads);
   CUtensorMap tmK, tmV, tmQ;
+  const uint64_t row = (uint64_t)head_dim * 2;
   const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
                              (uint64_t)num_blocks};
-  const uint64_t row = (uint64_t)head_dim * 2;
   const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
   const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
   const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads, (uint64_t)num_seqs};
@@ -779,13 +748,14 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
       !pa::encode_tmap_16bit(&tmQ, q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))
     return PA_ERR_CUDA;
 
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   pa::DecodeArgs a;
   a.out = out;
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
-  a.part_o = need ? static_cast<float*>(workspace) : nullptr;
-  a.part_ml = need ? static_cast<float*>(workspace) + (size_t)num_seqs * num_q_heads * parts * head_dim
-                   : nullptr;
+  a.counter = reinterpret_cast<int*>(ws);
+  a.part_o = partials ? reinterpret_cast<float*>(ws + pa::kWorkspaceHeader) : nullptr;
+  a.part_ml = partials ? a.part_o + (size_t)num_seqs * num_q_heads * parts * head_dim : nullptr;
   a.err = err;
   a.num_seqs = num_seqs;
   a.num_q_heads = num_q_heads;
@@ -797,24 +767,22 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   a.max_parts = parts;
   const long long cap_tbl = (long long)max_blocks_per_seq * block_size;
   a.seq_cap = (int)std::min<long long>(cap_tbl, max_seq_len);
-  a.slots_per_ring = 0;
+  a.ring_off = 0;
+  a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PA_F16)
-    return HB == 2 ? pa::dispatch_group<__half, 2>(G, tmK, tmV, tmQ, a, st)
-                   : pa::dispatch_group<__half, 1>(G, tmK, tmV, tmQ, a, st);
-  return HB == 2 ? pa::dispatch_group<__nv_bfloat16, 2>(G, tmK, tmV, tmQ, a, st)
-                 : pa::dispatch_group<__nv_bfloat16, 1>(G, tmK, tmV, tmQ, a, st);
+  return dtype == PA_F16 ? pa::dispatch_group<__half>(G, HB, tmK, tmV, tmQ, a, st)
+                         : pa::dispatch_group<__nv_bfloat16>(G, HB, tmK, tmV, tmQ, a, st);
 }
 
-// ---------------------------------------------------------------------------
 // Decode without any caller-provided scratch.
 //
 // Some callers cannot allocate device memory on their own: code that runs inside a
 // serving loop whose memory is entirely owned by an engine's pre-allocated pool (the
 // pool hands out KV blocks, not scratch buffers), plugins whose host framework forbids
 // raw cudaMalloc, and latency-critical paths where an allocation could synchronise the
-// device.  For them this entry point keeps the split-K partials in a fixed array that
+// device.  For them this entry point keeps its workspace (the work-item counter and the
+// split-K partials) in a fixed array that
 // lives in this file (kNoAllocScratchBytes on every GPU that loads the library, held
 // until the process exits) and otherwise runs exactly pa_decode.
 // ---------------------------------------------------------------------------
@@ -851,14 +819,11 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
   const size_t need =
       pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, partition_size);
   if (need > kNoAllocScratchBytes) return PA_ERR_WORKSPACE_TOO_SMALL;
-  void* scratch = nullptr;
-  if (need) {
-    scratch = scratch_for_current_device();
-    if (!scratch) return PA_ERR_CUDA;
-  }
+  void* scratch = scratch_for_current_device();
+  if (!scratch) return PA_ERR_CUDA;
   return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
                    num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size, num_blocks,
-                   max_seq_len, partition_size, scratch, need ? kNoAllocScratchBytes : 0, dtype,
+                   max_seq_len, partition_size, scratch, kNoAllocScratchBytes, dtype,
                    stream);
 }
 

@@ -18,8 +18,9 @@
 
 namespace pa {
 
-// Longest any single pipeline wait may take before the kernel gives up.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// Longest any single pipeline wait may take before the kernel gives up, in SM clock
+// cycles (the per-SM counter is cheap to read; ~2 s at B200 clocks).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
@@ -29,11 +30,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -86,13 +82,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and flags PA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitNs.
+// (and flags PA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       flag_error(err, PA_DEVERR_TIMEOUT);
       return false;
     }

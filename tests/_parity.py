@@ -67,7 +67,7 @@ def gpu_decode(batch: workloads.PagedBatch, partition_size=0, max_seq_len=None, 
     B, Hq, D = batch.q.shape
     msl = batch.max_seq_len if max_seq_len is None else max_seq_len
     ws_bytes = pa.pa_decode_workspace_size(B, Hq, D, msl, partition_size)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=batch.q.device) if ws_bytes else None
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=batch.q.device)
     out = torch.empty_like(batch.q)
     pa.pa_decode(out, batch.q, batch.k_cache, batch.v_cache, batch.block_tables, batch.seq_lens,
                  batch.scale, msl, partition_size, ws, stream=stream)

@@ -55,13 +55,17 @@ def test_status_strings(palib):
 
 
 def test_workspace_size_arithmetic(palib):
-    # one partition covers the sequence -> no scratch
-    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 0) == 0
-    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 512) == 0
+    H = 256  # header: the kernel's work-item counter
+    # one partition covers the sequence -> the header alone
+    assert palib.pa_decode_workspace_size(64, 32, 128, 64, 0) == H
+    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 512) == H
+    # automatic choice: sized for 64-token partitions, the smallest the library picks
+    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 0) == H + 64 * 32 * 8 * 130 * 4
     # 8000 tokens at 512 per partition -> 16 partitions of (128 + 2) fp32 per (seq, q-head)
-    assert palib.pa_decode_workspace_size(64, 32, 128, 8000, 512) == 64 * 32 * 16 * 130 * 4
-    assert palib.pa_decode_workspace_size(32, 64, 128, 32768, 512) == 32 * 64 * 64 * 130 * 4
-    assert palib.pa_decode_workspace_size(2, 8, 128, 100, 16) == 2 * 8 * 7 * 130 * 4
+    assert palib.pa_decode_workspace_size(64, 32, 128, 8000, 512) == H + 64 * 32 * 16 * 130 * 4
+    assert palib.pa_decode_workspace_size(32, 64, 128, 32768, 512) == H + 32 * 64 * 64 * 130 * 4
+    assert palib.pa_decode_workspace_size(2, 8, 128, 100, 16) == H + 2 * 8 * 7 * 130 * 4
+    assert palib.pa_decode_workspace_size(0, 8, 128, 100, 16) == 0  # invalid shape
     assert palib.pa_chunked_prefill_workspace_size(4, 512, 64, 128, 8000) == 0
 
 
@@ -99,8 +103,10 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(q=ctypes.c_void_p(4100)) == 1  # misaligned
     assert dec(dt=3) == 2
     assert dec(B=0) == 0                     # nothing to do
-    assert dec(maxlen=8000, P=512) == 3      # needs a workspace
+    assert dec(B=5000) == 2                  # more sequences than the schedule holds
+    assert dec(P=512) == 3                   # every call needs a workspace (item counter)
     assert dec(maxlen=8000, P=512, ws=p, wsb=100) == 3
+    assert dec(maxlen=8000, P=512, ws=ctypes.c_void_p(4096 + 16), wsb=1 << 24) == 1  # alignment
 
 
 def test_product_package_does_not_touch_oracle():

@@ -3,11 +3,11 @@
 Some callers of this library never call cudaMalloc themselves: their device memory
 belongs to an engine's pre-allocated KV pool or to a host framework that forbids raw
 allocations, or they run in a latency-critical loop where an allocation could
-synchronise the device.  pa_decode_noalloc serves them by keeping the split-K partials
-in a fixed array inside the library.  These checks run through the C ABI on a GPU:
-two calls in a row must reproduce pa_decode with a caller-provided workspace (within
-the parity tolerance), and sizes whose partials do not fit the array must be refused
-before anything is launched.  The file sorts last so a fail-fast run has already run
+synchronise the device.  pa_decode_noalloc serves them by keeping its workspace (the
+work-item counter and the split-K partials) in a fixed array inside the library.
+These checks run through the C ABI on a GPU: two calls in a row must reproduce
+pa_decode with a caller-provided workspace (within the parity tolerance), and sizes
+whose partials do not fit the array must be refused before anything is launched.  The file sorts last so a fail-fast run has already run
 every other test when it gets here.
 """
 import ctypes
@@ -41,10 +41,10 @@ def test_noalloc_matches_workspace_decode_twice():
         assert diff <= tol, diff
 
 
-def test_noalloc_single_partition_needs_no_scratch():
+def test_noalloc_single_partition():
     b = workloads.tiny_mha(device="cuda")[0]
     P.gpu_append(b)
-    ref = P.gpu_decode(b, partition_size=256)  # one partition: no workspace
+    ref = P.gpu_decode(b, partition_size=256)  # one partition: no merge pass
     out = torch.empty_like(b.q)
     pa.pa_decode_noalloc(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens, b.scale,
                          b.max_seq_len, partition_size=256)
