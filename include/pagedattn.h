@@ -92,13 +92,12 @@ PA_API pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cach
                                void* stream);
 
 /*
- * Bytes of scratch `pa_decode` needs: a 256-byte header (the kernel's work-item
- * counter, reset by pa_decode on the stream before every launch) followed, when some
- * sequence may span more than one partition, by the split-K partials: per (sequence,
- * q-head, partition) the normalised partial output (head_dim fp32) and its running max
- * and sum (2 fp32).  partition_size 0 sizes for the smallest partition the library may
- * choose (64 tokens), which covers whatever pa_decode picks.  Never 0 for a valid
- * shape; 0 means invalid arguments.
+ * Bytes of scratch `pa_decode` needs, as an upper bound valid for every kv-head count
+ * and GPU: merge records (8 bytes per sequence and q-head, padded to 256 bytes), then
+ * split-K partial rows of head_dim+2 fp32 (normalised partial output, running max and
+ * sum): (256 + num_seqs) * num_q_heads rows, plus, when partition_size > 0,
+ * num_seqs * num_q_heads * ceil(ceil(max_seq_len/16) / (partition_size/16)) +
+ * num_q_heads rows.  0 means invalid arguments.
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_seq_len,
                                 int partition_size);
@@ -116,12 +115,12 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   seq_lens      int32 [num_seqs] (device): tokens of each sequence, 0 gives zeros
  *   max_seq_len   host-side upper bound of seq_lens; sizes the grid and the
  *                 partition count.  A longer sequence sets PA_DEVERR_SEQ_TOO_LONG.
- *   partition_size  split-K partition in tokens (multiple of 16, at most 2048),
- *                 0 = library choice: 256 tokens, halved down to 64 while the batch
- *                 would give the SMs fewer than four work items each.
- *                 A work item is (sequence, partition, group of up to 8 kv-heads); a
- *                 persistent grid takes items largest-first from a device counter.
- *                 Sequences longer than one partition are merged by a log-sum-exp pass.
+ *   partition_size  0 = balanced split-K: the 16-token tiles of every (sequence, group of
+ *                 up to 8 kv-heads) are laid end to end and a persistent grid of one CTA
+ *                 per SM takes equal shares; a sequence held by one CTA is written
+ *                 directly, the others are merged by a log-sum-exp pass.  > 0 (a
+ *                 multiple of 16, at most 2048) also caps every share at that many
+ *                 tokens, using more CTAs.
  *   workspace     device scratch, 256-byte aligned, of at least
  *                 pa_decode_workspace_size(...) bytes; contents need no initialisation.
  *                 Calls that overlap on the GPU must not share a workspace.
@@ -141,7 +140,7 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that
  * forbids raw cudaMalloc) or who must not risk the device-wide synchronisation an
  * allocation can cause.  Arguments and results are those of pa_decode without the
- * workspace: the work-item counter and split-K partials go to a fixed array inside the library,
+ * workspace: the merge records and split-K partials go to a fixed array inside the library,
  * pa_decode_noalloc_scratch_bytes() long (32 MiB), which every GPU that loads the
  * library holds until the process exits.
  *  - Sizes whose partials need more than that (pa_decode_workspace_size(...) >

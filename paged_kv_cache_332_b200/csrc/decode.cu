@@ -16,26 +16,29 @@
 //    second box the same of V.  Measured on B200, boxes of one or two kv-heads (256 or
 //    512-byte runs scattered over randomly placed blocks) stream at 2.4-4.4 TB/s while
 //    whole 2 KB rows stream at 7 TB/s.
-//  * Work item = (sequence, partition of P tokens, group of HB kv-heads).  Items are
-//    ordered every full partition first, then each sequence's last partition largest
-//    first; a persistent grid of one CTA per SM hands them out through an atomic counter
-//    (a largest-first dynamic schedule).
-//  * One consumer warp per kv-head of the item handles all G q-heads of that kv-head
-//    over every tile of the item, so no two warps share an output and no merge inside
-//    the CTA is needed.  q.k: 8 lanes split a token's 128 dims (16 each, two 16-byte
-//    shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving exchange that
-//    sums all G heads at once.  Online softmax (running max m, sum l) in the log2 domain
-//    (q pre-scaled by scale*log2 e: one ex2 per logit); p.V with lanes over head_dim.
-//  * A staging warp claims items and, up to two items ahead, copies their block-table
-//    entries into shared memory (one coalesced read per 32 entries) and starts the TMA
-//    copy of their q rows.  A producer thread walks the tiles in order and issues the
-//    two boxes of each as soon as a slot of the shared ring frees (blocking waits take
-//    no issue slots from the consumers).
-//  * A sequence that fits one partition writes `out` directly; longer ones write
-//    normalised partials (o, m, l) to the caller's workspace, merged by a log-sum-exp pass
-//    (lse_reduce_kernel).
+//  * Balanced split-K.  The tiles of every (sequence, group of HB kv-heads) are laid end
+//    to end, and CTA c of a persistent grid (one per SM) takes the c-th equal share of
+//    that list.  Every CTA moves the same number of bytes, whatever the length mix, and
+//    a sequence is split only where a share boundary falls inside it.  The piece of a
+//    sequence that a CTA sees is a segment: a sequence held by one CTA is written to
+//    `out` directly; the others leave normalised partials (o, m, l) in the caller's
+//    workspace at slot c + group, merged by a log-sum-exp pass (lse_reduce_kernel).
+//    An explicit partition size caps the share, so no segment is longer.
+//  * One consumer warp per kv-head of the group handles all G q-heads of that kv-head,
+//    so no two warps share an output.  q.k: 8 lanes split a token's 128 dims (16 each,
+//    two 16-byte shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving
+//    exchange that sums all G heads at once.  Online softmax (running max m, sum l) in
+//    the log2 domain (q pre-scaled by scale*log2 e: one ex2 per logit); p.V with lanes
+//    over head_dim.  With G = 8 the consumers take registers from the producer side of
+//    the CTA (setmaxnreg) to hold 8 q rows without spilling.
+//  * A staging warp cuts the CTA's share into units of at most 128 tiles and, up to two
+//    units ahead, copies their block-table entries into shared memory (one coalesced
+//    read per 32 entries) and starts the TMA copy of their q rows.  A producer thread
+//    walks the tiles in order and issues the two boxes of each as soon as a slot of the
+//    shared ring frees (blocking waits take no issue slots from the consumers).
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
 #include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "pa_device.cuh"
@@ -47,12 +50,12 @@ struct DecodeArgs {
   void* out;
   const int32_t* block_tables;
   const int32_t* seq_lens;
-  float* part_o;   // [B, Hq, max_parts, 128]
-  float* part_ml;  // [B, Hq, max_parts, 2]   (max in log2 units, sum)
-  int* counter;    // dynamic item counter (zeroed before the launch)
+  float* part_o;   // [slots, HB*G, 128]   normalised partial outputs
+  float* part_ml;  // [slots, HB*G, 2]     (max in log2 units, sum)
+  int2* meta;      // [B * NHP]            (first slot, slot count) of each group
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
-  int part_size, max_parts, seq_cap;
+  int seq_cap;
   int ring_off, nslots;  // shared-memory offset of the tile ring and its slot count
   float qscale;          // scale * log2(e)
 };
@@ -60,24 +63,33 @@ struct DecodeArgs {
 constexpr int kD = 128;
 constexpr int kTileTok = 16;
 constexpr int kRowBytes = kD * 2;      // one token of one kv-head
-constexpr int kQSlots = 2;             // items staged ahead
+constexpr int kQSlots = 2;             // units staged ahead
 constexpr int kMaxSlots = 8;
-constexpr int kMaxTilesPerItem = 128;  // partition <= 2048 tokens
-constexpr int kSortBuckets = 128;      // = 32 lanes x 4 in the bucket scan
-constexpr int kWorkspaceHeader = 256;  // bytes: the item counter
+constexpr int kMaxTilesPerUnit = 128;
+constexpr int kMaxGrid = 256;          // persistent grid: min(SMs, this)
+// unit flags
+constexpr int kFirst = 1;   // first unit of a segment: load q, reset the softmax state
+constexpr int kLast = 2;    // last unit of a segment: write the result
+constexpr int kDirect = 4;  // the segment is the whole group: write `out`
 
 template <int G_, int HB_>
 struct DecodeCfg {
   static constexpr int G = G_;
-  static constexpr int HB = HB_;                  // kv-heads per item = consumer warps
-  static constexpr int GW = G;                    // q-heads per warp
-  static constexpr int THREADS = (HB + 2) * 32;   // + producer warp + staging warp
-  static constexpr int WARP_PROD = HB;
-  static constexpr int WARP_STAGE = HB + 1;
+  static constexpr int HB = HB_;                  // kv-heads per group = consumer warps
+  static constexpr int GW = G;                    // q-heads per consumer warp
+  static constexpr int WARP_PROD = 0;
+  static constexpr int WARP_STAGE = 1;
+  static constexpr int WARP_FILL = 2;             // zero-fills empty sequences
+  static constexpr int WARP_C0 = 4;               // first consumer warp
+  static constexpr int THREADS = 128 + HB * 32;
+  // G = 8 with eight consumer warps: 12 warps at launch get 168 registers each; the
+  // first warpgroup gives back down to 72 so each consumer can grow to 216
+  // (128*72 + 256*216 = 384*168).
+  static constexpr bool SPLIT_REGS = (HB == 8 && G == 8);
   static constexpr int DUPMASK = GW == 8 ? 0 : (GW == 4 ? 1 : (GW == 2 ? 3 : 7));
   static constexpr int TILE_BYTES = kTileTok * HB * kRowBytes;  // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
-  static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of an item
+  static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of a group
   // shared-memory carve-up (bytes); the sequence arrays and then the ring follow
   static constexpr int OFF_FULL = 0;
   static constexpr int OFF_EMPTY = OFF_FULL + kMaxSlots * 8;
@@ -85,15 +97,15 @@ struct DecodeCfg {
   static constexpr int OFF_QEMPTY = OFF_QFULL + kQSlots * 8;
   static constexpr int OFF_TFULL = OFF_QEMPTY + kQSlots * 8;
   static constexpr int OFF_TEMPTY = OFF_TFULL + kQSlots * 8;
-  static constexpr int OFF_ITEM = OFF_TEMPTY + kQSlots * 8;     // claimed item per slot
-  static constexpr int OFF_ABORT = OFF_ITEM + kQSlots * 4;
+  static constexpr int OFF_UNIT = OFF_TEMPTY + kQSlots * 8;     // 8 ints per staged unit
+  static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 32;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
-  static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerItem * 4;
+  static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerUnit * 4;
   static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;          // p pairs per warp
   static constexpr int OFF_A = OFF_P + HB * kTileTok * GW * 8;     // alpha per warp
-  static constexpr int OFF_SORT = ((OFF_A + HB * GW * 4 + 15) / 16) * 16;
-  static constexpr int OFF_SEQ = OFF_SORT + kSortBuckets * 4;       // 3 int arrays
+  static constexpr int OFF_SEQ = ((OFF_A + HB * GW * 4 + 15) / 16) * 16;  // 2B+1 ints
   static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
+  static_assert(!SPLIT_REGS || THREADS == 384, "register split assumes three warpgroups");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -185,33 +197,12 @@ __device__ __forceinline__ int lane_of_head(int jj) {
   return GW == 8 ? jj : (GW == 4 ? (((jj >> 1) << 2) | ((jj & 1) << 1)) : (GW == 2 ? jj * 4 : 0));
 }
 
-// The launch's item order: item i -> (sequence s, partition p, kv-head group hp).
-struct Schedule {
-  const int* fstart;  // [B+1] prefix of full partitions per sequence
-  const int* slen;    // [B]   clamped lengths
-  const int* order;   // [B]   sequences by size of their last partition, largest first
-  int B, NHP, P, nfull;
-  __device__ __forceinline__ void item(int i, int& s, int& p, int& hp) const {
-    const int sp = i / NHP;
-    hp = i - sp * NHP;
-    if (sp < nfull) {
-      int lo = 0, hi = B - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (fstart[mid] <= sp) lo = mid; else hi = mid - 1;
-      }
-      s = lo;
-      p = sp - fstart[lo];
-    } else {
-      s = order[sp - nfull];
-      p = fstart[s + 1] - fstart[s];  // the last partition
-    }
-  }
-  __device__ __forceinline__ int ntiles(int s, int p) const {
-    const int tok0 = p * P;
-    return cdiv(max(min(slen[s], tok0 + P) - tok0, 0), kTileTok);
-  }
-};
+
+// CTA holding global tile `pos` when T tiles are shared out over `grid` CTAs
+// (CTA c holds [c*T/grid, (c+1)*T/grid)).
+__device__ __forceinline__ int cta_of(int pos, int T, int grid) {
+  return (int)((((long long)pos + 1) * grid - 1) / T);
+}
 
 template <typename T, int G, int HB>
 __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
@@ -220,6 +211,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
                         const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
   using C = DecodeCfg<G, HB>;
   constexpr int GW = C::GW;
+  constexpr int HBG = HB * G;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
@@ -227,27 +219,24 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
   uint64_t* qempty = reinterpret_cast<uint64_t*>(smem + C::OFF_QEMPTY);
   uint64_t* tfull = reinterpret_cast<uint64_t*>(smem + C::OFF_TFULL);
   uint64_t* tempty = reinterpret_cast<uint64_t*>(smem + C::OFF_TEMPTY);
-  volatile int* item_of = reinterpret_cast<volatile int*>(smem + C::OFF_ITEM);
+  volatile int* unit = reinterpret_cast<volatile int*>(smem + C::OFF_UNIT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
   int* tbl = reinterpret_cast<int*>(smem + C::OFF_TBL);
   uint8_t* qbuf = smem + C::OFF_Q;
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
   float* abuf = reinterpret_cast<float*>(smem + C::OFF_A);
-  int* cursor = reinterpret_cast<int*>(smem + C::OFF_SORT);
   const int B = a.num_seqs;
-  int* fstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);
-  int* slen = fstart + B + 1;
-  int* order = slen + B;
+  int* sstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);  // [B+1] first tile of each sequence
+  int* slen = sstart + B + 1;                                // [B]   clamped lengths
   uint8_t* ring = smem + a.ring_off;
   const int nslots = a.nslots;
+  const int NHP = a.num_kv_heads / HB;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int P = a.part_size;
 
-  // ---- schedule: clamped lengths, full-partition prefix, last partitions by size
+  // ---- clamped lengths and the prefix of tiles over (sequence, head group)
   if (warp == 0) {
-    for (int b = lane; b < kSortBuckets; b += 32) cursor[b] = 0;
     const int per = (B + 31) / 32;
     const int lo = min(B, lane * per), hi = min(B, lo + per);
     int sum = 0;
@@ -256,7 +245,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
       const int L = clamp_len(raw, a.seq_cap);
       if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
       slen[s] = L;
-      sum += max(1, cdiv(L, P)) - 1;
+      sum += NHP * cdiv(L, kTileTok);
     }
     int incl = sum;
 #pragma unroll
@@ -266,47 +255,10 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
     }
     int run = incl - sum;
     for (int s = lo; s < hi; ++s) {
-      fstart[s] = run;
-      run += max(1, cdiv(slen[s], P)) - 1;
+      sstart[s] = run;
+      run += NHP * cdiv(slen[s], kTileTok);
     }
-    if (lane == 31) fstart[B] = incl;
-    __syncwarp();
-    // stable counting sort of the sequences by their last partition, largest first
-    auto bucket = [&](int s) {
-      const int L = slen[s];
-      const int r = L - (max(1, cdiv(L, P)) - 1) * P;  // 0..P
-      return (int)(((long long)(P - r) * kSortBuckets) / (P + 1));
-    };
-    for (int base = 0; base < B; base += 32) {
-      const int s = base + lane;
-      if (s < B) atomicAdd(&cursor[bucket(s)], 1);
-    }
-    __syncwarp();
-    {  // exclusive scan of the bucket counts, 4 buckets per lane
-      int c[4], tot = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) { c[j] = cursor[lane * 4 + j]; tot += c[j]; }
-      int inc = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += t;
-      }
-      int run2 = inc - tot;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) { cursor[lane * 4 + j] = run2; run2 += c[j]; }
-    }
-    __syncwarp();
-    for (int base = 0; base < B; base += 32) {
-      const int s = base + lane;
-      const int bk = s < B ? bucket(s) : kSortBuckets + lane;
-      const unsigned same = __match_any_sync(0xffffffffu, bk);
-      const int rank = __popc(same & ((1u << lane) - 1));
-      if (s < B) order[cursor[bk] + rank] = s;
-      __syncwarp();
-      if (s < B && rank == 0) cursor[bk] += __popc(same);
-      __syncwarp();
-    }
+    if (lane == 31) sstart[B] = incl;
   }
   if (threadIdx.x == C::WARP_STAGE * 32) {
     for (int i = 0; i < nslots; ++i) {
@@ -323,145 +275,193 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  const int NHP = a.num_kv_heads / HB;
-  Schedule sch{fstart, slen, order, B, NHP, P, fstart[B]};
-  const int total = (sch.nfull + B) * NHP;
+  const int Ttot = sstart[B];
+  // The launch sizes the grid for the longest possible batch; when the batch holds
+  // fewer tiles than CTAs, only the first Ttot CTAs take a share, so every share is
+  // non-empty and the segments of a group sit in consecutive CTAs (and slots).
+  const int grid = min((int)gridDim.x, max(Ttot, 1));
+  const int cta = blockIdx.x;
+  const int r0 = cta < grid ? (int)(((long long)cta * Ttot) / grid) : Ttot;
+  const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
 
-  if (warp == C::WARP_STAGE) {
-    // ===== staging warp: claims items; block-table entries + q rows, two items ahead =====
-    if (lane == 0) prefetch_tmap(&tmQ);
-    for (int k = 0;; ++k) {
-      const int qs = k % kQSlots;
-      const uint32_t par = ((k / kQSlots) & 1) ^ 1;
-      wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read item k-2's q
-      wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // its tiles were issued
-      int item = 0;
-      if (lane == 0) item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(a.counter, 1);
-      item = __shfl_sync(0xffffffffu, item, 0);
-      if (item >= total || *abort_flag) {  // tell the other warps there is no more work
-        if (lane == 0) {
-          item_of[qs] = -1;
-          mbar_arrive_expect_tx(&qfull[qs], 0);
-          mbar_arrive(&tfull[qs]);
-        }
-        break;
+  if (warp < C::WARP_C0) {
+    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    if (warp == C::WARP_FILL) {
+      // ===== empty sequences: no CTA visits them; zero their output and merge record =====
+      for (int s = cta; s < B; s += gridDim.x) {
+        if (slen[s] != 0) continue;
+        for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
+        T* ob = static_cast<T*>(a.out) + (long long)s * a.num_q_heads * kD;
+        for (int i = lane; i < a.num_q_heads * kD / 8; i += 32)
+          reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
       }
-      int s, p, hp;
-      sch.item(item, s, p, hp);
-      const int ntile = sch.ntiles(s, p);
-      const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
-      const int tok0 = p * P;
-      int ids[kMaxTilesPerItem / 32];
-#pragma unroll
-      for (int j = 0; j < kMaxTilesPerItem / 32; ++j) {
-        const int t = j * 32 + lane;
-        ids[j] = t < ntile ? __ldg(trow + ((tok0 + t * kTileTok) >> a.log2_bs)) : -1;
-      }
-#pragma unroll
-      for (int j = 0; j < kMaxTilesPerItem / 32; ++j) {
-        const int t = j * 32 + lane;
-        if (t < ntile) {
-          int id = ids[j];
-          if ((unsigned)id >= (unsigned)a.num_blocks) {
-            flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
-            id = -1;
-          }
-          tbl[qs * kMaxTilesPerItem + t] = id;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        item_of[qs] = item;
-        mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
-        tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HB * G, s, &qfull[qs]);
-        mbar_arrive(&tfull[qs]);
-      }
+      return;
     }
-    return;
-  }
-
-  if (warp == C::WARP_PROD) {
-    // ===== producer: one thread walks every tile in order into the shared ring =====
-    if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int bs_mask = (1 << a.log2_bs) - 1;
-      int cnt = 0;
+    if (warp == C::WARP_STAGE) {
+      // ===== staging warp: cuts the share into units; table entries + q, two units ahead =====
+      if (lane == 0) prefetch_tmap(&tmQ);
+      int pos = r0;
+      int s = 0;
+      if (pos < r1) {  // sequence holding pos: the last s with sstart[s] <= pos
+        int lo = 0, hi = B - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (sstart[mid] <= pos) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+      }
       for (int k = 0;; ++k) {
         const int qs = k % kQSlots;
-        wait_or_abort(&tfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-        const int item = item_of[qs];
-        if (item < 0 || *abort_flag) break;
-        int s, p, hp;
-        sch.item(item, s, p, hp);
-        const int ntile = sch.ntiles(s, p);
-        for (int t = 0; t < ntile; ++t, ++cnt) {
-          const int slot = cnt % nslots;
-          wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err);
-          const int bid = *abort_flag ? -1 : tbl[qs * kMaxTilesPerItem + t];
-          mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
-          if (bid >= 0) {
-            const int row = (p * P + t * kTileTok) & bs_mask;
-            uint8_t* dst = ring + slot * C::SLOT_BYTES;
-            tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
-            tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
+        const uint32_t par = ((k / kQSlots) & 1) ^ 1;
+        wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read unit k-2's q
+        wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // its tiles were issued
+        volatile int* u = unit + qs * 8;
+        if (pos >= r1 || *abort_flag) {  // tell the other warps there is no more work
+          if (lane == 0) {
+            u[0] = -1;
+            mbar_arrive_expect_tx(&qfull[qs], 0);
+            mbar_arrive(&tfull[qs]);
+          }
+          break;
+        }
+        const int nt = cdiv(slen[s], kTileTok);  // > 0: pos lies in this sequence
+        const int off = pos - sstart[s];
+        const int hp = off / nt;
+        const int t0 = off - hp * nt;
+        const int t1 = min(nt, t0 + min(r1 - pos, kMaxTilesPerUnit));
+        const int grp = s * NHP + hp;
+        const int gs = sstart[s] + hp * nt;  // the group's first and one-past-last tile
+        const int ge = gs + nt;
+        int flags = 0;
+        if (t0 == 0 || pos == r0) flags |= kFirst;
+        if (t1 == nt || pos + (t1 - t0) == r1) flags |= kLast;
+        if (gs >= r0 && ge <= r1) flags |= kDirect;
+        const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
+        int ids[kMaxTilesPerUnit / 32];
+  #pragma unroll
+        for (int j = 0; j < kMaxTilesPerUnit / 32; ++j) {
+          const int t = t0 + j * 32 + lane;
+          ids[j] = t < t1 ? __ldg(trow + ((t * kTileTok) >> a.log2_bs)) : -1;
+        }
+  #pragma unroll
+        for (int j = 0; j < kMaxTilesPerUnit / 32; ++j) {
+          const int i = j * 32 + lane;
+          if (t0 + i < t1) {
+            int id = ids[j];
+            if ((unsigned)id >= (unsigned)a.num_blocks) {
+              flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
+              id = -1;
+            }
+            tbl[qs * kMaxTilesPerUnit + i] = id;
           }
         }
-        mbar_arrive(&tempty[qs]);
+        __syncwarp();
+        if (lane == 0) {
+          if (t0 == 0) a.meta[grp] = make_int2(cta + grp, cta_of(ge - 1, Ttot, grid) - cta + 1);
+          u[0] = s;
+          u[1] = hp;
+          u[2] = t0;
+          u[3] = t1;
+          u[4] = flags;
+          u[5] = cta + grp;
+          if (flags & kFirst) {
+            mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
+            tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HBG, s, &qfull[qs]);
+          } else {
+            mbar_arrive_expect_tx(&qfull[qs], 0);
+          }
+          mbar_arrive(&tfull[qs]);
+        }
+        pos += t1 - t0;
+        while (s + 1 < B && sstart[s + 1] <= pos) ++s;
       }
+      return;
     }
-    return;
+
+    if (warp == C::WARP_PROD) {
+      // ===== producer: one thread walks every tile in order into the shared ring =====
+      if (lane == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        const int bs_mask = (1 << a.log2_bs) - 1;
+        int cnt = 0;
+        for (int k = 0;; ++k) {
+          const int qs = k % kQSlots;
+          wait_or_abort(&tfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
+          const volatile int* u = unit + qs * 8;
+          const int s = u[0];
+          if (s < 0 || *abort_flag) break;
+          const int hp = u[1], t0 = u[2], t1 = u[3];
+          for (int t = t0; t < t1; ++t, ++cnt) {
+            const int slot = cnt % nslots;
+            wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err);
+            const int bid = *abort_flag ? -1 : tbl[qs * kMaxTilesPerUnit + (t - t0)];
+            mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
+            if (bid >= 0) {
+              const int row = (t * kTileTok) & bs_mask;
+              uint8_t* dst = ring + slot * C::SLOT_BYTES;
+              tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
+              tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
+            }
+          }
+          mbar_arrive(&tempty[qs]);
+        }
+      }
+      return;
+    }
+
+    return;  // warp 3 idles
   }
+  if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
 
   // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
+  const int w = warp - C::WARP_C0;
   const int sub = lane & 7;
   const int tp = lane >> 3;
   const int hh = head_of_lane<GW>(lane);
   const bool writer = (lane & C::DUPMASK) == 0;
-  float2* pw = pbuf + warp * kTileTok * GW;
+  float2* pw = pbuf + w * kTileTok * GW;
   int cnt = 0;
+  float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
+  float m = -INFINITY, l = 0.f;
+  float2 acc[GW][2];
 
   for (int k = 0;; ++k) {
     const int qs = k % kQSlots;
     wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-    const int item = item_of[qs];
-    if (item < 0 || *abort_flag) break;
-    int s, p, hp;
-    sch.item(item, s, p, hp);
-    const int tok0 = p * P;
-    const int tok1 = min(slen[s], tok0 + P);
-    const int ntile = cdiv(max(tok1 - tok0, 0), kTileTok);
-
-    // q of this warp's G heads, dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8),
-    // as (even, odd) pairs, pre-scaled into the log2 domain
-    float2 q2[GW][8];
-    {
-      const uint8_t* qb = qbuf + qs * C::QBYTES + warp * G * kRowBytes;
+    const volatile int* u = unit + qs * 8;
+    const int s = u[0];
+    if (s < 0 || *abort_flag) break;
+    const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
+    if (flags & kFirst) {
+      // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
+      const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
 #pragma unroll
       for (int j = 0; j < GW; ++j) {
         const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
         const uint4 w1 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + 128 + sub * 16);
-        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float2 f = Elem<T>::unpack2(w[i]);
+          const float2 f = Elem<T>::unpack2(wd[i]);
           q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
         }
       }
+      m = -INFINITY;
+      l = 0.f;
+#pragma unroll
+      for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&qempty[qs]);
-    float m = -INFINITY, l = 0.f;
-    float2 acc[GW][2];
-#pragma unroll
-    for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+    const int L = slen[s];
 
-    for (int t = 0; t < ntile; ++t, ++cnt) {
+    for (int t = t0; t < t1; ++t, ++cnt) {
       const int slot = cnt % nslots;
       wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
-      const int nvalid = min(kTileTok, tok1 - (tok0 + t * kTileTok));
+      const int nvalid = min(kTileTok, L - t * kTileTok);
       // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + warp * kRowBytes;
+      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
       const uint8_t* Vs = Ks + C::TILE_BYTES;
 
       // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
@@ -472,10 +472,10 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
         const uint8_t* kr = Ks + rr * (HB * kRowBytes);
         const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
         const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
-        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         float2 kf[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(w[i]);
+        for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
         float d[GW];
 #pragma unroll
         for (int jj = 0; jj < GW; ++jj) {
@@ -502,12 +502,12 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
         if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
       }
       l = l * alpha + psum;
-      if (writer && tp == 0) abuf[warp * GW + hh] = alpha;
+      if (writer && tp == 0) abuf[w * GW + hh] = alpha;
       __syncwarp();
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int jj = 0; jj < GW; ++jj) {
-          const float al = abuf[warp * GW + jj];
+          const float al = abuf[w * GW + jj];
           const float2 a2 = make_float2(al, al);
           acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
           acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
@@ -533,24 +533,25 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
+    if (!(flags & kLast)) continue;
 
-    // ---- finish: l summed over the 4 token groups; m and l of every head to every lane
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
-    const int nparts = fstart[s + 1] - fstart[s] + 1;
+    // ---- end of segment: l summed over the 4 token groups; m and l of every head
+    float lt = l + __shfl_xor_sync(0xffffffffu, l, 8);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
 #pragma unroll
     for (int jj = 0; jj < GW; ++jj) {
-      const float lj = __shfl_sync(0xffffffffu, l, lane_of_head<GW>(jj));
+      const float lj = __shfl_sync(0xffffffffu, lt, lane_of_head<GW>(jj));
       const float mj = __shfl_sync(0xffffffffu, m, lane_of_head<GW>(jj));
       const float inv = lj > 0.f ? 1.f / lj : 0.f;
-      const int qh = (hp * HB + warp) * G + jj;
+      const int j = w * G + jj;  // q-head within the group
       const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
       const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
-      if (nparts == 1) {
-        T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + qh) * kD + lane * 4;
+      if (flags & kDirect) {
+        T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + hp * HBG + j) * kD +
+                lane * 4;
         *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
       } else {
-        const long long row = ((long long)s * a.num_q_heads + qh) * a.max_parts + p;
+        const long long row = (long long)pslot * HBG + j;
         *reinterpret_cast<float4*>(a.part_o + row * kD + lane * 4) = make_float4(o0, o1, o2, o3);
         if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
       }
@@ -559,33 +560,37 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 }
 
 // Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes
-// over head_dim.  o = sum_p w_p o_p / sum_p w_p with w_p = l_p * 2^(m_p - max m).
+// over head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - max m), over
+// the segments i of the (sequence, head group), which sit in consecutive slots.
 template <typename T>
-__global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= a.num_seqs * a.num_q_heads) return;
   const int s = gw / a.num_q_heads;
-  const int L = clamp_len(a.seq_lens[s], a.seq_cap);
-  const int n = max(1, cdiv(L, a.part_size));
+  const int qh = gw - s * a.num_q_heads;
+  const int nhp = a.num_q_heads / hbg;
+  const int j = qh % hbg;
+  const int2 mt = a.meta[s * nhp + qh / hbg];
+  const int n = mt.y;
   if (n <= 1) return;  // written by the decode kernel
-  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (long long)gw * a.max_parts;
+  const long long row0 = (long long)mt.x * hbg + j;
   float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, a.part_ml[(row0 + (long long)i * hbg) * 2]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* po = a.part_o + (long long)gw * a.max_parts * kD + lane * 4;
-  // eight partitions per round: all loads of a round are in flight together
+  // eight segments per round: all loads of a round are in flight together
   for (int i0 = 0; i0 < n; i0 += 8) {
     float2 mlv[8];
     float4 ov[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (i0 + u < n) {
-        mlv[u] = ml[i0 + u];
-        ov[u] = *reinterpret_cast<const float4*>(po + (long long)(i0 + u) * kD);
+        const long long row = row0 + (long long)(i0 + u) * hbg;
+        mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
+        ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
       }
     }
 #pragma unroll
@@ -603,38 +608,37 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
       make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
 }
 
-constexpr int kDefaultPartition = 256;
-constexpr int kMaxPartition = kMaxTilesPerItem * kTileTok;
+constexpr int kMaxPartition = kMaxTilesPerUnit * kTileTok;
 constexpr int kMaxSeqs = 4096;
 constexpr int kMaxSmem = 227 * 1024;
 
-// kv-heads per item: all of them up to eight (whole 2 KB rows for 8 heads of 128)
+// kv-heads per group: all of them up to eight (whole 2 KB rows for 8 heads of 128)
 inline int heads_per_item(int num_kv_heads) {
   for (int hb = 8; hb > 1; hb >>= 1)
     if (num_kv_heads % hb == 0) return hb;
   return 1;
 }
 
-// Library choice of the split-K partition: 256 tokens, halved (down to 64) while even
-// the upper bound on the work items (every sequence at max_seq_len) would leave fewer
-// than four items per SM for the dynamic schedule to balance.
-inline int choose_partition(int partition_size, int num_seqs, int num_kv_heads,
-                            int max_seq_len) {
-  if (partition_size > 0) return partition_size;
-  const long long groups = (long long)num_seqs * (num_kv_heads / heads_per_item(num_kv_heads));
-  const int sms = std::max(1, num_sms());
-  int P = kDefaultPartition;
-  while (P > 64 && groups * std::max(1, (max_seq_len + P - 1) / P) < 4LL * sms) P /= 2;
-  return P;
-}
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-inline int num_parts_host(int max_seq_len, int P) { return std::max(1, (max_seq_len + P - 1) / P); }
+// Workspace of one launch: merge records, then partial outputs, then (m, l) pairs.
+struct WsLayout {
+  size_t meta, part_o, part_ml, total;
+};
+inline WsLayout ws_layout(long long groups, long long slots, int hbg, int head_dim) {
+  WsLayout w;
+  w.meta = 0;
+  w.part_o = align256((size_t)groups * sizeof(int2));
+  w.part_ml = w.part_o + (size_t)slots * hbg * head_dim * sizeof(float);
+  w.total = w.part_ml + (size_t)slots * hbg * 2 * sizeof(float);
+  return w;
+}
 
 template <typename T, int G, int HB>
 pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
-                        DecodeArgs a, cudaStream_t stream) {
+                        DecodeArgs a, int grid, cudaStream_t stream) {
   using C = DecodeCfg<G, HB>;
-  const size_t ring_off = ((C::OFF_SEQ + (size_t)(3 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
+  const size_t ring_off = ((C::OFF_SEQ + (size_t)(2 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
   const long long room = (long long)kMaxSmem - (long long)ring_off;
   const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
   if (nslots < 2) return PA_ERR_UNSUPPORTED;
@@ -645,17 +649,12 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
-  const long long items_max = (long long)a.num_seqs * (a.num_kv_heads / HB) * a.max_parts;
-  const int sms = num_sms();
-  if (sms <= 0) return PA_ERR_CUDA;
-  const int grid = (int)std::min<long long>(items_max, sms);
-  if (cudaMemsetAsync(a.counter, 0, sizeof(int), stream) != cudaSuccess) return PA_ERR_CUDA;
   kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
-  if (a.max_parts > 1) {
+  if (grid > 1) {
     const int warps = a.num_seqs * a.num_q_heads;
-    lse_reduce_kernel<T><<<(warps + 7) / 8, 256, 0, stream>>>(a);
+    lse_reduce_kernel<T><<<(warps + 7) / 8, 256, 0, stream>>>(a, HB * G);
     if (check_launch() != PA_OK) return PA_ERR_CUDA;
     ++launches;
   }
@@ -665,24 +664,25 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
 
 template <typename T, int G>
 pa_status dispatch_hb(int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                      const CUtensorMap& tmQ, const DecodeArgs& a, cudaStream_t stream) {
+                      const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream) {
   switch (HB) {
-    case 1: return launch_decode<T, G, 1>(tmK, tmV, tmQ, a, stream);
-    case 2: return launch_decode<T, G, 2>(tmK, tmV, tmQ, a, stream);
-    case 4: return launch_decode<T, G, 4>(tmK, tmV, tmQ, a, stream);
-    case 8: return launch_decode<T, G, 8>(tmK, tmV, tmQ, a, stream);
+    case 1: return launch_decode<T, G, 1>(tmK, tmV, tmQ, a, grid, stream);
+    case 2: return launch_decode<T, G, 2>(tmK, tmV, tmQ, a, grid, stream);
+    case 4: return launch_decode<T, G, 4>(tmK, tmV, tmQ, a, grid, stream);
+    case 8: return launch_decode<T, G, 8>(tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
 
 template <typename T>
 pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                         const CUtensorMap& tmQ, const DecodeArgs& a, cudaStream_t stream) {
+                         const CUtensorMap& tmQ, const DecodeArgs& a, int grid,
+                         cudaStream_t stream) {
   switch (G) {
-    case 1: return dispatch_hb<T, 1>(HB, tmK, tmV, tmQ, a, stream);
-    case 2: return dispatch_hb<T, 2>(HB, tmK, tmV, tmQ, a, stream);
-    case 4: return dispatch_hb<T, 4>(HB, tmK, tmV, tmQ, a, stream);
-    case 8: return dispatch_hb<T, 8>(HB, tmK, tmV, tmQ, a, stream);
+    case 1: return dispatch_hb<T, 1>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 2: return dispatch_hb<T, 2>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 4: return dispatch_hb<T, 4>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 8: return dispatch_hb<T, 8>(HB, tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -691,13 +691,21 @@ pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMa
 
 extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim,
                                            int max_seq_len, int partition_size) {
-  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0) return 0;
-  // the automatic choice may pick down to 64 tokens; size for the most partitions
-  const int P = partition_size > 0 ? partition_size : 64;
-  const int parts = pa::num_parts_host(max_seq_len, P);
-  const size_t partials =
-      parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * sizeof(float) : 0;
-  return pa::kWorkspaceHeader + partials;
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_seq_len < 0 ||
+      partition_size < 0)
+    return 0;
+  // Bounds over every kv-head count: groups <= B*Hq; partial rows = (grid + groups) *
+  // (q-heads per group) <= grid*Hq + B*Hq, grid <= kMaxGrid + (tiles / tiles per
+  // partition when a partition is given).
+  const long long B = num_seqs, Hq = num_q_heads;
+  long long rows = ((long long)pa::kMaxGrid + B) * Hq;
+  if (partition_size > 0) {
+    const long long nt = (max_seq_len + pa::kTileTok - 1) / pa::kTileTok;
+    const long long tpp = std::max(1, partition_size / pa::kTileTok);
+    rows += B * Hq * ((nt + tpp - 1) / tpp) + Hq;
+  }
+  return pa::align256((size_t)B * Hq * sizeof(int2)) +
+         (size_t)rows * (head_dim + 2) * sizeof(float);
 }
 
 extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -724,16 +732,27 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
   if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
     return PA_ERR_INVALID_ARG;
-  const int P = pa::choose_partition(partition_size, num_seqs, num_kv_heads, max_seq_len);
-  const int parts = pa::num_parts_host(max_seq_len, P);
-  const size_t partials = parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * 4 : 0;
-  const size_t need = pa::kWorkspaceHeader + partials;
-  if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
+
+  const int HB = pa::heads_per_item(num_kv_heads);
+  const int NHP = num_kv_heads / HB;
+  const int HBG = HB * G;
+  const long long cap_tbl = (long long)max_blocks_per_seq * block_size;
+  const int seq_cap = (int)std::min<long long>(cap_tbl, max_seq_len);
+  const long long nt_max = (seq_cap + pa::kTileTok - 1) / pa::kTileTok;
+  const long long tiles_max = (long long)num_seqs * NHP * nt_max;
+  if (tiles_max > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
+  // persistent grid of one CTA per SM; an explicit partition caps each CTA's share
+  long long grid = std::min<long long>(std::max(1, pa::num_sms()), pa::kMaxGrid);
+  grid = std::max<long long>(1, std::min<long long>(grid, tiles_max));
+  if (partition_size > 0)
+    grid = std::max<long long>(grid, (tiles_max + partition_size / 16 - 1) / (partition_size / 16));
+  const long long groups = (long long)num_seqs * NHP;
+  const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
+  if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
   int* err = pa::device_error_flag();
   if (!err) return PA_ERR_CUDA;
 
-  const int HB = pa::heads_per_item(num_kv_heads);
   CUtensorMap tmK, tmV, tmQ;
   const uint64_t row = (uint64_t)head_dim * 2;
   const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
@@ -742,7 +761,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
   const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads, (uint64_t)num_seqs};
   const uint64_t qstr[2] = {row, row * num_q_heads};
-  const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)(HB * G), 1};
+  const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)HBG, 1};
   if (!pa::encode_tmap_16bit(&tmK, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !pa::encode_tmap_16bit(&tmV, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !pa::encode_tmap_16bit(&tmQ, q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -753,9 +772,9 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   a.out = out;
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
-  a.counter = reinterpret_cast<int*>(ws);
-  a.part_o = partials ? reinterpret_cast<float*>(ws + pa::kWorkspaceHeader) : nullptr;
-  a.part_ml = partials ? a.part_o + (size_t)num_seqs * num_q_heads * parts * head_dim : nullptr;
+  a.meta = reinterpret_cast<int2*>(ws + lay.meta);
+  a.part_o = reinterpret_cast<float*>(ws + lay.part_o);
+  a.part_ml = reinterpret_cast<float*>(ws + lay.part_ml);
   a.err = err;
   a.num_seqs = num_seqs;
   a.num_q_heads = num_q_heads;
@@ -763,16 +782,14 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   a.max_blocks = max_blocks_per_seq;
   a.log2_bs = block_size == 16 ? 4 : 5;
   a.num_blocks = num_blocks;
-  a.part_size = P;
-  a.max_parts = parts;
-  const long long cap_tbl = (long long)max_blocks_per_seq * block_size;
-  a.seq_cap = (int)std::min<long long>(cap_tbl, max_seq_len);
+  a.seq_cap = seq_cap;
   a.ring_off = 0;
   a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dtype == PA_F16 ? pa::dispatch_group<__half>(G, HB, tmK, tmV, tmQ, a, st)
-                         : pa::dispatch_group<__nv_bfloat16>(G, HB, tmK, tmV, tmQ, a, st);
+  return dtype == PA_F16
+             ? pa::dispatch_group<__half>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
+             : pa::dispatch_group<__nv_bfloat16>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
 }
 
 // Decode without any caller-provided scratch.
@@ -781,7 +798,7 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
 // serving loop whose memory is entirely owned by an engine's pre-allocated pool (the
 // pool hands out KV blocks, not scratch buffers), plugins whose host framework forbids
 // raw cudaMalloc, and latency-critical paths where an allocation could synchronise the
-// device.  For them this entry point keeps its workspace (the work-item counter and the
+// device.  For them this entry point keeps its workspace (the merge records and the
 // split-K partials) in a fixed array that
 // lives in this file (kNoAllocScratchBytes on every GPU that loads the library, held
 // until the process exits) and otherwise runs exactly pa_decode.

@@ -54,17 +54,26 @@ def test_status_strings(palib):
     assert palib.pa_status_string(99) == "PA_ERR_UNKNOWN"
 
 
+def _ws_bound(B, Hq, L, P, D=128):
+    """The documented upper bound: merge records (8 B per sequence and q-head, padded
+    to 256 B) and partial rows of D+2 fp32: (256 + B) * Hq, plus, with an explicit
+    partition, B * Hq * ceil(ceil(L/16) / (P/16)) + Hq."""
+    rows = (256 + B) * Hq
+    if P:
+        rows += B * Hq * -(-(-(-L // 16)) // (P // 16)) + Hq
+    return -(-(B * Hq * 8) // 256) * 256 + rows * (D + 2) * 4
+
+
 def test_workspace_size_arithmetic(palib):
-    H = 256  # header: the kernel's work-item counter
-    # one partition covers the sequence -> the header alone
-    assert palib.pa_decode_workspace_size(64, 32, 128, 64, 0) == H
-    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 512) == H
-    # automatic choice: sized for 64-token partitions, the smallest the library picks
-    assert palib.pa_decode_workspace_size(64, 32, 128, 512, 0) == H + 64 * 32 * 8 * 130 * 4
-    # 8000 tokens at 512 per partition -> 16 partitions of (128 + 2) fp32 per (seq, q-head)
-    assert palib.pa_decode_workspace_size(64, 32, 128, 8000, 512) == H + 64 * 32 * 16 * 130 * 4
-    assert palib.pa_decode_workspace_size(32, 64, 128, 32768, 512) == H + 32 * 64 * 64 * 130 * 4
-    assert palib.pa_decode_workspace_size(2, 8, 128, 100, 16) == H + 2 * 8 * 7 * 130 * 4
+    for B, Hq, L, P in [(64, 32, 64, 0), (64, 32, 8000, 0), (64, 32, 8000, 512),
+                        (32, 64, 32768, 512), (2, 8, 100, 16), (1, 1, 0, 0)]:
+        assert palib.pa_decode_workspace_size(B, Hq, 128, L, P) == _ws_bound(B, Hq, L, P)
+    # the balanced split needs no more scratch for longer sequences
+    assert palib.pa_decode_workspace_size(64, 32, 128, 8000, 0) == \
+        palib.pa_decode_workspace_size(64, 32, 128, 64, 0)
+    # 16 sequences x 64 q-heads, 32768 tokens, 512-token partitions: 64 partitions each
+    assert palib.pa_decode_workspace_size(16, 64, 128, 32768, 512) == \
+        16 * 64 * 8 + ((256 + 16) * 64 + 16 * 64 * 64 + 64) * 130 * 4
     assert palib.pa_decode_workspace_size(0, 8, 128, 100, 16) == 0  # invalid shape
     assert palib.pa_chunked_prefill_workspace_size(4, 512, 64, 128, 8000) == 0
 
@@ -104,7 +113,7 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(dt=3) == 2
     assert dec(B=0) == 0                     # nothing to do
     assert dec(B=5000) == 2                  # more sequences than the schedule holds
-    assert dec(P=512) == 3                   # every call needs a workspace (item counter)
+    assert dec(P=512) == 3                   # every call needs a workspace (merge records)
     assert dec(maxlen=8000, P=512, ws=p, wsb=100) == 3
     assert dec(maxlen=8000, P=512, ws=ctypes.c_void_p(4096 + 16), wsb=1 << 24) == 1  # alignment
 

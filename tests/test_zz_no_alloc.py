@@ -4,7 +4,7 @@ Some callers of this library never call cudaMalloc themselves: their device memo
 belongs to an engine's pre-allocated KV pool or to a host framework that forbids raw
 allocations, or they run in a latency-critical loop where an allocation could
 synchronise the device.  pa_decode_noalloc serves them by keeping its workspace (the
-work-item counter and the split-K partials) in a fixed array inside the library.
+merge records and the split-K partials) in a fixed array inside the library.
 These checks run through the C ABI on a GPU: two calls in a row must reproduce
 pa_decode with a caller-provided workspace (within the parity tolerance), and sizes
 whose partials do not fit the array must be refused before anything is launched.  The file sorts last so a fail-fast run has already run
