@@ -234,6 +234,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the merge pass may be scheduled now; it waits for this grid's results itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- clamped lengths and the prefix of tiles over (sequence, head group)
   if (warp == 0) {
@@ -564,6 +566,10 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 // the segments i of the (sequence, head group), which sit in consecutive slots.
 template <typename T>
 __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
+  // launched as a programmatic dependent of the decode kernel: its CTAs may start while
+  // the decode grid drains; this waits until that grid has finished and its writes are
+  // visible (a no-op when launched without the dependency)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= a.num_seqs * a.num_q_heads) return;
@@ -646,15 +652,24 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   a.nslots = nslots;
   const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
   auto kern = paged_decode_kernel<T, G, HB>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
   kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
   if (grid > 1) {
     const int warps = a.num_seqs * a.num_q_heads;
-    lse_reduce_kernel<T><<<(warps + 7) / 8, 256, 0, stream>>>(a, HB * G);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T>, a, HB * G) != cudaSuccess)
+      return PA_ERR_CUDA;
     if (check_launch() != PA_OK) return PA_ERR_CUDA;
     ++launches;
   }

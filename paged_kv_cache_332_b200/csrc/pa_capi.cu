@@ -1,6 +1,8 @@
 // Status strings, the per-device error flag, SM-count cache and TMA
 // descriptor encoding for libpagedattn.
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "pa_host.h"
 
@@ -51,6 +53,20 @@ int num_sms() {
     g_sms[d] = n;
   }
   return g_sms[d];
+}
+
+bool ensure_dynamic_smem(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> granted;
+  const int d = current_device();
+  if (d < 0) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  int& have = granted[{func, d}];
+  if (have >= bytes) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  have = bytes;
+  return true;
 }
 
 static bool load_encoder() {

@@ -15,6 +15,11 @@ int* device_error_flag();
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 
+// Allow `func` at least `bytes` of dynamic shared memory on the current device.  The
+// attribute is set once per (kernel, device) and only raised afterwards, so steady-state
+// calls cost a map lookup instead of a driver call.
+bool ensure_dynamic_smem(const void* func, int bytes);
+
 // Encode a 4-D tiled TMA descriptor over a KV cache
 // [num_blocks, block_size, num_kv_heads, head_dim] of 16-bit elements whose box is
 // `box_rows` consecutive tokens x head_dim of one kv-head of one block.

@@ -468,9 +468,7 @@ template <typename T, int G>
 pa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
                  cudaStream_t stream) {
   auto kern = chunked_prefill_kernel<T, G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES)) return PA_ERR_CUDA;
   const long long grid = (long long)a.num_seqs * a.num_kv_heads * a.qblocks;
   if (grid <= 0) return PA_OK;
   if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
