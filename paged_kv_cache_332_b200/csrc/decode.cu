@@ -29,8 +29,11 @@
 //    two 16-byte shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving
 //    exchange that sums all G heads at once.  Online softmax (running max m, sum l) in
 //    the log2 domain (q pre-scaled by scale*log2 e: one ex2 per logit); p.V with lanes
-//    over head_dim.  With G = 8 the consumers take registers from the producer side of
-//    the CTA (setmaxnreg) to hold 8 q rows without spilling.
+//    over head_dim.
+//  * G = 8 (LLaMA-70B-style GQA) is the exception: its two contractions cost 4 FMAs per
+//    byte of KV, more than the FP32 pipe sustains at HBM rate, so q.k and p.V of a tile
+//    run as mma.sync m16n8k16 tensor-core fragments (fp32 accumulate); the online
+//    softmax, masking and the split-K bookkeeping are the same.
 //  * A staging warp cuts the CTA's share into units of at most 128 tiles and, up to two
 //    units ahead, copies their block-table entries into shared memory (one coalesced
 //    read per 32 entries) and starts the TMA copy of their q rows.  A producer thread
@@ -82,11 +85,7 @@ struct DecodeCfg {
   static constexpr int WARP_FILL = 2;             // zero-fills empty sequences
   static constexpr int WARP_C0 = 4;               // first consumer warp
   static constexpr int THREADS = 128 + HB * 32;
-  // G = 8 with eight consumer warps: 12 warps at launch get 168 registers each; the
-  // first warpgroup gives back down to 72 so each consumer can grow to 216
-  // (128*72 + 256*216 = 384*168).
-  static constexpr bool SPLIT_REGS = (HB == 8 && G == 8);
-  static constexpr int DUPMASK = GW == 8 ? 0 : (GW == 4 ? 1 : (GW == 2 ? 3 : 7));
+  static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);  // CUDA-core path (G <= 4)
   static constexpr int TILE_BYTES = kTileTok * HB * kRowBytes;  // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
   static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of a group
@@ -105,7 +104,6 @@ struct DecodeCfg {
   static constexpr int OFF_A = OFF_P + HB * kTileTok * GW * 8;     // alpha per warp
   static constexpr int OFF_SEQ = ((OFF_A + HB * GW * 4 + 15) / 16) * 16;  // 2B+1 ints
   static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
-  static_assert(!SPLIT_REGS || THREADS == 384, "register split assumes three warpgroups");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -120,34 +118,10 @@ __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
 
 // Sum per-lane partial dot products over each 8-lane token group for GW heads at
 // once (halving exchange).  Returns the sum for head hh(lane):
-//   GW=8: hh = 4*bit2 + 2*bit1 + bit0;  GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;
+//   GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;
 //   GW=1: hh = 0.
 template <int GW>
 __device__ __forceinline__ float reduce_heads(const float (&d)[GW], int lane);
-
-template <>
-__device__ __forceinline__ float reduce_heads<8>(const float (&d)[8], int lane) {
-  const bool b2 = lane & 4;
-  float k[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float keep = b2 ? d[i + 4] : d[i];
-    const float send = b2 ? d[i] : d[i + 4];
-    k[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  const bool b1 = lane & 2;
-  float k2[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float keep = b1 ? k[i + 2] : k[i];
-    const float send = b1 ? k[i] : k[i + 2];
-    k2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  const bool b0 = lane & 1;
-  const float keep = b0 ? k2[1] : k2[0];
-  const float send = b0 ? k2[0] : k2[1];
-  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-}
 
 template <>
 __device__ __forceinline__ float reduce_heads<4>(const float (&d)[4], int lane) {
@@ -186,17 +160,58 @@ __device__ __forceinline__ float reduce_heads<1>(const float (&d)[1], int lane) 
 
 template <int GW>
 __device__ __forceinline__ int head_of_lane(int lane) {
-  return GW == 8 ? (lane & 7)
-                 : (GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1))
-                            : (GW == 2 ? ((lane >> 2) & 1) : 0));
+  return GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)) : (GW == 2 ? ((lane >> 2) & 1) : 0);
 }
 
 // A lane that holds head jj's value after reduce_heads (with tp = 0).
 template <int GW>
 __device__ __forceinline__ int lane_of_head(int jj) {
-  return GW == 8 ? jj : (GW == 4 ? (((jj >> 1) << 2) | ((jj & 1) << 1)) : (GW == 2 ? jj * 4 : 0));
+  return GW == 4 ? (((jj >> 1) << 2) | ((jj & 1) << 1)) : (GW == 2 ? jj * 4 : 0);
 }
 
+
+// mma.sync m16n8k16 with fp32 accumulate, A row-major / B column-major fragments, and
+// the packing of two fp32 values into one register of the element type.
+template <typename T>
+struct Mma;
+template <>
+struct Mma<__nv_bfloat16> {
+  static __device__ __forceinline__ void run(float (&d)[4], uint32_t a0, uint32_t a1,
+                                             uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+template <>
+struct Mma<__half> {
+  static __device__ __forceinline__ void run(float (&d)[4], uint32_t a0, uint32_t a1,
+                                             uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+// Transpose of an 8x8 matrix of 16-bit elements held as one fragment register per lane
+// (lane l: row l/4, columns 2(l%4), 2(l%4)+1).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  return d;
+}
 
 // CTA holding global tile `pos` when T tiles are shared out over `grid` CTAs
 // (CTA c holds [c*T/grid, (c+1)*T/grid)).
@@ -287,7 +302,6 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
   const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
 
   if (warp < C::WARP_C0) {
-    if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     if (warp == C::WARP_FILL) {
       // ===== empty sequences: no CTA visits them; zero their output and merge record =====
       for (int s = cta; s < B; s += gridDim.x) {
@@ -414,151 +428,320 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 
     return;  // warp 3 idles
   }
-  if constexpr (C::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
 
   // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
   const int w = warp - C::WARP_C0;
-  const int sub = lane & 7;
-  const int tp = lane >> 3;
-  const int hh = head_of_lane<GW>(lane);
-  const bool writer = (lane & C::DUPMASK) == 0;
-  float2* pw = pbuf + w * kTileTok * GW;
-  int cnt = 0;
-  float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
-  float m = -INFINITY, l = 0.f;
-  float2 acc[GW][2];
-
-  for (int k = 0;; ++k) {
-    const int qs = k % kQSlots;
-    wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-    const volatile int* u = unit + qs * 8;
-    const int s = u[0];
-    if (s < 0 || *abort_flag) break;
-    const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
-    if (flags & kFirst) {
-      // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
-      const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
+  if constexpr (G == 8) {
+    // Tensor-core consumer.  Per 16-token tile: S^T = K Q^T (M = 16 tokens, N = 8
+    // q-heads, K = 128 dims: 8 MMAs) and O^T += V^T P^T (M = 128 dims in 8 tiles, N = 8
+    // q-heads, K = 16 tokens: 8 MMAs).  Lane (g, tq) = (lane/4, lane%4) holds the logits
+    // of tokens g and g+8 for q-heads 2tq and 2tq+1, and the output of those two heads
+    // for dims [16g, 16g+16).  The contraction over dims may take the dims in any order
+    // as long as K and Q agree: k-step 2j (2j+1) uses the first (last) two dim pairs of
+    // the 16-byte chunk tq + 4j, so each fragment register is one aligned 32-bit read.
+    constexpr int RS = HB * kRowBytes;  // bytes between consecutive tokens of a tile
+    const int g = lane >> 2, tq = lane & 3;
+    uint32_t qf[8][2];  // Q^T fragments of the 8 k-steps
+    float oacc[8][4];   // O^T: [m-tile mt] dims 16g+mt / 16g+8+mt x heads 2tq, 2tq+1
+    float mh0 = -INFINITY, mh1 = -INFINITY, lh0 = 0.f, lh1 = 0.f;  // heads 2tq, 2tq+1
+    int cnt = 0;
+    for (int k = 0;; ++k) {
+      const int qs = k % kQSlots;
+      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
+      const volatile int* u = unit + qs * 8;
+      const int s = u[0];
+      if (s < 0 || *abort_flag) break;
+      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
+      if (flags & kFirst) {
+        const uint8_t* qrow = qbuf + qs * C::QBYTES + (w * G + g) * kRowBytes;
 #pragma unroll
-      for (int j = 0; j < GW; ++j) {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + 128 + sub * 16);
-        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 f = Elem<T>::unpack2(wd[i]);
-          q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
+        for (int j = 0; j < 4; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16);
+          qf[2 * j][0] = v.x;
+          qf[2 * j][1] = v.y;
+          qf[2 * j + 1][0] = v.z;
+          qf[2 * j + 1][1] = v.w;
         }
-      }
-      m = -INFINITY;
-      l = 0.f;
+        mh0 = mh1 = -INFINITY;
+        lh0 = lh1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&qempty[qs]);
-    const int L = slen[s];
-
-    for (int t = t0; t < t1; ++t, ++cnt) {
-      const int slot = cnt % nslots;
-      wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
-      const int nvalid = min(kTileTok, L - t * kTileTok);
-      // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-      const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
-      const uint8_t* Vs = Ks + C::TILE_BYTES;
-
-      // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
-      float x[4];
-#pragma unroll
-      for (int ps = 0; ps < 4; ++ps) {
-        const int rr = ps * 4 + tp;
-        const uint8_t* kr = Ks + rr * (HB * kRowBytes);
-        const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
-        const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        float2 kf[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
-        float d[GW];
-#pragma unroll
-        for (int jj = 0; jj < GW; ++jj) {
-          float2 e = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
-          d[jj] = e.x + e.y;
-        }
-        const float xv = reduce_heads<GW>(d, lane);
-        x[ps] = rr < nvalid ? xv : -INFINITY;
-      }
-      // ---- online softmax over the tile, per head hh
-      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float m_new = fmaxf(m, mx);
-      const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
-      m = m_new;
-      float psum = 0.f;
-#pragma unroll
-      for (int ps = 0; ps < 4; ++ps) {
-        const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
-        psum += pv;
-        if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
-      }
-      l = l * alpha + psum;
-      if (writer && tp == 0) abuf[w * GW + hh] = alpha;
-      __syncwarp();
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int jj = 0; jj < GW; ++jj) {
-          const float al = abuf[w * GW + jj];
-          const float2 a2 = make_float2(al, al);
-          acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
-          acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
-        }
-      }
-      // ---- p.V: lane owns dims [4*lane, 4*lane+4)
-      auto pv_row = [&](int tt) {
-        const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
-        const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
-#pragma unroll
-        for (int jj = 0; jj < GW; ++jj) {
-          const float2 pp = pw[tt * GW + jj];
-          acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
-          acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
-        }
-      };
-      if (nvalid == kTileTok) {
-#pragma unroll
-        for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
-      } else {
-        for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
+        for (int mt = 0; mt < 8; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
-    }
-    if (!(flags & kLast)) continue;
+      if (lane == 0) mbar_arrive(&qempty[qs]);
+      const int L = slen[s];
 
-    // ---- end of segment: l summed over the 4 token groups; m and l of every head
-    float lt = l + __shfl_xor_sync(0xffffffffu, l, 8);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+      for (int t = t0; t < t1; ++t, ++cnt) {
+        const int slot = cnt % nslots;
+        wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
+        const int nvalid = min(kTileTok, L - t * kTileTok);
+        // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
+        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+        const uint8_t* Vs = Ks + C::TILE_BYTES;
+
+        // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int jj = 0; jj < GW; ++jj) {
-      const float lj = __shfl_sync(0xffffffffu, lt, lane_of_head<GW>(jj));
-      const float mj = __shfl_sync(0xffffffffu, m, lane_of_head<GW>(jj));
-      const float inv = lj > 0.f ? 1.f / lj : 0.f;
-      const int j = w * G + jj;  // q-head within the group
-      const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
-      const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
-      if (flags & kDirect) {
-        T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + hp * HBG + j) * kD +
-                lane * 4;
-        *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
-      } else {
-        const long long row = (long long)pslot * HBG + j;
-        *reinterpret_cast<float4*>(a.part_o + row * kD + lane * 4) = make_float4(o0, o1, o2, o3);
-        if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
+        for (int j = 0; j < 4; ++j) {
+          const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
+          const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+          Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
+          Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+        }
+        // ---- online softmax over the tile (log2 domain), per head
+        const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
+        const float x0 = v0 ? sc[0] * a.qscale : -INFINITY;  // token g,   head 2tq
+        const float x1 = v0 ? sc[1] * a.qscale : -INFINITY;  // token g,   head 2tq+1
+        const float x2 = v8 ? sc[2] * a.qscale : -INFINITY;  // token g+8, head 2tq
+        const float x3 = v8 ? sc[3] * a.qscale : -INFINITY;  // token g+8, head 2tq+1
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = fmaxf(mh0, mx0), mn1 = fmaxf(mh1, mx1);
+        const float al0 = fast_exp2(mh0 - mn0), al1 = fast_exp2(mh1 - mn1);  // -inf -> 0
+        mh0 = mn0;
+        mh1 = mn1;
+        const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
+        const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+        lh0 = lh0 * al0 + (p0 + p2);
+        lh1 = lh1 * al1 + (p1 + p3);
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+          const float2 al = make_float2(al0, al1);
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            const float2 lo = __fmul2_rn(make_float2(oacc[mt][0], oacc[mt][1]), al);
+            const float2 hi = __fmul2_rn(make_float2(oacc[mt][2], oacc[mt][3]), al);
+            oacc[mt][0] = lo.x;
+            oacc[mt][1] = lo.y;
+            oacc[mt][2] = hi.x;
+            oacc[mt][3] = hi.y;
+          }
+        }
+        // ---- P^T fragments: [tokens 2tq, 2tq+1 | 8+2tq, 9+2tq] x head g
+        const uint32_t pb0 = transpose8x8(Mma<T>::pack(p0, p1));
+        const uint32_t pb1 = transpose8x8(Mma<T>::pack(p2, p3));
+        // ---- V^T fragments: dims [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9,
+        // paired along tokens; rows past the sequence end are zeroed (p is 0 there, but
+        // the block's unused rows may hold anything)
+        uint32_t vw[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+          const uint4 lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
+          const uint4 hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
+          const bool ok = tk < nvalid;
+          vw[i][0] = ok ? lo.x : 0u;
+          vw[i][1] = ok ? lo.y : 0u;
+          vw[i][2] = ok ? lo.z : 0u;
+          vw[i][3] = ok ? lo.w : 0u;
+          vw[i][4] = ok ? hi.x : 0u;
+          vw[i][5] = ok ? hi.y : 0u;
+          vw[i][6] = ok ? hi.z : 0u;
+          vw[i][7] = ok ? hi.w : 0u;
+        }
+        // ---- O^T += V^T P^T, m-tile mt: rows dims 16g+mt (g) and 16g+8+mt (g+8)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int r = mt >> 1;
+          const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
+          const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], sel);
+          const uint32_t a1 = __byte_perm(vw[0][4 + r], vw[1][4 + r], sel);
+          const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], sel);
+          const uint32_t a3 = __byte_perm(vw[2][4 + r], vw[3][4 + r], sel);
+          Mma<T>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      if (!(flags & kLast)) continue;
+
+      // ---- end of segment: sums over the 8 token rows g, then heads 2tq and 2tq+1
+      float lt0 = lh0, lt1 = lh1;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
+        lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
+      }
+      const float inv0 = lt0 > 0.f ? 1.f / lt0 : 0.f;
+      const float inv1 = lt1 > 0.f ? 1.f / lt1 : 0.f;
+      const int j0 = w * G + 2 * tq;  // q-heads j0, j0+1 within the group
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float inv = e ? inv1 : inv0;
+        if (flags & kDirect) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            pk[i] = Elem<T>::pack2(oacc[2 * i][e] * inv, oacc[2 * i + 1][e] * inv);
+            pk[4 + i] = Elem<T>::pack2(oacc[2 * i][2 + e] * inv, oacc[2 * i + 1][2 + e] * inv);
+          }
+          T* ob = static_cast<T*>(a.out) +
+                  ((long long)s * a.num_q_heads + hp * HBG + j0 + e) * kD + 16 * g;
+          reinterpret_cast<uint4*>(ob)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          reinterpret_cast<uint4*>(ob)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          const long long row = (long long)pslot * HBG + j0 + e;
+          float4* po = reinterpret_cast<float4*>(a.part_o + row * kD + 16 * g);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            po[i] = make_float4(oacc[4 * i][e] * inv, oacc[4 * i + 1][e] * inv,
+                                oacc[4 * i + 2][e] * inv, oacc[4 * i + 3][e] * inv);
+            po[2 + i] = make_float4(oacc[4 * i][2 + e] * inv, oacc[4 * i + 1][2 + e] * inv,
+                                    oacc[4 * i + 2][2 + e] * inv, oacc[4 * i + 3][2 + e] * inv);
+          }
+          if (g == 0)
+            *reinterpret_cast<float2*>(a.part_ml + row * 2) =
+                make_float2(e ? mh1 : mh0, e ? lt1 : lt0);
+        }
       }
     }
-  }
+    return;
+  } else {
+    const int sub = lane & 7;
+    const int tp = lane >> 3;
+    const int hh = head_of_lane<GW>(lane);
+    const bool writer = (lane & C::DUPMASK) == 0;
+    float2* pw = pbuf + w * kTileTok * GW;
+    int cnt = 0;
+    float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
+    float m = -INFINITY, l = 0.f;
+    float2 acc[GW][2];
+
+    for (int k = 0;; ++k) {
+      const int qs = k % kQSlots;
+      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
+      const volatile int* u = unit + qs * 8;
+      const int s = u[0];
+      if (s < 0 || *abort_flag) break;
+      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
+      if (flags & kFirst) {
+        // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
+        const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
+#pragma unroll
+        for (int j = 0; j < GW; ++j) {
+          const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + 128 + sub * 16);
+          const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 f = Elem<T>::unpack2(wd[i]);
+            q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
+          }
+        }
+        m = -INFINITY;
+        l = 0.f;
+#pragma unroll
+        for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qs]);
+      const int L = slen[s];
+
+      for (int t = t0; t < t1; ++t, ++cnt) {
+        const int slot = cnt % nslots;
+        wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
+        const int nvalid = min(kTileTok, L - t * kTileTok);
+        // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
+        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+        const uint8_t* Vs = Ks + C::TILE_BYTES;
+
+        // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
+        float x[4];
+#pragma unroll
+        for (int ps = 0; ps < 4; ++ps) {
+          const int rr = ps * 4 + tp;
+          const uint8_t* kr = Ks + rr * (HB * kRowBytes);
+          const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
+          const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          float2 kf[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
+          float d[GW];
+#pragma unroll
+          for (int jj = 0; jj < GW; ++jj) {
+            float2 e = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
+            d[jj] = e.x + e.y;
+          }
+          const float xv = reduce_heads<GW>(d, lane);
+          x[ps] = rr < nvalid ? xv : -INFINITY;
+        }
+        // ---- online softmax over the tile, per head hh
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m, mx);
+        const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
+        m = m_new;
+        float psum = 0.f;
+#pragma unroll
+        for (int ps = 0; ps < 4; ++ps) {
+          const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
+          psum += pv;
+          if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
+        }
+        l = l * alpha + psum;
+        if (writer && tp == 0) abuf[w * GW + hh] = alpha;
+        __syncwarp();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int jj = 0; jj < GW; ++jj) {
+            const float al = abuf[w * GW + jj];
+            const float2 a2 = make_float2(al, al);
+            acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
+            acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
+          }
+        }
+        // ---- p.V: lane owns dims [4*lane, 4*lane+4)
+        auto pv_row = [&](int tt) {
+          const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
+          const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
+#pragma unroll
+          for (int jj = 0; jj < GW; ++jj) {
+            const float2 pp = pw[tt * GW + jj];
+            acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
+            acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
+          }
+        };
+        if (nvalid == kTileTok) {
+#pragma unroll
+          for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
+        } else {
+          for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      if (!(flags & kLast)) continue;
+
+      // ---- end of segment: l summed over the 4 token groups; m and l of every head
+      float lt = l + __shfl_xor_sync(0xffffffffu, l, 8);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+#pragma unroll
+      for (int jj = 0; jj < GW; ++jj) {
+        const float lj = __shfl_sync(0xffffffffu, lt, lane_of_head<GW>(jj));
+        const float mj = __shfl_sync(0xffffffffu, m, lane_of_head<GW>(jj));
+        const float inv = lj > 0.f ? 1.f / lj : 0.f;
+        const int j = w * G + jj;  // q-head within the group
+        const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
+        const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
+        if (flags & kDirect) {
+          T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + hp * HBG + j) * kD +
+                  lane * 4;
+          *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
+        } else {
+          const long long row = (long long)pslot * HBG + j;
+          *reinterpret_cast<float4*>(a.part_o + row * kD + lane * 4) = make_float4(o0, o1, o2, o3);
+          if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
+        }
+      }
+    }
+  }  // G < 8
 }
 
 // Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes
