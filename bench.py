@@ -7,11 +7,11 @@ One step = one pass of the whole hot path over one batch of the workload:
 pa_reshape_and_cache of this step's new tokens, then pa_decode (split-K decode
 kernel + log-sum-exp merge) — and, for the mixed prefill workload,
 pa_chunked_prefill as well.  Inputs are seeded synthetic tensors already
-resident in HBM when the timed region starts; every workload except the tiny
-one reads more KV than the 126 MB L2 holds per step, and the tiny one flushes
-L2 between steps.  Times are CUDA-event times on the launching stream,
-bracketed by barrier + synchronize, max over ranks.  Rank 0 prints one JSON
-line.
+resident in HBM when the timed region starts; L2 is flushed (by reading a
+buffer twice its size) before every timed step and every timed call.  The step
+runs as one CUDA graph replay.  Times are CUDA-event times on the launching
+stream, bracketed by barrier + synchronize, max over ranks.  Rank 0 prints one
+JSON line.
 
 With --gpus N > 1 (launched by torch.distributed.run) every rank runs an
 independent replica of the workload (the sequences of a decode batch are
@@ -249,13 +249,17 @@ def run_ours(args, rank, world, device):
     dec = step.decode[0] if step.decode else None
     pre = step.prefill[0] if step.prefill else None
     kv_bytes = sum(b.k_cache.numel() * b.k_cache.element_size() * 2 for b in batches)
-    flush = None
-    if kv_bytes < 2 * L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    # L2 is flushed between timed iterations for every workload (outside the timed
+    # span), so no call finds the previous call's KV in the 126 MB L2.  The flush READS
+    # a buffer twice the size of L2: it leaves clean lines behind, so the timed kernel
+    # pays no write-back of the flush's own data.
+    flush_buf = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+
+    def l2_flush():
+        torch.sum(flush_buf)
 
     def one():
-        if flush is not None:
-            flush.fill_(1.0)
+        l2_flush()
         return step.run()
 
     # eager warm-up: first calls set up per-device state (error flag, kernel attributes)
@@ -274,7 +278,7 @@ def run_ours(args, rank, world, device):
     with torch.cuda.graph(g_step, stream=stream):
         step.run()
     # Per-call device time of pa_decode / pa_chunked_prefill: a graph of N calls, each
-    # bracketed by event-record nodes (and preceded by an L2 flush when the inputs fit L2).
+    # bracketed by event-record nodes and preceded by an L2 flush.
     n_kt = 8
     def timing_graph(kind):
         evs = [(torch.cuda.Event(enable_timing=True, external=True),
@@ -282,8 +286,7 @@ def run_ours(args, rank, world, device):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n_kt):
-                if flush is not None:
-                    flush.fill_(float(i))
+                l2_flush()
                 if kind == "decode":
                     step.run_decode(evs[i])
                 else:
@@ -293,8 +296,7 @@ def run_ours(args, rank, world, device):
     g_pre = timing_graph("prefill") if pre is not None else None
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            if flush is not None:
-                flush.fill_(1.0)
+            l2_flush()
             g_step.replay()
         for timed in (g_dec, g_pre):
             if timed is not None:
@@ -309,8 +311,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize(device)
         with torch.cuda.stream(stream):
             for i in range(args.steps):
-                if flush is not None:
-                    flush.fill_(float(i))
+                l2_flush()
                 ev[i][0].record(stream)
                 g_step.replay()
                 ev[i][1].record(stream)
@@ -378,8 +379,8 @@ def run_ours(args, rank, world, device):
     }
     cfg = {"workload": "+".join(b.name for b in batches), "parallelism": "replicas%d" % world,
            "launch": "each step replays one CUDA graph of the library calls",
-           "l2": "flushed between steps" if flush is not None else
-           "inputs larger than L2 (%.0f MB of KV cache per replica)" % (kv_bytes / 1e6)}
+           "l2": "flushed between timed steps and between timed calls (%.0f MB of KV cache "
+                 "per replica)" % (kv_bytes / 1e6)}
     if dec is not None:
         cfg.update(num_seqs=dec.num_seqs, q_heads=dec.num_q_heads, kv_heads=dec.num_kv_heads,
                    head_dim=dec.head_dim, block_size=dec.block_size,

@@ -100,9 +100,11 @@ struct DecodeCfg {
   static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 32;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
   static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerUnit * 4;
-  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;          // p pairs per warp
-  static constexpr int OFF_A = OFF_P + HB * kTileTok * GW * 8;     // alpha per warp
-  static constexpr int OFF_SEQ = ((OFF_A + HB * GW * 4 + 15) / 16) * 16;  // 2B+1 ints
+  // p pairs and alpha per warp (CUDA-core path only; the G = 8 path keeps them in
+  // registers, which leaves room for a third 64 KB ring slot)
+  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;
+  static constexpr int OFF_A = OFF_P + (G == 8 ? 0 : HB * kTileTok * GW * 8);
+  static constexpr int OFF_SEQ = ((OFF_A + (G == 8 ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 2B+1 ints
   static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
 };
 
@@ -745,8 +747,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 }
 
 // Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes
-// over head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - max m), over
-// the segments i of the (sequence, head group), which sit in consecutive slots.
+// over head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the
+// largest m_i, over the segments i of the (sequence, head group), which sit in
+// consecutive slots.
 template <typename T>
 __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
   // launched as a programmatic dependent of the decode kernel: its CTAs may start while
@@ -764,32 +767,37 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
   const int n = mt.y;
   if (n <= 1) return;  // written by the decode kernel
   const long long row0 = (long long)mt.x * hbg + j;
-  float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, a.part_ml[(row0 + (long long)i * hbg) * 2]);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float den = 0.f;
+  // one pass with a running maximum: up to eight segments per round, all loads of a
+  // round in flight together (most groups span fewer than eight CTAs: one round)
+  float M = -INFINITY, den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  // eight segments per round: all loads of a round are in flight together
   for (int i0 = 0; i0 < n; i0 += 8) {
     float2 mlv[8];
     float4 ov[8];
+    float Mr = -INFINITY;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (i0 + u < n) {
         const long long row = row0 + (long long)(i0 + u) * hbg;
         mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
         ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
+        Mr = fmaxf(Mr, mlv[u].x);
       }
     }
+    const float Mn = fmaxf(M, Mr);
+    if (Mn == -INFINITY) continue;  // only empty segments so far
+    const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
+    den *= sc;
+    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (i0 + u < n) {
-        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - M) * mlv[u].y;
+        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
         den += f;
         num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
       }
     }
+    M = Mn;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   T* ob = static_cast<T*>(a.out) + (long long)gw * kD + lane * 4;
