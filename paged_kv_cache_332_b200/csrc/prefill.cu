@@ -130,6 +130,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 consecutive columns of this thread's TMEM lane, waited for inside the same asm
+// statement, so no use of the registers can be scheduled before the data is there.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -243,102 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ======================== TMA producer ========================
-    if (lane == 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
-      const int bs_mask = (1 << a.log2_bs) - 1;
-      for (int kt = 0; kt < n_kt; ++kt) {
-        const int st = kt & 1;
-        const uint32_t ph = ((kt >> 1) & 1) ^ 1;
-        // block ids of the tile's eight 16-token runs (out of range -> zero fill)
-        int bid[8], row[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          const int pos = kt * kBN + r * 16;
-          bid[r] = a.num_blocks;  // past the tensor: TMA fills zeros
-          row[r] = pos & bs_mask;
-          if (pos < L) {
-            const int id = __ldg(trow + (pos >> a.log2_bs));
-            if ((unsigned)id < (unsigned)a.num_blocks) bid[r] = id;
-            else flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
-          }
-        }
-        wait_or_abort(&k_empty[st], ph, abort_flag, a.err);
-        mbar_arrive_expect_tx(&k_full[st], kTileBytes);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int kh = 0; kh < 2; ++kh)
-            tma_load_4d(smem + OFF_K + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmK,
-                        kh * 64, h, row[r], bid[r], &k_full[st]);
-        wait_or_abort(&v_empty[st], ph, abort_flag, a.err);
-        mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int kh = 0; kh < 2; ++kh)
-            tma_load_4d(smem + OFF_V + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmV,
-                        kh * 64, h, row[r], bid[r], &v_full[st]);
-      }
-    }
-  } else if (warp == 1) {
-    // ======================== MMA issuer ========================
-    if (lane == 0) {
-      constexpr bool BF = sizeof(T) == 2 && !std::is_same<T, __half>::value;
-      const uint32_t id_qk = idesc_f16(BF, false);
-      const uint32_t id_pv = idesc_f16(BF, true);
-      const uint32_t sQ = smem_u32(smem + OFF_Q);
-      const uint32_t sK = smem_u32(smem + OFF_K);
-      const uint32_t sV = smem_u32(smem + OFF_V);
-      auto issue_s = [&](int mt, int kt) {
-        const int st = kt & 1;
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t da = sw128_desc(sQ + mt * kTileBytes + off, 16, 1024);
-          const uint64_t db = sw128_desc(sK + st * kTileBytes + off, 16, 1024);
-          mma_ss(tmem + mt * 128, da, db, id_qk, kk > 0);
-        }
-        mma_commit(&s_full[mt]);
-      };
-      auto issue_pv = [&](int mt, int kt) {
-        const int st = kt & 1;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t db = sw128_desc(sV + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
-          mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (kt > 0 || kk > 0));
-        }
-      };
-      wait_or_abort(q_full, 0, abort_flag, a.err);
-      tc_fence_after();
-      if (n_kt > 0) {
-        wait_or_abort(&k_full[0], 0, abort_flag, a.err);
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        mma_commit(&k_empty[0]);
-      }
-      for (int kt = 0; kt < n_kt; ++kt) {
-        const int st = kt & 1;
-        const bool more = kt + 1 < n_kt;
-        wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
-        if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
-        for (int mt = 0; mt < 2; ++mt) {
-          wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
-          tc_fence_after();
-          issue_pv(mt, kt);
-          if (more) issue_s(mt, kt + 1);
-        }
-        if (more) mma_commit(&k_empty[(kt + 1) & 1]);
-        mma_commit(&v_empty[st]);
-      }
-      mma_commit(&o_full[0]);
-      mma_commit(&o_full[1]);
-    }
-  } else if (warp >= 4) {
+  if (warp >= 4) {
+    // softmax warpgroups: 208 registers each thread (one S row of 128 fp32 in registers)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
     // ======================== softmax warpgroups ========================
     const int mt = (warp - 4) >> 2;
     const int wq = warp & 3;              // TMEM lane quarter
@@ -373,19 +308,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_or_abort(&s_full[mt], kt & 1, abort_flag, a.err);
       tc_fence_after();
       const int key0 = kt * kBN;
-      const bool need_mask = key0 + kBN - 1 > wlim;
-      float v[32];
-      float mx = -INFINITY;
+      // the whole S row (128 keys) in registers: one pass over TMEM
+      float v[kBN];
+      tmem_ld64(t_s, v);
+      tmem_ld64(t_s + 64, v + 64);
+      if (key0 + kBN - 1 > wlim) {  // causal diagonal or sequence end in this tile
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(t_s + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = (need_mask && key0 + c * 32 + i > limit) ? -INFINITY : v[i];
-          mx = fmaxf(mx, x);
-        }
+        for (int i = 0; i < kBN; ++i)
+          if (key0 + i > limit) v[i] = -INFINITY;
       }
-      mx *= a.qscale;
+      // row max as a tree of independent maxima (no 128-long dependency chain)
+      float mx8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(v[j], v[j + 8]);
+#pragma unroll
+      for (int i = 16; i < kBN; i += 8)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(mx8[j], v[i + j]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                       a.qscale;
       // lazy reference max: move it only when this tile exceeds it by more than 8
       float alpha = 1.f;
       if (mx > m_ref + 8.f) {
@@ -395,28 +337,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          tmem_ld32(t_o + c * 32, v);
+          float o[32];
+          tmem_ld32(t_o + c * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(t_o + c * 32, v);
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_o + c * 32, o);
         }
       }
-      float sum = 0.f;
+      // p = 2^(x*qscale - m_ref); masked keys hold -inf and give 0 (the offset is kept
+      // finite while every key so far was masked)
+      const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        tmem_ld32(t_s + c * 32, v);
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const bool k0 = !(need_mask && key0 + c * 32 + i > limit);
-          const bool k1 = !(need_mask && key0 + c * 32 + i + 1 > limit);
-          const float p0 = k0 ? fast_exp2(fmaf(v[i], a.qscale, -m_ref)) : 0.f;
-          const float p1 = k1 ? fast_exp2(fmaf(v[i + 1], a.qscale, -m_ref)) : 0.f;
-          sum += p0 + p1;
+          const float p0 = fast_exp2(fmaf(v[c * 32 + i], a.qscale, nm));
+          const float p1 = fast_exp2(fmaf(v[c * 32 + i + 1], a.qscale, nm));
+          sum8[(i >> 1) & 7] += p0 + p1;
           w[i >> 1] = pack16<T>(p0, p1);
         }
         tmem_st16(t_s + c * 16, w);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * alpha + sum;
       // keys past the sequence end in the last tile: clear their V rows
       if (mt == 0 && kt == n_kt - 1 && L < key0 + kBN) {
@@ -453,6 +398,107 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 4; ++j)
           *reinterpret_cast<uint4*>(orow + c * 32 + j * 8) =
               make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      }
+    }
+  
+  } else {
+    // producer / MMA issuer / two idle warps: 88 registers each thread
+    // (128 x 88 + 256 x 208 = 384 x 168, the registers the CTA is launched with)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    if (warp == 0) {
+      // ======================== TMA producer ========================
+      if (lane == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
+        const int bs_mask = (1 << a.log2_bs) - 1;
+        for (int kt = 0; kt < n_kt; ++kt) {
+          const int st = kt & 1;
+          const uint32_t ph = ((kt >> 1) & 1) ^ 1;
+          // block ids of the tile's eight 16-token runs (out of range -> zero fill)
+          int bid[8], row[8];
+  #pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const int pos = kt * kBN + r * 16;
+            bid[r] = a.num_blocks;  // past the tensor: TMA fills zeros
+            row[r] = pos & bs_mask;
+            if (pos < L) {
+              const int id = __ldg(trow + (pos >> a.log2_bs));
+              if ((unsigned)id < (unsigned)a.num_blocks) bid[r] = id;
+              else flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
+            }
+          }
+          wait_or_abort(&k_empty[st], ph, abort_flag, a.err);
+          mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+  #pragma unroll
+          for (int r = 0; r < 8; ++r)
+  #pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+              tma_load_4d(smem + OFF_K + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmK,
+                          kh * 64, h, row[r], bid[r], &k_full[st]);
+          wait_or_abort(&v_empty[st], ph, abort_flag, a.err);
+          mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+  #pragma unroll
+          for (int r = 0; r < 8; ++r)
+  #pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+              tma_load_4d(smem + OFF_V + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmV,
+                          kh * 64, h, row[r], bid[r], &v_full[st]);
+        }
+      }
+    } else if (warp == 1) {
+      // ======================== MMA issuer ========================
+      if (lane == 0) {
+        constexpr bool BF = sizeof(T) == 2 && !std::is_same<T, __half>::value;
+        const uint32_t id_qk = idesc_f16(BF, false);
+        const uint32_t id_pv = idesc_f16(BF, true);
+        const uint32_t sQ = smem_u32(smem + OFF_Q);
+        const uint32_t sK = smem_u32(smem + OFF_K);
+        const uint32_t sV = smem_u32(smem + OFF_V);
+        auto issue_s = [&](int mt, int kt) {
+          const int st = kt & 1;
+  #pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            const uint64_t da = sw128_desc(sQ + mt * kTileBytes + off, 16, 1024);
+            const uint64_t db = sw128_desc(sK + st * kTileBytes + off, 16, 1024);
+            mma_ss(tmem + mt * 128, da, db, id_qk, kk > 0);
+          }
+          mma_commit(&s_full[mt]);
+        };
+        auto issue_pv = [&](int mt, int kt) {
+          const int st = kt & 1;
+  #pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t db = sw128_desc(sV + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
+            mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (kt > 0 || kk > 0));
+          }
+        };
+        wait_or_abort(q_full, 0, abort_flag, a.err);
+        tc_fence_after();
+        if (n_kt > 0) {
+          wait_or_abort(&k_full[0], 0, abort_flag, a.err);
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          mma_commit(&k_empty[0]);
+        }
+        for (int kt = 0; kt < n_kt; ++kt) {
+          const int st = kt & 1;
+          const bool more = kt + 1 < n_kt;
+          wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
+          if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
+          for (int mt = 0; mt < 2; ++mt) {
+            wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
+            tc_fence_after();
+            issue_pv(mt, kt);
+            if (more) issue_s(mt, kt + 1);
+          }
+          if (more) mma_commit(&k_empty[(kt + 1) & 1]);
+          mma_commit(&v_empty[st]);
+        }
+        mma_commit(&o_full[0]);
+        mma_commit(&o_full[1]);
       }
     }
   }
