@@ -58,18 +58,26 @@ def measured_peaks():
                 source="fallback")
 
 
-def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu record, or None when the
-    kernel source changed since the capture (or no capture matches)."""
+def kernel_source_sha(path: str, start: str, end: str) -> str:
+    """sha256 of a kernel's source text: from the line holding `start` up to `end`."""
     import hashlib
+    with open(os.path.join(ROOT, path), encoding="utf-8") as f:
+        text = f.read()
+    i = text.index(start)
+    j = text.index(end, i)
+    return hashlib.sha256(text[i:j].encode()).hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu record, or None when the kernel's
+    source text changed since the capture (or no capture matches the workload)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f).get(kernel)
         if not rec or rec.get("workload") != workload:
             return None
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
+        h = kernel_source_sha(rec["source"], rec["region_start"], rec["region_end"])
         return int(rec["dram_bytes_per_launch"]) if h.startswith(rec["source_sha256_prefix"]) else None
     except Exception:
         return None
