@@ -412,22 +412,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmV);
         const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
         const int bs_mask = (1 << a.log2_bs) - 1;
+        // block-table entries of a tile's eight 16-token runs, read one tile ahead so
+        // that their latency overlaps the previous tile's waits and copies
+        auto table_ids = [&](int kt, int (&id)[8]) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const int pos = kt * kBN + r * 16;
+            id[r] = pos < L ? __ldg(trow + (pos >> a.log2_bs)) : -1;
+          }
+        };
+        int next_id[8];
+        if (n_kt > 0) table_ids(0, next_id);
         for (int kt = 0; kt < n_kt; ++kt) {
           const int st = kt & 1;
           const uint32_t ph = ((kt >> 1) & 1) ^ 1;
           // block ids of the tile's eight 16-token runs (out of range -> zero fill)
           int bid[8], row[8];
-  #pragma unroll
+#pragma unroll
           for (int r = 0; r < 8; ++r) {
             const int pos = kt * kBN + r * 16;
+            const int id = next_id[r];
             bid[r] = a.num_blocks;  // past the tensor: TMA fills zeros
             row[r] = pos & bs_mask;
             if (pos < L) {
-              const int id = __ldg(trow + (pos >> a.log2_bs));
               if ((unsigned)id < (unsigned)a.num_blocks) bid[r] = id;
               else flag_error(a.err, PA_DEVERR_BLOCK_RANGE);
             }
           }
+          if (kt + 1 < n_kt) table_ids(kt + 1, next_id);
           wait_or_abort(&k_empty[st], ph, abort_flag, a.err);
           mbar_arrive_expect_tx(&k_full[st], kTileBytes);
   #pragma unroll
