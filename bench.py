@@ -3,9 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = one pass of the whole hot path over one batch of the workload:
-pa_reshape_and_cache of this step's new tokens, then pa_decode (split-K decode
-kernel + log-sum-exp merge) — and, for the mixed prefill workload,
+One step = one pass of the whole hot path over one batch of the workload: the
+append of this step's new tokens and the decode attention, as one
+pa_decode_append call (decode kernel with the append + log-sum-exp merge) — and,
+for the mixed prefill workload, pa_reshape_and_cache of the chunk tokens and
 pa_chunked_prefill as well.  Inputs are seeded synthetic tensors already
 resident in HBM when the timed region starts; L2 is flushed (by reading a
 buffer twice its size) before every timed step and every timed call.  The step
@@ -186,6 +187,9 @@ class Step:
         self.batches = batches
         self.decode = [b for b in batches if b.query_start_loc is None]
         self.prefill = [b for b in batches if b.query_start_loc is not None]
+        # a decode batch whose every sequence appends one token runs pa_decode_append
+        # (the append inside the decode launch); others append with pa_reshape_and_cache
+        self.fused = {id(b): int(b.k_new.shape[0]) == b.num_seqs for b in self.decode}
         self.ws = {}
         self.out = {}
         for b in batches:
@@ -215,9 +219,15 @@ class Step:
         for b in self.decode:
             if record is not None:
                 record[0].record(self.stream)
-            self.pa.pa_decode(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
-                              b.seq_lens, b.scale, self.max_len[id(b)], 0, self.ws[id(b)],
-                              stream=self.stream)
+            if self.fused[id(b)]:
+                self.pa.pa_decode_append(self.out[id(b)], b.q, b.k_new, b.v_new, b.k_cache,
+                                         b.v_cache, b.block_tables, b.seq_lens, b.scale,
+                                         self.max_len[id(b)], 0, self.ws[id(b)],
+                                         stream=self.stream)
+            else:
+                self.pa.pa_decode(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
+                                  b.seq_lens, b.scale, self.max_len[id(b)], 0, self.ws[id(b)],
+                                  stream=self.stream)
             n += self.pa.pa_last_launch_count()
             if record is not None:
                 record[1].record(self.stream)
@@ -228,6 +238,8 @@ class Step:
         Returns the number of kernels launched."""
         n = 0
         for b in self.batches:
+            if self.fused.get(id(b)):
+                continue  # appended inside its decode launch
             self.pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping,
                                          stream=self.stream)
             n += self.pa.pa_last_launch_count()
@@ -302,11 +314,41 @@ def run_ours(args, rank, world, device):
         return g, evs
     g_dec = timing_graph("decode") if dec is not None else None
     g_pre = timing_graph("prefill") if pre is not None else None
+    # The pages' indirection comparison: the same decode with identity tables (each
+    # sequence's blocks contiguous and in order), when the pool holds every sequence's
+    # blocks without sharing.
+    g_ident = g_paged = None
+    if dec is not None:
+        nb = [-(-int(L) // dec.block_size) for L in dec.seq_lens.tolist()]
+        if sum(nb) <= dec.num_blocks:
+            ident = torch.zeros_like(dec.block_tables)
+            off = 0
+            for i, n in enumerate(nb):
+                ident[i, :n] = torch.arange(off, off + n, dtype=torch.int32, device=device)
+                off += n
+            out_ident = torch.empty_like(dec.q)
+
+            def decode_graph(tables):
+                evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                        torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_kt)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n_kt):
+                        l2_flush()
+                        evs[i][0].record(stream)
+                        pa.pa_decode(out_ident, dec.q, dec.k_cache, dec.v_cache, tables,
+                                     dec.seq_lens, dec.scale, step.max_len[id(dec)], 0,
+                                     step.ws[id(dec)], stream=stream)
+                        evs[i][1].record(stream)
+                return g, evs
+            g_paged = decode_graph(dec.block_tables)
+            g, evs = decode_graph(ident)
+            g_ident = (g, evs)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             l2_flush()
             g_step.replay()
-        for timed in (g_dec, g_pre):
+        for timed in (g_dec, g_pre, g_ident, g_paged):
             if timed is not None:
                 timed[0].replay()
     torch.cuda.synchronize(device)
@@ -336,6 +378,8 @@ def run_ours(args, rank, world, device):
             return [a.elapsed_time(b) for a, b in events]
         dec_ms = kernel_ms(g_dec)
         pre_ms = kernel_ms(g_pre)
+        ident_ms = kernel_ms(g_ident)
+        paged_ms = kernel_ms(g_paged)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     local_ms = sum(step_ms)
     launches = per_step_launches * args.steps
@@ -396,15 +440,24 @@ def run_ours(args, rank, world, device):
     line["config"] = cfg
     if dec is not None:
         ab = decode_algorithmic_bytes(dec)
+        if step.fused[id(dec)]:  # the append inside the launch: read k/v_new, write the slots
+            ab += 2 * 2 * dec.num_seqs * dec.num_kv_heads * dec.head_dim * dec.q.element_size()
         dmean = statistics.mean(dec_ms)
         ach = ab / (dmean / 1e3) / 1e9
-        line["roofline"] = {"kernel": "pa_decode (paged_decode_kernel + lse_reduce_kernel)",
+        line["roofline"] = {"kernel": ("pa_decode_append" if step.fused[id(dec)] else "pa_decode")
+                                      + " (paged_decode_kernel + lse_reduce_kernel)",
                             "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                             "peak_source": peaks["source"], "unit": "GB/s",
                             "frac": round(ach / peaks["hbm_gbs"], 4),
                             "frac_of_8TBs_spec": round(ach / 8000.0, 4),
                             "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
                             "traffic": recorded_traffic("paged_decode_kernel", dec.name)}
+        if ident_ms:
+            im, pm = statistics.mean(ident_ms), statistics.mean(paged_ms)
+            line["indirection"] = {"paged_ms": round(pm, 5), "identity_tables_ms": round(im, 5),
+                                   "overhead": round(pm / im - 1, 4),
+                                   "note": "pa_decode with the workload's tables vs each "
+                                           "sequence's blocks contiguous and in order"}
         line["context_tokens_per_s"] = round(world * int(dec.seq_lens.sum().item()) * args.steps
                                              / (total_ms / 1e3), 1)
     if pre is not None:

@@ -135,6 +135,32 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     size_t workspace_bytes, pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode_append — pa_reshape_and_cache of each sequence's new token followed by
+ * pa_decode, in one launch.  [P1] "PagedAttention 的 CUDA Kernel 实现" and "工程边界与架构
+ * 取舍": a decode step appends the token it produced (its K/V go into the slot of position
+ * seq_len-1 through the block table) and then attends over the whole cache.
+ *
+ *   k_new, v_new  [num_seqs, num_kv_heads, head_dim] in `dtype`, 16-byte aligned: the new
+ *                 token of sequence s, written bitwise to
+ *                 k_cache/v_cache[table[s][(L-1)/bs], (L-1)%bs, :, :] with L = seq_lens[s]
+ *                 (L counts the new token), and attended to by the same call.
+ *   everything else as pa_decode (same workspace size).
+ * A sequence with L = 0 appends nothing; one whose L exceeds its table (flagged
+ * PA_DEVERR_SEQ_TOO_LONG) or whose last table entry is out of range (flagged
+ * PA_DEVERR_BLOCK_RANGE) appends nothing.  The appended slot must not be read by another
+ * sequence of the same call (true whenever shared blocks are full, as with copy-on-write
+ * prefix sharing).  Result and cache contents equal pa_reshape_and_cache (slot of
+ * position L-1) followed by pa_decode.
+ */
+PA_API pa_status pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, float scale,
+                                  int block_size, int num_blocks, int max_seq_len,
+                                  int partition_size, void* workspace, size_t workspace_bytes,
+                                  pa_dtype dtype, void* stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The paper has no counterpart to this call; it exists for callers whose device memory
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that

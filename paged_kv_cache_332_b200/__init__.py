@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
-    "pa_decode_workspace_size", "pa_decode", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
+    "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
+    "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
     "PA_DEVERR",
@@ -40,6 +41,8 @@ _SIGS = [
     ("pa_decode_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_decode", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f, _i32, _i32,
                          _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_decode_append", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                                _f, _i32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
     ("pa_decode_noalloc", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f,
                                  _i32, _i32, _i32, _i32, _i32, _vp]),
     ("pa_decode_noalloc_scratch_bytes", _sz, []),
@@ -146,6 +149,23 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_l
                            int(max_seq_len), int(partition_size), _ptr(workspace), ws_bytes,
                            _dtype_code(k_cache), _stream(stream)),
            "pa_decode")
+
+
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, scale,
+                     max_seq_len, partition_size=0, workspace=None, stream=None):
+    """pa_decode with each sequence's new token (``k_new``/``v_new`` [B, Hkv, D])
+    written into its cache slot (position seq_len-1 through the table) in the same
+    launch; equals pa_reshape_and_cache followed by pa_decode."""
+    N, bs, Hkv, D = k_cache.shape
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_decode_append(_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                  _ptr(v_cache), _i32tensor(block_tables, "block_tables"),
+                                  block_tables.shape[1], _i32tensor(seq_lens, "seq_lens"), B, Hq,
+                                  Hkv, D, float(scale), bs, N, int(max_seq_len),
+                                  int(partition_size), _ptr(workspace), ws_bytes,
+                                  _dtype_code(k_cache), _stream(stream)),
+           "pa_decode_append")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

@@ -56,6 +56,12 @@ struct DecodeArgs {
   float* part_o;   // [slots, HB*G, 128]   normalised partial outputs
   float* part_ml;  // [slots, HB*G, 2]     (max in log2 units, sum)
   int2* meta;      // [B * NHP]            (first slot, slot count) of each group
+  // append in the same launch (k_new != nullptr): the step's new token of each sequence,
+  // [B, Hkv, 128], written into its cache slot at position seq_len-1 before it is read
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int seq_cap;
@@ -96,7 +102,8 @@ struct DecodeCfg {
   static constexpr int OFF_QEMPTY = OFF_QFULL + kQSlots * 8;
   static constexpr int OFF_TFULL = OFF_QEMPTY + kQSlots * 8;
   static constexpr int OFF_TEMPTY = OFF_TFULL + kQSlots * 8;
-  static constexpr int OFF_UNIT = OFF_TEMPTY + kQSlots * 8;     // 8 ints per staged unit
+  static constexpr int OFF_ADONE = OFF_TEMPTY + kQSlots * 8;    // append of a unit written
+  static constexpr int OFF_UNIT = OFF_ADONE + kQSlots * 8;      // 8 ints per staged unit
   static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 32;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
   static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerUnit * 4;
@@ -236,6 +243,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
   uint64_t* qempty = reinterpret_cast<uint64_t*>(smem + C::OFF_QEMPTY);
   uint64_t* tfull = reinterpret_cast<uint64_t*>(smem + C::OFF_TFULL);
   uint64_t* tempty = reinterpret_cast<uint64_t*>(smem + C::OFF_TEMPTY);
+  uint64_t* adone = reinterpret_cast<uint64_t*>(smem + C::OFF_ADONE);
   volatile int* unit = reinterpret_cast<volatile int*>(smem + C::OFF_UNIT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
   int* tbl = reinterpret_cast<int*>(smem + C::OFF_TBL);
@@ -289,6 +297,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
       mbar_init(&qempty[i], HB);
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 1);
+      mbar_init(&adone[i], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -374,6 +383,35 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           }
         }
         __syncwarp();
+        // The unit holding a sequence's last tile also writes the step's new token (K and
+        // V rows of the group's kv-heads, one 2 KB run each for 8 heads) into its slot.
+        // The rows are loaded now, the unit is published, and the stores follow; the
+        // producer waits for them (adone) only before copying that last tile.
+        constexpr int kAppendVecs = (HB * 16 + 31) / 32;  // 16-byte vectors per lane
+        uint4 kv_k[kAppendVecs], kv_v[kAppendVecs];
+        uint4* kd = nullptr;
+        uint4* vd = nullptr;
+        bool append = false;
+        if (a.k_new != nullptr && t1 == nt) {
+          const int raw = __ldg(a.seq_lens + s);
+          const int bid = tbl[qs * kMaxTilesPerUnit + (t1 - 1 - t0)];
+          if (raw == slen[s] && bid >= 0) {
+            append = true;
+            const int row = (raw - 1) & ((1 << a.log2_bs) - 1);
+            const size_t dst = ((((size_t)bid << a.log2_bs) + row) * a.num_kv_heads + hp * HB) * 16;
+            const size_t src = ((size_t)s * a.num_kv_heads + hp * HB) * 16;  // in 16-byte units
+            kd = static_cast<uint4*>(a.k_cache) + dst;
+            vd = static_cast<uint4*>(a.v_cache) + dst;
+#pragma unroll
+            for (int j = 0; j < kAppendVecs; ++j) {
+              const int i = j * 32 + lane;
+              if (i < HB * 16) {
+                kv_k[j] = __ldg(static_cast<const uint4*>(a.k_new) + src + i);
+                kv_v[j] = __ldg(static_cast<const uint4*>(a.v_new) + src + i);
+              }
+            }
+          }
+        }
         if (lane == 0) {
           if (t0 == 0) a.meta[grp] = make_int2(cta + grp, cta_of(ge - 1, Ttot, grid) - cta + 1);
           u[0] = s;
@@ -382,6 +420,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           u[3] = t1;
           u[4] = flags;
           u[5] = cta + grp;
+          u[6] = append ? 1 : 0;
           if (flags & kFirst) {
             mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
             tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HBG, s, &qfull[qs]);
@@ -390,6 +429,19 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           }
           mbar_arrive(&tfull[qs]);
         }
+        if (append) {
+#pragma unroll
+          for (int j = 0; j < kAppendVecs; ++j) {
+            const int i = j * 32 + lane;
+            if (i < HB * 16) {
+              kd[i] = kv_k[j];
+              vd[i] = kv_v[j];
+            }
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // before the TMA reads
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&adone[qs]);  // every unit, so phases stay one per unit
         pos += t1 - t0;
         while (s + 1 < B && sstart[s + 1] <= pos) ++s;
       }
@@ -409,9 +461,12 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           const volatile int* u = unit + qs * 8;
           const int s = u[0];
           if (s < 0 || *abort_flag) break;
-          const int hp = u[1], t0 = u[2], t1 = u[3];
+          const int hp = u[1], t0 = u[2], t1 = u[3], append = u[6];
           for (int t = t0; t < t1; ++t, ++cnt) {
             const int slot = cnt % nslots;
+            // the new token's row is in the last tile: its stores must have landed
+            if (append && t == t1 - 1)
+              wait_or_abort(&adone[qs], (k / kQSlots) & 1, abort_flag, a.err);
             wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err);
             const int bid = *abort_flag ? -1 : tbl[qs * kMaxTilesPerUnit + (t - t0)];
             mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
@@ -914,13 +969,14 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int he
          (size_t)rows * (head_dim + 2) * sizeof(float);
 }
 
-extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                               const int32_t* block_tables, int max_blocks_per_seq,
-                               const int32_t* seq_lens, int num_seqs, int num_q_heads,
-                               int num_kv_heads, int head_dim, float scale, int block_size,
-                               int num_blocks, int max_seq_len, int partition_size,
-                               void* workspace, size_t workspace_bytes, pa_dtype dtype,
-                               void* stream) {
+namespace {
+// pa_decode, and pa_decode_append when k_new / v_new are given
+pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v_new,
+                      const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                      int num_q_heads, int num_kv_heads, int head_dim, float scale,
+                      int block_size, int num_blocks, int max_seq_len, int partition_size,
+                      void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0 ||
@@ -938,6 +994,8 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
   if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
     return PA_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_INVALID_ARG;
+  if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return PA_ERR_INVALID_ARG;
 
   const int HB = pa::heads_per_item(num_kv_heads);
   const int NHP = num_kv_heads / HB;
@@ -979,6 +1037,10 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
   a.meta = reinterpret_cast<int2*>(ws + lay.meta);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_cache = const_cast<void*>(k_cache);
+  a.v_cache = const_cast<void*>(v_cache);
   a.part_o = reinterpret_cast<float*>(ws + lay.part_o);
   a.part_ml = reinterpret_cast<float*>(ws + lay.part_ml);
   a.err = err;
@@ -996,6 +1058,35 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
   return dtype == PA_F16
              ? pa::dispatch_group<__half>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
              : pa::dispatch_group<__nv_bfloat16>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
+}
+}  // namespace
+
+extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, float scale, int block_size,
+                               int num_blocks, int max_seq_len, int partition_size,
+                               void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                               void* stream) {
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                     seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
+                     num_blocks, max_seq_len, partition_size, workspace, workspace_bytes, dtype,
+                     stream);
+}
+
+extern "C" pa_status pa_decode_append(void* out, const void* q, const void* k_new,
+                                      const void* v_new, void* k_cache, void* v_cache,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, float scale, int block_size,
+                                      int num_blocks, int max_seq_len, int partition_size,
+                                      void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                                      void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
+  return decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                     seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
+                     num_blocks, max_seq_len, partition_size, workspace, workspace_bytes, dtype,
+                     stream);
 }
 
 // Decode without any caller-provided scratch.

@@ -118,6 +118,22 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(maxlen=8000, P=512, ws=ctypes.c_void_p(4096 + 16), wsb=1 << 24) == 1  # alignment
 
 
+def test_append_decode_arguments_rejected_on_host(palib):
+    L = _raw(palib)
+    p = ctypes.c_void_p(4096)
+
+    def app(kn=p, vn=p, B=2, D=128, ws=None, wsb=0):
+        return L.pa_decode_append(p, p, kn, vn, p, p, p, 8, p, B, 8, 8, D, 0.1, 16, 16, 100, 512,
+                                  ws, wsb, 0, None)
+    assert app(kn=None) == 1                     # new K missing
+    assert app(vn=None) == 1                     # new V missing
+    assert app(kn=ctypes.c_void_p(4100)) == 1    # misaligned
+    assert app(D=64) == 2                        # head_dim must be 128
+    assert app(B=0) == 0                         # nothing to do
+    assert app() == 3                            # needs a workspace
+    assert palib.pa_last_launch_count() == 0
+
+
 def test_product_package_does_not_touch_oracle():
     # the product path never imports the oracle
     pkg = os.path.join(ROOT, "paged_kv_cache_332_b200")
