@@ -193,3 +193,83 @@ def to_f64(t):
     """fp16/bf16/fp32 torch tensor -> fp64 numpy array (exact)."""
     import torch
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) KV cache
+# ---------------------------------------------------------------------------
+# [P1] "工程边界与架构取舍", on quantization and KV-cache precision: storing the cache in
+# FP8 instead of FP16 halves its memory (at some accuracy cost on long sequences).
+# The pages fix no format, scale granularity or rounding.  Readings:
+#  - the e4m3 format with no infinities: 1 sign bit, 4 exponent bits (bias 7), 3
+#    mantissa bits; exponent field 0 holds the subnormals 2^-6 * m/8; the largest finite
+#    value is 1.75 * 2^8 = 448; codes 0x7F and 0xFF are NaN;
+#  - one fp32 scale per kv-head for K and one for V: a stored code c stands for
+#    value(c) * scale;
+#  - quantisation computes x * (1 / scale) in fp32 (the reciprocal rounded to fp32,
+#    then the product rounded to fp32), rounds to the nearest e4m3 value, ties to the
+#    even code, and saturates to +-448.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code):
+    """fp64 value of e4m3 codes (array of 0..255): (-1)^s 2^(e-7) (1 + m/8) for
+    exponent field e > 0, (-1)^s 2^-6 (m/8) for e = 0; 0x7F and 0xFF are NaN."""
+    c = np.asarray(code).astype(np.int64) & 0xFF
+    s, e, m = (c >> 7) & 1, (c >> 3) & 0xF, c & 7
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    val = np.where(s == 1, -mag, mag)
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+# the 127 non-negative finite values (codes 0x00..0x7E), increasing
+_E4M3_POS = e4m3_value(np.arange(0x7F))
+
+
+def e4m3_round(x):
+    """Nearest e4m3 code (uint8) to each fp64 value: the nearest of the finite values,
+    ties to the even code (last mantissa bit 0), magnitudes past 448 saturate to 448,
+    the sign kept (a negative value that rounds to zero gives 0x80); NaN gives 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 1, 0x7E)  # _POS[hi-1] < a <= _POS[hi]
+    lo = hi - 1
+    d_lo, d_hi = a - _E4M3_POS[lo], _E4M3_POS[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    mag = np.where(pick_hi, hi, lo)
+    mag = np.where(a == 0, 0, mag)
+    code = np.where(np.signbit(x), mag | 0x80, mag)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def quantize_e4m3(x, scale):
+    """Codes of ``x`` (fp16/bf16/fp32 values as an array) with per-kv-head ``scale``
+    broadcast against it: e4m3_round(float32(x) * float32(1/float32(scale)))."""
+    inv = (np.float32(1.0) / np.asarray(scale, dtype=np.float32)).astype(np.float32)
+    y = (np.asarray(x, dtype=np.float32) * inv).astype(np.float32)
+    return e4m3_round(y.astype(np.float64))
+
+
+def reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale):
+    """reshape_and_cache into uint8 e4m3 caches [N, bs, Hkv, D]: token t's rows
+    k[t], v[t] ([Hkv, D], the values of the step's fp16/bf16 K/V) are quantised with
+    the per-head scales (``k_scale``/``v_scale`` [Hkv]) and stored at slot
+    ``slot_mapping[t]`` (negative = padding, skipped), in place."""
+    bs = k_cache.shape[1]
+    ks = np.asarray(k_scale, dtype=np.float32)[:, None]
+    vs = np.asarray(v_scale, dtype=np.float32)[:, None]
+    for t, slot in enumerate(np.asarray(slot_mapping)):
+        if slot < 0:
+            continue
+        b, r = divmod(int(slot), bs)
+        k_cache[b, r] = quantize_e4m3(k[t], ks)
+        v_cache[b, r] = quantize_e4m3(v[t], vs)
+
+
+def dequantize_cache(cache_codes, scale):
+    """fp64 values of an e4m3 cache [N, bs, Hkv, D] with per-kv-head ``scale`` [Hkv]:
+    value(code) * scale.  Attention over an FP8 cache is the attention of the oracle
+    above over these values."""
+    return e4m3_value(cache_codes) * np.asarray(scale, dtype=np.float64)[None, None, :, None]
