@@ -161,6 +161,45 @@ PA_API pa_status pa_decode_append(void* out, const void* q, const void* k_new, c
                                   pa_dtype dtype, void* stream);
 
 /*
+ * FP8 (e4m3) KV cache.  [P1] "工程边界与架构取舍", on quantization and KV-cache precision:
+ * an FP8 cache takes half the memory of FP16 (and decode, which reads the whole cache,
+ * half the bytes).  The pages fix no format; this library stores e4m3 codes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, subnormals, no infinities, largest
+ * finite 448) with one fp32 scale per kv-head for K and one for V: code c stands for
+ * value(c) * scale[h].  Caches are uint8 [num_blocks, block_size, num_kv_heads,
+ * head_dim]; k_scale / v_scale are device fp32 [num_kv_heads].
+ */
+
+/*
+ * pa_reshape_and_cache_fp8 — pa_reshape_and_cache into e4m3 caches: element x of
+ * kv-head h of token t (k / v in `dtype`, [T, num_kv_heads, head_dim]) is stored as the
+ * e4m3 code nearest to x * (1 / scale[h]) computed in fp32 (reciprocal, then product),
+ * ties to even, saturated to +-448.  Slot handling and errors as pa_reshape_and_cache.
+ */
+PA_API pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache,
+                                          void* v_cache, const int32_t* slot_mapping,
+                                          const float* k_scale, const float* v_scale,
+                                          int num_tokens, int num_kv_heads, int head_dim,
+                                          int num_blocks, int block_size, pa_dtype dtype,
+                                          void* stream);
+
+/*
+ * pa_decode_fp8 — pa_decode over e4m3 caches: the result is the attention over the
+ * dequantised values value(code) * scale[h], with q and out in `dtype`.  q.k and p.V
+ * run as mma.sync fragments in f16 (e4m3 values are exact in f16; q is rounded to f16
+ * once; P is rounded to f16); the K scale multiplies the logits and the V scale the
+ * output, both in fp32.  Arguments, limits, workspace and errors as pa_decode.
+ */
+PA_API pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* seq_lens, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, float scale, int block_size,
+                               int num_blocks, int max_seq_len, int partition_size,
+                               void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                               void* stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The paper has no counterpart to this call; it exists for callers whose device memory
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that

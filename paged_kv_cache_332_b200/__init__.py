@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
     "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8",
     "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
@@ -43,6 +44,10 @@ _SIGS = [
                          _i32, _i32, _vp, _sz, _i32, _vp]),
     ("pa_decode_append", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                                 _f, _i32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_reshape_and_cache_fp8", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                        _i32, _i32, _vp]),
+    ("pa_decode_fp8", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                             _f, _i32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
     ("pa_decode_noalloc", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f,
                                  _i32, _i32, _i32, _i32, _i32, _vp]),
     ("pa_decode_noalloc_scratch_bytes", _sz, []),
@@ -166,6 +171,49 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_l
                                   int(partition_size), _ptr(workspace), ws_bytes,
                                   _dtype_code(k_cache), _stream(stream)),
            "pa_decode_append")
+
+
+def _f32tensor(t, what):
+    if t.dtype != torch.float32:
+        raise TypeError("%s must be float32" % what)
+    return _ptr(t)
+
+
+def _u8cache(t, what):
+    if t.dtype != torch.uint8:
+        raise TypeError("%s must be a uint8 (e4m3 code) tensor" % what)
+    return _ptr(t)
+
+
+def pa_reshape_and_cache_fp8(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None):
+    """Quantise ``k``/``v`` [T, Hkv, D] (fp16/bf16) to e4m3 codes with the per-kv-head
+    fp32 scales and scatter them into the uint8 caches [N, bs, Hkv, D]."""
+    N, bs, Hkv, D = k_cache.shape
+    _check(lib().pa_reshape_and_cache_fp8(_ptr(k), _ptr(v), _u8cache(k_cache, "k_cache"),
+                                          _u8cache(v_cache, "v_cache"),
+                                          _i32tensor(slot_mapping, "slot_mapping"),
+                                          _f32tensor(k_scale, "k_scale"),
+                                          _f32tensor(v_scale, "v_scale"), k.shape[0], Hkv, D, N,
+                                          bs, _dtype_code(k), _stream(stream)),
+           "pa_reshape_and_cache_fp8")
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_lens, scale,
+                  max_seq_len, partition_size=0, workspace=None, stream=None):
+    """pa_decode over uint8 e4m3 caches with per-kv-head fp32 scales; ``q``/``out``
+    fp16/bf16 [B, Hq, D]."""
+    N, bs, Hkv, D = k_cache.shape
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_decode_fp8(_ptr(out), _ptr(q), _u8cache(k_cache, "k_cache"),
+                               _u8cache(v_cache, "v_cache"), _f32tensor(k_scale, "k_scale"),
+                               _f32tensor(v_scale, "v_scale"),
+                               _i32tensor(block_tables, "block_tables"), block_tables.shape[1],
+                               _i32tensor(seq_lens, "seq_lens"), B, Hq, Hkv, D, float(scale), bs,
+                               N, int(max_seq_len), int(partition_size), _ptr(workspace),
+                               ws_bytes, _dtype_code(q), _stream(stream)),
+           "pa_decode_fp8")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

@@ -40,9 +40,12 @@
 //    walks the tiles in order and issues the two boxes of each as soon as a slot of the
 //    shared ring frees (blocking waits take no issue slots from the consumers).
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
+#include <cuda_fp8.h>
+
 #include <algorithm>
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "pa_device.cuh"
 #include "pa_host.h"
@@ -62,6 +65,9 @@ struct DecodeArgs {
   const void* v_new;
   void* k_cache;
   void* v_cache;
+  // FP8 (e4m3) cache: fp32 scale of each kv-head's K and V codes, [Hkv]
+  const float* k_scale;
+  const float* v_scale;
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int seq_cap;
@@ -81,10 +87,13 @@ constexpr int kFirst = 1;   // first unit of a segment: load q, reset the softma
 constexpr int kLast = 2;    // last unit of a segment: write the result
 constexpr int kDirect = 4;  // the segment is the whole group: write `out`
 
-template <int G_, int HB_>
+template <int G_, int HB_, bool F8_>
 struct DecodeCfg {
   static constexpr int G = G_;
   static constexpr int HB = HB_;                  // kv-heads per group = consumer warps
+  static constexpr bool F8 = F8_;                 // e4m3 cache (else fp16/bf16)
+  static constexpr bool MMA = F8 || G == 8;       // tensor-core consumers
+  static constexpr int KROW = kD * (F8 ? 1 : 2);  // one token of one kv-head in the cache
   static constexpr int GW = G;                    // q-heads per consumer warp
   static constexpr int WARP_PROD = 0;
   static constexpr int WARP_STAGE = 1;
@@ -92,7 +101,7 @@ struct DecodeCfg {
   static constexpr int WARP_C0 = 4;               // first consumer warp
   static constexpr int THREADS = 128 + HB * 32;
   static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);  // CUDA-core path (G <= 4)
-  static constexpr int TILE_BYTES = kTileTok * HB * kRowBytes;  // K (or V) of a tile
+  static constexpr int TILE_BYTES = kTileTok * HB * KROW;       // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
   static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of a group
   // shared-memory carve-up (bytes); the sequence arrays and then the ring follow
@@ -110,8 +119,8 @@ struct DecodeCfg {
   // p pairs and alpha per warp (CUDA-core path only; the G = 8 path keeps them in
   // registers, which leaves room for a third 64 KB ring slot)
   static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;
-  static constexpr int OFF_A = OFF_P + (G == 8 ? 0 : HB * kTileTok * GW * 8);
-  static constexpr int OFF_SEQ = ((OFF_A + (G == 8 ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 2B+1 ints
+  static constexpr int OFF_A = OFF_P + (MMA ? 0 : HB * kTileTok * GW * 8);
+  static constexpr int OFF_SEQ = ((OFF_A + (MMA ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 2B+1 ints
   static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
 };
 
@@ -214,6 +223,14 @@ struct Mma<__half> {
   }
 };
 
+// Two e4m3 codes (low 16 bits of x; the lower code first) -> their f16 values as one
+// f16x2 register.  Exact: every e4m3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
+  const __half2_raw h =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(x & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // Transpose of an 8x8 matrix of 16-bit elements held as one fragment register per lane
 // (lane l: row l/4, columns 2(l%4), 2(l%4)+1).
 __device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
@@ -228,12 +245,12 @@ __device__ __forceinline__ int cta_of(int pos, int T, int grid) {
   return (int)((((long long)pos + 1) * grid - 1) / T);
 }
 
-template <typename T, int G, int HB>
-__global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
+template <typename T, int G, int HB, bool F8>
+__global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
-  using C = DecodeCfg<G, HB>;
+  using C = DecodeCfg<G, HB, F8>;
   constexpr int GW = C::GW;
   constexpr int HBG = HB * G;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -488,15 +505,20 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 
   // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
   const int w = warp - C::WARP_C0;
-  if constexpr (G == 8) {
-    // Tensor-core consumer.  Per 16-token tile: S^T = K Q^T (M = 16 tokens, N = 8
+  if constexpr (C::MMA) {
+    // Tensor-core consumer (G = 8, and every G on an FP8 cache).  Per 16-token tile: S^T = K Q^T (M = 16 tokens, N = 8
     // q-heads, K = 128 dims: 8 MMAs) and O^T += V^T P^T (M = 128 dims in 8 tiles, N = 8
     // q-heads, K = 16 tokens: 8 MMAs).  Lane (g, tq) = (lane/4, lane%4) holds the logits
     // of tokens g and g+8 for q-heads 2tq and 2tq+1, and the output of those two heads
     // for dims [16g, 16g+16).  The contraction over dims may take the dims in any order
     // as long as K and Q agree: k-step 2j (2j+1) uses the first (last) two dim pairs of
     // the 16-byte chunk tq + 4j, so each fragment register is one aligned 32-bit read.
-    constexpr int RS = HB * kRowBytes;  // bytes between consecutive tokens of a tile
+    // FP8: the same tile with e4m3 K/V converted to f16 on the way into the fragments
+    // (exact: every e4m3 value is an f16 value), q rounded to f16 once per segment, the
+    // K scale folded into the logit scale and the V scale into the final normalisation;
+    // with G < 8 the q-heads past G are zero columns of the MMAs and are not written.
+    using MT = typename std::conditional<F8, __half, T>::type;  // MMA operand type
+    constexpr int RS = HB * C::KROW;  // bytes between consecutive tokens of a tile
     const int g = lane >> 2, tq = lane & 3;
     uint32_t qf[8][2];  // Q^T fragments of the 8 k-steps
     float oacc[8][4];   // O^T: [m-tile mt] dims 16g+mt / 16g+8+mt x heads 2tq, 2tq+1
@@ -511,13 +533,35 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
       const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
       if (flags & kFirst) {
         const uint8_t* qrow = qbuf + qs * C::QBYTES + (w * G + g) * kRowBytes;
+        if constexpr (F8) {
+          // k-step 4c+i takes dims 4i..4i+3 of the 16-dim chunk tq + 4c (one 32-bit
+          // word of e4m3 codes); Q takes the same dims, as f16 pairs
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16);
-          qf[2 * j][0] = v.x;
-          qf[2 * j][1] = v.y;
-          qf[2 * j + 1][0] = v.z;
-          qf[2 * j + 1][1] = v.w;
+          for (int c = 0; c < 2; ++c) {
+            const uint8_t* src = qrow + (tq + 4 * c) * 32;
+            uint32_t wq[8];
+            *reinterpret_cast<uint4*>(wq) = *reinterpret_cast<const uint4*>(src);
+            *reinterpret_cast<uint4*>(wq + 4) = *reinterpret_cast<const uint4*>(src + 16);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 f = Elem<T>::unpack2(wq[i]);
+              wq[i] = g < G ? Mma<__half>::pack(f.x, f.y) : 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              qf[4 * c + i][0] = wq[2 * i];
+              qf[4 * c + i][1] = wq[2 * i + 1];
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16);
+            qf[2 * j][0] = v.x;
+            qf[2 * j][1] = v.y;
+            qf[2 * j + 1][0] = v.z;
+            qf[2 * j + 1][1] = v.w;
+          }
         }
         mh0 = mh1 = -INFINITY;
         lh0 = lh1 = 0.f;
@@ -527,30 +571,46 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&qempty[qs]);
       const int L = slen[s];
+      const int kvh = hp * HB + w;
+      const float lsc = F8 ? a.qscale * __ldg(a.k_scale + kvh) : a.qscale;
 
       for (int t = t0; t < t1; ++t, ++cnt) {
         const int slot = cnt % nslots;
         wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
         const int nvalid = min(kTileTok, L - t * kTileTok);
         // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * C::KROW;
         const uint8_t* Vs = Ks + C::TILE_BYTES;
 
         // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (F8) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
-          const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
-          Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
-          Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+          for (int c = 0; c < 2; ++c) {
+            const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * c) * 16);
+            const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * c) * 16);
+            const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              Mma<__half>::run(sc, e4m3x2_to_f16x2(wa[i]), e4m3x2_to_f16x2(wb[i]),
+                               e4m3x2_to_f16x2(wa[i] >> 16), e4m3x2_to_f16x2(wb[i] >> 16),
+                               qf[4 * c + i][0], qf[4 * c + i][1]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
+            const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+            Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
+            Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+          }
         }
         // ---- online softmax over the tile (log2 domain), per head
         const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
-        const float x0 = v0 ? sc[0] * a.qscale : -INFINITY;  // token g,   head 2tq
-        const float x1 = v0 ? sc[1] * a.qscale : -INFINITY;  // token g,   head 2tq+1
-        const float x2 = v8 ? sc[2] * a.qscale : -INFINITY;  // token g+8, head 2tq
-        const float x3 = v8 ? sc[3] * a.qscale : -INFINITY;  // token g+8, head 2tq+1
+        const float x0 = v0 ? sc[0] * lsc : -INFINITY;  // token g,   head 2tq
+        const float x1 = v0 ? sc[1] * lsc : -INFINITY;  // token g,   head 2tq+1
+        const float x2 = v8 ? sc[2] * lsc : -INFINITY;  // token g+8, head 2tq
+        const float x3 = v8 ? sc[3] * lsc : -INFINITY;  // token g+8, head 2tq+1
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -578,8 +638,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           }
         }
         // ---- P^T fragments: [tokens 2tq, 2tq+1 | 8+2tq, 9+2tq] x head g
-        const uint32_t pb0 = transpose8x8(Mma<T>::pack(p0, p1));
-        const uint32_t pb1 = transpose8x8(Mma<T>::pack(p2, p3));
+        const uint32_t pb0 = transpose8x8(Mma<MT>::pack(p0, p1));
+        const uint32_t pb1 = transpose8x8(Mma<MT>::pack(p2, p3));
         // ---- V^T fragments: dims [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9,
         // paired along tokens; rows past the sequence end are zeroed (p is 0 there, but
         // the block's unused rows may hold anything)
@@ -587,8 +647,17 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-          const uint4 lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
-          const uint4 hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
+          uint4 lo, hi;
+          if constexpr (F8) {  // 16 e4m3 codes -> 8 f16 pairs
+            const uint4 c8 = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 16);
+            lo = make_uint4(e4m3x2_to_f16x2(c8.x), e4m3x2_to_f16x2(c8.x >> 16),
+                            e4m3x2_to_f16x2(c8.y), e4m3x2_to_f16x2(c8.y >> 16));
+            hi = make_uint4(e4m3x2_to_f16x2(c8.z), e4m3x2_to_f16x2(c8.z >> 16),
+                            e4m3x2_to_f16x2(c8.w), e4m3x2_to_f16x2(c8.w >> 16));
+          } else {
+            lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
+            hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
+          }
           const bool ok = tk < nvalid;
           vw[i][0] = ok ? lo.x : 0u;
           vw[i][1] = ok ? lo.y : 0u;
@@ -608,7 +677,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
           const uint32_t a1 = __byte_perm(vw[0][4 + r], vw[1][4 + r], sel);
           const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], sel);
           const uint32_t a3 = __byte_perm(vw[2][4 + r], vw[3][4 + r], sel);
-          Mma<T>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+          Mma<MT>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
@@ -622,11 +691,13 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB>::THREADS, 1)
         lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
         lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
       }
-      const float inv0 = lt0 > 0.f ? 1.f / lt0 : 0.f;
-      const float inv1 = lt1 > 0.f ? 1.f / lt1 : 0.f;
+      const float vsc = F8 ? __ldg(a.v_scale + kvh) : 1.f;
+      const float inv0 = lt0 > 0.f ? vsc / lt0 : 0.f;
+      const float inv1 = lt1 > 0.f ? vsc / lt1 : 0.f;
       const int j0 = w * G + 2 * tq;  // q-heads j0, j0+1 within the group
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
+        if (2 * tq + e >= G) continue;  // a zero column (G < 8)
         const float inv = e ? inv1 : inv0;
         if (flags & kDirect) {
           uint32_t pk[8];
@@ -886,10 +957,10 @@ inline WsLayout ws_layout(long long groups, long long slots, int hbg, int head_d
   return w;
 }
 
-template <typename T, int G, int HB>
+template <typename T, int G, int HB, bool F8>
 pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                         DecodeArgs a, int grid, cudaStream_t stream) {
-  using C = DecodeCfg<G, HB>;
+  using C = DecodeCfg<G, HB, F8>;
   const size_t ring_off = ((C::OFF_SEQ + (size_t)(2 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
   const long long room = (long long)kMaxSmem - (long long)ring_off;
   const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
@@ -897,7 +968,7 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   a.ring_off = (int)ring_off;
   a.nslots = nslots;
   const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
-  auto kern = paged_decode_kernel<T, G, HB>;
+  auto kern = paged_decode_kernel<T, G, HB, F8>;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
   kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
@@ -923,27 +994,27 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   return PA_OK;
 }
 
-template <typename T, int G>
+template <typename T, int G, bool F8>
 pa_status dispatch_hb(int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                       const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream) {
   switch (HB) {
-    case 1: return launch_decode<T, G, 1>(tmK, tmV, tmQ, a, grid, stream);
-    case 2: return launch_decode<T, G, 2>(tmK, tmV, tmQ, a, grid, stream);
-    case 4: return launch_decode<T, G, 4>(tmK, tmV, tmQ, a, grid, stream);
-    case 8: return launch_decode<T, G, 8>(tmK, tmV, tmQ, a, grid, stream);
+    case 1: return launch_decode<T, G, 1, F8>(tmK, tmV, tmQ, a, grid, stream);
+    case 2: return launch_decode<T, G, 2, F8>(tmK, tmV, tmQ, a, grid, stream);
+    case 4: return launch_decode<T, G, 4, F8>(tmK, tmV, tmQ, a, grid, stream);
+    case 8: return launch_decode<T, G, 8, F8>(tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
 
-template <typename T>
+template <typename T, bool F8>
 pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const CUtensorMap& tmQ, const DecodeArgs& a, int grid,
                          cudaStream_t stream) {
   switch (G) {
-    case 1: return dispatch_hb<T, 1>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 2: return dispatch_hb<T, 2>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 4: return dispatch_hb<T, 4>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 8: return dispatch_hb<T, 8>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 1: return dispatch_hb<T, 1, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 2: return dispatch_hb<T, 2, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 4: return dispatch_hb<T, 4, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 8: return dispatch_hb<T, 8, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -972,7 +1043,8 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int he
 namespace {
 // pa_decode, and pa_decode_append when k_new / v_new are given
 pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v_new,
-                      const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const void* k_cache, const void* v_cache, const float* k_scale,
+                      const float* v_scale, const int32_t* block_tables,
                       int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
                       int num_q_heads, int num_kv_heads, int head_dim, float scale,
                       int block_size, int num_blocks, int max_seq_len, int partition_size,
@@ -996,6 +1068,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     return PA_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_INVALID_ARG;
   if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return PA_ERR_INVALID_ARG;
+  const bool f8 = k_scale != nullptr;
+  if (f8 && (!v_scale || k_new)) return PA_ERR_INVALID_ARG;
 
   const int HB = pa::heads_per_item(num_kv_heads);
   const int NHP = num_kv_heads / HB;
@@ -1019,15 +1093,18 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
 
   CUtensorMap tmK, tmV, tmQ;
   const uint64_t row = (uint64_t)head_dim * 2;
+  const uint64_t crow = (uint64_t)head_dim * (f8 ? 1 : 2);  // one kv-head of one token
   const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
                              (uint64_t)num_blocks};
-  const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const uint64_t cstr[3] = {crow, crow * num_kv_heads, crow * num_kv_heads * block_size};
   const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
   const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads, (uint64_t)num_seqs};
   const uint64_t qstr[2] = {row, row * num_q_heads};
   const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)HBG, 1};
-  if (!pa::encode_tmap_16bit(&tmK, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !pa::encode_tmap_16bit(&tmV, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  const CUtensorMapDataType ct =
+      f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  if (!pa::encode_tmap(&tmK, ct, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !pa::encode_tmap(&tmV, ct, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !pa::encode_tmap_16bit(&tmQ, q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))
     return PA_ERR_CUDA;
 
@@ -1041,6 +1118,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.v_new = v_new;
   a.k_cache = const_cast<void*>(k_cache);
   a.v_cache = const_cast<void*>(v_cache);
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   a.part_o = reinterpret_cast<float*>(ws + lay.part_o);
   a.part_ml = reinterpret_cast<float*>(ws + lay.part_ml);
   a.err = err;
@@ -1055,9 +1134,13 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (f8)
+    return dtype == PA_F16
+               ? pa::dispatch_group<__half, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
+               : pa::dispatch_group<__nv_bfloat16, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
   return dtype == PA_F16
-             ? pa::dispatch_group<__half>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
-             : pa::dispatch_group<__nv_bfloat16>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
+             ? pa::dispatch_group<__half, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
+             : pa::dispatch_group<__nv_bfloat16, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
 }
 }  // namespace
 
@@ -1068,8 +1151,8 @@ extern "C" pa_status pa_decode(void* out, const void* q, const void* k_cache, co
                                int num_blocks, int max_seq_len, int partition_size,
                                void* workspace, size_t workspace_bytes, pa_dtype dtype,
                                void* stream) {
-  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                     seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr, block_tables,
+                     max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
                      num_blocks, max_seq_len, partition_size, workspace, workspace_bytes, dtype,
                      stream);
 }
@@ -1083,10 +1166,25 @@ extern "C" pa_status pa_decode_append(void* out, const void* q, const void* k_ne
                                       void* workspace, size_t workspace_bytes, pa_dtype dtype,
                                       void* stream) {
   if (num_seqs > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
-  return decode_impl(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                     seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
+  return decode_impl(out, q, k_new, v_new, k_cache, v_cache, nullptr, nullptr, block_tables,
+                     max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, scale, block_size,
                      num_blocks, max_seq_len, partition_size, workspace, workspace_bytes, dtype,
                      stream);
+}
+
+extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const float* k_scale,
+                                   const float* v_scale, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, float scale,
+                                   int block_size, int num_blocks, int max_seq_len,
+                                   int partition_size, void* workspace, size_t workspace_bytes,
+                                   pa_dtype dtype, void* stream) {
+  if (num_seqs > 0 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, k_scale, v_scale, block_tables,
+                     max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                     scale, block_size, num_blocks, max_seq_len, partition_size, workspace,
+                     workspace_bytes, dtype, stream);
 }
 
 // Decode without any caller-provided scratch.

@@ -83,9 +83,9 @@ static bool load_encoder() {
   return true;
 }
 
-bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
-                       const uint64_t* strides_bytes, const uint32_t* box,
-                       CUtensorMapSwizzle swizzle) {
+bool encode_tmap(CUtensorMap* out, CUtensorMapDataType type, const void* base, int rank,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle) {
   if (!load_encoder() || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
   cuuint32_t bx[5], es[5];
@@ -95,10 +95,17 @@ bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint6
     es[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, rank, const_cast<void*>(base), d,
-                        st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+  CUresult r = g_encode(out, type, rank, const_cast<void*>(base), d, st, bx, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapSwizzle swizzle) {
+  return encode_tmap(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, base, rank, dims, strides_bytes, box,
+                     swizzle);
 }
 
 bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,

@@ -28,6 +28,11 @@ bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int 
 
 // Encode a tiled TMA descriptor over a row-major tensor of 16-bit elements.
 // dims/box innermost first; strides_bytes[i] is the stride of dimension i+1.
+// Encode a tiled TMA descriptor of `type` elements (rank <= 5, dims innermost first,
+// strides in bytes for dims 1.., element strides 1, no interleave, L2 promotion 256 B).
+bool encode_tmap(CUtensorMap* out, CUtensorMapDataType type, const void* base, int rank,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle);
 bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint64_t* dims,
                        const uint64_t* strides_bytes, const uint32_t* box,
                        CUtensorMapSwizzle swizzle);

@@ -134,6 +134,25 @@ def test_append_decode_arguments_rejected_on_host(palib):
     assert palib.pa_last_launch_count() == 0
 
 
+def test_fp8_arguments_rejected_on_host(palib):
+    L = _raw(palib)
+    p = ctypes.c_void_p(4096)
+    nul = None
+    # scatter: missing scales, odd block size, bad source type
+    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, nul, p, 4, 8, 128, 16, 16, 0, nul) == 1
+    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 4, 8, 128, 16, 24, 0, nul) == 2
+    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 4, 8, 128, 16, 16, 7, nul) == 2
+    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 0, 8, 128, 16, 16, 0, nul) == 0
+
+    def dec(ks=p, vs=p, B=2, ws=None, wsb=0):
+        return L.pa_decode_fp8(p, p, p, p, ks, vs, p, 8, p, B, 8, 8, 128, 0.1, 16, 16, 100, 512,
+                               ws, wsb, 0, None)
+    assert dec(ks=None) == 1 and dec(vs=None) == 1
+    assert dec(B=0) == 0
+    assert dec() == 3  # needs a workspace
+    assert palib.pa_last_launch_count() == 0
+
+
 def test_product_package_does_not_touch_oracle():
     # the product path never imports the oracle
     pkg = os.path.join(ROOT, "paged_kv_cache_332_b200")

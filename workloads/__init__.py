@@ -108,6 +108,10 @@ class PagedBatch:
     query_start_loc: Optional[torch.Tensor] = None
     shared_prefix_blocks: int = 0
     group_size: int = 1
+    # FP8 (e4m3) caches: k_cache / v_cache hold uint8 codes, these the fp32 per-kv-head
+    # scales; None for fp16/bf16 caches
+    k_scale: Optional[torch.Tensor] = None
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def num_seqs(self) -> int:
@@ -319,6 +323,39 @@ def prefill_plus_decode(seed=1005, device="cpu", scale=1.0, n_prefill=4, n_decod
     return [p, d]
 
 
+def with_fp8_cache(batch: PagedBatch, seed: int = 77) -> PagedBatch:
+    """The same batch (tables, lengths, q, new K/V) over an FP8 (e4m3) cache: every
+    cache slot holds a seeded random e4m3 code of magnitude code 0x00..0x48 (values 0..4,
+    subnormals included) with a random sign, and each kv-head has its own fp32 scales
+    (K: 0.25 * (1 + h/Hkv), V: 0.5 * (1 + h/(2 Hkv))).  The step's new K/V stay in the
+    batch's fp16/bf16 type: appending them quantises them."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    shape = tuple(batch.k_cache.shape)
+
+    def codes():
+        mag = rng.integers(0, 0x49, size=shape, dtype=np.int64)
+        sign = rng.integers(0, 2, size=shape, dtype=np.int64) << 7
+        return torch.from_numpy((mag | sign).astype(np.uint8)).to(batch.k_cache.device)
+
+    kc, vc = codes(), codes()
+    H = batch.num_kv_heads
+    hs = np.arange(H, dtype=np.float64)
+    ks = torch.tensor(0.25 * (1 + hs / H), dtype=torch.float32, device=batch.k_cache.device)
+    vs = torch.tensor(0.5 * (1 + hs / (2 * H)), dtype=torch.float32, device=batch.k_cache.device)
+    return dataclasses.replace(batch, name=batch.name + "_fp8kv", k_cache=kc, v_cache=vc,
+                               k_scale=ks, v_scale=vs)
+
+
+def mixed_lengths_fp8(seed=1003, device="cpu", scale=1.0, batch=64):
+    """The mixed-length batch of ``mixed_lengths`` with an FP8 (e4m3) KV cache."""
+    return [with_fp8_cache(mixed_lengths(seed=seed, device=device, scale=scale, batch=batch)[0])]
+
+
+def llama70b_fp8(seed=1002, device="cpu", scale=1.0):
+    """The LLaMA-70B-shaped batch of ``llama70b_uniform`` with an FP8 (e4m3) KV cache."""
+    return [with_fp8_cache(llama70b_uniform(seed=seed, device=device, scale=scale)[0])]
+
+
 WORKLOADS = {
     "tiny": tiny_mha,
     "llama70b": llama70b_uniform,
@@ -326,6 +363,8 @@ WORKLOADS = {
     "shared16": lambda **kw: shared_prefix(block_size=16, **kw),
     "shared32": lambda **kw: shared_prefix(block_size=32, **kw),
     "prefill_decode": prefill_plus_decode,
+    "mixed_fp8": mixed_lengths_fp8,
+    "llama70b_fp8": llama70b_fp8,
 }
 
 
