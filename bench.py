@@ -85,11 +85,15 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 def decode_algorithmic_bytes(b: workloads.PagedBatch) -> int:
-    """KV of every token at its exact length, q and out, table rows, seq_lens."""
+    """KV of every token at its exact length, q and out, table rows, seq_lens (plus the
+    per-kv-head scales of an FP8 cache)."""
     e = b.q.element_size()
+    ekv = b.k_cache.element_size()
     lens = b.seq_lens.cpu().numpy().astype(np.int64)
     B = len(lens)
-    kv = int(lens.sum()) * 2 * b.num_kv_heads * b.head_dim * e
+    kv = int(lens.sum()) * 2 * b.num_kv_heads * b.head_dim * ekv
+    if b.k_scale is not None:
+        kv += 2 * 4 * b.num_kv_heads
     qo = 2 * B * b.num_q_heads * b.head_dim * e
     tables = B * int(math.ceil(int(lens.max()) / b.block_size)) * 4
     return kv + qo + tables + 4 * B
@@ -189,7 +193,8 @@ class Step:
         self.prefill = [b for b in batches if b.query_start_loc is not None]
         # a decode batch whose every sequence appends one token runs pa_decode_append
         # (the append inside the decode launch); others append with pa_reshape_and_cache
-        self.fused = {id(b): int(b.k_new.shape[0]) == b.num_seqs for b in self.decode}
+        self.fused = {id(b): int(b.k_new.shape[0]) == b.num_seqs and b.k_scale is None
+                      for b in self.decode}
         self.ws = {}
         self.out = {}
         for b in batches:
@@ -219,7 +224,11 @@ class Step:
         for b in self.decode:
             if record is not None:
                 record[0].record(self.stream)
-            if self.fused[id(b)]:
+            if b.k_scale is not None:
+                self.pa.pa_decode_fp8(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.k_scale,
+                                      b.v_scale, b.block_tables, b.seq_lens, b.scale,
+                                      self.max_len[id(b)], 0, self.ws[id(b)], stream=self.stream)
+            elif self.fused[id(b)]:
                 self.pa.pa_decode_append(self.out[id(b)], b.q, b.k_new, b.v_new, b.k_cache,
                                          b.v_cache, b.block_tables, b.seq_lens, b.scale,
                                          self.max_len[id(b)], 0, self.ws[id(b)],
@@ -240,8 +249,13 @@ class Step:
         for b in self.batches:
             if self.fused.get(id(b)):
                 continue  # appended inside its decode launch
-            self.pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache, b.slot_mapping,
-                                         stream=self.stream)
+            if b.k_scale is not None:
+                self.pa.pa_reshape_and_cache_fp8(b.k_new, b.v_new, b.k_cache, b.v_cache,
+                                                 b.slot_mapping, b.k_scale, b.v_scale,
+                                                 stream=self.stream)
+            else:
+                self.pa.pa_reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache,
+                                             b.slot_mapping, stream=self.stream)
             n += self.pa.pa_last_launch_count()
         n += self.run_prefill()
         n += self.run_decode()
@@ -336,9 +350,15 @@ def run_ours(args, rank, world, device):
                     for i in range(n_kt):
                         l2_flush()
                         evs[i][0].record(stream)
-                        pa.pa_decode(out_ident, dec.q, dec.k_cache, dec.v_cache, tables,
-                                     dec.seq_lens, dec.scale, step.max_len[id(dec)], 0,
-                                     step.ws[id(dec)], stream=stream)
+                        if dec.k_scale is not None:
+                            pa.pa_decode_fp8(out_ident, dec.q, dec.k_cache, dec.v_cache,
+                                             dec.k_scale, dec.v_scale, tables, dec.seq_lens,
+                                             dec.scale, step.max_len[id(dec)], 0,
+                                             step.ws[id(dec)], stream=stream)
+                        else:
+                            pa.pa_decode(out_ident, dec.q, dec.k_cache, dec.v_cache, tables,
+                                         dec.seq_lens, dec.scale, step.max_len[id(dec)], 0,
+                                         step.ws[id(dec)], stream=stream)
                         evs[i][1].record(stream)
                 return g, evs
             g_paged = decode_graph(dec.block_tables)
@@ -424,7 +444,8 @@ def run_ours(args, rank, world, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if batches[0].dtype == torch.bfloat16 else "fp16",
+        "dtype": ("bf16" if batches[0].dtype == torch.bfloat16 else "fp16")
+                 + ("; KV cache e4m3" if any(b.k_scale is not None for b in batches) else ""),
         "data": "synthetic (seeded N(0,1) q/K/V, FIFO free-list block tables)",
         "impl": "ours",
         "gpu_launches": launches,
@@ -444,7 +465,8 @@ def run_ours(args, rank, world, device):
             ab += 2 * 2 * dec.num_seqs * dec.num_kv_heads * dec.head_dim * dec.q.element_size()
         dmean = statistics.mean(dec_ms)
         ach = ab / (dmean / 1e3) / 1e9
-        line["roofline"] = {"kernel": ("pa_decode_append" if step.fused[id(dec)] else "pa_decode")
+        line["roofline"] = {"kernel": ("pa_decode_fp8" if dec.k_scale is not None else
+                                       "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
                                       + " (paged_decode_kernel + lse_reduce_kernel)",
                             "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                             "peak_source": peaks["source"], "unit": "GB/s",
@@ -501,11 +523,16 @@ def cpu_baseline(batches, args, budget_s=None):
         L = int(lens[s])
         nblk = -(-L // b.block_size)
         ids = bt[0, :nblk].long().to(b.k_cache.device)
-        kc = opa.to_f64(b.k_cache.index_select(0, ids))
-        vc = opa.to_f64(b.v_cache.index_select(0, ids))
+        kc = b.k_cache.index_select(0, ids).cpu()
+        vc = b.v_cache.index_select(0, ids).cpu()
         tbl = np.arange(nblk, dtype=np.int32)[None, :]
         q = opa.to_f64(b.q[s:s + 1])
         t0 = time.perf_counter()
+        if b.k_scale is not None:  # FP8 cache: the oracle dequantises, then attends
+            kc = opa.dequantize_cache(kc.numpy(), b.k_scale.cpu().numpy())
+            vc = opa.dequantize_cache(vc.numpy(), b.v_scale.cpu().numpy())
+        else:
+            kc, vc = opa.to_f64(kc), opa.to_f64(vc)
         opa.paged_decode(q, kc, vc, tbl, np.array([L]), b.scale)
         t_used += time.perf_counter() - t0
         ctx_done += L
