@@ -25,6 +25,7 @@ path computes) on the host cores, on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -263,14 +264,6 @@ class Step:
         return n
 
 
-def host_inputs(b: workloads.PagedBatch):
-    """Pinned host copies of a step's per-step inputs (everything but the cache)."""
-    names = ["q", "k_new", "v_new", "slot_mapping", "seq_lens", "block_tables"]
-    if b.query_start_loc is not None:
-        names.append("query_start_loc")
-    return {n: getattr(b, n).cpu().pin_memory() for n in names}
-
-
 # ---------------------------------------------------------------- arms
 
 def run_ours(args, rank, world, device):
@@ -405,25 +398,83 @@ def run_ours(args, rank, world, device):
     launches = per_step_launches * args.steps
     total_ms = aggregate_max(local_ms, device)
 
-    # ---- end to end: per-step H2D of the step's inputs from pinned host
-    # memory, the C-ABI calls, D2H of the outputs
-    hosts = [host_inputs(b) for b in batches]
-    outs_h = [torch.empty(step.out[id(b)].shape, dtype=b.q.dtype).pin_memory() for b in batches]
-    h2d = sum(t.numel() * t.element_size() for h in hosts for t in h.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    # ---- end to end through the C ABI: every step uploads that step's inputs (q, new
+    # K/V, slot mapping, lengths, block tables) from pinned host memory and reads the
+    # outputs back.  The inputs of a step are packed into one pinned buffer and one device
+    # staging buffer (one copy each way per step); two staging buffers alternate, so the
+    # upload of step i+1 runs on a copy stream while step i computes.
     e2e_steps = max(3, min(args.steps, 20))
+    fields = ["q", "k_new", "v_new", "slot_mapping", "seq_lens", "block_tables",
+              "query_start_loc"]
+
+    def packed_layout():
+        offs, off = [], 0
+        for bb in batches:
+            o = {}
+            for n in fields:
+                t = getattr(bb, n)
+                if t is None:
+                    continue
+                o[n] = off
+                off += -(-t.numel() * t.element_size() // 256) * 256
+            offs.append(o)
+        return offs, off
+    offs, in_bytes = packed_layout()
+    host_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+    for bb, o in zip(batches, offs):
+        for n, off in o.items():
+            t = getattr(bb, n).contiguous().view(-1).view(torch.uint8).cpu()
+            host_in[off:off + t.numel()].copy_(t)
+
+    def staged_step():
+        dev_in = host_in.to(device)  # the Step reads lengths from it when it sizes itself
+        views = []
+        for bb, o in zip(batches, offs):
+            kw = {}
+            for n, off in o.items():
+                t = getattr(bb, n)
+                nbytes = t.numel() * t.element_size()
+                kw[n] = dev_in[off:off + nbytes].view(t.dtype).view(t.shape)
+            views.append(dataclasses.replace(bb, **kw))
+        st = Step(views, pa, stream)
+        outs = [st.out[id(v)] for v in views]
+        out_bytes = sum(t.numel() * t.element_size() for t in outs)
+        dev_out = torch.empty(out_bytes, dtype=torch.uint8, device=device)
+        off = 0
+        for v, t in zip(views, outs):
+            nbytes = t.numel() * t.element_size()
+            st.out[id(v)] = dev_out[off:off + nbytes].view(t.dtype).view(t.shape)
+            off += nbytes
+        host_out = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+        return dev_in, st, dev_out, host_out
+    stages = [staged_step() for _ in range(2)]
+    h2d = in_bytes
+    d2h = stages[0][2].numel()
+    copy_stream = torch.cuda.Stream(device=device)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    with torch.cuda.stream(stream):  # warm the staged calls once (first-call set-up)
+        for dev_in, st, dev_out, host_out in stages:
+            dev_in.copy_(host_in, non_blocking=True)
+            st.run()
     barrier()
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
+        copy_stream.wait_event(e0)
         for i in range(e2e_steps):
-            for b, h in zip(batches, hosts):
-                for n, t in h.items():
-                    getattr(b, n).copy_(t, non_blocking=True)
-            step.run()
-            for b, o in zip(batches, outs_h):
-                o.copy_(step.out[id(b)], non_blocking=True)
+            j = i % 2
+            dev_in, st, dev_out, host_out = stages[j]
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(done[j])  # step i-2 is done with this buffer
+                dev_in.copy_(host_in, non_blocking=True)
+                ready[j].record(copy_stream)
+            stream.wait_event(ready[j])
+            st.run()
+            host_out.copy_(dev_out, non_blocking=True)
+            done[j].record(stream)
         e1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
@@ -494,7 +545,10 @@ def run_ours(args, rank, world, device):
                                     "flop_per_launch": fl, "ms_per_launch": round(pmean, 5),
                                     "traffic": None}
     line["e2e"] = {"value": round(world * tokens * e2e_steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                   "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+                   "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                   "note": "eager C-ABI calls; each step's inputs packed in one pinned buffer and "
+                           "uploaded on a copy stream while the previous step computes (two "
+                           "staging buffers); outputs copied back every step"}
     line["clocks"] = clocks.summary()
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batches, args)
