@@ -202,7 +202,10 @@ class Step:
             self.out[id(b)] = torch.empty_like(b.q)
             if b.query_start_loc is None:
                 n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
-                self.ws[id(b)] = torch.empty(n, dtype=torch.uint8, device=b.q.device)
+            else:
+                n = pa.pa_chunked_prefill_workspace_size(b.num_seqs, b.max_query_len, b.num_q_heads,
+                                                         b.head_dim, b.max_seq_len)
+            self.ws[id(b)] = torch.empty(n, dtype=torch.uint8, device=b.q.device)
         self.max_len = {id(b): b.max_seq_len for b in batches}
         self.max_q = {id(b): b.max_query_len for b in batches}
         self.launches = 0
@@ -214,7 +217,7 @@ class Step:
                 record[0].record(self.stream)
             self.pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
                                        b.seq_lens, b.query_start_loc, b.scale, self.max_q[id(b)],
-                                       self.max_len[id(b)], None, stream=self.stream)
+                                       self.max_len[id(b)], self.ws[id(b)], stream=self.stream)
             n += self.pa.pa_last_launch_count()
             if record is not None:
                 record[1].record(self.stream)

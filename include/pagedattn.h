@@ -228,7 +228,12 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
 /* Size in bytes of the fixed scratch array pa_decode_noalloc uses (per device). */
 PA_API size_t pa_decode_noalloc_scratch_bytes(void);
 
-/* Bytes of scratch pa_chunked_prefill needs (0 in this version: no split-K). */
+/*
+ * Bytes of the optional pa_chunked_prefill workspace that lets it split its last wave
+ * (see pa_chunked_prefill): per split item 2 halves x 256 rows of head_dim+2 fp32 plus a
+ * 256-entry int32 row map, for up to min(128, num_seqs * num_q_heads *
+ * ceil(max_query_len / 32)) items.  0 means invalid arguments.
+ */
 PA_API size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len, int num_q_heads,
                                          int head_dim, int max_seq_len);
 
@@ -245,6 +250,14 @@ PA_API size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len,
  *                     attends to keys 0 .. that position, inclusive.
  *   max_query_len     host-side upper bound of the chunk lengths
  *   max_seq_len       host-side upper bound of seq_lens
+ *   workspace         optional (NULL allowed), 256-byte aligned device scratch of
+ *                     pa_chunked_prefill_workspace_size(...) bytes.  With it, when the
+ *                     last wave of (sequence, kv-head, query block) CTAs would fill at
+ *                     most half of the SMs, each of those items runs as two CTAs over
+ *                     the two halves of its keys and a second launch merges their
+ *                     normalised partials (log-sum-exp); the result differs from the
+ *                     unsplit one only by rounding.  Calls that overlap on the GPU must
+ *                     not share a workspace.
  */
 PA_API pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* block_tables, int max_blocks_per_seq,

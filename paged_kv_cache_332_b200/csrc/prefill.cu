@@ -59,6 +59,14 @@ struct Args {
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int max_query_len, seq_cap, qblocks;
   float qscale;  // scale * log2(e)
+  // wave tail: the last `split_items` items (after `whole_items`) run as two CTAs each,
+  // one per half of the item's key tiles, writing normalised partials that
+  // merge_split_kernel combines ([split item][half][256 rows] fp32 rows and (m, l);
+  // rowmap [split item][256 rows]: the output row, -1 for rows past the chunk)
+  int whole_items, split_items;
+  float* part_o;
+  float* part_ml;
+  int* rowmap;
 };
 
 // shared memory carve-up
@@ -226,10 +234,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- which (sequence, kv-head, query block)
-  const int qb = blockIdx.x % a.qblocks;
-  const int h = (blockIdx.x / a.qblocks) % a.num_kv_heads;
-  const int s = blockIdx.x / (a.qblocks * a.num_kv_heads);
+  // the merge of split items may be scheduled now; it waits for this grid itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---- which (sequence, kv-head, query block), and which part of its keys
+  int item = blockIdx.x, part = -1;  // part -1: all keys; 0 / 1: first / second half
+  if (a.split_items > 0 && (int)blockIdx.x >= a.whole_items) {
+    const int j = blockIdx.x - a.whole_items;
+    item = a.whole_items + (j >> 1);
+    part = j & 1;
+  }
+  const int sidx = item - a.whole_items;  // index among the split items (part >= 0)
+  auto mark_rows_unused = [&]() {         // a split item that writes no rows
+    if (part == 0)
+      for (int i = threadIdx.x; i < 2 * kM; i += blockDim.x) a.rowmap[sidx * 2 * kM + i] = -1;
+  };
+  const int qb = item % a.qblocks;
+  const int h = (item / a.qblocks) % a.num_kv_heads;
+  const int s = item / (a.qblocks * a.num_kv_heads);
   const int q_begin = a.qsl[s];
   const int n = a.qsl[s + 1] - q_begin;
   const int Lraw = a.seq_lens[s];
@@ -239,12 +261,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && qb == 0 && h == 0)
       flag_error(a.err, (n < 0 || n > L || n > a.max_query_len) ? PA_DEVERR_QUERY_LAYOUT
                                                                : PA_DEVERR_SEQ_TOO_LONG);
-    if (n < 0 || n > L || n > a.max_query_len) return;
+    if (n < 0 || n > L || n > a.max_query_len) {
+      mark_rows_unused();
+      return;
+    }
   }
-  if (q0 >= n) return;  // this query block is past the chunk (uniform for the CTA)
-  // keys any row of this CTA can see: [0, kv_end)
+  if (q0 >= n) {  // this query block is past the chunk (uniform for the CTA)
+    mark_rows_unused();
+    return;
+  }
+  // keys any row of this CTA can see: [0, kv_end); this CTA takes tiles [kt_lo, kt_hi)
   const int kv_end = min(L, L - n + min(n, q0 + 2 * MQ));
-  const int n_kt = (kv_end + kBN - 1) / kBN;
+  const int n_kt_all = (kv_end + kBN - 1) / kBN;
+  const int kt_lo = part == 1 ? n_kt_all / 2 : 0;
+  const int kt_hi = part == 0 ? n_kt_all / 2 : n_kt_all;
+  const int n_kt = kt_hi - kt_lo;  // tiles here; loops below count them from 0
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 8);  // one arrival per softmax warp once its Q rows are in place
@@ -307,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kt = 0; kt < n_kt; ++kt) {
       wait_or_abort(&s_full[mt], kt & 1, abort_flag, a.err);
       tc_fence_after();
-      const int key0 = kt * kBN;
+      const int key0 = (kt_lo + kt) * kBN;
       // the whole S row (128 keys) in registers: one pass over TMEM
       float v[kBN];
       tmem_ld64(t_s, v);
@@ -364,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * alpha + sum;
       // keys past the sequence end in the last tile: clear their V rows
-      if (mt == 0 && kt == n_kt - 1 && L < key0 + kBN) {
+      if (mt == 0 && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
         wait_or_abort(&v_full[kt & 1], (kt >> 1) & 1, abort_flag, a.err);
         uint8_t* vt = smem + OFF_V + (kt & 1) * kTileBytes;
         const int first = L - key0;  // first row to clear
@@ -384,23 +415,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_or_abort(&o_full[mt], 0, abort_flag, a.err);
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    T* orow = static_cast<T*>(a.out) +
-              ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD;
+    if (part < 0) {
+      T* orow = static_cast<T*>(a.out) +
+                ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      tmem_ld32(t_o + c * 32, v);
-      if (row_valid && n_kt > 0) {
-        uint32_t w[16];
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(t_o + c * 32, v);
+        if (row_valid && n_kt > 0) {
+          uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) w[i >> 1] = pack16<T>(v[i] * inv, v[i + 1] * inv);
+          for (int i = 0; i < 32; i += 2) w[i >> 1] = pack16<T>(v[i] * inv, v[i + 1] * inv);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(orow + c * 32 + j * 8) =
-              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(orow + c * 32 + j * 8) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        }
       }
+    } else {
+      // half of a split item: normalised partial row and its (reference max, sum)
+      const bool any = n_kt > 0 && l > 0.f;
+      const long long prow = (long long)(sidx * 2 + part) * 2 * kM + mt * kM + r;
+      float* po = a.part_o + prow * kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(t_o + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(po + c * 32 + j * 4) =
+              any ? make_float4(v[4 * j] * inv, v[4 * j + 1] * inv, v[4 * j + 2] * inv,
+                                v[4 * j + 3] * inv)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      *reinterpret_cast<float2*>(a.part_ml + prow * 2) =
+          any ? make_float2(m_ref, l) : make_float2(-INFINITY, 0.f);
+      if (part == 0)
+        a.rowmap[sidx * 2 * kM + mt * kM + r] =
+            row_valid && n_kt_all > 0
+                ? (int)(((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)))
+                : -1;
     }
-  
   } else {
     // producer / MMA issuer / two idle warps: 88 registers each thread
     // (128 x 88 + 256 x 208 = 384 x 168, the registers the CTA is launched with)
@@ -417,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto table_ids = [&](int kt, int (&id)[8]) {
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
-            const int pos = kt * kBN + r * 16;
+            const int pos = (kt_lo + kt) * kBN + r * 16;
             id[r] = pos < L ? __ldg(trow + (pos >> a.log2_bs)) : -1;
           }
         };
@@ -430,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int bid[8], row[8];
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
-            const int pos = kt * kBN + r * 16;
+            const int pos = (kt_lo + kt) * kBN + r * 16;
             const int id = next_id[r];
             bid[r] = a.num_blocks;  // past the tensor: TMA fills zeros
             row[r] = pos & bs_mask;
@@ -522,28 +577,98 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merge of the two halves of each split item: one warp per output row, lanes over
+// head_dim; o = (w0 o0 + w1 o1) / (w0 + w1), w_i = l_i 2^(m_i - max m).
+template <typename T>
+__global__ void __launch_bounds__(256) merge_split_kernel(const Args a) {
+  // a programmatic dependent of the prefill grid: wait for its partials
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= a.split_items * 2 * kM) return;
+  const int dst = a.rowmap[row];
+  if (dst < 0) return;
+  const int sidx = row / (2 * kM), rr = row - sidx * 2 * kM;
+  const long long p0 = (long long)(sidx * 2) * 2 * kM + rr, p1 = p0 + 2 * kM;
+  const float2 ml0 = *reinterpret_cast<const float2*>(a.part_ml + p0 * 2);
+  const float2 ml1 = *reinterpret_cast<const float2*>(a.part_ml + p1 * 2);
+  const float4 o0 = *reinterpret_cast<const float4*>(a.part_o + p0 * kD + lane * 4);
+  const float4 o1 = *reinterpret_cast<const float4*>(a.part_o + p1 * kD + lane * 4);
+  const float M = fmaxf(ml0.x, ml1.x);
+  const float w0 = ml0.x == -INFINITY ? 0.f : ml0.y * fast_exp2(ml0.x - M);
+  const float w1 = ml1.x == -INFINITY ? 0.f : ml1.y * fast_exp2(ml1.x - M);
+  const float inv = w0 + w1 > 0.f ? 1.f / (w0 + w1) : 0.f;
+  T* ob = static_cast<T*>(a.out) + (long long)dst * kD + lane * 4;
+  *reinterpret_cast<uint2*>(ob) =
+      make_uint2(pack16<T>((w0 * o0.x + w1 * o1.x) * inv, (w0 * o0.y + w1 * o1.y) * inv),
+                 pack16<T>((w0 * o0.z + w1 * o1.z) * inv, (w0 * o0.w + w1 * o1.w) * inv));
+}
+
+// Workspace of the wave-tail split for `split` items.
+inline size_t split_bytes(long long split) {
+  return (size_t)split * 2 * kM * (2 * (kD + 2) * sizeof(float) + sizeof(int));
+}
+
 template <typename T, int G>
-pa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
-                 cudaStream_t stream) {
+pa_status launch(const CUtensorMap& tk, const CUtensorMap& tv, Args a, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream) {
   auto kern = chunked_prefill_kernel<T, G>;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES)) return PA_ERR_CUDA;
-  const long long grid = (long long)a.num_seqs * a.num_kv_heads * a.qblocks;
-  if (grid <= 0) return PA_OK;
-  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  const long long items = (long long)a.num_seqs * a.num_kv_heads * a.qblocks;
+  if (items <= 0) return PA_OK;
+  if (items > 0x3fffffffLL) return PA_ERR_UNSUPPORTED;
+  // One CTA per SM: the items run in waves of `sms`.  When the last wave is at most half
+  // full, its items run as two CTAs each (one per half of the keys), so that wave takes
+  // about half as long; this needs the caller's workspace.
+  const int sms = std::max(1, num_sms());
+  long long split = 0;
+  const long long rem = items % sms;
+  if (workspace && rem > 0 && 2 * rem <= sms && workspace_bytes >= split_bytes(rem) &&
+      !((uintptr_t)workspace & 255))
+    split = rem;
+  a.whole_items = (int)(items - split);
+  a.split_items = (int)split;
+  if (split) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.part_o = reinterpret_cast<float*>(ws);
+    a.part_ml = a.part_o + (size_t)split * 2 * 2 * kM * kD;
+    a.rowmap = reinterpret_cast<int*>(a.part_ml + (size_t)split * 2 * 2 * kM * 2);
+  } else {
+    a.part_o = a.part_ml = nullptr;
+    a.rowmap = nullptr;
+  }
+  const long long grid = items + split;
   kern<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(tk, tv, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
-  set_launch_count(1);
+  int launches = 1;
+  if (split) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    const long long warps = split * 2 * kM;
+    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, merge_split_kernel<T>, a) != cudaSuccess) return PA_ERR_CUDA;
+    if (check_launch() != PA_OK) return PA_ERR_CUDA;
+    ++launches;
+  }
+  set_launch_count(launches);
   return PA_OK;
 }
 
 template <typename T>
 pa_status dispatch(int G, const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
-                   cudaStream_t stream) {
+                   void* ws, size_t wsb, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch<T, 1>(tk, tv, a, stream);
-    case 2: return launch<T, 2>(tk, tv, a, stream);
-    case 4: return launch<T, 4>(tk, tv, a, stream);
-    case 8: return launch<T, 8>(tk, tv, a, stream);
+    case 1: return launch<T, 1>(tk, tv, a, ws, wsb, stream);
+    case 2: return launch<T, 2>(tk, tv, a, ws, wsb, stream);
+    case 4: return launch<T, 4>(tk, tv, a, ws, wsb, stream);
+    case 8: return launch<T, 8>(tk, tv, a, ws, wsb, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -551,7 +676,17 @@ pa_status dispatch(int G, const CUtensorMap& tk, const CUtensorMap& tv, const Ar
 }  // namespace prefill
 }  // namespace pa
 
-extern "C" size_t pa_chunked_prefill_workspace_size(int, int, int, int, int) { return 0; }
+extern "C" size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len,
+                                                    int num_q_heads, int head_dim,
+                                                    int max_seq_len) {
+  (void)head_dim;
+  (void)max_seq_len;
+  if (num_seqs <= 0 || max_query_len <= 0 || num_q_heads <= 0) return 0;
+  // at most half a wave of items is split (SMs <= 256), and never more items than exist
+  // (query blocks hold at least 32 queries; kv-heads <= q-heads)
+  const long long items = (long long)num_seqs * num_q_heads * ((max_query_len + 31) / 32);
+  return pa::prefill::split_bytes(std::min<long long>(128, items));
+}
 
 extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache,
                                         const void* v_cache, const int32_t* block_tables,
@@ -561,8 +696,6 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
                                         int head_dim, float scale, int block_size, int num_blocks,
                                         int max_seq_len, void* workspace, size_t workspace_bytes,
                                         pa_dtype dtype, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   pa::set_launch_count(0);
   if (num_seqs < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
@@ -607,7 +740,11 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_seq_len);
   a.qblocks = (max_query_len + 2 * MQ - 1) / (2 * MQ);
   a.qscale = scale * 1.4426950408889634f;
+  // the split's row map stores output row numbers as int
+  const long long rows = (long long)num_seqs * max_query_len * num_q_heads;
+  if (rows > 0x7fffffffLL) workspace = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dtype == PA_F16 ? pa::prefill::dispatch<__half>(G, tk, tv, a, st)
-                         : pa::prefill::dispatch<__nv_bfloat16>(G, tk, tv, a, st);
+  return dtype == PA_F16
+             ? pa::prefill::dispatch<__half>(G, tk, tv, a, workspace, workspace_bytes, st)
+             : pa::prefill::dispatch<__nv_bfloat16>(G, tk, tv, a, workspace, workspace_bytes, st);
 }

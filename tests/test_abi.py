@@ -75,7 +75,11 @@ def test_workspace_size_arithmetic(palib):
     assert palib.pa_decode_workspace_size(16, 64, 128, 32768, 512) == \
         16 * 64 * 8 + ((256 + 16) * 64 + 16 * 64 * 64 + 64) * 130 * 4
     assert palib.pa_decode_workspace_size(0, 8, 128, 100, 16) == 0  # invalid shape
-    assert palib.pa_chunked_prefill_workspace_size(4, 512, 64, 128, 8000) == 0
+    # prefill's optional wave-tail split: <= 128 items of 2 halves x 256 rows
+    per_item = 256 * (2 * 130 * 4 + 4)  # 2 halves x 256 rows of 130 fp32, 256 row ids
+    assert palib.pa_chunked_prefill_workspace_size(4, 512, 64, 128, 8000) == 128 * per_item
+    assert palib.pa_chunked_prefill_workspace_size(1, 32, 2, 128, 100) == 2 * per_item
+    assert palib.pa_chunked_prefill_workspace_size(0, 32, 2, 128, 100) == 0
 
 
 def _raw(palib):

@@ -128,3 +128,38 @@ def test_prefill_full_size_sampled_rows():
                                            p.scale))
                     got.append(out[int(qsl[s]) + i, hq])
     P.compare(torch.stack(got), np.stack(want), p.dtype, "chunked prefill full size, sampled")
+
+
+def _prefill_with_workspace(b):
+    ws = torch.empty(pa.pa_chunked_prefill_workspace_size(b.num_seqs, b.max_query_len,
+                                                          b.num_q_heads, 128, b.max_seq_len),
+                     dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(b.q)
+    pa.pa_chunked_prefill(out, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
+                          b.query_start_loc, b.scale, b.max_query_len, b.max_seq_len, ws)
+    return out, pa.pa_last_launch_count()
+
+
+@pytest.mark.parametrize("lens,qlens", [
+    ([300, 400, 250, 500], [160, 160, 160, 160]),   # 160 items: a 12-item tail wave on 148 SMs
+    ([300, 40, 250, 500], [160, 10, 160, 33]),      # ragged chunks: split items with no rows
+    ([700], [64]),                                  # 16 items: every item split
+])
+def test_prefill_wave_tail_split(lens, qlens):
+    """With the optional workspace the last wave's items run as two halves of their keys
+    and are merged; the result matches the oracle and the unsplit call."""
+    bc = _batch(lens, qlens, 8, torch.bfloat16, Hkv=8, seed=31)
+    b = bc.to(DEV)
+    P.gpu_append(b)
+    plain = P.gpu_prefill(b)
+    split, launches = _prefill_with_workspace(b)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    qblocks = -(-max(qlens) // 32)
+    items = len(lens) * 8 * qblocks
+    tail = items % sms
+    assert launches == (2 if 0 < 2 * tail <= sms else 1)
+    ref = P.oracle_prefill(bc)
+    P.compare(split, ref, bc.dtype, "prefill with the wave tail split")
+    assert (split.float() - plain.float()).abs().max().item() <= P.TOL[bc.dtype]
