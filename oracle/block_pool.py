@@ -1,0 +1,90 @@
+"""Plain oracle of block-table maintenance (test infrastructure only: only tests/,
+the package entry's smoke check and bench.py's baseline may use it; the library never
+imports it).
+
+Source — page "大模型推理内存优化从 KV Cache 分页到连续批处理的工程实践", section
+"生产级推理引擎的内存管理与调度": a pool of physical blocks keeps its free block ids in a
+FIFO queue (a new pool holds 0..N-1 in order; allocating pops the front, freeing pushes
+the id on the back); the scheduler gives a sequence a new block when the blocks it needs
+for its tokens (integer ceiling of tokens / block size) exceed the blocks it owns, and
+when no block is free that sequence is preempted for this step while later sequences
+are still considered; a finished sequence returns all its blocks to the pool.
+
+Readings where the page is silent:
+- a step may append several tokens to a sequence (a prefill chunk); the sequence gets
+  all the blocks it needs or none (preempted: nothing allocated, no slots);
+- sequences are served in index order; a sequence's blocks are freed in table order,
+  sequences in index order;
+- the free queue is a ring of N entries with a head (next id to allocate) and a count;
+- a token at position p of sequence s lands in slot table[s][p // bs] * bs + p % bs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def blocks_needed(num_tokens, block_size):
+    """Integer ceiling of tokens / block size (the scheduler's block count)."""
+    return (num_tokens + block_size - 1) // block_size
+
+
+class BlockPool:
+    """The FIFO free-block queue as a ring: ``ring[(head + i) % N]`` for i < count are
+    the free ids, the front first."""
+
+    def __init__(self, num_blocks):
+        self.n = int(num_blocks)
+        self.ring = np.arange(self.n, dtype=np.int64)
+        self.head = 0
+        self.count = self.n
+
+    def available(self):
+        return self.count
+
+    def allocate(self):
+        """Pop the front id (None when empty)."""
+        if self.count == 0:
+            return None
+        b = int(self.ring[self.head])
+        self.head = (self.head + 1) % self.n
+        self.count -= 1
+        return b
+
+    def free(self, block_id):
+        """Push ``block_id`` on the back."""
+        assert self.count < self.n
+        self.ring[(self.head + self.count) % self.n] = block_id
+        self.count += 1
+
+
+def allocate_step(pool, block_tables, owned, seq_lens, q_lens, block_size):
+    """One step of appends: sequence s (index order) holds ``seq_lens[s]`` tokens in
+    ``owned[s]`` blocks and appends ``q_lens[s]`` tokens.  If it needs more blocks than
+    it owns it pops them from the pool, all or none.  Updates ``block_tables`` and
+    ``owned`` in place; returns (slot_mapping int64 [sum q_lens], granted bool [B]).
+    A preempted sequence's slots are -1 and its table is unchanged."""
+    B = len(seq_lens)
+    slots, granted = [], np.zeros(B, dtype=bool)
+    for s in range(B):
+        L, q = int(seq_lens[s]), int(q_lens[s])
+        extra = max(0, blocks_needed(L + q, block_size) - int(owned[s]))
+        ok = extra <= pool.available() and int(owned[s]) + extra <= block_tables.shape[1]
+        if ok:
+            for _ in range(extra):
+                block_tables[s, owned[s]] = pool.allocate()
+                owned[s] += 1
+        granted[s] = ok
+        for p in range(L, L + q):
+            slots.append(int(block_tables[s, p // block_size]) * block_size + p % block_size
+                         if ok else -1)
+    return np.asarray(slots, dtype=np.int64), granted
+
+
+def free_sequences(pool, block_tables, owned, finished):
+    """Return every block of each finished sequence to the pool (sequences in index
+    order, blocks in table order) and set its owned count to 0."""
+    for s in range(len(owned)):
+        if finished[s]:
+            for j in range(int(owned[s])):
+                pool.free(int(block_tables[s, j]))
+            owned[s] = 0
