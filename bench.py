@@ -269,6 +269,57 @@ class Step:
 
 # ---------------------------------------------------------------- arms
 
+def block_pool_timing(pa, dec, stream, device, n=8):
+    """Device time of the block-table calls for one decode step of ``dec``'s sequences:
+    pa_block_allocate with one new token per sequence (sequences at a block boundary take
+    a block) and pa_block_free of every 16th sequence.  Pool, tables and owned counts are
+    restored from a snapshot before each timed call, so every call does the same work."""
+    B, bs = dec.num_seqs, dec.block_size
+    lens = dec.seq_lens
+    max_blocks = -(-(int(lens.max()) + 1) // bs)
+    n_blocks = int(((lens + 1 + bs - 1) // bs).sum()) + B
+    ring = torch.empty(n_blocks, dtype=torch.int32, device=device)
+    state = torch.empty(2, dtype=torch.int32, device=device)
+    tables = torch.zeros((B, max_blocks), dtype=torch.int32, device=device)
+    owned = torch.zeros(B, dtype=torch.int32, device=device)
+    zeros = torch.zeros(B, dtype=torch.int32, device=device)
+    ones = torch.ones(B, dtype=torch.int32, device=device)
+    slots = torch.empty(max(int(lens.sum()), B, 1), dtype=torch.int32, device=device)
+    granted = torch.empty(B, dtype=torch.int32, device=device)
+    finished = (torch.arange(B, device=device) % 16 == 0).to(torch.int32)
+    with torch.cuda.stream(stream):
+        pa.pa_block_pool_init(ring, state, stream=stream)
+        # prompts: every sequence's first seq_lens tokens
+        pa.pa_block_allocate(ring, state, tables, owned, zeros, lens, bs, slots, granted,
+                             stream=stream)
+    torch.cuda.synchronize(device)
+    snap = [t.clone() for t in (ring, state, tables, owned)]
+    new_blocks = int(((lens % bs) == 0).sum())
+
+    def timed(call):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n + 2)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                for dst, src in zip((ring, state, tables, owned), snap):
+                    dst.copy_(src)
+                a.record(stream)
+                call()
+                b.record(stream)
+        torch.cuda.synchronize(device)
+        return statistics.mean(a.elapsed_time(b) for a, b in evs[2:]) * 1e3
+
+    alloc_us = timed(lambda: pa.pa_block_allocate(ring, state, tables, owned, lens, ones, bs,
+                                                  slots, granted, stream=stream))
+    free_us = timed(lambda: pa.pa_block_free(ring, state, tables, owned, finished,
+                                             stream=stream))
+    return {"allocate_us": round(alloc_us, 2), "free_us": round(free_us, 2), "num_seqs": B,
+            "new_blocks_per_allocate": new_blocks, "freed_seqs": int(finished.sum()),
+            "bound": "latency (one CTA per call; a few KB of table traffic)",
+            "note": "pa_block_allocate: one token per sequence; pa_block_free: every 16th "
+                    "sequence; state restored before each of %d timed calls" % n}
+
+
 def run_ours(args, rank, world, device):
     import paged_kv_cache_332_b200 as pa
     pa.lib()  # fails loudly if the library is missing
@@ -483,6 +534,8 @@ def run_ours(args, rank, world, device):
     barrier()
     e2e_ms = aggregate_max(e0.elapsed_time(e1), device)
 
+    pool_line = block_pool_timing(pa, dec, stream, device) if dec is not None else None
+
     # ---- metric
     tokens = sum(b.num_seqs for b in step.decode) + sum(int(b.q.shape[0]) for b in step.prefill)
     value = world * tokens * args.steps / (total_ms / 1e3)
@@ -552,6 +605,8 @@ def run_ours(args, rank, world, device):
                    "note": "eager C-ABI calls; each step's inputs packed in one pinned buffer and "
                            "uploaded on a copy stream while the previous step computes (two "
                            "staging buffers); outputs copied back every step"}
+    if pool_line is not None:
+        line["block_pool"] = pool_line
     line["clocks"] = clocks.summary()
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batches, args)

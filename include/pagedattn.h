@@ -69,6 +69,8 @@ typedef enum {
 #define PA_DEVERR_QUERY_LAYOUT 0x8  /* prefill: query_start_loc not monotone, q_len > seq_len
                                        or q_len > max_query_len */
 #define PA_DEVERR_TIMEOUT      0x10 /* an in-kernel pipeline wait gave up (never expected) */
+#define PA_DEVERR_POOL         0x20 /* block pool: state out of range, or more blocks freed
+                                       than the ring holds (nothing changed) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 PA_API const char* pa_status_string(int status);
@@ -197,6 +199,55 @@ PA_API pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, co
                                int num_kv_heads, int head_dim, float scale, int block_size,
                                int num_blocks, int max_seq_len, int partition_size,
                                void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                               void* stream);
+
+/*
+ * Device-side block-table maintenance.  [P1] "生产级推理引擎的内存管理与调度": a pool
+ * keeps the free block ids in a FIFO queue (a new pool holds 0..N-1 in order; allocation
+ * pops the front, freeing pushes the back); a sequence gets new blocks when the blocks
+ * its tokens need, ceil(tokens / block_size), exceed the blocks it owns; with too few
+ * free blocks it is preempted for the step while later sequences are still served; a
+ * finished sequence returns its blocks.  The queue lives on the device as a ring
+ * `ring` int32 [num_blocks] with `state` int32 [2] = {head, count}; the free ids are
+ * ring[(head + i) % num_blocks], i < count, the front first.  All arguments are device
+ * pointers; each call is one kernel on `stream`.
+ */
+
+/* pa_block_pool_init — ring = 0..num_blocks-1, head = 0, count = num_blocks. */
+PA_API pa_status pa_block_pool_init(int32_t* ring, int32_t* state, int num_blocks, void* stream);
+
+/*
+ * pa_block_allocate — one step of appends.  Sequence s holds seq_lens[s] tokens in
+ * blocks_owned[s] blocks (the first entries of its block_tables row) and appends
+ * q_lens[s] tokens.  In index order, a sequence that needs more blocks takes all of them
+ * from the front of the ring (appended to its table, blocks_owned updated) or, if the
+ * ring holds fewer than it needs or its table row is too short, none (granted[s] = 0).
+ *   slot_mapping  int32 [sum q_lens] out: the slot of every appended token, sequences in
+ *                 index order (positions seq_lens[s] .. seq_lens[s]+q_lens[s]-1), -1 for a
+ *                 sequence not granted — ready for pa_reshape_and_cache
+ *   granted       int32 [num_seqs] out
+ * seq_lens is not updated (the caller adds q_lens of granted sequences).  Limits:
+ * num_seqs <= 4096, block_size 16 or 32.  Device-side errors (PA_DEVERR_POOL, read with
+ * pa_get_device_error): a state that is not {0 <= head < num_blocks, 0 <= count <=
+ * num_blocks} changes nothing; a sequence with a negative length or a blocks_owned[s]
+ * outside [0, max_blocks_per_seq] is not granted.
+ */
+PA_API pa_status pa_block_allocate(int32_t* ring, int32_t* state, int num_blocks,
+                                   int32_t* block_tables, int max_blocks_per_seq,
+                                   int32_t* blocks_owned, const int32_t* seq_lens,
+                                   const int32_t* q_lens, int num_seqs, int block_size,
+                                   int32_t* slot_mapping, int32_t* granted, void* stream);
+
+/*
+ * pa_block_free — every sequence with finished[s] != 0 returns its blocks_owned[s]
+ * blocks to the back of the ring (sequences in index order, blocks in table order) and
+ * gets blocks_owned[s] = 0.  Returning more blocks than the ring can hold, or a state
+ * that is not a pool state, changes nothing and sets PA_DEVERR_POOL.  Limits:
+ * num_seqs <= 4096.
+ */
+PA_API pa_status pa_block_free(int32_t* ring, int32_t* state, int num_blocks,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               int32_t* blocks_owned, const int32_t* finished, int num_seqs,
                                void* stream);
 
 /*

@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
     "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
-    "pa_reshape_and_cache_fp8", "pa_decode_fp8",
+    "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_block_pool_init", "pa_block_allocate",
+    "pa_block_free",
     "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
@@ -32,7 +33,7 @@ library_path = os.path.join(_HERE, "libpagedattn.so")
 PA_OK = 0
 PA_F16, PA_BF16 = 0, 1
 PA_DEVERR = {"SLOT_RANGE": 0x1, "BLOCK_RANGE": 0x2, "SEQ_TOO_LONG": 0x4, "QUERY_LAYOUT": 0x8,
-             "TIMEOUT": 0x10}
+             "TIMEOUT": 0x10, "POOL": 0x20}
 
 # (name, restype, argtypes) of every entry point declared in include/pagedattn.h
 _vp, _i32, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -48,6 +49,10 @@ _SIGS = [
                                         _i32, _i32, _vp]),
     ("pa_decode_fp8", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                              _f, _i32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+    ("pa_block_pool_init", _i32, [_vp, _vp, _i32, _vp]),
+    ("pa_block_allocate", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _vp, _vp,
+                                 _vp]),
+    ("pa_block_free", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
     ("pa_decode_noalloc", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f,
                                  _i32, _i32, _i32, _i32, _i32, _vp]),
     ("pa_decode_noalloc_scratch_bytes", _sz, []),
@@ -214,6 +219,37 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_
                                N, int(max_seq_len), int(partition_size), _ptr(workspace),
                                ws_bytes, _dtype_code(q), _stream(stream)),
            "pa_decode_fp8")
+
+
+def pa_block_pool_init(ring, state, stream=None):
+    """Fill the device ring (int32 [N]) with 0..N-1 and state (int32 [2]) with {0, N}."""
+    _check(lib().pa_block_pool_init(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                                    ring.numel(), _stream(stream)), "pa_block_pool_init")
+
+
+def pa_block_allocate(ring, state, block_tables, blocks_owned, seq_lens, q_lens, block_size,
+                      slot_mapping, granted, stream=None):
+    """One step of appends on the device pool: grows ``block_tables``/``blocks_owned`` in
+    place and writes ``slot_mapping`` (int32 [sum q_lens]) and ``granted`` (int32 [B])."""
+    _check(lib().pa_block_allocate(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                                   ring.numel(), _i32tensor(block_tables, "block_tables"),
+                                   block_tables.shape[1], _i32tensor(blocks_owned, "blocks_owned"),
+                                   _i32tensor(seq_lens, "seq_lens"), _i32tensor(q_lens, "q_lens"),
+                                   seq_lens.numel(), int(block_size),
+                                   _i32tensor(slot_mapping, "slot_mapping"),
+                                   _i32tensor(granted, "granted"), _stream(stream)),
+           "pa_block_allocate")
+
+
+def pa_block_free(ring, state, block_tables, blocks_owned, finished, stream=None):
+    """Return the blocks of every sequence with ``finished[s] != 0`` (int32 [B]) to the
+    back of the device ring."""
+    _check(lib().pa_block_free(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                               ring.numel(), _i32tensor(block_tables, "block_tables"),
+                               block_tables.shape[1], _i32tensor(blocks_owned, "blocks_owned"),
+                               _i32tensor(finished, "finished"), finished.numel(),
+                               _stream(stream)),
+           "pa_block_free")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

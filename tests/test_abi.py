@@ -157,6 +157,27 @@ def test_fp8_arguments_rejected_on_host(palib):
     assert palib.pa_last_launch_count() == 0
 
 
+def test_block_pool_arguments_rejected_on_host(palib):
+    L = _raw(palib)
+    p = ctypes.c_void_p(4096)
+    nul = None
+    assert L.pa_block_pool_init(p, p, 0, nul) == 1          # empty pool
+    assert L.pa_block_pool_init(nul, p, 8, nul) == 1        # ring missing
+
+    def alloc(ring=p, n=64, mb=8, B=4, bs=16, slots=p):
+        return L.pa_block_allocate(ring, p, n, p, mb, p, p, p, B, bs, slots, p, nul)
+    assert alloc(n=0) == 1 and alloc(mb=0) == 1 and alloc(B=-1) == 1
+    assert alloc(bs=8) == 2                                  # block size 16 or 32
+    assert alloc(B=4097) == 2                                # one CTA's limit
+    assert alloc(B=0) == 0                                   # nothing to do
+    assert alloc(ring=nul) == 1 and alloc(slots=nul) == 1
+
+    def free(n=64, B=4, fin=p):
+        return L.pa_block_free(p, p, n, p, 8, p, fin, B, nul)
+    assert free(n=0) == 1 and free(B=4097) == 2 and free(B=0) == 0 and free(fin=nul) == 1
+    assert palib.pa_last_launch_count() == 0
+
+
 def test_product_package_does_not_touch_oracle():
     # the product path never imports the oracle
     pkg = os.path.join(ROOT, "paged_kv_cache_332_b200")
