@@ -85,14 +85,23 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
-def decode_algorithmic_bytes(b: workloads.PagedBatch) -> int:
+def decode_algorithmic_bytes(b: workloads.PagedBatch, shared: bool = False) -> int:
     """KV of every token at its exact length, q and out, table rows, seq_lens (plus the
-    per-kv-head scales of an FP8 cache)."""
+    per-kv-head scales of an FP8 cache).  With ``shared``, the tokens of a group's shared
+    prefix count once per group (and the group arrays are added)."""
     e = b.q.element_size()
     ekv = b.k_cache.element_size()
     lens = b.seq_lens.cpu().numpy().astype(np.int64)
     B = len(lens)
-    kv = int(lens.sum()) * 2 * b.num_kv_heads * b.head_dim * ekv
+    tokens = int(lens.sum())
+    if shared:
+        gs = b.group_starts.cpu().numpy().astype(np.int64)
+        pl = b.prefix_lens.cpu().numpy().astype(np.int64)
+        tokens -= int(((gs[1:] - gs[:-1] - 1).clip(min=0) * pl).sum())
+        extra = 4 * (len(gs) + len(pl))
+    else:
+        extra = 0
+    kv = tokens * 2 * b.num_kv_heads * b.head_dim * ekv + extra
     if b.k_scale is not None:
         kv += 2 * 4 * b.num_kv_heads
     qo = 2 * B * b.num_q_heads * b.head_dim * e
@@ -194,13 +203,25 @@ class Step:
         self.prefill = [b for b in batches if b.query_start_loc is not None]
         # a decode batch whose every sequence appends one token runs pa_decode_append
         # (the append inside the decode launch); others append with pa_reshape_and_cache
+        # a batch whose sequences share prompt blocks runs pa_decode_shared_prefix (the
+        # shared blocks read once per group), after pa_reshape_and_cache
+        self.shared = {id(b): b.group_starts is not None and b.k_scale is None
+                       for b in self.decode}
         self.fused = {id(b): int(b.k_new.shape[0]) == b.num_seqs and b.k_scale is None
-                      for b in self.decode}
+                      and not self.shared[id(b)] for b in self.decode}
+        self.group_bounds = {}
+        for b in self.decode:
+            if self.shared[id(b)]:
+                sizes = (b.group_starts[1:] - b.group_starts[:-1]).cpu()
+                self.group_bounds[id(b)] = (int(sizes.max()), int(b.prefix_lens.max()))
         self.ws = {}
         self.out = {}
         for b in batches:
             self.out[id(b)] = torch.empty_like(b.q)
-            if b.query_start_loc is None:
+            if b.query_start_loc is None and self.shared[id(b)]:
+                n = pa.pa_decode_shared_prefix_workspace_size(b.num_seqs, b.num_q_heads,
+                                                              b.head_dim, b.max_seq_len)
+            elif b.query_start_loc is None:
                 n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
             else:
                 n = pa.pa_chunked_prefill_workspace_size(b.num_seqs, b.max_query_len, b.num_q_heads,
@@ -232,6 +253,12 @@ class Step:
                 self.pa.pa_decode_fp8(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.k_scale,
                                       b.v_scale, b.block_tables, b.seq_lens, b.scale,
                                       self.max_len[id(b)], 0, self.ws[id(b)], stream=self.stream)
+            elif self.shared[id(b)]:
+                mg, mp = self.group_bounds[id(b)]
+                self.pa.pa_decode_shared_prefix(self.out[id(b)], b.q, b.k_cache, b.v_cache,
+                                                b.block_tables, b.seq_lens, b.group_starts,
+                                                b.prefix_lens, b.scale, self.max_len[id(b)], mg,
+                                                mp, self.ws[id(b)], stream=self.stream)
             elif self.fused[id(b)]:
                 self.pa.pa_decode_append(self.out[id(b)], b.q, b.k_new, b.v_new, b.k_cache,
                                          b.v_cache, b.block_tables, b.seq_lens, b.scale,
@@ -297,17 +324,26 @@ def block_pool_timing(pa, dec, stream, device, n=8):
     new_blocks = int(((lens % bs) == 0).sum())
 
     def timed(call):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(n + 2)]
+        # captured as one graph (restore, event, call, event) x n, so the host's launch
+        # latency stays out of the device time between the events
+        evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
         with torch.cuda.stream(stream):
+            call()  # first-call set-up outside the capture
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
             for a, b in evs:
                 for dst, src in zip((ring, state, tables, owned), snap):
                     dst.copy_(src)
                 a.record(stream)
                 call()
                 b.record(stream)
+        with torch.cuda.stream(stream):
+            g.replay()  # warm
+            g.replay()
         torch.cuda.synchronize(device)
-        return statistics.mean(a.elapsed_time(b) for a, b in evs[2:]) * 1e3
+        return statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
 
     alloc_us = timed(lambda: pa.pa_block_allocate(ring, state, tables, owned, lens, ones, bs,
                                                   slots, granted, stream=stream))
@@ -459,7 +495,7 @@ def run_ours(args, rank, world, device):
     # upload of step i+1 runs on a copy stream while step i computes.
     e2e_steps = max(3, min(args.steps, 20))
     fields = ["q", "k_new", "v_new", "slot_mapping", "seq_lens", "block_tables",
-              "query_start_loc"]
+              "query_start_loc", "group_starts", "prefix_lens"]
 
     def packed_layout():
         offs, off = [], 0
@@ -570,17 +606,28 @@ def run_ours(args, rank, world, device):
         ab = decode_algorithmic_bytes(dec)
         if step.fused[id(dec)]:  # the append inside the launch: read k/v_new, write the slots
             ab += 2 * 2 * dec.num_seqs * dec.num_kv_heads * dec.head_dim * dec.q.element_size()
+        shared = step.shared[id(dec)]
+        if shared:  # the shared blocks are read once per group
+            ab_unshared = ab
+            ab = decode_algorithmic_bytes(dec, shared=True)
         dmean = statistics.mean(dec_ms)
         ach = ab / (dmean / 1e3) / 1e9
-        line["roofline"] = {"kernel": ("pa_decode_fp8" if dec.k_scale is not None else
-                                       "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
-                                      + " (paged_decode_kernel + lse_reduce_kernel)",
+        kname = ("pa_decode_fp8" if dec.k_scale is not None else
+                 "pa_decode_shared_prefix" if shared else
+                 "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
+        kparts = (" (chunked_prefill_kernel prefix pass + paged_decode_kernel + lse_reduce_kernel)"
+                  if shared else " (paged_decode_kernel + lse_reduce_kernel)")
+        line["roofline"] = {"kernel": kname + kparts,
                             "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                             "peak_source": peaks["source"], "unit": "GB/s",
                             "frac": round(ach / peaks["hbm_gbs"], 4),
                             "frac_of_8TBs_spec": round(ach / 8000.0, 4),
                             "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
                             "traffic": recorded_traffic("paged_decode_kernel", dec.name)}
+        if shared:
+            line["roofline"]["algorithmic_bytes_unshared"] = ab_unshared
+            line["roofline"]["note"] = ("bytes count each shared prefix block once per group; "
+                                        "algorithmic_bytes_unshared counts it once per member")
         if ident_ms:
             im, pm = statistics.mean(ident_ms), statistics.mean(paged_ms)
             line["indirection"] = {"paged_ms": round(pm, 5), "identity_tables_ms": round(im, 5),

@@ -9,7 +9,8 @@
  *        the block table), "工程边界与架构取舍" (decode is memory-bound and reads
  *        the whole cache; long prompts are prefilled in chunks).
  *   [P2] "KV Cache管理优化：大模型推理显存瓶颈突破" (intelliparadigm), 2.1 (one
- *        pre-allocated pool, no per-request allocation), 2.2 (blocks of 16-32 tokens).
+ *        pre-allocated pool, no per-request allocation), 2.2 (blocks of 16-32 tokens),
+ *        4.1 (blocks shared across sequences by reference counting).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -71,6 +72,9 @@ typedef enum {
 #define PA_DEVERR_TIMEOUT      0x10 /* an in-kernel pipeline wait gave up (never expected) */
 #define PA_DEVERR_POOL         0x20 /* block pool: state out of range, or more blocks freed
                                        than the ring holds (nothing changed) */
+#define PA_DEVERR_PREFIX       0x40 /* shared-prefix decode: a prefix length negative, not a
+                                       multiple of block_size, above max_prefix_len or
+                                       above a member's seq_len */
 
 /* Human-readable name of a status code (static string, never NULL). */
 PA_API const char* pa_status_string(int status);
@@ -200,6 +204,44 @@ PA_API pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, co
                                int num_blocks, int max_seq_len, int partition_size,
                                void* workspace, size_t workspace_bytes, pa_dtype dtype,
                                void* stream);
+
+/*
+ * pa_decode_shared_prefix — pa_decode for a batch in which groups of sequences share the
+ * first tokens of their context (parallel sampling or beam search over one prompt: [P1]
+ * "KV Cache 的内存开销与分页机制", block-level sharing of prefix blocks, and [P2] 4.1,
+ * reference-counted blocks that several block tables point at).  The result is
+ * pa_decode's, within the same tolerance; the shared blocks are read once per group
+ * instead of once per member.
+ *   group_starts  int32 [num_groups + 1], device: group g is the sequences
+ *                 group_starts[g] .. group_starts[g+1]-1 (ascending, within [0, num_seqs]);
+ *                 sequences outside every group share nothing
+ *   prefix_lens   int32 [num_groups], device: tokens shared by the members of group g, a
+ *                 multiple of block_size, at most max_prefix_len and each member's seq_len;
+ *                 the first prefix_lens[g] / block_size table entries of the members hold
+ *                 the same K/V (normally the same physical blocks); they are read through
+ *                 the table row of the group's first member
+ *   max_group_size, max_prefix_len  host bounds (grid sizing)
+ * Three launches: the prefix pass (the tcgen05 prefill kernel with the members' q-heads
+ * of one kv-head as the rows of an M-tile, no causal mask, the prefix cut into up to 8
+ * pieces that write normalised partial rows), the decode kernel over each sequence's
+ * keys after its prefix, and the log-sum-exp merge of both.  Workspace: at least
+ * pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len)
+ * bytes, 256-byte aligned.  An invalid prefix sets PA_DEVERR_PREFIX (outputs of its
+ * group unspecified).  fp16/bf16 caches; other limits as pa_decode (partition_size 0).
+ * With num_groups, max_group_size or max_prefix_len 0 it is pa_decode.
+ */
+PA_API size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+                                                     int max_seq_len);
+PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* seq_lens,
+                                         int num_seqs, const int32_t* group_starts,
+                                         const int32_t* prefix_lens, int num_groups,
+                                         int max_group_size, int max_prefix_len, int num_q_heads,
+                                         int num_kv_heads, int head_dim, float scale,
+                                         int block_size, int num_blocks, int max_seq_len,
+                                         void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                                         void* stream);
 
 /*
  * Device-side block-table maintenance.  [P1] "生产级推理引擎的内存管理与调度": a pool

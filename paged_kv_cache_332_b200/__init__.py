@@ -20,7 +20,7 @@ __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
     "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_block_pool_init", "pa_block_allocate",
-    "pa_block_free",
+    "pa_block_free", "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
     "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
@@ -33,7 +33,7 @@ library_path = os.path.join(_HERE, "libpagedattn.so")
 PA_OK = 0
 PA_F16, PA_BF16 = 0, 1
 PA_DEVERR = {"SLOT_RANGE": 0x1, "BLOCK_RANGE": 0x2, "SEQ_TOO_LONG": 0x4, "QUERY_LAYOUT": 0x8,
-             "TIMEOUT": 0x10, "POOL": 0x20}
+             "TIMEOUT": 0x10, "POOL": 0x20, "PREFIX": 0x40}
 
 # (name, restype, argtypes) of every entry point declared in include/pagedattn.h
 _vp, _i32, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
@@ -53,6 +53,10 @@ _SIGS = [
     ("pa_block_allocate", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _vp, _vp,
                                  _vp]),
     ("pa_block_free", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
+    ("pa_decode_shared_prefix_workspace_size", _sz, [_i32, _i32, _i32, _i32]),
+    ("pa_decode_shared_prefix", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
+                                       _i32, _i32, _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp,
+                                       _sz, _i32, _vp]),
     ("pa_decode_noalloc", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _f,
                                  _i32, _i32, _i32, _i32, _i32, _vp]),
     ("pa_decode_noalloc_scratch_bytes", _sz, []),
@@ -250,6 +254,30 @@ def pa_block_free(ring, state, block_tables, blocks_owned, finished, stream=None
                                _i32tensor(finished, "finished"), finished.numel(),
                                _stream(stream)),
            "pa_block_free")
+
+
+def pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len):
+    return int(lib().pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim,
+                                                            max_seq_len))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, group_starts,
+                            prefix_lens, scale, max_seq_len, max_group_size, max_prefix_len,
+                            workspace=None, stream=None):
+    """pa_decode for groups of sequences sharing a prefix: ``group_starts`` int32
+    [G+1] (group g = sequences group_starts[g] .. group_starts[g+1]-1), ``prefix_lens``
+    int32 [G] (shared tokens, multiples of the block size); ``workspace`` at least
+    :func:`pa_decode_shared_prefix_workspace_size` bytes."""
+    N, bs, Hkv, D = k_cache.shape
+    B, Hq, _ = q.shape
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _i32tensor(block_tables, "block_tables"),
+        block_tables.shape[1], _i32tensor(seq_lens, "seq_lens"), B,
+        _i32tensor(group_starts, "group_starts"), _i32tensor(prefix_lens, "prefix_lens"),
+        prefix_lens.numel(), int(max_group_size), int(max_prefix_len), Hq, Hkv, D, float(scale),
+        bs, N, int(max_seq_len), _ptr(workspace), ws_bytes, _dtype_code(k_cache), _stream(stream)),
+        "pa_decode_shared_prefix")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

@@ -68,6 +68,16 @@ struct DecodeArgs {
   // FP8 (e4m3) cache: fp32 scale of each kv-head's K and V codes, [Hkv]
   const float* k_scale;
   const float* v_scale;
+  // shared-prefix decode (num_groups > 0): sequences [group_starts[g], group_starts[g+1])
+  // share their first prefix_lens[g] tokens.  The prefix pass left the attention of every
+  // member's q-heads over those tokens in pre_o / pre_ml ([pre_chunks][B * Hq rows],
+  // normalised rows and (max in log2 units, sum)); this launch reads only the keys after
+  // a sequence's prefix and the merge folds both parts together.
+  const int32_t* group_starts;
+  const int32_t* prefix_lens;
+  const float* pre_o;
+  const float* pre_ml;
+  int num_groups, pre_chunks;
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int seq_cap;
@@ -120,12 +130,27 @@ struct DecodeCfg {
   // registers, which leaves room for a third 64 KB ring slot)
   static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;
   static constexpr int OFF_A = OFF_P + (MMA ? 0 : HB * kTileTok * GW * 8);
-  static constexpr int OFF_SEQ = ((OFF_A + (MMA ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 2B+1 ints
+  static constexpr int OFF_SEQ = ((OFF_A + (MMA ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 3B+1 ints
   static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+// merge records: (first slot, slot count | kHasPrefix when prefix partials join the merge)
+constexpr int kHasPrefix = 1 << 30;
+
+// Shared-prefix length of sequence s: prefix_lens[g] of the group holding s (the last g
+// with group_starts[g] <= s, if s < group_starts[g+1]), else 0.
+__device__ __forceinline__ int shared_prefix_of(const DecodeArgs& a, int s) {
+  if (a.num_groups <= 0 || s < __ldg(a.group_starts)) return 0;
+  int lo = 0, hi = a.num_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a.group_starts + mid) <= s) lo = mid; else hi = mid - 1;
+  }
+  return s < __ldg(a.group_starts + lo + 1) ? __ldg(a.prefix_lens + lo) : 0;
+}
 
 // Bounded wait that turns into a no-op once any warp of the CTA gave up.
 __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
@@ -270,6 +295,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
   const int B = a.num_seqs;
   int* sstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);  // [B+1] first tile of each sequence
   int* slen = sstart + B + 1;                                // [B]   clamped lengths
+  int* sfirst = slen + B;  // [B] first tile after the shared prefix (0 without one)
   uint8_t* ring = smem + a.ring_off;
   const int nslots = a.nslots;
   const int NHP = a.num_kv_heads / HB;
@@ -289,7 +315,15 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       const int L = clamp_len(raw, a.seq_cap);
       if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
       slen[s] = L;
-      sum += NHP * cdiv(L, kTileTok);
+      int first = 0;
+      if (a.num_groups > 0) {
+        const int p = shared_prefix_of(a, s);
+        if ((p < 0 || p > L || (p & ((1 << a.log2_bs) - 1))) && blockIdx.x == 0)
+          flag_error(a.err, PA_DEVERR_PREFIX);
+        first = clamp_len(p, L) / kTileTok;
+      }
+      sfirst[s] = first;
+      sum += NHP * (cdiv(L, kTileTok) - first);
     }
     int incl = sum;
 #pragma unroll
@@ -300,7 +334,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     int run = incl - sum;
     for (int s = lo; s < hi; ++s) {
       sstart[s] = run;
-      run += NHP * cdiv(slen[s], kTileTok);
+      run += NHP * (cdiv(slen[s], kTileTok) - sfirst[s]);
     }
     if (lane == 31) sstart[B] = incl;
   }
@@ -333,8 +367,11 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     if (warp == C::WARP_FILL) {
       // ===== empty sequences: no CTA visits them; zero their output and merge record =====
       for (int s = cta; s < B; s += gridDim.x) {
-        if (slen[s] != 0) continue;
-        for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
+        if (cdiv(slen[s], kTileTok) != sfirst[s]) continue;
+        // no keys of its own: a sequence with a shared prefix takes the prefix part alone
+        const int pre = sfirst[s] > 0 ? kHasPrefix : 0;
+        for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, pre);
+        if (pre) continue;
         T* ob = static_cast<T*>(a.out) + (long long)s * a.num_q_heads * kD;
         for (int i = lane; i < a.num_q_heads * kD / 8; i += 32)
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -368,18 +405,20 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           }
           break;
         }
-        const int nt = cdiv(slen[s], kTileTok);  // > 0: pos lies in this sequence
+        const int nt = cdiv(slen[s], kTileTok);
+        const int ts = sfirst[s];         // tiles [ts, nt) are read here
+        const int cnt = nt - ts;          // > 0: pos lies in this sequence
         const int off = pos - sstart[s];
-        const int hp = off / nt;
-        const int t0 = off - hp * nt;
+        const int hp = off / cnt;
+        const int t0 = ts + off - hp * cnt;
         const int t1 = min(nt, t0 + min(r1 - pos, kMaxTilesPerUnit));
         const int grp = s * NHP + hp;
-        const int gs = sstart[s] + hp * nt;  // the group's first and one-past-last tile
-        const int ge = gs + nt;
+        const int gs = sstart[s] + hp * cnt;  // the group's first and one-past-last tile
+        const int ge = gs + cnt;
         int flags = 0;
-        if (t0 == 0 || pos == r0) flags |= kFirst;
+        if (t0 == ts || pos == r0) flags |= kFirst;
         if (t1 == nt || pos + (t1 - t0) == r1) flags |= kLast;
-        if (gs >= r0 && ge <= r1) flags |= kDirect;
+        if (gs >= r0 && ge <= r1 && ts == 0) flags |= kDirect;
         const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
         int ids[kMaxTilesPerUnit / 32];
   #pragma unroll
@@ -430,7 +469,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           }
         }
         if (lane == 0) {
-          if (t0 == 0) a.meta[grp] = make_int2(cta + grp, cta_of(ge - 1, Ttot, grid) - cta + 1);
+          if (t0 == ts)
+            a.meta[grp] = make_int2(cta + grp, (cta_of(ge - 1, Ttot, grid) - cta + 1) |
+                                                   (ts > 0 ? kHasPrefix : 0));
           u[0] = s;
           u[1] = hp;
           u[2] = t0;
@@ -890,23 +931,32 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
   const int nhp = a.num_q_heads / hbg;
   const int j = qh % hbg;
   const int2 mt = a.meta[s * nhp + qh / hbg];
-  const int n = mt.y;
-  if (n <= 1) return;  // written by the decode kernel
+  const int n = mt.y & (kHasPrefix - 1);                 // segments of this launch
+  const int npre = (mt.y & kHasPrefix) ? a.pre_chunks : 0;  // shared-prefix partials
+  if (n <= 1 && npre == 0) return;  // written by the decode kernel
+  const int total = n + npre;
   const long long row0 = (long long)mt.x * hbg + j;
+  const long long prow_stride = (long long)a.num_seqs * a.num_q_heads;
   // one pass with a running maximum: up to eight segments per round, all loads of a
   // round in flight together (most groups span fewer than eight CTAs: one round)
   float M = -INFINITY, den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < n; i0 += 8) {
+  for (int i0 = 0; i0 < total; i0 += 8) {
     float2 mlv[8];
     float4 ov[8];
     float Mr = -INFINITY;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      if (i0 + u < n) {
-        const long long row = row0 + (long long)(i0 + u) * hbg;
+      const int i = i0 + u;
+      if (i < n) {
+        const long long row = row0 + (long long)i * hbg;
         mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
         ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
+        Mr = fmaxf(Mr, mlv[u].x);
+      } else if (i < total) {
+        const long long row = (long long)(i - n) * prow_stride + gw;
+        mlv[u] = *reinterpret_cast<const float2*>(a.pre_ml + row * 2);
+        ov[u] = *reinterpret_cast<const float4*>(a.pre_o + row * kD + lane * 4);
         Mr = fmaxf(Mr, mlv[u].x);
       }
     }
@@ -917,7 +967,7 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
     num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      if (i0 + u < n) {
+      if (i0 + u < total) {
         const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
         den += f;
         num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
@@ -961,7 +1011,7 @@ template <typename T, int G, int HB, bool F8>
 pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                         DecodeArgs a, int grid, cudaStream_t stream) {
   using C = DecodeCfg<G, HB, F8>;
-  const size_t ring_off = ((C::OFF_SEQ + (size_t)(2 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
+  const size_t ring_off = ((C::OFF_SEQ + (size_t)(3 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
   const long long room = (long long)kMaxSmem - (long long)ring_off;
   const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
   if (nslots < 2) return PA_ERR_UNSUPPORTED;
@@ -973,7 +1023,7 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
-  if (grid > 1) {
+  if (grid > 1 || a.num_groups > 0) {
     const int warps = a.num_seqs * a.num_q_heads;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1041,14 +1091,23 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int he
 }
 
 namespace {
-// pa_decode, and pa_decode_append when k_new / v_new are given
+// Groups of sequences sharing a prefix (pa_decode_shared_prefix).
+struct SharedPrefixArgs {
+  const int32_t* group_starts;
+  const int32_t* prefix_lens;
+  int num_groups, max_group_size, max_prefix_len;
+};
+
+// pa_decode, pa_decode_append when k_new / v_new are given, pa_decode_fp8 with scales,
+// pa_decode_shared_prefix with `sp`
 pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v_new,
                       const void* k_cache, const void* v_cache, const float* k_scale,
                       const float* v_scale, const int32_t* block_tables,
                       int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
                       int num_q_heads, int num_kv_heads, int head_dim, float scale,
                       int block_size, int num_blocks, int max_seq_len, int partition_size,
-                      void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream) {
+                      void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream,
+                      const SharedPrefixArgs* sp = nullptr) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0 ||
@@ -1086,7 +1145,16 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     grid = std::max<long long>(grid, (tiles_max + partition_size / 16 - 1) / (partition_size / 16));
   const long long groups = (long long)num_seqs * NHP;
   const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
-  if (!workspace || workspace_bytes < lay.total) return PA_ERR_WORKSPACE_TOO_SMALL;
+  // shared prefix: the prefix pass's partial rows follow the decode workspace
+  int chunks = 0;
+  size_t pre_off = 0, need = lay.total;
+  if (sp) {
+    chunks = pa::shared_prefix_chunks(sp->num_groups, num_kv_heads, G, sp->max_group_size,
+                                      sp->max_prefix_len);
+    pre_off = pa::align256(lay.total);
+    need = pre_off + (size_t)chunks * num_seqs * num_q_heads * (head_dim + 2) * sizeof(float);
+  }
+  if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
   int* err = pa::device_error_flag();
   if (!err) return PA_ERR_CUDA;
@@ -1133,7 +1201,34 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.ring_off = 0;
   a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
+  a.group_starts = a.prefix_lens = nullptr;
+  a.pre_o = a.pre_ml = nullptr;
+  a.num_groups = a.pre_chunks = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sp) {
+    // pass 1: every group's prefix, once for all its members (tensor cores); pass 2 (the
+    // decode kernel below) reads each sequence's own keys; the merge combines them
+    float* pre_o = reinterpret_cast<float*>(ws + pre_off);
+    float* pre_ml = pre_o + (size_t)chunks * num_seqs * num_q_heads * head_dim;
+    const pa_status ps = pa::shared_prefix_pass(
+        q, k_cache, v_cache, block_tables, max_blocks_per_seq, sp->group_starts,
+        sp->prefix_lens, sp->num_groups, sp->max_group_size, sp->max_prefix_len, num_seqs,
+        num_q_heads, num_kv_heads, scale, block_size, num_blocks, chunks, pre_o, pre_ml, dtype,
+        err, st);
+    if (ps != PA_OK) return ps;
+    a.group_starts = sp->group_starts;
+    a.prefix_lens = sp->prefix_lens;
+    a.num_groups = sp->num_groups;
+    a.pre_o = pre_o;
+    a.pre_ml = pre_ml;
+    a.pre_chunks = chunks;
+    const pa_status ds =
+        dtype == PA_F16
+            ? pa::dispatch_group<__half, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
+            : pa::dispatch_group<__nv_bfloat16, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
+    if (ds == PA_OK) pa::set_launch_count(pa::launch_count() + 1);
+    return ds;
+  }
   if (f8)
     return dtype == PA_F16
                ? pa::dispatch_group<__half, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
@@ -1240,3 +1335,36 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
 }
 
 extern "C" size_t pa_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads,
+                                                         int head_dim, int max_seq_len) {
+  const size_t base = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
+  if (base == 0) return 0;
+  return pa::align256(base) + (size_t)pa::kMaxPrefixChunks * num_seqs * num_q_heads *
+                                  (head_dim + 2) * sizeof(float);
+}
+
+extern "C" pa_status pa_decode_shared_prefix(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+    const int32_t* group_starts, const int32_t* prefix_lens, int num_groups, int max_group_size,
+    int max_prefix_len, int num_q_heads, int num_kv_heads, int head_dim, float scale,
+    int block_size, int num_blocks, int max_seq_len, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, void* stream) {
+  pa::set_launch_count(0);
+  if (num_groups < 0 || max_group_size < 0 || max_prefix_len < 0 || num_seqs < 0 ||
+      num_groups > num_seqs || max_group_size > num_seqs)
+    return PA_ERR_INVALID_ARG;
+  if (num_groups == 0 || max_group_size == 0 || max_prefix_len == 0)  // nothing shared
+    return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
+                       block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len, 0,
+                       workspace, workspace_bytes, dtype, stream);
+  if (!group_starts || !prefix_lens) return PA_ERR_INVALID_ARG;
+  const SharedPrefixArgs sp = {group_starts, prefix_lens, num_groups, max_group_size,
+                               max_prefix_len};
+  return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr, block_tables,
+                     max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                     scale, block_size, num_blocks, max_seq_len, 0, workspace, workspace_bytes,
+                     dtype, stream, &sp);
+}

@@ -120,6 +120,7 @@ bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int 
 }
 
 void set_launch_count(int n) { g_last_launches = n; }
+int launch_count() { return g_last_launches; }
 
 }  // namespace pa
 

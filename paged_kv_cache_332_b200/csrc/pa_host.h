@@ -39,6 +39,22 @@ bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint6
 
 // Launch accounting for pa_last_launch_count().
 void set_launch_count(int n);
+int launch_count();
+
+// Shared-prefix decode, first pass (prefill.cu): the attention of every member's q-heads
+// over its group's shared prefix, on the tcgen05 prefill kernel (the members' queries of
+// one kv-head form the rows of one M-tile), as `chunks` pieces of normalised partial rows
+// in pre_o [chunks][q_rows * num_q_heads][128] and (max, sum) in pre_ml.
+constexpr int kMaxPrefixChunks = 8;
+int shared_prefix_chunks(int num_groups, int num_kv_heads, int G, int max_group_size,
+                         int max_prefix_len);
+pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* group_starts, const int32_t* prefix_lens,
+                             int num_groups, int max_group_size, int max_prefix_len, int q_rows,
+                             int num_q_heads, int num_kv_heads, float scale, int block_size,
+                             int num_blocks, int chunks, float* pre_o, float* pre_ml,
+                             pa_dtype dtype, int* err, cudaStream_t stream);
 
 inline pa_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -67,6 +67,15 @@ struct Args {
   float* part_o;
   float* part_ml;
   int* rowmap;
+  // shared-prefix pass of the decode (prefix_chunks > 0): item "sequence" s is group s,
+  // whose queries are the decode rows qsl[s] .. qsl[s+1]-1 (one per member, q_rows rows
+  // in all) and whose keys are the first seq_lens[s] tokens, read through the table row
+  // of member qsl[s] and visible to every row (no causal mask).  The keys are cut into
+  // prefix_chunks pieces of whole tiles; each piece writes normalised partial rows and
+  // (max in log2 units, sum) to pre_o / pre_ml [piece][q_rows * num_q_heads].
+  int prefix_chunks, q_rows;
+  float* pre_o;
+  float* pre_ml;
 };
 
 // shared memory carve-up
@@ -239,7 +248,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- which (sequence, kv-head, query block), and which part of its keys
   int item = blockIdx.x, part = -1;  // part -1: all keys; 0 / 1: first / second half
-  if (a.split_items > 0 && (int)blockIdx.x >= a.whole_items) {
+  const bool pmode = a.prefix_chunks > 0;
+  int piece = 0;
+  if (pmode) {
+    piece = item % a.prefix_chunks;
+    item /= a.prefix_chunks;
+  } else if (a.split_items > 0 && (int)blockIdx.x >= a.whole_items) {
     const int j = blockIdx.x - a.whole_items;
     item = a.whole_items + (j >> 1);
     part = j & 1;
@@ -257,7 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int Lraw = a.seq_lens[s];
   const int L = Lraw < 0 ? 0 : (Lraw > a.seq_cap ? a.seq_cap : Lraw);
   const int q0 = qb * 2 * MQ;
-  if (n < 0 || n > L || n > a.max_query_len || Lraw != L) {
+  if (pmode) {
+    // a group: members qsl[s] .. qsl[s+1]-1, prefix a multiple of the block size
+    const bool layout_bad = n < 0 || n > a.max_query_len || q_begin < 0 || q_begin + n > a.q_rows;
+    const bool prefix_bad = Lraw != L || (L & ((1 << a.log2_bs) - 1));
+    if ((layout_bad || prefix_bad) && threadIdx.x == 0 && qb == 0 && h == 0 && piece == 0)
+      flag_error(a.err, layout_bad ? PA_DEVERR_QUERY_LAYOUT : PA_DEVERR_PREFIX);
+    if (layout_bad) return;
+  } else if (n < 0 || n > L || n > a.max_query_len || Lraw != L) {
     if (threadIdx.x == 0 && qb == 0 && h == 0)
       flag_error(a.err, (n < 0 || n > L || n > a.max_query_len) ? PA_DEVERR_QUERY_LAYOUT
                                                                : PA_DEVERR_SEQ_TOO_LONG);
@@ -271,10 +292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   // keys any row of this CTA can see: [0, kv_end); this CTA takes tiles [kt_lo, kt_hi)
-  const int kv_end = min(L, L - n + min(n, q0 + 2 * MQ));
+  const int kv_end = pmode ? L : min(L, L - n + min(n, q0 + 2 * MQ));
   const int n_kt_all = (kv_end + kBN - 1) / kBN;
-  const int kt_lo = part == 1 ? n_kt_all / 2 : 0;
-  const int kt_hi = part == 0 ? n_kt_all / 2 : n_kt_all;
+  const int kt_lo = pmode ? (int)((long long)piece * n_kt_all / a.prefix_chunks)
+                          : (part == 1 ? n_kt_all / 2 : 0);
+  const int kt_hi = pmode ? (int)((long long)(piece + 1) * n_kt_all / a.prefix_chunks)
+                          : (part == 0 ? n_kt_all / 2 : n_kt_all);
   const int n_kt = kt_hi - kt_lo;  // tiles here; loops below count them from 0
 
   if (threadIdx.x == 0) {
@@ -311,7 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = wq * 32 + lane;         // row of the M-tile
     const int qi = q0 + mt * MQ + r / G;  // query index within the chunk
     const bool row_valid = qi < n;
-    const int limit = L - n + min(qi, n - 1);  // last visible key (inclusive)
+    // last visible key (inclusive): causal, or the whole prefix for the shared-prefix pass
+    const int limit = pmode ? L - 1 : L - n + min(qi, n - 1);
     const uint32_t t_s = tmem + ((uint32_t)(wq * 32) << 16) + mt * 128;
     const uint32_t t_o = tmem + ((uint32_t)(wq * 32) << 16) + 256 + mt * 128;
     // lowest limit in the warp decides whether a tile needs the causal mask
@@ -415,7 +439,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_or_abort(&o_full[mt], 0, abort_flag, a.err);
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (part < 0) {
+    if (pmode) {
+      // one piece of a group's prefix: normalised partial row and (reference max, sum)
+      const bool any = n_kt > 0 && l > 0.f;
+      const long long prow = (long long)piece * a.q_rows * a.num_q_heads +
+                             (long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(t_o + c * 32, v);
+        if (row_valid) {
+          float* po = a.pre_o + prow * kD + c * 32;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(po + j * 4) =
+                any ? make_float4(v[4 * j] * inv, v[4 * j + 1] * inv, v[4 * j + 2] * inv,
+                                  v[4 * j + 3] * inv)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      if (row_valid)
+        *reinterpret_cast<float2*>(a.pre_ml + prow * 2) =
+            any ? make_float2(m_ref, l) : make_float2(-INFINITY, 0.f);
+    } else if (part < 0) {
       T* orow = static_cast<T*>(a.out) +
                 ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD;
 #pragma unroll
@@ -465,7 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
+        // the shared-prefix pass reads a group's prefix through its first member's row
+        const int32_t* trow = a.block_tables + (long long)(pmode ? q_begin : s) * a.max_blocks;
         const int bs_mask = (1 << a.log2_bs) - 1;
         // block-table entries of a tile's eight 16-token runs, read one tile ahead so
         // that their latency overlaps the previous tile's waits and copies
@@ -673,7 +720,85 @@ pa_status dispatch(int G, const CUtensorMap& tk, const CUtensorMap& tv, const Ar
   }
 }
 
+template <typename T, int G>
+pa_status launch_prefix(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
+                        long long grid, cudaStream_t stream) {
+  auto kern = chunked_prefill_kernel<T, G>;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES)) return PA_ERR_CUDA;
+  kern<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(tk, tv, a);
+  return check_launch();
+}
+
 }  // namespace prefill
+
+int shared_prefix_chunks(int num_groups, int num_kv_heads, int G, int max_group_size,
+                         int max_prefix_len) {
+  const long long qblocks = (max_group_size + 2 * (prefill::kM / G) - 1) / (2 * (prefill::kM / G));
+  const long long items = std::max<long long>(1, (long long)num_groups * num_kv_heads * qblocks);
+  const long long tiles = (std::max(0, max_prefix_len) + prefill::kBN - 1) / prefill::kBN;
+  const long long fill = std::max<long long>(1, num_sms() / items);  // pieces that fill one wave
+  return (int)std::max<long long>(1, std::min<long long>({(long long)kMaxPrefixChunks, fill, tiles}));
+}
+
+pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* group_starts, const int32_t* prefix_lens,
+                             int num_groups, int max_group_size, int max_prefix_len, int q_rows,
+                             int num_q_heads, int num_kv_heads, float scale, int block_size,
+                             int num_blocks, int chunks, float* pre_o, float* pre_ml,
+                             pa_dtype dtype, int* err, cudaStream_t stream) {
+  const int G = num_q_heads / num_kv_heads;
+  const int MQ = prefill::kM / G;
+  CUtensorMap tk, tv;
+  const uint64_t row = (uint64_t)prefill::kD * 2;
+  const uint64_t cdims[4] = {(uint64_t)prefill::kD, (uint64_t)num_kv_heads, (uint64_t)block_size,
+                             (uint64_t)num_blocks};
+  const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+  const uint32_t cbox[4] = {64, 1, 16, 1};
+  if (!encode_tmap_16bit(&tk, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap_16bit(&tv, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B))
+    return PA_ERR_CUDA;
+  prefill::Args a = {};
+  a.out = nullptr;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.seq_lens = prefix_lens;
+  a.qsl = group_starts;
+  a.err = err;
+  a.num_seqs = num_groups;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.log2_bs = block_size == 16 ? 4 : 5;
+  a.num_blocks = num_blocks;
+  a.max_query_len = max_group_size;
+  a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_prefix_len);
+  a.qblocks = (max_group_size + 2 * MQ - 1) / (2 * MQ);
+  a.qscale = scale * 1.4426950408889634f;
+  a.whole_items = 0;
+  a.split_items = 0;
+  a.part_o = a.part_ml = nullptr;
+  a.rowmap = nullptr;
+  a.prefix_chunks = chunks;
+  a.q_rows = q_rows;
+  a.pre_o = pre_o;
+  a.pre_ml = pre_ml;
+  const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * chunks;
+  if (grid <= 0) return PA_OK;
+  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  auto go = [&](auto tag) -> pa_status {
+    using T = decltype(tag);
+    switch (G) {
+      case 1: return prefill::launch_prefix<T, 1>(tk, tv, a, grid, stream);
+      case 2: return prefill::launch_prefix<T, 2>(tk, tv, a, grid, stream);
+      case 4: return prefill::launch_prefix<T, 4>(tk, tv, a, grid, stream);
+      case 8: return prefill::launch_prefix<T, 8>(tk, tv, a, grid, stream);
+      default: return PA_ERR_UNSUPPORTED;
+    }
+  };
+  return dtype == PA_F16 ? go(__half{}) : go(__nv_bfloat16{});
+}
+
 }  // namespace pa
 
 extern "C" size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_len,
@@ -740,6 +865,9 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_seq_len);
   a.qblocks = (max_query_len + 2 * MQ - 1) / (2 * MQ);
   a.qscale = scale * 1.4426950408889634f;
+  a.prefix_chunks = 0;
+  a.q_rows = 0;
+  a.pre_o = a.pre_ml = nullptr;
   // the split's row map stores output row numbers as int
   const long long rows = (long long)num_seqs * max_query_len * num_q_heads;
   if (rows > 0x7fffffffLL) workspace = nullptr;

@@ -157,6 +157,25 @@ def test_fp8_arguments_rejected_on_host(palib):
     assert palib.pa_last_launch_count() == 0
 
 
+def test_shared_prefix_arguments_rejected_on_host(palib):
+    L = _raw(palib)
+    p = ctypes.c_void_p(4096)
+    nul = None
+
+    def dec(B=8, gs=p, pl=p, ng=2, mg=4, mp=256, ws=None, wsb=0):
+        return L.pa_decode_shared_prefix(p, p, p, p, p, 32, p, B, gs, pl, ng, mg, mp, 32, 8, 128,
+                                         0.1, 16, 1000, 512, ws, wsb, 0, nul)
+    assert dec(ng=-1) == 1 and dec(mg=-1) == 1 and dec(mp=-1) == 1
+    assert dec(ng=9) == 1 and dec(mg=9) == 1       # more groups / members than sequences
+    assert dec(gs=nul) == 1 and dec(pl=nul) == 1
+    assert dec(B=0, ng=0, mg=0) == 0               # nothing to do
+    assert dec() == 3 and dec(mp=0) == 3            # needs a workspace (shared or plain)
+    base = palib.pa_decode_workspace_size(8, 32, 128, 512, 0)
+    assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 128, 512) >= base + 8 * 8 * 32 * 130 * 4
+    assert palib.pa_decode_shared_prefix_workspace_size(0, 32, 128, 512) == 0
+    assert palib.pa_last_launch_count() == 0
+
+
 def test_block_pool_arguments_rejected_on_host(palib):
     L = _raw(palib)
     p = ctypes.c_void_p(4096)

@@ -112,6 +112,11 @@ class PagedBatch:
     # scales; None for fp16/bf16 caches
     k_scale: Optional[torch.Tensor] = None
     v_scale: Optional[torch.Tensor] = None
+    # groups of consecutive sequences sharing their first blocks: int32 [groups + 1]
+    # (group g = sequences group_starts[g] .. group_starts[g+1]-1) and the shared token
+    # count of each group, int32 [groups]; None without sharing
+    group_starts: Optional[torch.Tensor] = None
+    prefix_lens: Optional[torch.Tensor] = None
 
     @property
     def num_seqs(self) -> int:
@@ -219,6 +224,25 @@ def make_batch(name: str, *, seq_lens: List[int], q_lens: Optional[List[int]] = 
     qsl[1:] = np.cumsum(q_lens)
     is_prefill = any(ql > 1 for ql in q_lens) if prefill is None else prefill
 
+    gs_t = pl_t = None
+    if shared_groups and all(g == list(range(g[0], g[0] + len(g))) for g in shared_groups):
+        starts = sorted(g[0] for g in shared_groups)
+        ends = {g[0]: g[0] + len(g) for g in shared_groups}
+        if all(ends[a] <= b for a, b in zip(starts, starts[1:])):
+            bounds = [x for a in starts for x in (a, ends[a])]
+            # gaps between groups become groups with nothing shared
+            gstarts, plens = [], []
+            prev_end = None
+            for i in range(0, len(bounds), 2):
+                if gstarts and bounds[i] != prev_end:
+                    gstarts.append(prev_end)
+                    plens.append(0)
+                gstarts.append(bounds[i])
+                plens.append(shared_prefix_tokens)
+                prev_end = bounds[i + 1]
+            gstarts.append(prev_end)
+            gs_t = torch.tensor(np.asarray(gstarts, dtype=np.int32), device=device)
+            pl_t = torch.tensor(np.asarray(plens, dtype=np.int32), device=device)
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     cshape = (num_blocks, block_size, num_kv_heads, head_dim)
@@ -239,6 +263,7 @@ def make_batch(name: str, *, seq_lens: List[int], q_lens: Optional[List[int]] = 
         query_start_loc=torch.from_numpy(qsl).to(device) if is_prefill else None,
         shared_prefix_blocks=(shared_prefix_tokens // block_size) if shared_groups else 0,
         group_size=len(shared_groups[0]) if shared_groups else 1,
+        group_starts=gs_t, prefix_lens=pl_t,
     )
 
 
