@@ -1146,13 +1146,13 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   const long long groups = (long long)num_seqs * NHP;
   const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
   // shared prefix: the prefix pass's partial rows follow the decode workspace
-  int chunks = 0;
+  pa::SharedPrefixPlan plan = {};
   size_t pre_off = 0, need = lay.total;
   if (sp) {
-    chunks = pa::shared_prefix_chunks(sp->num_groups, num_kv_heads, G, sp->max_group_size,
-                                      sp->max_prefix_len);
+    plan = pa::plan_shared_prefix(sp->num_groups, num_kv_heads, G, sp->max_group_size,
+                                  sp->max_prefix_len);
     pre_off = pa::align256(lay.total);
-    need = pre_off + (size_t)chunks * num_seqs * num_q_heads * (head_dim + 2) * sizeof(float);
+    need = pre_off + (size_t)plan.slots * num_seqs * num_q_heads * (head_dim + 2) * sizeof(float);
   }
   if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
@@ -1209,11 +1209,11 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     // pass 1: every group's prefix, once for all its members (tensor cores); pass 2 (the
     // decode kernel below) reads each sequence's own keys; the merge combines them
     float* pre_o = reinterpret_cast<float*>(ws + pre_off);
-    float* pre_ml = pre_o + (size_t)chunks * num_seqs * num_q_heads * head_dim;
+    float* pre_ml = pre_o + (size_t)plan.slots * num_seqs * num_q_heads * head_dim;
     const pa_status ps = pa::shared_prefix_pass(
         q, k_cache, v_cache, block_tables, max_blocks_per_seq, sp->group_starts,
         sp->prefix_lens, sp->num_groups, sp->max_group_size, sp->max_prefix_len, num_seqs,
-        num_q_heads, num_kv_heads, scale, block_size, num_blocks, chunks, pre_o, pre_ml, dtype,
+        num_q_heads, num_kv_heads, scale, block_size, num_blocks, plan, pre_o, pre_ml, dtype,
         err, st);
     if (ps != PA_OK) return ps;
     a.group_starts = sp->group_starts;
@@ -1221,7 +1221,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     a.num_groups = sp->num_groups;
     a.pre_o = pre_o;
     a.pre_ml = pre_ml;
-    a.pre_chunks = chunks;
+    a.pre_chunks = plan.slots;
     const pa_status ds =
         dtype == PA_F16
             ? pa::dispatch_group<__half, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)

@@ -44,17 +44,23 @@ int launch_count();
 // Shared-prefix decode, first pass (prefill.cu): the attention of every member's q-heads
 // over its group's shared prefix, on the tcgen05 prefill kernel (the members' queries of
 // one kv-head form the rows of one M-tile), as `chunks` pieces of normalised partial rows
-// in pre_o [chunks][q_rows * num_q_heads][128] and (max, sum) in pre_ml.
-constexpr int kMaxPrefixChunks = 8;
-int shared_prefix_chunks(int num_groups, int num_kv_heads, int G, int max_group_size,
-                         int max_prefix_len);
+// in pre_o [slots][q_rows * num_q_heads][128] and (max, sum) in pre_ml.
+constexpr int kMaxPrefixChunks = 8;  // partial slots at most
+struct SharedPrefixPlan {
+  int ksplit;   // groups fit one M-tile: the two M-tiles take alternate key tiles
+  int qblocks;  // query blocks per (group, kv-head)
+  int pieces;   // key pieces per (group, kv-head, query block)
+  int slots;    // partial rows per output row: pieces (x 2 with ksplit)
+};
+SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
+                                    int max_prefix_len);
 pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* block_tables, int max_blocks_per_seq,
                              const int32_t* group_starts, const int32_t* prefix_lens,
                              int num_groups, int max_group_size, int max_prefix_len, int q_rows,
                              int num_q_heads, int num_kv_heads, float scale, int block_size,
-                             int num_blocks, int chunks, float* pre_o, float* pre_ml,
-                             pa_dtype dtype, int* err, cudaStream_t stream);
+                             int num_blocks, const SharedPrefixPlan& plan, float* pre_o,
+                             float* pre_ml, pa_dtype dtype, int* err, cudaStream_t stream);
 
 inline pa_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -73,7 +73,10 @@ struct Args {
   // of member qsl[s] and visible to every row (no causal mask).  The keys are cut into
   // prefix_chunks pieces of whole tiles; each piece writes normalised partial rows and
   // (max in log2 units, sum) to pre_o / pre_ml [piece][q_rows * num_q_heads].
-  int prefix_chunks, q_rows;
+  // With ksplit (shared-prefix pass, every group within one M-tile of rows) the two
+  // M-tiles hold the same rows and take alternate key tiles, two independent softmax
+  // chains per CTA; each writes its own partial (piece 2 * piece + M-tile).
+  int prefix_chunks, q_rows, ksplit;
   float* pre_o;
   float* pre_ml;
 };
@@ -270,7 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = a.qsl[s + 1] - q_begin;
   const int Lraw = a.seq_lens[s];
   const int L = Lraw < 0 ? 0 : (Lraw > a.seq_cap ? a.seq_cap : Lraw);
-  const int q0 = qb * 2 * MQ;
+  const bool ksplit = pmode && a.ksplit;
+  const int q0 = qb * (ksplit ? MQ : 2 * MQ);
   if (pmode) {
     // a group: members qsl[s] .. qsl[s+1]-1, prefix a multiple of the block size
     const bool layout_bad = n < 0 || n > a.max_query_len || q_begin < 0 || q_begin + n > a.q_rows;
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int mt = (warp - 4) >> 2;
     const int wq = warp & 3;              // TMEM lane quarter
     const int r = wq * 32 + lane;         // row of the M-tile
-    const int qi = q0 + mt * MQ + r / G;  // query index within the chunk
+    const int qi = q0 + (ksplit ? 0 : mt * MQ) + r / G;  // query index within the chunk
     const bool row_valid = qi < n;
     // last visible key (inclusive): causal, or the whole prefix for the shared-prefix pass
     const int limit = pmode ? L - 1 : L - n + min(qi, n - 1);
@@ -359,8 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(q_full);
     }
     float m_ref = -INFINITY, l = 0.f;
-    for (int kt = 0; kt < n_kt; ++kt) {
-      wait_or_abort(&s_full[mt], kt & 1, abort_flag, a.err);
+    // tiles kt of this M-tile (all of them; with ksplit, those with kt % 2 == mt), and
+    // j counts them
+    for (int kt = ksplit ? mt : 0, j = 0; kt < n_kt; kt += ksplit ? 2 : 1, ++j) {
+      wait_or_abort(&s_full[mt], j & 1, abort_flag, a.err);
       tc_fence_after();
       const int key0 = (kt_lo + kt) * kBN;
       // the whole S row (128 keys) in registers: one pass over TMEM
@@ -389,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = fast_exp2(m_ref - mx);  // m_ref = -inf -> 0
         m_ref = mx;
       }
-      if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -419,11 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * alpha + sum;
       // keys past the sequence end in the last tile: clear their V rows
-      if (mt == 0 && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
+      if ((ksplit || mt == 0) && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
         wait_or_abort(&v_full[kt & 1], (kt >> 1) & 1, abort_flag, a.err);
         uint8_t* vt = smem + OFF_V + (kt & 1) * kTileBytes;
         const int first = L - key0;  // first row to clear
-        for (int i = threadIdx.x - 128; i < (kBN - first) * 16; i += 128) {
+        for (int i = threadIdx.x & 127; i < (kBN - first) * 16; i += 128) {
           const int rr = first + i / 16, chunk = i % 16;  // 16 x 16 B per row (two halves)
           *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + rr * 128 + (chunk & 7) * 16) =
               make_uint4(0, 0, 0, 0);
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (pmode) {
       // one piece of a group's prefix: normalised partial row and (reference max, sum)
       const bool any = n_kt > 0 && l > 0.f;
-      const long long prow = (long long)piece * a.q_rows * a.num_q_heads +
+      const long long prow = (long long)(ksplit ? 2 * piece + mt : piece) * a.q_rows * a.num_q_heads +
                              (long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -580,39 +586,68 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&s_full[mt]);
         };
-        auto issue_pv = [&](int mt, int kt) {
+        auto issue_pv = [&](int mt, int kt, bool acc) {
           const int st = kt & 1;
   #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint64_t db = sw128_desc(sV + st * kTileBytes + kk * 2048, kHalfBytes, 1024);
-            mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (kt > 0 || kk > 0));
+            mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (acc || kk > 0));
           }
         };
         wait_or_abort(q_full, 0, abort_flag, a.err);
         tc_fence_after();
-        if (n_kt > 0) {
-          wait_or_abort(&k_full[0], 0, abort_flag, a.err);
-          tc_fence_after();
-          issue_s(0, 0);
-          issue_s(1, 0);
-          mma_commit(&k_empty[0]);
-        }
-        for (int kt = 0; kt < n_kt; ++kt) {
-          const int st = kt & 1;
-          const bool more = kt + 1 < n_kt;
-          wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
-          if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
-          for (int mt = 0; mt < 2; ++mt) {
-            wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
+        if (ksplit) {
+          // two chains: M-tile mt takes tiles mt, mt + 2, ... (stage mt of each ring)
+          for (int mt = 0; mt < 2 && mt < n_kt; ++mt) {
+            wait_or_abort(&k_full[mt], 0, abort_flag, a.err);
             tc_fence_after();
-            issue_pv(mt, kt);
-            if (more) issue_s(mt, kt + 1);
+            issue_s(mt, mt);
+            mma_commit(&k_empty[mt]);
           }
-          if (more) mma_commit(&k_empty[(kt + 1) & 1]);
-          mma_commit(&v_empty[st]);
+          for (int j = 0; 2 * j < n_kt; ++j) {
+            for (int mt = 0; mt < 2; ++mt) {
+              const int kt = 2 * j + mt;
+              if (kt >= n_kt) break;
+              wait_or_abort(&p_full[mt], j & 1, abort_flag, a.err);
+              wait_or_abort(&v_full[mt], j & 1, abort_flag, a.err);
+              tc_fence_after();
+              issue_pv(mt, kt, j > 0);
+              mma_commit(&v_empty[mt]);
+              if (kt + 2 < n_kt) {
+                wait_or_abort(&k_full[mt], (j + 1) & 1, abort_flag, a.err);
+                tc_fence_after();
+                issue_s(mt, kt + 2);
+                mma_commit(&k_empty[mt]);
+              }
+            }
+          }
+          mma_commit(&o_full[0]);
+          mma_commit(&o_full[1]);
+        } else {
+          if (n_kt > 0) {
+            wait_or_abort(&k_full[0], 0, abort_flag, a.err);
+            tc_fence_after();
+            issue_s(0, 0);
+            issue_s(1, 0);
+            mma_commit(&k_empty[0]);
+          }
+          for (int kt = 0; kt < n_kt; ++kt) {
+            const int st = kt & 1;
+            const bool more = kt + 1 < n_kt;
+            wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
+            if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
+            for (int mt = 0; mt < 2; ++mt) {
+              wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
+              tc_fence_after();
+              issue_pv(mt, kt, kt > 0);
+              if (more) issue_s(mt, kt + 1);
+            }
+            if (more) mma_commit(&k_empty[(kt + 1) & 1]);
+            mma_commit(&v_empty[st]);
+          }
+          mma_commit(&o_full[0]);
+          mma_commit(&o_full[1]);
         }
-        mma_commit(&o_full[0]);
-        mma_commit(&o_full[1]);
       }
     }
   }
@@ -731,13 +766,22 @@ pa_status launch_prefix(const CUtensorMap& tk, const CUtensorMap& tv, const Args
 
 }  // namespace prefill
 
-int shared_prefix_chunks(int num_groups, int num_kv_heads, int G, int max_group_size,
-                         int max_prefix_len) {
-  const long long qblocks = (max_group_size + 2 * (prefill::kM / G) - 1) / (2 * (prefill::kM / G));
-  const long long items = std::max<long long>(1, (long long)num_groups * num_kv_heads * qblocks);
+SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
+                                    int max_prefix_len) {
+  SharedPrefixPlan p;
+  const int MQ = prefill::kM / G;
+  // groups that fit one M-tile of rows: both M-tiles take the same rows, alternate tiles
+  p.ksplit = max_group_size <= MQ ? 1 : 0;
+  p.qblocks = p.ksplit ? 1 : (max_group_size + 2 * MQ - 1) / (2 * MQ);
+  const long long items = std::max<long long>(1, (long long)num_groups * num_kv_heads * p.qblocks);
   const long long tiles = (std::max(0, max_prefix_len) + prefill::kBN - 1) / prefill::kBN;
   const long long fill = std::max<long long>(1, num_sms() / items);  // pieces that fill one wave
-  return (int)std::max<long long>(1, std::min<long long>({(long long)kMaxPrefixChunks, fill, tiles}));
+  const long long per_piece = p.ksplit ? 2 : 1;                        // partials per piece
+  p.pieces = (int)std::max<long long>(
+      1, std::min<long long>({kMaxPrefixChunks / per_piece, fill,
+                              std::max<long long>(1, tiles / per_piece)}));
+  p.slots = p.pieces * (int)per_piece;
+  return p;
 }
 
 pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
@@ -745,10 +789,9 @@ pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_c
                              const int32_t* group_starts, const int32_t* prefix_lens,
                              int num_groups, int max_group_size, int max_prefix_len, int q_rows,
                              int num_q_heads, int num_kv_heads, float scale, int block_size,
-                             int num_blocks, int chunks, float* pre_o, float* pre_ml,
-                             pa_dtype dtype, int* err, cudaStream_t stream) {
+                             int num_blocks, const SharedPrefixPlan& plan, float* pre_o,
+                             float* pre_ml, pa_dtype dtype, int* err, cudaStream_t stream) {
   const int G = num_q_heads / num_kv_heads;
-  const int MQ = prefill::kM / G;
   CUtensorMap tk, tv;
   const uint64_t row = (uint64_t)prefill::kD * 2;
   const uint64_t cdims[4] = {(uint64_t)prefill::kD, (uint64_t)num_kv_heads, (uint64_t)block_size,
@@ -773,17 +816,18 @@ pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_c
   a.num_blocks = num_blocks;
   a.max_query_len = max_group_size;
   a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_prefix_len);
-  a.qblocks = (max_group_size + 2 * MQ - 1) / (2 * MQ);
+  a.qblocks = plan.qblocks;
   a.qscale = scale * 1.4426950408889634f;
   a.whole_items = 0;
   a.split_items = 0;
   a.part_o = a.part_ml = nullptr;
   a.rowmap = nullptr;
-  a.prefix_chunks = chunks;
+  a.prefix_chunks = plan.pieces;
+  a.ksplit = plan.ksplit;
   a.q_rows = q_rows;
   a.pre_o = pre_o;
   a.pre_ml = pre_ml;
-  const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * chunks;
+  const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * plan.pieces;
   if (grid <= 0) return PA_OK;
   if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
   auto go = [&](auto tag) -> pa_status {
@@ -866,6 +910,7 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   a.qblocks = (max_query_len + 2 * MQ - 1) / (2 * MQ);
   a.qscale = scale * 1.4426950408889634f;
   a.prefix_chunks = 0;
+  a.ksplit = 0;
   a.q_rows = 0;
   a.pre_o = a.pre_ml = nullptr;
   // the split's row map stores output row numbers as int
