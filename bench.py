@@ -209,6 +209,12 @@ class Step:
                        for b in self.decode}
         self.fused = {id(b): int(b.k_new.shape[0]) == b.num_seqs and b.k_scale is None
                       and not self.shared[id(b)] for b in self.decode}
+        # a varlen batch mixing rows of one query and longer chunks runs
+        # pa_attention_varlen (decode kernel + prefill kernel in one call)
+        self.varlen = {}
+        for b in self.prefill:
+            ql = (b.query_start_loc[1:] - b.query_start_loc[:-1]).cpu()
+            self.varlen[id(b)] = bool((ql == 1).any()) and bool((ql > 1).any())
         self.group_bounds = {}
         for b in self.decode:
             if self.shared[id(b)]:
@@ -223,6 +229,9 @@ class Step:
                                                               b.head_dim, b.max_seq_len)
             elif b.query_start_loc is None:
                 n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
+            elif self.varlen[id(b)]:
+                n = pa.pa_attention_varlen_workspace_size(b.num_seqs, b.max_query_len,
+                                                          b.num_q_heads, b.head_dim, b.max_seq_len)
             else:
                 n = pa.pa_chunked_prefill_workspace_size(b.num_seqs, b.max_query_len, b.num_q_heads,
                                                          b.head_dim, b.max_seq_len)
@@ -236,9 +245,16 @@ class Step:
         for b in self.prefill:
             if record is not None:
                 record[0].record(self.stream)
-            self.pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache, b.block_tables,
-                                       b.seq_lens, b.query_start_loc, b.scale, self.max_q[id(b)],
-                                       self.max_len[id(b)], self.ws[id(b)], stream=self.stream)
+            if self.varlen[id(b)]:
+                self.pa.pa_attention_varlen(self.out[id(b)], b.q, b.k_cache, b.v_cache,
+                                            b.block_tables, b.seq_lens, b.query_start_loc,
+                                            b.scale, self.max_q[id(b)], self.max_len[id(b)],
+                                            self.ws[id(b)], stream=self.stream)
+            else:
+                self.pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache,
+                                           b.block_tables, b.seq_lens, b.query_start_loc, b.scale,
+                                           self.max_q[id(b)], self.max_len[id(b)], self.ws[id(b)],
+                                           stream=self.stream)
             n += self.pa.pa_last_launch_count()
             if record is not None:
                 record[1].record(self.stream)
@@ -636,7 +652,29 @@ def run_ours(args, rank, world, device):
                                            "sequence's blocks contiguous and in order"}
         line["context_tokens_per_s"] = round(world * int(dec.seq_lens.sum().item()) * args.steps
                                              / (total_ms / 1e3), 1)
-    if pre is not None:
+    if pre is not None and step.varlen[id(pre)]:
+        # one call, two kernels in sequence: its speed of light is the decode rows' bytes
+        # at the HBM peak plus the chunks' flops at the tensor peak
+        ql = (pre.query_start_loc[1:] - pre.query_start_loc[:-1]).cpu().numpy()
+        lens = pre.seq_lens.cpu().numpy().astype(np.int64)
+        dec_rows = ql == 1
+        e = pre.q.element_size()
+        dec_bytes = int(lens[dec_rows].sum()) * 2 * pre.num_kv_heads * pre.head_dim * e + \
+            2 * int(dec_rows.sum()) * pre.num_q_heads * pre.head_dim * e + \
+            int(dec_rows.sum()) * int(math.ceil(int(lens.max()) / pre.block_size)) * 4
+        fl = 4 * pre.head_dim * pre.num_q_heads * sum(
+            sum(int(L) - int(n) + i + 1 for i in range(int(n))) for L, n in zip(lens, ql) if n > 1)
+        pmean = statistics.mean(pre_ms)
+        ideal_ms = (dec_bytes / (peaks["hbm_gbs"] * 1e9) + fl / (peaks["bf16_tflops"] * 1e12)) * 1e3
+        line["roofline"] = {"kernel": "pa_attention_varlen (paged_decode_kernel + lse_reduce_kernel"
+                                      " + chunked_prefill_kernel)",
+                            "bound": "hbm (decode rows) then tensor (chunks)",
+                            "achieved": round(ideal_ms / pmean, 4), "peak": 1.0,
+                            "unit": "fraction of the serial speed of light",
+                            "frac": round(ideal_ms / pmean, 4), "ms_per_launch": round(pmean, 5),
+                            "ideal_ms": round(ideal_ms, 5), "decode_bytes": dec_bytes,
+                            "chunk_flop": fl, "peak_source": peaks["source"], "traffic": None}
+    elif pre is not None:
         fl = prefill_flops(pre)
         pmean = statistics.mean(pre_ms)
         tf = fl / (pmean / 1e3) / 1e12

@@ -244,6 +244,31 @@ PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k
                                          void* stream);
 
 /*
+ * pa_attention_varlen — one call for a continuous-batching step that mixes decode
+ * sequences and prefill chunks ([P1] "工程边界与架构取舍": long prompts are prefilled in
+ * chunks with decode steps in between).  Layout as pa_chunked_prefill: sequence s has
+ * n = query_start_loc[s+1] - query_start_loc[s] query rows (its last n tokens, already
+ * cached), q / out [num_q_rows, num_q_heads, 128].  Sequences with n == 1 run on the
+ * decode kernel (reading q and writing out at row query_start_loc[s]), those with n > 1
+ * on the tcgen05 prefill kernel; the result of each row is that of pa_chunked_prefill.
+ * The call launches both kernels (and their merges) on `stream`: a single launch for
+ * both is not built, since each kernel's CTA needs ~200 KB of shared memory and the two
+ * could not share an SM.  Workspace: at least pa_attention_varlen_workspace_size(...)
+ * bytes, 256-byte aligned.  Limits as pa_decode and pa_chunked_prefill; a decode row
+ * outside [0, num_q_rows) sets PA_DEVERR_QUERY_LAYOUT and is skipped.
+ */
+PA_API size_t pa_attention_varlen_workspace_size(int num_seqs, int max_query_len, int num_q_heads,
+                                                 int head_dim, int max_seq_len);
+PA_API pa_status pa_attention_varlen(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     int max_blocks_per_seq, const int32_t* seq_lens,
+                                     const int32_t* query_start_loc, int num_seqs, int num_q_rows,
+                                     int max_query_len, int num_q_heads, int num_kv_heads,
+                                     int head_dim, float scale, int block_size, int num_blocks,
+                                     int max_seq_len, void* workspace, size_t workspace_bytes,
+                                     pa_dtype dtype, void* stream);
+
+/*
  * Device-side block-table maintenance.  [P1] "生产级推理引擎的内存管理与调度": a pool
  * keeps the free block ids in a FIFO queue (a new pool holds 0..N-1 in order; allocation
  * pops the front, freeing pushes the back); a sequence gets new blocks when the blocks

@@ -21,6 +21,7 @@ __all__ = [
     "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_block_pool_init", "pa_block_allocate",
     "pa_block_free", "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
+    "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
     "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
@@ -54,6 +55,9 @@ _SIGS = [
                                  _vp]),
     ("pa_block_free", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
     ("pa_decode_shared_prefix_workspace_size", _sz, [_i32, _i32, _i32, _i32]),
+    ("pa_attention_varlen_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
+    ("pa_attention_varlen", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32,
+                                   _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
     ("pa_decode_shared_prefix", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
                                        _i32, _i32, _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp,
                                        _sz, _i32, _vp]),
@@ -278,6 +282,29 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, gr
         prefix_lens.numel(), int(max_group_size), int(max_prefix_len), Hq, Hkv, D, float(scale),
         bs, N, int(max_seq_len), _ptr(workspace), ws_bytes, _dtype_code(k_cache), _stream(stream)),
         "pa_decode_shared_prefix")
+
+
+def pa_attention_varlen_workspace_size(num_seqs, max_query_len, num_q_heads, head_dim,
+                                       max_seq_len):
+    return int(lib().pa_attention_varlen_workspace_size(num_seqs, max_query_len, num_q_heads,
+                                                        head_dim, max_seq_len))
+
+
+def pa_attention_varlen(out, q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, scale,
+                        max_query_len, max_seq_len, workspace=None, stream=None):
+    """A mixed step: rows of one query (decode) on the decode kernel, chunks on the
+    prefill kernel.  ``q``/``out`` [rows, Hq, D]; ``query_start_loc`` int32 [B+1];
+    ``workspace`` at least :func:`pa_attention_varlen_workspace_size` bytes."""
+    N, bs, Hkv, D = k_cache.shape
+    rows, Hq, _ = q.shape
+    B = seq_lens.numel()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().pa_attention_varlen(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _i32tensor(block_tables, "block_tables"),
+        block_tables.shape[1], _i32tensor(seq_lens, "seq_lens"),
+        _i32tensor(query_start_loc, "query_start_loc"), B, rows, int(max_query_len), Hq, Hkv, D,
+        float(scale), bs, N, int(max_seq_len), _ptr(workspace), ws_bytes, _dtype_code(k_cache),
+        _stream(stream)), "pa_attention_varlen")
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, max_seq_len,

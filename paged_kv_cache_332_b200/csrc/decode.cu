@@ -78,6 +78,10 @@ struct DecodeArgs {
   const float* pre_o;
   const float* pre_ml;
   int num_groups, pre_chunks;
+  // varlen batch (qsl != nullptr): only sequences with one query row (qsl[s+1]-qsl[s] == 1)
+  // are served here, reading q and writing out at row qsl[s] of num_q_rows
+  const int32_t* qsl;
+  int num_q_rows;
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int seq_cap;
@@ -316,14 +320,22 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
       slen[s] = L;
       int first = 0;
-      if (a.num_groups > 0) {
+      if (a.qsl != nullptr) {  // varlen: decode rows only; the others are prefill chunks
+        const int q0 = __ldg(a.qsl + s), nq = __ldg(a.qsl + s + 1) - q0;
+        if (nq != 1) first = -1;
+        else if (q0 < 0 || q0 >= a.num_q_rows) {
+          if (blockIdx.x == 0) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
+          first = -1;
+        }
+      }
+      if (first == 0 && a.num_groups > 0) {
         const int p = shared_prefix_of(a, s);
         if ((p < 0 || p > L || (p & ((1 << a.log2_bs) - 1))) && blockIdx.x == 0)
           flag_error(a.err, PA_DEVERR_PREFIX);
         first = clamp_len(p, L) / kTileTok;
       }
       sfirst[s] = first;
-      sum += NHP * (cdiv(L, kTileTok) - first);
+      sum += first < 0 ? 0 : NHP * (cdiv(L, kTileTok) - first);
     }
     int incl = sum;
 #pragma unroll
@@ -334,7 +346,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     int run = incl - sum;
     for (int s = lo; s < hi; ++s) {
       sstart[s] = run;
-      run += NHP * (cdiv(slen[s], kTileTok) - sfirst[s]);
+      run += sfirst[s] < 0 ? 0 : NHP * (cdiv(slen[s], kTileTok) - sfirst[s]);
     }
     if (lane == 31) sstart[B] = incl;
   }
@@ -367,12 +379,17 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     if (warp == C::WARP_FILL) {
       // ===== empty sequences: no CTA visits them; zero their output and merge record =====
       for (int s = cta; s < B; s += gridDim.x) {
+        if (sfirst[s] < 0) {  // not served by this kernel: no merge, no output
+          for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
+          continue;
+        }
         if (cdiv(slen[s], kTileTok) != sfirst[s]) continue;
         // no keys of its own: a sequence with a shared prefix takes the prefix part alone
         const int pre = sfirst[s] > 0 ? kHasPrefix : 0;
         for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, pre);
         if (pre) continue;
-        T* ob = static_cast<T*>(a.out) + (long long)s * a.num_q_heads * kD;
+        const int orow = a.qsl ? __ldg(a.qsl + s) : s;
+        T* ob = static_cast<T*>(a.out) + (long long)orow * a.num_q_heads * kD;
         for (int i = lane; i < a.num_q_heads * kD / 8; i += 32)
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -479,9 +496,10 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           u[4] = flags;
           u[5] = cta + grp;
           u[6] = append ? 1 : 0;
+          u[7] = a.qsl ? __ldg(a.qsl + s) : s;  // q / out row
           if (flags & kFirst) {
             mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
-            tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HBG, s, &qfull[qs]);
+            tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HBG, u[7], &qfull[qs]);
           } else {
             mbar_arrive_expect_tx(&qfull[qs], 0);
           }
@@ -571,7 +589,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       const volatile int* u = unit + qs * 8;
       const int s = u[0];
       if (s < 0 || *abort_flag) break;
-      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
+      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5], orow = u[7];
       if (flags & kFirst) {
         const uint8_t* qrow = qbuf + qs * C::QBYTES + (w * G + g) * kRowBytes;
         if constexpr (F8) {
@@ -748,7 +766,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
             pk[4 + i] = Elem<T>::pack2(oacc[2 * i][2 + e] * inv, oacc[2 * i + 1][2 + e] * inv);
           }
           T* ob = static_cast<T*>(a.out) +
-                  ((long long)s * a.num_q_heads + hp * HBG + j0 + e) * kD + 16 * g;
+                  ((long long)orow * a.num_q_heads + hp * HBG + j0 + e) * kD + 16 * g;
           reinterpret_cast<uint4*>(ob)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           reinterpret_cast<uint4*>(ob)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         } else {
@@ -785,7 +803,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       const volatile int* u = unit + qs * 8;
       const int s = u[0];
       if (s < 0 || *abort_flag) break;
-      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5];
+      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5], orow = u[7];
       if (flags & kFirst) {
         // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
         const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
@@ -900,7 +918,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
         const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
         const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
         if (flags & kDirect) {
-          T* ob = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + hp * HBG + j) * kD +
+          T* ob = static_cast<T*>(a.out) + ((long long)orow * a.num_q_heads + hp * HBG + j) * kD +
                   lane * 4;
           *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
         } else {
@@ -976,7 +994,8 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
     M = Mn;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  T* ob = static_cast<T*>(a.out) + (long long)gw * kD + lane * 4;
+  const long long orow = a.qsl ? __ldg(a.qsl + s) : s;
+  T* ob = static_cast<T*>(a.out) + (orow * a.num_q_heads + qh) * kD + lane * 4;
   *reinterpret_cast<uint2*>(ob) =
       make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
 }
@@ -1107,7 +1126,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
                       int num_q_heads, int num_kv_heads, int head_dim, float scale,
                       int block_size, int num_blocks, int max_seq_len, int partition_size,
                       void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream,
-                      const SharedPrefixArgs* sp = nullptr) {
+                      const SharedPrefixArgs* sp = nullptr, const int32_t* qsl = nullptr,
+                      int num_q_rows = 0) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0 ||
@@ -1166,7 +1186,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
                              (uint64_t)num_blocks};
   const uint64_t cstr[3] = {crow, crow * num_kv_heads, crow * num_kv_heads * block_size};
   const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
-  const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads, (uint64_t)num_seqs};
+  const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads,
+                             (uint64_t)(qsl ? num_q_rows : num_seqs)};
   const uint64_t qstr[2] = {row, row * num_q_heads};
   const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)HBG, 1};
   const CUtensorMapDataType ct =
@@ -1204,6 +1225,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.group_starts = a.prefix_lens = nullptr;
   a.pre_o = a.pre_ml = nullptr;
   a.num_groups = a.pre_chunks = 0;
+  a.qsl = qsl;
+  a.num_q_rows = qsl ? num_q_rows : num_seqs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (sp) {
     // pass 1: every group's prefix, once for all its members (tensor cores); pass 2 (the
@@ -1367,4 +1390,53 @@ extern "C" pa_status pa_decode_shared_prefix(
                      max_blocks_per_seq, seq_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
                      scale, block_size, num_blocks, max_seq_len, 0, workspace, workspace_bytes,
                      dtype, stream, &sp);
+}
+
+// Mixed varlen batch: decode rows on the decode kernel, prefill chunks on the tcgen05
+// prefill kernel, in one call.
+extern "C" size_t pa_attention_varlen_workspace_size(int num_seqs, int max_query_len,
+                                                     int num_q_heads, int head_dim,
+                                                     int max_seq_len) {
+  const size_t d = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
+  if (d == 0) return 0;
+  return pa::align256(d) + pa_chunked_prefill_workspace_size(num_seqs, max_query_len,
+                                                             num_q_heads, head_dim, max_seq_len);
+}
+
+extern "C" pa_status pa_attention_varlen(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+    const int32_t* query_start_loc, int num_seqs, int num_q_rows, int max_query_len,
+    int num_q_heads, int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
+    int max_seq_len, void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream) {
+  pa::set_launch_count(0);
+  if (num_seqs < 0 || num_q_rows < 0 || max_query_len < 0) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_q_rows == 0 || max_query_len == 0) return PA_OK;
+  if (!query_start_loc) return PA_ERR_INVALID_ARG;
+  if (num_q_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
+  const size_t dws = pa::align256(
+      pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0));
+  if (!workspace || workspace_bytes < dws) return PA_ERR_WORKSPACE_TOO_SMALL;
+  // the rows of one query: the decode kernel (it skips the others)
+  pa_status st = decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
+                             block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                             num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len,
+                             0, workspace, dws, dtype, stream, nullptr, query_start_loc,
+                             num_q_rows);
+  if (st != PA_OK) return st;
+  int launches = pa::launch_count();
+  if (max_query_len > 1) {
+    // the chunks: the prefill kernel (it skips the rows of one query)
+    const size_t rest = workspace_bytes - dws;
+    st = pa::chunked_prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                  seq_lens, query_start_loc, num_seqs, max_query_len,
+                                  num_q_heads, num_kv_heads, head_dim, scale, block_size,
+                                  num_blocks, max_seq_len,
+                                  rest ? static_cast<uint8_t*>(workspace) + dws : nullptr, rest,
+                                  dtype, stream, true);
+    if (st != PA_OK) return st;
+    launches += pa::launch_count();
+  }
+  pa::set_launch_count(launches);
+  return PA_OK;
 }

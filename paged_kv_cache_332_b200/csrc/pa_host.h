@@ -52,6 +52,16 @@ struct SharedPrefixPlan {
   int pieces;   // key pieces per (group, kv-head, query block)
   int slots;    // partial rows per output row: pieces (x 2 with ksplit)
 };
+// pa_chunked_prefill; with skip_single, sequences of one query row are left out (the
+// varlen call serves them with the decode kernel).
+pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* seq_lens, const int32_t* query_start_loc,
+                               int num_seqs, int max_query_len, int num_q_heads, int num_kv_heads,
+                               int head_dim, float scale, int block_size, int num_blocks,
+                               int max_seq_len, void* workspace, size_t workspace_bytes,
+                               pa_dtype dtype, void* stream, bool skip_single);
+
 SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
                                     int max_prefix_len);
 pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,

@@ -79,6 +79,8 @@ struct Args {
   int prefix_chunks, q_rows, ksplit;
   float* pre_o;
   float* pre_ml;
+  // varlen call: sequences with a single query row are left to the decode kernel
+  int skip_single;
 };
 
 // shared memory carve-up
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return;
     }
   }
-  if (q0 >= n) {  // this query block is past the chunk (uniform for the CTA)
+  if (q0 >= n || (a.skip_single && n == 1)) {  // past the chunk, or a decode row
     mark_rows_unused();
     return;
   }
@@ -827,6 +829,7 @@ pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_c
   a.q_rows = q_rows;
   a.pre_o = pre_o;
   a.pre_ml = pre_ml;
+  a.skip_single = 0;
   const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * plan.pieces;
   if (grid <= 0) return PA_OK;
   if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
@@ -857,14 +860,14 @@ extern "C" size_t pa_chunked_prefill_workspace_size(int num_seqs, int max_query_
   return pa::prefill::split_bytes(std::min<long long>(128, items));
 }
 
-extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache,
-                                        const void* v_cache, const int32_t* block_tables,
-                                        int max_blocks_per_seq, const int32_t* seq_lens,
-                                        const int32_t* query_start_loc, int num_seqs,
-                                        int max_query_len, int num_q_heads, int num_kv_heads,
-                                        int head_dim, float scale, int block_size, int num_blocks,
-                                        int max_seq_len, void* workspace, size_t workspace_bytes,
-                                        pa_dtype dtype, void* stream) {
+namespace pa {
+pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* seq_lens, const int32_t* query_start_loc,
+                               int num_seqs, int max_query_len, int num_q_heads, int num_kv_heads,
+                               int head_dim, float scale, int block_size, int num_blocks,
+                               int max_seq_len, void* workspace, size_t workspace_bytes,
+                               pa_dtype dtype, void* stream, bool skip_single) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
@@ -911,6 +914,7 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   a.qscale = scale * 1.4426950408889634f;
   a.prefix_chunks = 0;
   a.ksplit = 0;
+  a.skip_single = skip_single ? 1 : 0;
   a.q_rows = 0;
   a.pre_o = a.pre_ml = nullptr;
   // the split's row map stores output row numbers as int
@@ -920,4 +924,19 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   return dtype == PA_F16
              ? pa::prefill::dispatch<__half>(G, tk, tv, a, workspace, workspace_bytes, st)
              : pa::prefill::dispatch<__nv_bfloat16>(G, tk, tv, a, workspace, workspace_bytes, st);
+}
+}  // namespace pa
+
+extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* seq_lens,
+                                        const int32_t* query_start_loc, int num_seqs,
+                                        int max_query_len, int num_q_heads, int num_kv_heads,
+                                        int head_dim, float scale, int block_size, int num_blocks,
+                                        int max_seq_len, void* workspace, size_t workspace_bytes,
+                                        pa_dtype dtype, void* stream) {
+  return pa::chunked_prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                  seq_lens, query_start_loc, num_seqs, max_query_len, num_q_heads,
+                                  num_kv_heads, head_dim, scale, block_size, num_blocks,
+                                  max_seq_len, workspace, workspace_bytes, dtype, stream, false);
 }

@@ -348,6 +348,20 @@ def prefill_plus_decode(seed=1005, device="cpu", scale=1.0, n_prefill=4, n_decod
     return [p, d]
 
 
+def varlen_step(seed=1006, device="cpu", scale=1.0, n_prefill=4, n_decode=32):
+    """The chunked-prefill + long-decode step of ``prefill_plus_decode`` as ONE varlen
+    batch over one cache: 4 sequences with a 512-token chunk over 8000-token contexts
+    and 32 decode rows of 32768 tokens; 64 q / 8 kv heads, bf16, block 16."""
+    chunk = max(2, int(512 * scale))
+    total = max(chunk, int(8000 * scale))
+    dec_len = max(1, int(32768 * scale))
+    lens = [total] * n_prefill + [dec_len] * n_decode
+    return [make_batch("varlen_4x512_ctx8000_plus_32x32768_bf16", seq_lens=lens,
+                       q_lens=[chunk] * n_prefill + [1] * n_decode, num_q_heads=64,
+                       num_kv_heads=8, block_size=16, num_blocks=_pool_size(lens, 16),
+                       dtype=torch.bfloat16, seed=seed, device=device, prefill=True)]
+
+
 def with_fp8_cache(batch: PagedBatch, seed: int = 77) -> PagedBatch:
     """The same batch (tables, lengths, q, new K/V) over an FP8 (e4m3) cache: every
     cache slot holds a seeded random e4m3 code of magnitude code 0x00..0x48 (values 0..4,
@@ -388,6 +402,7 @@ WORKLOADS = {
     "shared16": lambda **kw: shared_prefix(block_size=16, **kw),
     "shared32": lambda **kw: shared_prefix(block_size=32, **kw),
     "prefill_decode": prefill_plus_decode,
+    "varlen": varlen_step,
     "mixed_fp8": mixed_lengths_fp8,
     "llama70b_fp8": llama70b_fp8,
 }
