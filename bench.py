@@ -212,9 +212,11 @@ class Step:
         # a varlen batch mixing rows of one query and longer chunks runs
         # pa_attention_varlen (decode kernel + prefill kernel in one call)
         self.varlen = {}
+        self.chunk_seqs = {}
         for b in self.prefill:
             ql = (b.query_start_loc[1:] - b.query_start_loc[:-1]).cpu()
             self.varlen[id(b)] = bool((ql == 1).any()) and bool((ql > 1).any())
+            self.chunk_seqs[id(b)] = int((ql > 1).sum())
         self.group_bounds = {}
         for b in self.decode:
             if self.shared[id(b)]:
@@ -249,7 +251,8 @@ class Step:
                 self.pa.pa_attention_varlen(self.out[id(b)], b.q, b.k_cache, b.v_cache,
                                             b.block_tables, b.seq_lens, b.query_start_loc,
                                             b.scale, self.max_q[id(b)], self.max_len[id(b)],
-                                            self.ws[id(b)], stream=self.stream)
+                                            self.ws[id(b)], stream=self.stream,
+                                            max_chunk_seqs=self.chunk_seqs[id(b)])
             else:
                 self.pa.pa_chunked_prefill(self.out[id(b)], b.q, b.k_cache, b.v_cache,
                                            b.block_tables, b.seq_lens, b.query_start_loc, b.scale,

@@ -253,9 +253,13 @@ PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k
  * on the tcgen05 prefill kernel; the result of each row is that of pa_chunked_prefill.
  * The call launches both kernels (and their merges) on `stream`: a single launch for
  * both is not built, since each kernel's CTA needs ~200 KB of shared memory and the two
- * could not share an SM.  Workspace: at least pa_attention_varlen_workspace_size(...)
- * bytes, 256-byte aligned.  Limits as pa_decode and pa_chunked_prefill; a decode row
- * outside [0, num_q_rows) sets PA_DEVERR_QUERY_LAYOUT and is skipped.
+ * could not share an SM.  The decode kernel also lists the sequences with more than one
+ * query row, and the prefill grid covers max_chunk_seqs of them (a host bound on their
+ * number, like max_query_len; negative = num_seqs; more chunks than the bound set
+ * PA_DEVERR_QUERY_LAYOUT and the extra ones are not computed).  Workspace: at least
+ * pa_attention_varlen_workspace_size(...) bytes, 256-byte aligned.  Limits as pa_decode
+ * and pa_chunked_prefill; a decode row outside [0, num_q_rows) sets
+ * PA_DEVERR_QUERY_LAYOUT and is skipped.
  */
 PA_API size_t pa_attention_varlen_workspace_size(int num_seqs, int max_query_len, int num_q_heads,
                                                  int head_dim, int max_seq_len);
@@ -263,10 +267,10 @@ PA_API pa_status pa_attention_varlen(void* out, const void* q, const void* k_cac
                                      const void* v_cache, const int32_t* block_tables,
                                      int max_blocks_per_seq, const int32_t* seq_lens,
                                      const int32_t* query_start_loc, int num_seqs, int num_q_rows,
-                                     int max_query_len, int num_q_heads, int num_kv_heads,
-                                     int head_dim, float scale, int block_size, int num_blocks,
-                                     int max_seq_len, void* workspace, size_t workspace_bytes,
-                                     pa_dtype dtype, void* stream);
+                                     int max_query_len, int max_chunk_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, float scale, int block_size,
+                                     int num_blocks, int max_seq_len, void* workspace,
+                                     size_t workspace_bytes, pa_dtype dtype, void* stream);
 
 /*
  * Device-side block-table maintenance.  [P1] "生产级推理引擎的内存管理与调度": a pool

@@ -57,7 +57,8 @@ _SIGS = [
     ("pa_decode_shared_prefix_workspace_size", _sz, [_i32, _i32, _i32, _i32]),
     ("pa_attention_varlen_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_attention_varlen", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32,
-                                   _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
+                                   _i32, _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32,
+                                   _vp]),
     ("pa_decode_shared_prefix", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32,
                                        _i32, _i32, _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp,
                                        _sz, _i32, _vp]),
@@ -291,9 +292,11 @@ def pa_attention_varlen_workspace_size(num_seqs, max_query_len, num_q_heads, hea
 
 
 def pa_attention_varlen(out, q, k_cache, v_cache, block_tables, seq_lens, query_start_loc, scale,
-                        max_query_len, max_seq_len, workspace=None, stream=None):
+                        max_query_len, max_seq_len, workspace=None, stream=None,
+                        max_chunk_seqs=-1):
     """A mixed step: rows of one query (decode) on the decode kernel, chunks on the
     prefill kernel.  ``q``/``out`` [rows, Hq, D]; ``query_start_loc`` int32 [B+1];
+    ``max_chunk_seqs`` a bound on the sequences with more than one row (-1: B);
     ``workspace`` at least :func:`pa_attention_varlen_workspace_size` bytes."""
     N, bs, Hkv, D = k_cache.shape
     rows, Hq, _ = q.shape
@@ -302,7 +305,8 @@ def pa_attention_varlen(out, q, k_cache, v_cache, block_tables, seq_lens, query_
     _check(lib().pa_attention_varlen(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _i32tensor(block_tables, "block_tables"),
         block_tables.shape[1], _i32tensor(seq_lens, "seq_lens"),
-        _i32tensor(query_start_loc, "query_start_loc"), B, rows, int(max_query_len), Hq, Hkv, D,
+        _i32tensor(query_start_loc, "query_start_loc"), B, rows, int(max_query_len),
+        int(max_chunk_seqs), Hq, Hkv, D,
         float(scale), bs, N, int(max_seq_len), _ptr(workspace), ws_bytes, _dtype_code(k_cache),
         _stream(stream)), "pa_attention_varlen")
 

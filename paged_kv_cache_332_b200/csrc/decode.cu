@@ -82,6 +82,10 @@ struct DecodeArgs {
   // are served here, reading q and writing out at row qsl[s] of num_q_rows
   const int32_t* qsl;
   int num_q_rows;
+  // varlen: CTA 0 also lists the sequences with more than one query row for the prefill
+  // kernel that follows (chunk_ids[0..n), n = chunk_ids[chunk_cap] <= chunk_cap)
+  int32_t* chunk_ids;
+  int chunk_cap;
   int* err;
   int num_seqs, num_q_heads, num_kv_heads, max_blocks, log2_bs, num_blocks;
   int seq_cap;
@@ -349,6 +353,26 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       run += sfirst[s] < 0 ? 0 : NHP * (cdiv(slen[s], kTileTok) - sfirst[s]);
     }
     if (lane == 31) sstart[B] = incl;
+    if (a.chunk_ids != nullptr && blockIdx.x == 0) {
+      int c = 0;
+      for (int s = lo; s < hi; ++s) c += (__ldg(a.qsl + s + 1) - __ldg(a.qsl + s)) > 1;
+      int ci = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, ci, o);
+        if (lane >= o) ci += t;
+      }
+      int r = ci - c;
+      for (int s = lo; s < hi; ++s)
+        if (__ldg(a.qsl + s + 1) - __ldg(a.qsl + s) > 1) {
+          if (r < a.chunk_cap) a.chunk_ids[r] = s;
+          ++r;
+        }
+      if (lane == 31) {
+        a.chunk_ids[a.chunk_cap] = min(ci, a.chunk_cap);
+        if (ci > a.chunk_cap) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
+      }
+    }
   }
   if (threadIdx.x == C::WARP_STAGE * 32) {
     for (int i = 0; i < nslots; ++i) {
@@ -934,31 +958,18 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
 // Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes
 // over head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the
 // largest m_i, over the segments i of the (sequence, head group), which sit in
-// consecutive slots.
-template <typename T>
-__global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
-  // launched as a programmatic dependent of the decode kernel: its CTAs may start while
-  // the decode grid drains; this waits until that grid has finished and its writes are
-  // visible (a no-op when launched without the dependency)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= a.num_seqs * a.num_q_heads) return;
-  const int s = gw / a.num_q_heads;
-  const int qh = gw - s * a.num_q_heads;
-  const int nhp = a.num_q_heads / hbg;
-  const int j = qh % hbg;
-  const int2 mt = a.meta[s * nhp + qh / hbg];
-  const int n = mt.y & (kHasPrefix - 1);                 // segments of this launch
-  const int npre = (mt.y & kHasPrefix) ? a.pre_chunks : 0;  // shared-prefix partials
-  if (n <= 1 && npre == 0) return;  // written by the decode kernel
-  const int total = n + npre;
-  const long long row0 = (long long)mt.x * hbg + j;
+// consecutive slots, and the sequence's shared-prefix partials.
+//
+// Fold the segments of one output row into (M, den, num): the n slots of this launch
+// (rows row0 + i * hbg) and, with PRE, the npre shared-prefix partials (row gw of each).
+// One pass with a running maximum: up to eight segments per round, all loads of a round
+// in flight together (most groups span fewer than eight CTAs: one round).
+template <bool PRE>
+__device__ __forceinline__ void fold_segments(const DecodeArgs& a, long long row0, int hbg,
+                                              int n, int npre, int gw, int lane, float& M,
+                                              float& den, float4& num) {
+  const int total = n + (PRE ? npre : 0);
   const long long prow_stride = (long long)a.num_seqs * a.num_q_heads;
-  // one pass with a running maximum: up to eight segments per round, all loads of a
-  // round in flight together (most groups span fewer than eight CTAs: one round)
-  float M = -INFINITY, den = 0.f;
-  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int i0 = 0; i0 < total; i0 += 8) {
     float2 mlv[8];
     float4 ov[8];
@@ -966,15 +977,16 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int i = i0 + u;
-      if (i < n) {
-        const long long row = row0 + (long long)i * hbg;
-        mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
-        ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
-        Mr = fmaxf(Mr, mlv[u].x);
-      } else if (i < total) {
-        const long long row = (long long)(i - n) * prow_stride + gw;
-        mlv[u] = *reinterpret_cast<const float2*>(a.pre_ml + row * 2);
-        ov[u] = *reinterpret_cast<const float4*>(a.pre_o + row * kD + lane * 4);
+      if (i < total) {
+        if (!PRE || i < n) {
+          const long long row = row0 + (long long)i * hbg;
+          mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
+          ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
+        } else {
+          const long long row = (long long)(i - n) * prow_stride + gw;
+          mlv[u] = *reinterpret_cast<const float2*>(a.pre_ml + row * 2);
+          ov[u] = *reinterpret_cast<const float4*>(a.pre_o + row * kD + lane * 4);
+        }
         Mr = fmaxf(Mr, mlv[u].x);
       }
     }
@@ -993,6 +1005,32 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int
     }
     M = Mn;
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
+  // launched as a programmatic dependent of the decode kernel: its CTAs may start while
+  // the decode grid drains; this waits until that grid has finished and its writes are
+  // visible (a no-op when launched without the dependency)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= a.num_seqs * a.num_q_heads) return;
+  const int s = gw / a.num_q_heads;
+  const int qh = gw - s * a.num_q_heads;
+  const int nhp = a.num_q_heads / hbg;
+  const int j = qh % hbg;
+  const int2 mt = a.meta[s * nhp + qh / hbg];
+  const int n = mt.y & (kHasPrefix - 1);                 // segments of this launch
+  const int npre = (mt.y & kHasPrefix) ? a.pre_chunks : 0;  // shared-prefix partials
+  if (n <= 1 && npre == 0) return;  // written by the decode kernel
+  const long long row0 = (long long)mt.x * hbg + j;
+  float M = -INFINITY, den = 0.f;
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (npre == 0)
+    fold_segments<false>(a, row0, hbg, n, 0, gw, lane, M, den, num);
+  else
+    fold_segments<true>(a, row0, hbg, n, npre, gw, lane, M, den, num);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   const long long orow = a.qsl ? __ldg(a.qsl + s) : s;
   T* ob = static_cast<T*>(a.out) + (orow * a.num_q_heads + qh) * kD + lane * 4;
@@ -1127,7 +1165,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
                       int block_size, int num_blocks, int max_seq_len, int partition_size,
                       void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream,
                       const SharedPrefixArgs* sp = nullptr, const int32_t* qsl = nullptr,
-                      int num_q_rows = 0) {
+                      int num_q_rows = 0, int32_t* chunk_ids = nullptr, int chunk_cap = 0) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0 ||
@@ -1227,6 +1265,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.num_groups = a.pre_chunks = 0;
   a.qsl = qsl;
   a.num_q_rows = qsl ? num_q_rows : num_seqs;
+  a.chunk_ids = chunk_ids;
+  a.chunk_cap = chunk_cap;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (sp) {
     // pass 1: every group's prefix, once for all its members (tensor cores); pass 2 (the
@@ -1399,41 +1439,49 @@ extern "C" size_t pa_attention_varlen_workspace_size(int num_seqs, int max_query
                                                      int max_seq_len) {
   const size_t d = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
   if (d == 0) return 0;
-  return pa::align256(d) + pa_chunked_prefill_workspace_size(num_seqs, max_query_len,
-                                                             num_q_heads, head_dim, max_seq_len);
+  return pa::align256(d) + pa::align256((size_t)(num_seqs + 1) * sizeof(int32_t)) +
+         pa_chunked_prefill_workspace_size(num_seqs, max_query_len, num_q_heads, head_dim,
+                                           max_seq_len);
 }
 
 extern "C" pa_status pa_attention_varlen(
     void* out, const void* q, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
     const int32_t* query_start_loc, int num_seqs, int num_q_rows, int max_query_len,
-    int num_q_heads, int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
-    int max_seq_len, void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream) {
+    int max_chunk_seqs, int num_q_heads, int num_kv_heads, int head_dim, float scale,
+    int block_size, int num_blocks, int max_seq_len, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, void* stream) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_rows < 0 || max_query_len < 0) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0 || num_q_rows == 0 || max_query_len == 0) return PA_OK;
   if (!query_start_loc) return PA_ERR_INVALID_ARG;
   if (num_q_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
+  // a bound on the sequences with more than one query row (negative: num_seqs)
+  const int cap = max_query_len > 1 ? (max_chunk_seqs < 0 ? num_seqs
+                                                          : std::min(max_chunk_seqs, num_seqs))
+                                    : 0;
   const size_t dws = pa::align256(
       pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0));
-  if (!workspace || workspace_bytes < dws) return PA_ERR_WORKSPACE_TOO_SMALL;
-  // the rows of one query: the decode kernel (it skips the others)
+  const size_t lws = pa::align256((size_t)(num_seqs + 1) * sizeof(int32_t));
+  if (!workspace || workspace_bytes < dws + lws) return PA_ERR_WORKSPACE_TOO_SMALL;
+  int32_t* chunk_ids =
+      cap > 0 ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + dws) : nullptr;
+  // the rows of one query: the decode kernel (it skips the others, and lists the chunks)
   pa_status st = decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
                              block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                              num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len,
                              0, workspace, dws, dtype, stream, nullptr, query_start_loc,
-                             num_q_rows);
+                             num_q_rows, chunk_ids, cap);
   if (st != PA_OK) return st;
   int launches = pa::launch_count();
-  if (max_query_len > 1) {
-    // the chunks: the prefill kernel (it skips the rows of one query)
-    const size_t rest = workspace_bytes - dws;
-    st = pa::chunked_prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                  seq_lens, query_start_loc, num_seqs, max_query_len,
-                                  num_q_heads, num_kv_heads, head_dim, scale, block_size,
-                                  num_blocks, max_seq_len,
-                                  rest ? static_cast<uint8_t*>(workspace) + dws : nullptr, rest,
-                                  dtype, stream, true);
+  if (cap > 0) {
+    // the chunks: the prefill kernel over the listed sequences
+    const size_t rest = workspace_bytes - dws - lws;
+    st = pa::chunked_prefill_impl(
+        out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc,
+        num_seqs, max_query_len, num_q_heads, num_kv_heads, head_dim, scale, block_size,
+        num_blocks, max_seq_len, rest ? static_cast<uint8_t*>(workspace) + dws + lws : nullptr,
+        rest, dtype, stream, true, chunk_ids, cap);
     if (st != PA_OK) return st;
     launches += pa::launch_count();
   }

@@ -53,14 +53,17 @@ struct SharedPrefixPlan {
   int slots;    // partial rows per output row: pieces (x 2 with ksplit)
 };
 // pa_chunked_prefill; with skip_single, sequences of one query row are left out (the
-// varlen call serves them with the decode kernel).
+// varlen call serves them with the decode kernel); with chunk_ids (a device list of the
+// sequences with more than one query row, its length at chunk_ids[chunk_cap]) the grid
+// covers chunk_cap sequences of that list instead of all num_seqs.
 pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* block_tables, int max_blocks_per_seq,
                                const int32_t* seq_lens, const int32_t* query_start_loc,
                                int num_seqs, int max_query_len, int num_q_heads, int num_kv_heads,
                                int head_dim, float scale, int block_size, int num_blocks,
                                int max_seq_len, void* workspace, size_t workspace_bytes,
-                               pa_dtype dtype, void* stream, bool skip_single);
+                               pa_dtype dtype, void* stream, bool skip_single,
+                               const int32_t* chunk_ids, int chunk_cap);
 
 SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
                                     int max_prefix_len);

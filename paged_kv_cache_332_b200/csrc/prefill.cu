@@ -79,8 +79,12 @@ struct Args {
   int prefix_chunks, q_rows, ksplit;
   float* pre_o;
   float* pre_ml;
-  // varlen call: sequences with a single query row are left to the decode kernel
+  // varlen call: sequences with a single query row are left to the decode kernel.  With
+  // chunk_ids, item "sequence" r is the r-th sequence with more than one query row,
+  // chunk_ids[r] (chunk_ids[chunk_cap] holds how many; num_seqs = chunk_cap)
   int skip_single;
+  const int32_t* chunk_ids;
+  int chunk_cap;
 };
 
 // shared memory carve-up
@@ -270,7 +274,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   const int qb = item % a.qblocks;
   const int h = (item / a.qblocks) % a.num_kv_heads;
-  const int s = item / (a.qblocks * a.num_kv_heads);
+  int s = item / (a.qblocks * a.num_kv_heads);
+  if (a.chunk_ids != nullptr) {
+    if (s >= __ldg(a.chunk_ids + a.chunk_cap)) {  // fewer chunks than the bound
+      mark_rows_unused();
+      return;
+    }
+    s = __ldg(a.chunk_ids + s);
+  }
   const int q_begin = a.qsl[s];
   const int n = a.qsl[s + 1] - q_begin;
   const int Lraw = a.seq_lens[s];
@@ -830,6 +841,8 @@ pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_c
   a.pre_o = pre_o;
   a.pre_ml = pre_ml;
   a.skip_single = 0;
+  a.chunk_ids = nullptr;
+  a.chunk_cap = 0;
   const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * plan.pieces;
   if (grid <= 0) return PA_OK;
   if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
@@ -867,7 +880,8 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
                                int num_seqs, int max_query_len, int num_q_heads, int num_kv_heads,
                                int head_dim, float scale, int block_size, int num_blocks,
                                int max_seq_len, void* workspace, size_t workspace_bytes,
-                               pa_dtype dtype, void* stream, bool skip_single) {
+                               pa_dtype dtype, void* stream, bool skip_single,
+                               const int32_t* chunk_ids, int chunk_cap) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
@@ -902,7 +916,7 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
   a.seq_lens = seq_lens;
   a.qsl = query_start_loc;
   a.err = err;
-  a.num_seqs = num_seqs;
+  a.num_seqs = chunk_ids ? chunk_cap : num_seqs;
   a.num_q_heads = num_q_heads;
   a.num_kv_heads = num_kv_heads;
   a.max_blocks = max_blocks_per_seq;
@@ -915,6 +929,8 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
   a.prefix_chunks = 0;
   a.ksplit = 0;
   a.skip_single = skip_single ? 1 : 0;
+  a.chunk_ids = chunk_ids;
+  a.chunk_cap = chunk_cap;
   a.q_rows = 0;
   a.pre_o = a.pre_ml = nullptr;
   // the split's row map stores output row numbers as int
@@ -938,5 +954,6 @@ extern "C" pa_status pa_chunked_prefill(void* out, const void* q, const void* k_
   return pa::chunked_prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                   seq_lens, query_start_loc, num_seqs, max_query_len, num_q_heads,
                                   num_kv_heads, head_dim, scale, block_size, num_blocks,
-                                  max_seq_len, workspace, workspace_bytes, dtype, stream, false);
+                                  max_seq_len, workspace, workspace_bytes, dtype, stream, false,
+                                  nullptr, 0);
 }

@@ -182,15 +182,15 @@ def test_varlen_arguments_rejected_on_host(palib):
     nul = None
 
     def call(B=4, rows=10, mq=5, qsl=p, ws=None, wsb=0):
-        return L.pa_attention_varlen(p, p, p, p, p, 32, p, qsl, B, rows, mq, 32, 8, 128, 0.1, 16,
-                                     1000, 512, ws, wsb, 0, nul)
+        return L.pa_attention_varlen(p, p, p, p, p, 32, p, qsl, B, rows, mq, -1, 32, 8, 128, 0.1,
+                                     16, 1000, 512, ws, wsb, 0, nul)
     assert call(B=-1) == 1 and call(rows=-1) == 1 and call(mq=-1) == 1
     assert call(B=0) == 0 and call(rows=0) == 0 and call(mq=0) == 0   # nothing to do
     assert call(qsl=nul) == 1
     assert call() == 3                                                  # needs a workspace
     d = palib.pa_decode_workspace_size(4, 32, 128, 512, 0)
     pf = palib.pa_chunked_prefill_workspace_size(4, 5, 32, 128, 512)
-    assert palib.pa_attention_varlen_workspace_size(4, 5, 32, 128, 512) >= d + pf
+    assert palib.pa_attention_varlen_workspace_size(4, 5, 32, 128, 512) >= d + pf + 5 * 4
     assert palib.pa_last_launch_count() == 0
 
 

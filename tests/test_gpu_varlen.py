@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _varlen(b, rows=None, qsl=None):
+def _varlen(b, rows=None, qsl=None, max_chunk_seqs=-1):
     B, Hq, D = b.num_seqs, b.num_q_heads, b.head_dim
     mq = b.max_query_len
     ws = torch.empty(pa.pa_attention_varlen_workspace_size(B, mq, Hq, D, b.max_seq_len),
@@ -28,7 +28,7 @@ def _varlen(b, rows=None, qsl=None):
     out = torch.full_like(q, float("nan"))
     pa.pa_attention_varlen(out, q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
                            b.query_start_loc if qsl is None else qsl, b.scale, mq, b.max_seq_len,
-                           ws)
+                           ws, max_chunk_seqs=max_chunk_seqs)
     return out
 
 
@@ -55,6 +55,27 @@ def test_mixed_step_matches_oracle(G, dtype, bs):
     assert pa.pa_get_device_error() == 0
     assert launches >= 3  # decode + its merge + prefill
     P.compare(out, P.oracle_prefill(bc), bc.dtype, "mixed varlen step G=%d" % G)
+
+
+def test_chunk_bound_exact_and_too_small():
+    lens = [300, 40, 700, 129, 2000, 90]
+    q_lens = [1, 40, 1, 64, 1, 33]  # three chunks
+    bc = _batch("varlen_bound", lens, q_lens, 4, torch.float16, seed=31)
+    b = bc.to(DEV)
+    P.gpu_append(b)
+    ref = P.oracle_prefill(bc)
+    out = _varlen(b, max_chunk_seqs=3)  # the exact count: a grid over the three chunks
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == 0
+    P.compare(out, ref, bc.dtype, "varlen, chunk bound exact")
+    out = _varlen(b, max_chunk_seqs=2)  # too small: flagged, the third chunk not computed
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() & pa.PA_DEVERR["QUERY_LAYOUT"]
+    qsl = bc.query_start_loc.tolist()
+    first_two = list(range(qsl[1], qsl[2])) + list(range(qsl[3], qsl[4]))
+    decode_rows = [qsl[0], qsl[2], qsl[4]]
+    keep = sorted(first_two + decode_rows)
+    P.compare(out[keep], ref[keep], bc.dtype, "varlen, rows inside the bound")
 
 
 def test_decode_rows_only_equal_pa_decode_bitwise():
