@@ -1,0 +1,87 @@
+"""Host-side logic with no GPU: the seeded workloads' sharing and varlen structure, the
+bench's algorithmic-byte counts (checked against an independent count of the cache
+slots a step actually reads), and how the bench routes each batch to a library call."""
+import numpy as np
+import pytest
+import torch
+
+import bench
+import workloads
+
+
+def _slots_read(b):
+    """Distinct (physical block, offset) slots a decode step reads: every position
+    below each sequence's length, through its table."""
+    bt = b.block_tables.cpu().numpy()
+    seen = set()
+    for s, L in enumerate(b.seq_lens.cpu().numpy()):
+        for p in range(int(L)):
+            seen.add((int(bt[s, p // b.block_size]), p % b.block_size))
+    return seen
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_shared_prompt_groups_and_tables(bs):
+    b = workloads.shared_prefix(block_size=bs, scale=1 / 8)[0]
+    assert b.group_starts.tolist() == list(range(0, 65, 8))
+    assert b.prefix_lens.tolist() == [256] * 8
+    bt = b.block_tables.numpy()
+    npre = 256 // bs
+    for g in range(8):
+        rows = bt[8 * g:8 * g + 8, :npre]
+        assert (rows == rows[0]).all()                 # the members share the prefix blocks
+    owned = [set(bt[s, npre:-(-int(L) // bs)].tolist()) for s, L in enumerate(b.seq_lens.numpy())]
+    for i in range(64):
+        for j in range(i + 1, 64):
+            assert not owned[i] & owned[j]             # the rest is private
+
+
+def test_groups_with_gaps_between_them():
+    b = workloads.make_batch("gaps", seq_lens=[40, 60, 70, 80, 90, 100, 50], num_q_heads=8,
+                             num_kv_heads=2, block_size=16, num_blocks=64, dtype=torch.float16,
+                             seed=1, shared_groups=[[1, 2], [4, 5]], shared_prefix_tokens=32)
+    assert b.group_starts.tolist() == [1, 3, 4, 6]
+    assert b.prefix_lens.tolist() == [32, 0, 32]
+
+
+def test_unique_bytes_of_a_shared_step_match_the_slots_read():
+    b = workloads.shared_prefix(block_size=16, scale=1 / 8)[0]
+    row = 2 * b.num_kv_heads * b.head_dim * b.k_cache.element_size()  # K and V of one slot
+    e = b.q.element_size()
+    B = b.num_seqs
+    rest = 2 * B * b.num_q_heads * b.head_dim * e + \
+        B * int(np.ceil(int(b.seq_lens.max()) / b.block_size)) * 4 + 4 * B
+    unique = len(_slots_read(b)) * row + rest
+    arrays = 4 * (b.group_starts.numel() + b.prefix_lens.numel())
+    assert bench.decode_algorithmic_bytes(b, shared=True) == unique + arrays
+    every = int(b.seq_lens.sum()) * row + rest
+    assert bench.decode_algorithmic_bytes(b) == every
+    assert every > 2 * unique
+
+
+def test_varlen_step_structure():
+    b = workloads.varlen_step(scale=1 / 16)[0]
+    ql = (b.query_start_loc[1:] - b.query_start_loc[:-1]).tolist()
+    assert ql == [32] * 4 + [1] * 32
+    assert b.q.shape[0] == sum(ql) and b.slot_mapping.numel() == sum(ql)
+
+
+def test_bench_routes_each_batch_to_its_call():
+    import paged_kv_cache_332_b200 as pa
+    shared = workloads.shared_prefix(block_size=16, scale=1 / 8)[0]
+    mixed = workloads.mixed_lengths(scale=1 / 8)[0]
+    fp8 = workloads.mixed_lengths_fp8(scale=1 / 8)[0]
+    varlen = workloads.varlen_step(scale=1 / 16)[0]
+    pre, dec = workloads.prefill_plus_decode(scale=1 / 16)
+    st = bench.Step([shared, mixed, fp8, varlen, pre, dec], pa, None)
+    assert st.shared[id(shared)] and not st.fused[id(shared)]
+    assert st.fused[id(mixed)] and not st.shared[id(mixed)]
+    assert not st.fused[id(fp8)] and not st.shared[id(fp8)]
+    assert st.varlen[id(varlen)] and st.chunk_seqs[id(varlen)] == 4
+    assert not st.varlen[id(pre)]
+    assert st.group_bounds[id(shared)] == (8, 256)
+    # every batch got a workspace of the size its call asks for
+    assert st.ws[id(shared)].numel() == pa.pa_decode_shared_prefix_workspace_size(
+        64, 32, 128, shared.max_seq_len)
+    assert st.ws[id(varlen)].numel() == pa.pa_attention_varlen_workspace_size(
+        36, 32, 64, 128, varlen.max_seq_len)
