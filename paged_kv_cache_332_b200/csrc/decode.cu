@@ -1464,8 +1464,10 @@ extern "C" pa_status pa_attention_varlen(
       pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0));
   const size_t lws = pa::align256((size_t)(num_seqs + 1) * sizeof(int32_t));
   if (!workspace || workspace_bytes < dws + lws) return PA_ERR_WORKSPACE_TOO_SMALL;
-  int32_t* chunk_ids =
-      cap > 0 ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + dws) : nullptr;
+  // listed whenever chunks may exist, so that more of them than the bound is flagged
+  int32_t* chunk_ids = max_query_len > 1
+                           ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + dws)
+                           : nullptr;
   // the rows of one query: the decode kernel (it skips the others, and lists the chunks)
   pa_status st = decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
                              block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
