@@ -39,6 +39,13 @@
 //    read per 32 entries) and starts the TMA copy of their q rows.  A producer thread
 //    walks the tiles in order and issues the two boxes of each as soon as a slot of the
 //    shared ring frees (blocking waits take no issue slots from the consumers).
+// Two more modes share the kernel:
+//  * shared prefixes (pa_decode_shared_prefix): a sequence whose first tokens are shared
+//    with its group reads only its tiles after the prefix; the prefix pass (prefill.cu)
+//    left the attention over the prefix as partials, and the merge folds them in;
+//  * varlen rows (pa_attention_varlen): only sequences with one query row are served,
+//    q and out rows come from query_start_loc, and CTA 0 lists the other sequences for
+//    the prefill kernel that follows.
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
 #include <cuda_fp8.h>
 

@@ -31,6 +31,10 @@
 //  * Keys at or past L in the last tile: K is masked in the softmax; V rows are
 //    zero-filled (TMA out-of-range fill for whole runs, a shared-memory clear for the
 //    tail of a partial block) so that 0 * (stale value) never reaches the sum.
+// The same kernel is the first pass of the shared-prefix decode: the "sequence" is a
+// group, its queries the members' decode rows, its keys the shared prefix with no causal
+// mask, and its output normalised partial rows; when the group fits one M-tile the two
+// M-tiles take alternate key tiles as two independent softmax chains.
 // Every wait is bounded; on a timeout the CTA flags PA_DEVERR_TIMEOUT, runs to its end
 // without further waits and frees its TMEM.
 #include <algorithm>
