@@ -702,8 +702,11 @@ def run_ours(args, rank, world, device):
 
 
 def cpu_baseline(batches, args, budget_s=None):
-    """Time the oracle, as it stands, on a bounded sample of the workload and
-    scale to the metric (decoded tokens per second of a full step)."""
+    """Time the oracle, as it stands, on a bounded sample of the workload and scale to
+    the metric (query rows of a full step per second: decoded tokens plus chunk rows).
+    The work of a sequence is its (query row, visible key) pairs; sequences of every
+    batch are drawn in a seeded order until the budget is spent, and the time is scaled
+    by the pairs of the whole step over the pairs done."""
     import oracle.paged_attention as opa
     try:
         from threadpoolctl import threadpool_limits
@@ -711,43 +714,62 @@ def cpu_baseline(batches, args, budget_s=None):
     except Exception:  # pragma: no cover
         limiter = None
     budget_s = budget_s if budget_s is not None else args.cpu_budget
-    dec = [b for b in batches if b.query_start_loc is None]
-    b = dec[0] if dec else batches[0]
-    lens = b.seq_lens.cpu().numpy()
-    order = np.random.Generator(np.random.PCG64(0)).permutation(len(lens))
-    t_used, ctx_done, seqs_done = 0.0, 0, 0
-    for s in order:
-        s = int(s)
-        sub_t0 = time.perf_counter()
+    units, total_pairs, total_rows = [], 0, 0
+    for bi, b in enumerate(batches):
+        lens = b.seq_lens.cpu().numpy().astype(np.int64)
+        if b.query_start_loc is None:
+            ql = np.ones(len(lens), dtype=np.int64)
+        else:
+            qsl = b.query_start_loc.cpu().numpy().astype(np.int64)
+            ql = qsl[1:] - qsl[:-1]
+        for s in range(len(lens)):
+            n, L = int(ql[s]), int(lens[s])
+            pairs = n * L - n * (n - 1) // 2  # row i of n sees L - n + i + 1 keys
+            units.append((bi, s, n, L, pairs))
+            total_pairs += pairs
+            total_rows += n
+    order = np.random.Generator(np.random.PCG64(0)).permutation(len(units))
+    t_used, pairs_done, seqs_done = 0.0, 0, 0
+    for k in order:
+        bi, s, n, L, pairs = units[int(k)]
+        if n == 0:
+            continue
+        b = batches[bi]
         bt = b.block_tables[s:s + 1].cpu()
-        L = int(lens[s])
         nblk = -(-L // b.block_size)
         ids = bt[0, :nblk].long().to(b.k_cache.device)
         kc = b.k_cache.index_select(0, ids).cpu()
         vc = b.v_cache.index_select(0, ids).cpu()
         tbl = np.arange(nblk, dtype=np.int32)[None, :]
-        q = opa.to_f64(b.q[s:s + 1])
+        if b.query_start_loc is None:
+            q = opa.to_f64(b.q[s:s + 1])
+        else:
+            q0 = int(b.query_start_loc[s])
+            q = opa.to_f64(b.q[q0:q0 + n])
         t0 = time.perf_counter()
         if b.k_scale is not None:  # FP8 cache: the oracle dequantises, then attends
             kc = opa.dequantize_cache(kc.numpy(), b.k_scale.cpu().numpy())
             vc = opa.dequantize_cache(vc.numpy(), b.v_scale.cpu().numpy())
         else:
             kc, vc = opa.to_f64(kc), opa.to_f64(vc)
-        opa.paged_decode(q, kc, vc, tbl, np.array([L]), b.scale)
+        if b.query_start_loc is None:
+            opa.paged_decode(q, kc, vc, tbl, np.array([L]), b.scale)
+        else:
+            opa.chunked_prefill(q, kc, vc, tbl, np.array([L]), np.array([0, n]), b.scale)
         t_used += time.perf_counter() - t0
-        ctx_done += L
+        pairs_done += pairs
         seqs_done += 1
         if t_used >= budget_s:
             break
     if limiter is not None:
         limiter.unregister() if hasattr(limiter, "unregister") else None
-    total_ctx = int(lens.sum())
-    est_step_s = t_used * total_ctx / max(ctx_done, 1)
-    value = b.num_seqs / est_step_s
+    est_step_s = t_used * total_pairs / max(pairs_done, 1)
+    value = total_rows / est_step_s
     return {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d sequences of %s (%d of %d context tokens), oracle time %.1f s "
-                      "scaled by context tokens to one full step" % (seqs_done, len(lens), b.name,
-                                                                     ctx_done, total_ctx, t_used)}
+            "sample": "%d of %d sequences of %s (%d of %d query-key pairs), oracle time %.1f s "
+                      "scaled by query-key pairs to one full step"
+                      % (seqs_done, len(units), "+".join(b.name for b in batches), pairs_done,
+                         total_pairs, t_used)}
 
 
 def run_reference(args, rank, world):
@@ -765,12 +787,11 @@ def run_reference(args, rank, world):
         vals.append(last["value"])
     wall = time.perf_counter() - t0
     value = statistics.mean(vals)
-    dec = [b for b in batches if b.query_start_loc is None]
-    b = dec[0] if dec else batches[0]
+    rows = sum(b.num_seqs if b.query_start_loc is None else int(b.q.shape[0]) for b in batches)
     line = {
         "metric": "paged decode tokens/s (one layer) and achieved HBM GB/s of pa_decode",
         "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(b.num_seqs / value * 1e3, 3),
+        "warmup": args.warmup, "ms_per_step": round(rows / value * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded N(0,1) q/K/V, FIFO free-list block tables)",
         "impl": "reference",
