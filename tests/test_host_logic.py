@@ -85,3 +85,18 @@ def test_bench_routes_each_batch_to_its_call():
         64, 32, 128, shared.max_seq_len)
     assert st.ws[id(varlen)].numel() == pa.pa_attention_varlen_workspace_size(
         36, 32, 64, 128, varlen.max_seq_len)
+
+
+def test_cpu_baseline_covers_decode_rows_and_chunks():
+    import types
+    args = types.SimpleNamespace(cpu_budget=0.2)
+    r = bench.cpu_baseline(workloads.tiny_mha(), args)
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
+    assert "4 of 4 sequences" in r["sample"]
+    pre, dec = workloads.prefill_plus_decode(scale=1 / 64)
+    r = bench.cpu_baseline([pre, dec], args, budget_s=60)
+    # everything fits the budget: all 36 sequences and every (query row, key) pair
+    lens = pre.seq_lens.numpy()
+    n = int(pre.query_start_loc[1] - pre.query_start_loc[0])
+    pairs = int(sum(n * L - n * (n - 1) // 2 for L in lens)) + int(dec.seq_lens.sum())
+    assert "36 of 36 sequences" in r["sample"] and "(%d of %d" % (pairs, pairs) in r["sample"]
