@@ -323,7 +323,7 @@ PA_API pa_status pa_block_free(int32_t* ring, int32_t* state, int num_blocks,
 
 /*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
- * The paper has no counterpart to this call; it exists for callers whose device memory
+ * The pages have no counterpart to this call; it exists for callers whose device memory
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that
  * forbids raw cudaMalloc) or who must not risk the device-wide synchronisation an
  * allocation can cause.  Arguments and results are those of pa_decode without the
