@@ -275,6 +275,10 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, gr
     :func:`pa_decode_shared_prefix_workspace_size` bytes."""
     N, bs, Hkv, D = k_cache.shape
     B, Hq, _ = q.shape
+    if group_starts.numel() != prefix_lens.numel() + 1:
+        raise ValueError("group_starts needs one more entry than prefix_lens")
+    if seq_lens.numel() != B or block_tables.shape[0] != B:
+        raise ValueError("q, seq_lens and block_tables disagree on the number of sequences")
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().pa_decode_shared_prefix(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _i32tensor(block_tables, "block_tables"),
@@ -301,6 +305,10 @@ def pa_attention_varlen(out, q, k_cache, v_cache, block_tables, seq_lens, query_
     N, bs, Hkv, D = k_cache.shape
     rows, Hq, _ = q.shape
     B = seq_lens.numel()
+    if query_start_loc.numel() != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("query_start_loc needs B + 1 entries and block_tables B rows")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().pa_attention_varlen(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _i32tensor(block_tables, "block_tables"),

@@ -100,3 +100,21 @@ def test_cpu_baseline_covers_decode_rows_and_chunks():
     n = int(pre.query_start_loc[1] - pre.query_start_loc[0])
     pairs = int(sum(n * L - n * (n - 1) // 2 for L in lens)) + int(dec.seq_lens.sum())
     assert "36 of 36 sequences" in r["sample"] and "(%d of %d" % (pairs, pairs) in r["sample"]
+
+
+def test_bindings_check_array_lengths_before_any_call():
+    import paged_kv_cache_332_b200 as pa
+    b = workloads.shared_prefix(block_size=16, scale=1 / 8)[0]
+    with pytest.raises(ValueError):
+        pa.pa_decode_shared_prefix(b.q, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
+                                   b.group_starts[:-1], b.prefix_lens, b.scale, 300, 8, 256)
+    with pytest.raises(ValueError):
+        pa.pa_decode_shared_prefix(b.q, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens[:5],
+                                   b.group_starts, b.prefix_lens, b.scale, 300, 8, 256)
+    v = workloads.varlen_step(scale=1 / 16)[0]
+    with pytest.raises(ValueError):
+        pa.pa_attention_varlen(v.q, v.q, v.k_cache, v.v_cache, v.block_tables, v.seq_lens,
+                               v.query_start_loc[:-1], v.scale, 32, 2048)
+    with pytest.raises(ValueError):
+        pa.pa_attention_varlen(v.q[:5], v.q, v.k_cache, v.v_cache, v.block_tables, v.seq_lens,
+                               v.query_start_loc, v.scale, 32, 2048)
