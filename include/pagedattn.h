@@ -17,7 +17,8 @@
  *  - Every tensor pointer is a DEVICE pointer owned by the caller, contiguous in the
  *    stated row-major layout; the library keeps no reference after the call returns.
  *  - KV caches: k_cache, v_cache [num_blocks, block_size, num_kv_heads, head_dim] of
- *    fp16 or bf16 (PA_F16 / PA_BF16); the two caches share one layout.
+ *    fp16 or bf16 (PA_F16 / PA_BF16), or of e4m3 codes for the *_fp8 calls; the two
+ *    caches share one layout.
  *  - Block tables: int32 [num_seqs, max_blocks_per_seq]; entry j of row s is the
  *    physical block that holds tokens j*block_size .. j*block_size+block_size-1 of
  *    sequence s.  Entries past a sequence's last block are never read.
@@ -27,7 +28,9 @@
  *    up to 4096 sequences per decode call.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and never synchronise the host.  The library allocates no device memory
- *    on any call; scratch space comes from the caller (`workspace`).
+ *    on any call; scratch space comes from the caller (`workspace`), or from the fixed
+ *    array of pa_decode_noalloc.  pa_last_launch_count() tells how many kernels the
+ *    calling thread's last call launched.
  *  - Return value: PA_OK once the kernels are launched, or an error found on the host
  *    before any launch (nothing is launched then).
  *  - Errors that depend on device data (a slot or block id outside the cache, a
