@@ -118,3 +118,26 @@ def test_bindings_check_array_lengths_before_any_call():
     with pytest.raises(ValueError):
         pa.pa_attention_varlen(v.q[:5], v.q, v.k_cache, v.v_cache, v.block_tables, v.seq_lens,
                                v.query_start_loc, v.scale, 32, 2048)
+
+
+def test_input_recipes_match_their_descriptions():
+    m = workloads.mixed_lengths()[0]
+    lens = m.seq_lens.numpy()
+    assert len(lens) == 64 and lens.min() >= 50 and lens.max() <= 8000
+    assert (m.num_q_heads, m.num_kv_heads, m.block_size, m.dtype) == (32, 8, 16, torch.bfloat16)
+    # log-uniform: about half of the lengths below the geometric mean sqrt(50 * 8000) = 632
+    assert 20 <= int((lens < 632).sum()) <= 44
+    # every slot of the step's appended token is that sequence's position L-1
+    bt = m.block_tables.numpy()
+    sm = m.slot_mapping.numpy()
+    assert all(sm[s] == bt[s, (L - 1) // 16] * 16 + (L - 1) % 16 for s, L in enumerate(lens))
+    ll = workloads.llama70b_uniform()[0]
+    assert ll.seq_lens.tolist() == [4096] * 16 and ll.num_blocks == 4096
+    assert sorted(ll.block_tables.numpy().ravel().tolist()) == list(range(4096))  # the pool exactly
+    assert (ll.num_q_heads, ll.num_kv_heads, ll.dtype) == (64, 8, torch.float16)
+    sp = workloads.shared_prefix()[0]
+    suffix = sp.seq_lens.numpy() - 2048
+    assert suffix.min() >= 1 and suffix.max() <= 512
+    pre, dec = workloads.prefill_plus_decode()
+    assert pre.seq_lens.tolist() == [8000] * 4 and pre.max_query_len == 512
+    assert dec.seq_lens.tolist() == [32768] * 32 and dec.num_q_heads == 64
