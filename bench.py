@@ -696,7 +696,7 @@ def run_ours(args, rank, world, device):
     if pool_line is not None:
         line["block_pool"] = pool_line
     line["clocks"] = clocks.summary()
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the oracle at N = 1 only
         line["cpu_baseline"] = cpu_baseline(batches, args)
     return line
 
