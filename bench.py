@@ -43,6 +43,10 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+DEFAULT_WORKLOAD = "mixed"
+# measured beside the default workload: LLaMA-2-70B-shaped decode, shared prompts (block
+# size 16 and 32), chunked prefill + long decode (two calls, and one varlen call), tiny
+OTHERS = ("llama70b", "shared16", "shared32", "prefill_decode", "varlen", "tiny")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -228,7 +232,8 @@ class Step:
             self.out[id(b)] = torch.empty_like(b.q)
             if b.query_start_loc is None and self.shared[id(b)]:
                 n = pa.pa_decode_shared_prefix_workspace_size(b.num_seqs, b.num_q_heads,
-                                                              b.head_dim, b.max_seq_len)
+                                                              b.num_kv_heads, b.head_dim,
+                                                              b.max_seq_len)
             elif b.query_start_loc is None:
                 n = pa.pa_decode_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, b.max_seq_len, 0)
             elif self.varlen[id(b)]:
@@ -311,6 +316,160 @@ class Step:
         n += self.run_decode()
         self.launches += n
         return n
+
+
+SPLIT_K = ("balanced split-K (partition_size 0): the 16-token tiles of every (sequence, "
+           "kv-head group) laid end to end, each CTA of a persistent grid (one per SM) takes "
+           "an equal share; a group split over several CTAs is merged by log-sum-exp")
+
+
+def rooflines(step, dec_ms, pre_ms, peaks):
+    """The roofline objects of one workload: `roofline` for its decode call (HBM) or, for
+    a varlen step, the call's serial speed of light; `roofline_prefill` (tensor cores) for
+    a separate chunked-prefill call."""
+    out = {}
+    dec = step.decode[0] if step.decode else None
+    pre = step.prefill[0] if step.prefill else None
+    if dec is not None:
+        ab = decode_algorithmic_bytes(dec)
+        if step.fused[id(dec)]:  # the append inside the launch: read k/v_new, write the slots
+            ab += 2 * 2 * dec.num_seqs * dec.num_kv_heads * dec.head_dim * dec.q.element_size()
+        shared = step.shared[id(dec)]
+        if shared:  # the shared blocks are read once per group
+            ab_unshared = ab
+            ab = decode_algorithmic_bytes(dec, shared=True)
+        dmean = statistics.mean(dec_ms)
+        ach = ab / (dmean / 1e3) / 1e9
+        kname = ("pa_decode_fp8" if dec.k_scale is not None else
+                 "pa_decode_shared_prefix" if shared else
+                 "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
+        kparts = (" (chunked_prefill_kernel prefix pass + zero_tickets_kernel + paged_decode_kernel,"
+                  " merge inside the decode launch)"
+                  if shared else " (zero_tickets_kernel + paged_decode_kernel, merge inside the "
+                                 "decode launch)")
+        out["roofline"] = {"kernel": kname + kparts,
+                           "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                           "peak_source": peaks["source"], "unit": "GB/s",
+                           "frac": round(ach / peaks["hbm_gbs"], 4),
+                           "frac_of_8TBs_spec": round(ach / 8000.0, 4),
+                           "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
+                           "traffic": recorded_traffic("paged_decode_kernel", dec.name)}
+        if shared:
+            out["roofline"]["algorithmic_bytes_unshared"] = ab_unshared
+            out["roofline"]["note"] = ("bytes count each shared prefix block once per group; "
+                                       "algorithmic_bytes_unshared counts it once per member")
+    if pre is not None and step.varlen[id(pre)]:
+        # one call: its speed of light is the decode rows' bytes at the HBM peak plus the
+        # chunks' flops at the tensor peak
+        ql = (pre.query_start_loc[1:] - pre.query_start_loc[:-1]).cpu().numpy()
+        lens = pre.seq_lens.cpu().numpy().astype(np.int64)
+        dec_rows = ql == 1
+        e = pre.q.element_size()
+        dec_bytes = int(lens[dec_rows].sum()) * 2 * pre.num_kv_heads * pre.head_dim * e + \
+            2 * int(dec_rows.sum()) * pre.num_q_heads * pre.head_dim * e + \
+            int(dec_rows.sum()) * int(math.ceil(int(lens.max()) / pre.block_size)) * 4
+        fl = 4 * pre.head_dim * pre.num_q_heads * sum(
+            sum(int(L) - int(n) + i + 1 for i in range(int(n))) for L, n in zip(lens, ql) if n > 1)
+        pmean = statistics.mean(pre_ms)
+        ideal_ms = (dec_bytes / (peaks["hbm_gbs"] * 1e9) + fl / (peaks["bf16_tflops"] * 1e12)) * 1e3
+        out["roofline"] = {"kernel": "pa_attention_varlen (zero_tickets_kernel + paged_decode_kernel"
+                                     " + chunked_prefill_kernel)",
+                           "bound": "hbm (decode rows) then tensor (chunks)",
+                           "achieved": round(ideal_ms / pmean, 4), "peak": 1.0,
+                           "unit": "fraction of the serial speed of light",
+                           "frac": round(ideal_ms / pmean, 4), "ms_per_launch": round(pmean, 5),
+                           "ideal_ms": round(ideal_ms, 5), "decode_bytes": dec_bytes,
+                           "chunk_flop": fl, "peak_source": peaks["source"], "traffic": None}
+    elif pre is not None:
+        fl = prefill_flops(pre)
+        pmean = statistics.mean(pre_ms)
+        tf = fl / (pmean / 1e3) / 1e12
+        peak_tf = peaks["bf16_tflops"]
+        out["roofline_prefill"] = {"kernel": "pa_chunked_prefill (chunked_prefill_kernel, tcgen05)",
+                                   "bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
+                                   "peak_source": peaks["source"] + " bf16 dense burst",
+                                   "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4),
+                                   "flop_per_launch": fl, "ms_per_launch": round(pmean, 5),
+                                   "traffic": None}
+    return out
+
+
+def step_tokens(step):
+    return sum(b.num_seqs for b in step.decode) + sum(int(b.q.shape[0]) for b in step.prefill)
+
+
+def measure_other(name, args, device, pa, stream, l2_flush, peaks):
+    """One more workload in the same process: its step replayed as a CUDA graph (tokens/s,
+    L2 flushed before every step) and its decode / prefill calls timed one by one for the
+    roofline, inside one clock record."""
+    batches = workloads.WORKLOADS[name](device=device)
+    step = Step(batches, pa, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            l2_flush()
+            step.run()
+    torch.cuda.synchronize(device)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        step.run()
+    timed = {k: timing_graph(step, k, stream, l2_flush) for k, bb in
+             (("decode", step.decode), ("prefill", step.prefill)) if bb}
+    steps = max(3, min(args.steps, 20))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            l2_flush()
+            g_step.replay()
+        for g, _ in timed.values():
+            g.replay()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clocks:
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                l2_flush()
+                ev[i][0].record(stream)
+                g_step.replay()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        ms = {}
+        for k, (g, evs) in timed.items():
+            with torch.cuda.stream(stream):
+                g.replay()
+            torch.cuda.synchronize(device)
+            ms[k] = [a.elapsed_time(b) for a, b in evs]
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    r = rooflines(step, ms.get("decode", []), ms.get("prefill", []), peaks)
+    res = {"value": round(step_tokens(step) / (step_ms / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(step_ms, 5), "steps": steps,
+           "workload": "+".join(b.name for b in batches), "clocks": clocks.summary()}
+    for k in ("roofline", "roofline_prefill"):
+        if k in r:
+            res[k] = {kk: r[k][kk] for kk in ("kernel", "achieved", "unit", "frac",
+                                              "ms_per_launch") if kk in r[k]}
+    del g_step, timed, step, batches
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    return res
+
+
+N_KERNEL_TIMED = 8
+
+
+def timing_graph(step, kind, stream, l2_flush):
+    """A graph of N calls of the step's decode (or prefill) calls, each bracketed by
+    event-record nodes and preceded by an L2 flush."""
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(N_KERNEL_TIMED)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(N_KERNEL_TIMED):
+            l2_flush()
+            if kind == "decode":
+                step.run_decode(evs[i])
+            else:
+                step.run_prefill(evs[i])
+    return g, evs
 
 
 # ---------------------------------------------------------------- arms
@@ -415,21 +574,9 @@ def run_ours(args, rank, world, device):
         step.run()
     # Per-call device time of pa_decode / pa_chunked_prefill: a graph of N calls, each
     # bracketed by event-record nodes and preceded by an L2 flush.
-    n_kt = 8
-    def timing_graph(kind):
-        evs = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_kt)]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n_kt):
-                l2_flush()
-                if kind == "decode":
-                    step.run_decode(evs[i])
-                else:
-                    step.run_prefill(evs[i])
-        return g, evs
-    g_dec = timing_graph("decode") if dec is not None else None
-    g_pre = timing_graph("prefill") if pre is not None else None
+    n_kt = N_KERNEL_TIMED
+    g_dec = timing_graph(step, "decode", stream, l2_flush) if dec is not None else None
+    g_pre = timing_graph(step, "prefill", stream, l2_flush) if pre is not None else None
     # The pages' indirection comparison: the same decode with identity tables (each
     # sequence's blocks contiguous and in order), when the pool holds every sequence's
     # blocks without sharing.
@@ -559,13 +706,26 @@ def run_ours(args, rank, world, device):
     stages = [staged_step() for _ in range(2)]
     h2d = in_bytes
     d2h = stages[0][2].numel()
+    # uploads and read-backs on two copy streams of their own, so an upload never waits
+    # behind the previous step's read-back
     copy_stream = torch.cuda.Stream(device=device)
+    back_stream = torch.cuda.Stream(device=device)
     ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
     done = [torch.cuda.Event() for _ in range(2)]
     with torch.cuda.stream(stream):  # warm the staged calls once (first-call set-up)
         for dev_in, st, dev_out, host_out in stages:
             dev_in.copy_(host_in, non_blocking=True)
             st.run()
+    torch.cuda.synchronize(device)
+    # each staging buffer's step as a CUDA graph of the same library calls, as an engine
+    # that captures its decode step would run them
+    graphs = []
+    for dev_in, st, dev_out, host_out in stages:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            st.run()
+        graphs.append(g)
     barrier()
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -577,17 +737,26 @@ def run_ours(args, rank, world, device):
             dev_in, st, dev_out, host_out = stages[j]
             with torch.cuda.stream(copy_stream):
                 if i >= 2:
-                    copy_stream.wait_event(done[j])  # step i-2 is done with this buffer
+                    copy_stream.wait_event(computed[j])  # step i-2 has read its inputs
                 dev_in.copy_(host_in, non_blocking=True)
                 ready[j].record(copy_stream)
             stream.wait_event(ready[j])
-            st.run()
-            host_out.copy_(dev_out, non_blocking=True)
-            done[j].record(stream)
+            if i >= 2:
+                stream.wait_event(done[j])  # step i-2's outputs are back on the host
+            graphs[j].replay()
+            computed[j].record(stream)
+            with torch.cuda.stream(back_stream):
+                # the read-back runs beside the next step's compute
+                back_stream.wait_event(computed[j])
+                host_out.copy_(dev_out, non_blocking=True)
+                done[j].record(back_stream)
+        for j in range(min(2, e2e_steps)):
+            stream.wait_event(done[j])
         e1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
     e2e_ms = aggregate_max(e0.elapsed_time(e1), device)
+    del graphs
 
     pool_line = block_pool_timing(pa, dec, stream, device) if dec is not None else None
 
@@ -615,38 +784,15 @@ def run_ours(args, rank, world, device):
     cfg = {"workload": "+".join(b.name for b in batches), "parallelism": "replicas%d" % world,
            "launch": "each step replays one CUDA graph of the library calls",
            "l2": "flushed between timed steps and between timed calls (%.0f MB of KV cache "
-                 "per replica)" % (kv_bytes / 1e6)}
+                 "per replica)" % (kv_bytes / 1e6),
+           "split_k": SPLIT_K}
     if dec is not None:
         cfg.update(num_seqs=dec.num_seqs, q_heads=dec.num_q_heads, kv_heads=dec.num_kv_heads,
                    head_dim=dec.head_dim, block_size=dec.block_size,
                    context_tokens=int(dec.seq_lens.sum().item()))
     line["config"] = cfg
+    line.update(rooflines(step, dec_ms, pre_ms, peaks))
     if dec is not None:
-        ab = decode_algorithmic_bytes(dec)
-        if step.fused[id(dec)]:  # the append inside the launch: read k/v_new, write the slots
-            ab += 2 * 2 * dec.num_seqs * dec.num_kv_heads * dec.head_dim * dec.q.element_size()
-        shared = step.shared[id(dec)]
-        if shared:  # the shared blocks are read once per group
-            ab_unshared = ab
-            ab = decode_algorithmic_bytes(dec, shared=True)
-        dmean = statistics.mean(dec_ms)
-        ach = ab / (dmean / 1e3) / 1e9
-        kname = ("pa_decode_fp8" if dec.k_scale is not None else
-                 "pa_decode_shared_prefix" if shared else
-                 "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
-        kparts = (" (chunked_prefill_kernel prefix pass + paged_decode_kernel + lse_reduce_kernel)"
-                  if shared else " (paged_decode_kernel + lse_reduce_kernel)")
-        line["roofline"] = {"kernel": kname + kparts,
-                            "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
-                            "peak_source": peaks["source"], "unit": "GB/s",
-                            "frac": round(ach / peaks["hbm_gbs"], 4),
-                            "frac_of_8TBs_spec": round(ach / 8000.0, 4),
-                            "algorithmic_bytes": ab, "ms_per_launch": round(dmean, 5),
-                            "traffic": recorded_traffic("paged_decode_kernel", dec.name)}
-        if shared:
-            line["roofline"]["algorithmic_bytes_unshared"] = ab_unshared
-            line["roofline"]["note"] = ("bytes count each shared prefix block once per group; "
-                                        "algorithmic_bytes_unshared counts it once per member")
         if ident_ms:
             im, pm = statistics.mean(ident_ms), statistics.mean(paged_ms)
             line["indirection"] = {"paged_ms": round(pm, 5), "identity_tables_ms": round(im, 5),
@@ -655,47 +801,22 @@ def run_ours(args, rank, world, device):
                                            "sequence's blocks contiguous and in order"}
         line["context_tokens_per_s"] = round(world * int(dec.seq_lens.sum().item()) * args.steps
                                              / (total_ms / 1e3), 1)
-    if pre is not None and step.varlen[id(pre)]:
-        # one call, two kernels in sequence: its speed of light is the decode rows' bytes
-        # at the HBM peak plus the chunks' flops at the tensor peak
-        ql = (pre.query_start_loc[1:] - pre.query_start_loc[:-1]).cpu().numpy()
-        lens = pre.seq_lens.cpu().numpy().astype(np.int64)
-        dec_rows = ql == 1
-        e = pre.q.element_size()
-        dec_bytes = int(lens[dec_rows].sum()) * 2 * pre.num_kv_heads * pre.head_dim * e + \
-            2 * int(dec_rows.sum()) * pre.num_q_heads * pre.head_dim * e + \
-            int(dec_rows.sum()) * int(math.ceil(int(lens.max()) / pre.block_size)) * 4
-        fl = 4 * pre.head_dim * pre.num_q_heads * sum(
-            sum(int(L) - int(n) + i + 1 for i in range(int(n))) for L, n in zip(lens, ql) if n > 1)
-        pmean = statistics.mean(pre_ms)
-        ideal_ms = (dec_bytes / (peaks["hbm_gbs"] * 1e9) + fl / (peaks["bf16_tflops"] * 1e12)) * 1e3
-        line["roofline"] = {"kernel": "pa_attention_varlen (paged_decode_kernel + lse_reduce_kernel"
-                                      " + chunked_prefill_kernel)",
-                            "bound": "hbm (decode rows) then tensor (chunks)",
-                            "achieved": round(ideal_ms / pmean, 4), "peak": 1.0,
-                            "unit": "fraction of the serial speed of light",
-                            "frac": round(ideal_ms / pmean, 4), "ms_per_launch": round(pmean, 5),
-                            "ideal_ms": round(ideal_ms, 5), "decode_bytes": dec_bytes,
-                            "chunk_flop": fl, "peak_source": peaks["source"], "traffic": None}
-    elif pre is not None:
-        fl = prefill_flops(pre)
-        pmean = statistics.mean(pre_ms)
-        tf = fl / (pmean / 1e3) / 1e12
-        peak_tf = peaks["bf16_tflops"]
-        line["roofline_prefill"] = {"kernel": "pa_chunked_prefill (chunked_prefill_kernel, tcgen05)",
-                                    "bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
-                                    "peak_source": peaks["source"] + " bf16 dense burst",
-                                    "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4),
-                                    "flop_per_launch": fl, "ms_per_launch": round(pmean, 5),
-                                    "traffic": None}
     line["e2e"] = {"value": round(world * tokens * e2e_steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                   "note": "eager C-ABI calls; each step's inputs packed in one pinned buffer and "
-                           "uploaded on a copy stream while the previous step computes (two "
-                           "staging buffers); outputs copied back every step"}
+                   "note": "the C-ABI calls of each step replayed as a CUDA graph; each step's "
+                           "inputs packed in one pinned buffer and uploaded on a copy stream "
+                           "while the previous step computes (two staging buffers); outputs "
+                           "copied back to pinned host memory every step on a second copy "
+                           "stream"}
     if pool_line is not None:
         line["block_pool"] = pool_line
     line["clocks"] = clocks.summary()
+    if args.others and args.workload == DEFAULT_WORKLOAD:
+        # the other workloads of the method's configurations, measured in this process
+        del stages
+        torch.cuda.empty_cache()
+        line["other_workloads"] = {
+            n: measure_other(n, args, device, pa, stream, l2_flush, peaks) for n in OTHERS}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the oracle at N = 1 only
         line["cpu_baseline"] = cpu_baseline(batches, args)
     return line
@@ -709,10 +830,12 @@ def cpu_baseline(batches, args, budget_s=None):
     by the pairs of the whole step over the pairs done."""
     import oracle.paged_attention as opa
     try:
-        from threadpoolctl import threadpool_limits
+        from threadpoolctl import threadpool_info, threadpool_limits
+        blas_threads = max([p.get("num_threads", 0) for p in threadpool_info()
+                            if p.get("user_api") == "blas"] or [0])
         limiter = threadpool_limits(1)
     except Exception:  # pragma: no cover
-        limiter = None
+        limiter, blas_threads = None, None
     budget_s = budget_s if budget_s is not None else args.cpu_budget
     units, total_pairs, total_rows = [], 0, 0
     for bi, b in enumerate(batches):
@@ -766,6 +889,8 @@ def cpu_baseline(batches, args, budget_s=None):
     est_step_s = t_used * total_pairs / max(pairs_done, 1)
     value = total_rows / est_step_s
     return {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "host_cores": os.cpu_count(), "blas_threads": blas_threads,
+            "threads_used": "1 (the oracle runs single-threaded: BLAS pool limited to 1)",
             "sample": "%d of %d sequences of %s (%d of %d query-key pairs), oracle time %.1f s "
                       "scaled by query-key pairs to one full step"
                       % (seqs_done, len(units), "+".join(b.name for b in batches), pairs_done,
@@ -797,6 +922,7 @@ def run_reference(args, rank, world):
         "impl": "reference",
         "config": {"workload": "+".join(x.name for x in batches), "parallelism": "replicas%d" % world},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "host_cores": last["host_cores"], "blas_threads": last["blas_threads"],
                          "sample": last["sample"] + "; each step a bounded sample, %.1f s wall" % wall},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -809,11 +935,13 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixed", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-step-budget", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-others", dest="others", action="store_false",
+                    help="skip the other workloads measured beside the default one")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -32,7 +32,11 @@
  *    array of pa_decode_noalloc.  pa_last_launch_count() tells how many kernels the
  *    calling thread's last call launched.
  *  - Return value: PA_OK once the kernels are launched, or an error found on the host
- *    before any launch (nothing is launched then).
+ *    before any launch (nothing is launched then).  PA_ERR_CUDA reports a failed launch
+ *    or tensor-map encoding; a call of two kernels may have queued the first when the
+ *    second fails to launch.  A launching call first clears a non-sticky CUDA error left
+ *    pending on the calling thread by earlier work (cudaGetLastError), so its status
+ *    reports its own launches only.
  *  - Errors that depend on device data (a slot or block id outside the cache, a
  *    sequence longer than its table or than max_seq_len, an inconsistent
  *    query_start_loc) never fault or trap: the kernel skips the offending rows (their
@@ -102,7 +106,8 @@ PA_API pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cach
 
 /*
  * Bytes of scratch `pa_decode` needs, as an upper bound valid for every kv-head count
- * and GPU: merge records (8 bytes per sequence and q-head, padded to 256 bytes), then
+ * and GPU: merge tickets (bounded by 8 bytes per sequence and q-head, padded to 256
+ * bytes), then
  * split-K partial rows of head_dim+2 fp32 (normalised partial output, running max and
  * sum): (256 + num_seqs) * num_q_heads rows, plus, when partition_size > 0,
  * num_seqs * num_q_heads * ceil(ceil(max_seq_len/16) / (partition_size/16)) +
@@ -127,12 +132,16 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   partition_size  0 = balanced split-K: the 16-token tiles of every (sequence, group of
  *                 up to 8 kv-heads) are laid end to end and a persistent grid of one CTA
  *                 per SM takes equal shares; a sequence held by one CTA is written
- *                 directly, the others are merged by a log-sum-exp pass.  > 0 (a
+ *                 directly; the pieces of the others leave normalised partials, and the
+ *                 last piece of each (sequence, kv-head) to finish, found by an atomic
+ *                 ticket, merges them by log-sum-exp inside the same launch.  > 0 (a
  *                 multiple of 16, at most 2048) also caps every share at that many
  *                 tokens, using more CTAs.
  *   workspace     device scratch, 256-byte aligned, of at least
- *                 pa_decode_workspace_size(...) bytes; contents need no initialisation.
- *                 Calls that overlap on the GPU must not share a workspace.
+ *                 pa_decode_workspace_size(...) bytes; contents need no initialisation
+ *                 (a small kernel launched first zeroes the tickets; the decode kernel
+ *                 starts as its programmatic dependent).  Calls that overlap on the GPU
+ *                 must not share a workspace.
  * Limits: head_dim 128, block_size 16 or 32, G = num_q_heads/num_kv_heads in
  * {1, 2, 4, 8}, num_seqs <= 4096 (else PA_ERR_UNSUPPORTED).
  */
@@ -224,16 +233,22 @@ PA_API pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, co
  *                 the same K/V (normally the same physical blocks); they are read through
  *                 the table row of the group's first member
  *   max_group_size, max_prefix_len  host bounds (grid sizing)
- * Three launches: the prefix pass (the tcgen05 prefill kernel with the members' q-heads
- * of one kv-head as the rows of an M-tile, no causal mask, the prefix cut into up to 8
- * pieces that write normalised partial rows), the decode kernel over each sequence's
- * keys after its prefix, and the log-sum-exp merge of both.  Workspace: at least
- * pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len)
- * bytes, 256-byte aligned.  An invalid prefix sets PA_DEVERR_PREFIX (outputs of its
- * group unspecified).  fp16/bf16 caches; other limits as pa_decode (partition_size 0).
- * With num_groups, max_group_size or max_prefix_len 0 it is pa_decode.
+ * Two launches: the ticket zeroing, then one decode grid over a schedule that holds
+ * every sequence's keys after its prefix and, appended to the batch, the "chunks": each
+ * group's members cut into runs of 16 / G, whose q-heads make 16 rows per kv-head, over the
+ * group's prefix (read through the table row of its first member).  A chunk's tiles are
+ * whole blocks, as for any sequence; its consumer warps run the 16 rows as two tensor-core
+ * tiles, so the prefix is read once per chunk (two chunks of one group are scheduled side
+ * by side, and the second read is served by L2).  The last piece of each (member, kv-head)
+ * to finish, own keys or chunk, merges both parts by log-sum-exp.  Workspace: at least
+ * pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+ * max_seq_len) bytes, 256-byte aligned.  An invalid prefix sets PA_DEVERR_PREFIX (outputs
+ * of its group unspecified).  fp16/bf16 caches, num_seqs <= 2048 (else
+ * PA_ERR_UNSUPPORTED); other limits as pa_decode (partition_size 0).  With num_groups,
+ * max_group_size or max_prefix_len 0 it is pa_decode.
  */
-PA_API size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+PA_API size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads,
+                                                     int num_kv_heads, int head_dim,
                                                      int max_seq_len);
 PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
                                          const void* v_cache, const int32_t* block_tables,
@@ -254,9 +269,8 @@ PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k
  * cached), q / out [num_q_rows, num_q_heads, 128].  Sequences with n == 1 run on the
  * decode kernel (reading q and writing out at row query_start_loc[s]), those with n > 1
  * on the tcgen05 prefill kernel; the result of each row is that of pa_chunked_prefill.
- * The call launches both kernels (and their merges) on `stream`: a single launch for
- * both is not built, since each kernel's CTA needs ~200 KB of shared memory and the two
- * could not share an SM.  The decode kernel also lists the sequences with more than one
+ * The call launches both kernels (and their merges) on `stream`.  The decode kernel
+ * also lists the sequences with more than one
  * query row, and the prefill grid covers max_chunk_seqs of them (a host bound on their
  * number, like max_query_len; negative = num_seqs; more chunks than the bound set
  * PA_DEVERR_QUERY_LAYOUT and the extra ones are not computed).  Workspace: at least
@@ -285,10 +299,18 @@ PA_API pa_status pa_attention_varlen(void* out, const void* q, const void* k_cac
  * `ring` int32 [num_blocks] with `state` int32 [2] = {head, count}; the free ids are
  * ring[(head + i) % num_blocks], i < count, the front first.  All arguments are device
  * pointers; each call is one kernel on `stream`.
+ *
+ * Shared blocks ([P2] 4.1, reference-counted blocks; [P1] "KV Cache 的内存开销与分页机制",
+ * blocks shared by sequences of one prompt): `block_refs` int32 [num_blocks] holds the
+ * number of table entries that refer to each block (0 for a free block).  Pass the same
+ * array to every call of a pool, or NULL to every call; without it every block belongs
+ * to exactly one sequence and pa_block_share is unavailable.
  */
 
-/* pa_block_pool_init — ring = 0..num_blocks-1, head = 0, count = num_blocks. */
-PA_API pa_status pa_block_pool_init(int32_t* ring, int32_t* state, int num_blocks, void* stream);
+/* pa_block_pool_init — ring = 0..num_blocks-1, head = 0, count = num_blocks, and
+ * block_refs (if not NULL) all 0. */
+PA_API pa_status pa_block_pool_init(int32_t* ring, int32_t* state, int32_t* block_refs,
+                                    int num_blocks, void* stream);
 
 /*
  * pa_block_allocate — one step of appends.  Sequence s holds seq_lens[s] tokens in
@@ -300,29 +322,54 @@ PA_API pa_status pa_block_pool_init(int32_t* ring, int32_t* state, int num_block
  *                 index order (positions seq_lens[s] .. seq_lens[s]+q_lens[s]-1), -1 for a
  *                 sequence not granted — ready for pa_reshape_and_cache
  *   granted       int32 [num_seqs] out
+ * Each block handed out gets block_refs[b] = 1 (when block_refs is not NULL).
  * seq_lens is not updated (the caller adds q_lens of granted sequences).  Limits:
  * num_seqs <= 4096, block_size 16 or 32.  Device-side errors (PA_DEVERR_POOL, read with
  * pa_get_device_error): a state that is not {0 <= head < num_blocks, 0 <= count <=
  * num_blocks} changes nothing; a sequence with a negative length or a blocks_owned[s]
  * outside [0, max_blocks_per_seq] is not granted.
  */
-PA_API pa_status pa_block_allocate(int32_t* ring, int32_t* state, int num_blocks,
-                                   int32_t* block_tables, int max_blocks_per_seq,
-                                   int32_t* blocks_owned, const int32_t* seq_lens,
-                                   const int32_t* q_lens, int num_seqs, int block_size,
-                                   int32_t* slot_mapping, int32_t* granted, void* stream);
+PA_API pa_status pa_block_allocate(int32_t* ring, int32_t* state, int32_t* block_refs,
+                                   int num_blocks, int32_t* block_tables,
+                                   int max_blocks_per_seq, int32_t* blocks_owned,
+                                   const int32_t* seq_lens, const int32_t* q_lens, int num_seqs,
+                                   int block_size, int32_t* slot_mapping, int32_t* granted,
+                                   void* stream);
 
 /*
- * pa_block_free — every sequence with finished[s] != 0 returns its blocks_owned[s]
- * blocks to the back of the ring (sequences in index order, blocks in table order) and
- * gets blocks_owned[s] = 0.  Returning more blocks than the ring can hold, or a state
- * that is not a pool state, changes nothing and sets PA_DEVERR_POOL.  Limits:
- * num_seqs <= 4096.
+ * pa_block_free — every sequence with finished[s] != 0 releases its blocks_owned[s]
+ * table entries and gets blocks_owned[s] = 0.  Without block_refs each released block
+ * goes to the back of the ring (sequences in index order, blocks in table order).  With
+ * block_refs each entry drops one reference, and a block goes to the back of the ring at
+ * the release that brings its count to zero, in that same order (a block shared by two
+ * finished sequences returns once, at the later one's entry).  Returning more blocks than
+ * the ring can hold, or a state that is not a pool state, leaves ring, state and counts
+ * unchanged and sets PA_DEVERR_POOL; so does a table entry outside [0, num_blocks)
+ * (skipped) or a count that would fall below zero (the block stays out of the ring).
+ * Limits: num_seqs <= 4096.
  */
-PA_API pa_status pa_block_free(int32_t* ring, int32_t* state, int num_blocks,
-                               const int32_t* block_tables, int max_blocks_per_seq,
-                               int32_t* blocks_owned, const int32_t* finished, int num_seqs,
-                               void* stream);
+PA_API pa_status pa_block_free(int32_t* ring, int32_t* state, int32_t* block_refs,
+                               int num_blocks, const int32_t* block_tables,
+                               int max_blocks_per_seq, int32_t* blocks_owned,
+                               const int32_t* finished, int num_seqs, void* stream);
+
+/*
+ * pa_block_share — prompt sharing ([P2] 4.1; [P1] "KV Cache 的内存开销与分页机制": the
+ * sequences sampled from one prompt share its blocks).  For each pair i, sequence
+ * dst_seqs[i], which must own no block, takes the first num_shared[i] blocks of sequence
+ * src_seqs[i]'s table row (blocks_owned[dst] = num_shared[i]); each of those blocks gains
+ * one reference in block_refs (required).  Appends to dst then go to new blocks once the
+ * shared ones are full (share whole blocks: dst's length is num_shared * block_size).
+ *   src_seqs, dst_seqs, num_shared  int32 [num_pairs], sequence indices in [0, num_seqs)
+ * A pair whose dst owns blocks, whose count is negative or above what src owns, whose
+ * src equals dst or lies outside the batch, or whose src row holds an id outside
+ * [0, num_blocks), is skipped and sets PA_DEVERR_POOL.  Pairs are applied in parallel: a
+ * sequence may be dst of one pair only, and no dst may be another pair's src.
+ */
+PA_API pa_status pa_block_share(int32_t* block_refs, int num_blocks, int32_t* block_tables,
+                                int max_blocks_per_seq, int32_t* blocks_owned, int num_seqs,
+                                const int32_t* src_seqs, const int32_t* dst_seqs,
+                                const int32_t* num_shared, int num_pairs, void* stream);
 
 /*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
@@ -330,17 +377,20 @@ PA_API pa_status pa_block_free(int32_t* ring, int32_t* state, int num_blocks,
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that
  * forbids raw cudaMalloc) or who must not risk the device-wide synchronisation an
  * allocation can cause.  Arguments and results are those of pa_decode without the
- * workspace: the merge records and split-K partials go to a fixed array inside the library,
+ * workspace: the merge tickets and split-K partials go to a fixed array inside the library,
  * pa_decode_noalloc_scratch_bytes() long (32 MiB), which every GPU that loads the
  * library holds until the process exits.
  *  - Sizes whose partials need more than that (pa_decode_workspace_size(...) >
  *    pa_decode_noalloc_scratch_bytes()) return PA_ERR_WORKSPACE_TOO_SMALL and launch
  *    nothing.
  *  - The first call on a device looks up that device's array address (with the device
- *    current); make that first call before any stream capture.
+ *    current); make that first call before any stream capture.  The address is kept for
+ *    the life of the process: after cudaDeviceReset, or anything else that destroys the
+ *    device's primary context, do not call this function again in that process.
  *  - Every call on a device shares the one array and leaves its last contents there;
- *    nothing in it needs to start at zero.  Calls that overlap on the GPU (different
- *    streams, no ordering between them) race on the array: order them.
+ *    each call zeroes the part that must start at zero (the merge tickets) itself.
+ *    Calls that overlap on the GPU (different streams, no ordering between them) race
+ *    on the array: order them.
  *  - The call itself allocates no memory.
  */
 PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
@@ -402,6 +452,22 @@ PA_API pa_status pa_get_device_error(void* stream, int32_t* code);
 /* Number of kernel launches the most recent call on this host thread issued (0 when it
  * returned an error before launching).  For launch accounting in benchmarks. */
 PA_API int pa_last_launch_count(void);
+
+/*
+ * pa_testing_wait_fault — testing hook for the bounded pipeline waits (no counterpart
+ * on the pages).  Every wait inside the kernels gives up after a limit (about 2 s of SM
+ * cycles), flags PA_DEVERR_TIMEOUT, stops issuing copies and arrivals, waits (bounded)
+ * for its copies and tensor-core products in flight, frees its tensor memory and exits,
+ * so that a lost arrival can never hang the GPU.  This hook makes the calling thread's
+ * next launch of one kernel withhold one arrival, so the path can be exercised:
+ *   kernel  1: the next paged decode kernel (CTA 0's first K/V tile is never copied nor
+ *              announced); 2: the next chunked-prefill kernel (CTA 0's first K tile);
+ *              0: clear the hook
+ *   wait_limit_cycles  the wait limit of that one launch (> 0), in SM clock cycles
+ * The launch then ends with PA_DEVERR_TIMEOUT set and unspecified outputs; later calls
+ * are unaffected.  One-shot: the hook clears itself when that launch takes it.
+ */
+PA_API pa_status pa_testing_wait_fault(int kernel, long long wait_limit_cycles);
 
 #ifdef __cplusplus
 }

@@ -9,6 +9,9 @@ the id on the back); the scheduler gives a sequence a new block when the blocks 
 for its tokens (integer ceiling of tokens / block size) exceed the blocks it owns, and
 when no block is free that sequence is preempted for this step while later sequences
 are still considered; a finished sequence returns all its blocks to the pool.
+Page "KV Cache管理优化：大模型推理显存瓶颈突破", section 4.1: a block may be shared by
+several sequences (a common prompt) and carries a reference count; releasing a
+reference frees the block only when the count reaches zero.
 
 Readings where the page is silent:
 - a step may append several tokens to a sequence (a prefill chunk); the sequence gets
@@ -16,7 +19,11 @@ Readings where the page is silent:
 - sequences are served in index order; a sequence's blocks are freed in table order,
   sequences in index order;
 - the free queue is a ring of N entries with a head (next id to allocate) and a count;
-- a token at position p of sequence s lands in slot table[s][p // bs] * bs + p % bs.
+- a token at position p of sequence s lands in slot table[s][p // bs] * bs + p % bs;
+- sharing gives a sequence that owns no block the first k blocks of another sequence's
+  table (one more reference each); when finished sequences release their blocks, in
+  the order above, a block returns to the pool at the release that drops its count to
+  zero.
 """
 from __future__ import annotations
 
@@ -37,6 +44,7 @@ class BlockPool:
         self.ring = np.arange(self.n, dtype=np.int64)
         self.head = 0
         self.count = self.n
+        self.refs = np.zeros(self.n, dtype=np.int64)  # references held on each block
 
     def available(self):
         return self.count
@@ -48,6 +56,7 @@ class BlockPool:
         b = int(self.ring[self.head])
         self.head = (self.head + 1) % self.n
         self.count -= 1
+        self.refs[b] = 1
         return b
 
     def free(self, block_id):
@@ -80,11 +89,35 @@ def allocate_step(pool, block_tables, owned, seq_lens, q_lens, block_size):
     return np.asarray(slots, dtype=np.int64), granted
 
 
+def share_blocks(pool, block_tables, owned, src, dst, num_shared):
+    """For each pair i (in order): sequence dst[i], which owns no block, takes the first
+    num_shared[i] blocks of sequence src[i]'s table, each gaining one reference.  A pair
+    whose dst owns blocks, whose count is negative or above what src owns, or whose src
+    is dst, is skipped.  Returns a bool array: the pairs applied."""
+    done = np.zeros(len(src), dtype=bool)
+    for i in range(len(src)):
+        a, b, k = int(src[i]), int(dst[i]), int(num_shared[i])
+        if a == b or owned[b] != 0 or k < 0 or k > owned[a]:
+            continue
+        for j in range(k):
+            blk = int(block_tables[a, j])
+            block_tables[b, j] = blk
+            pool.refs[blk] += 1
+        owned[b] = k
+        done[i] = True
+    return done
+
+
 def free_sequences(pool, block_tables, owned, finished):
-    """Return every block of each finished sequence to the pool (sequences in index
-    order, blocks in table order) and set its owned count to 0."""
+    """Release every block of each finished sequence (sequences in index order, blocks in
+    table order): a block goes back to the pool when its last reference is released.
+    Sets the owned counts of the finished sequences to 0."""
     for s in range(len(owned)):
         if finished[s]:
             for j in range(int(owned[s])):
-                pool.free(int(block_tables[s, j]))
+                b = int(block_tables[s, j])
+                assert pool.refs[b] > 0, "block %d released more often than it was held" % b
+                pool.refs[b] -= 1
+                if pool.refs[b] == 0:
+                    pool.free(b)
             owned[s] = 0

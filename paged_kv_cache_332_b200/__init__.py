@@ -20,11 +20,12 @@ __all__ = [
     "PagedAttnError", "lib", "library_path", "pa_status_string", "pa_reshape_and_cache",
     "pa_decode_workspace_size", "pa_decode", "pa_decode_append", "pa_decode_noalloc",
     "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_block_pool_init", "pa_block_allocate",
-    "pa_block_free", "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
+    "pa_block_free", "pa_block_share", "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
     "pa_attention_varlen_workspace_size", "pa_attention_varlen",
     "pa_decode_noalloc_scratch_bytes",
     "pa_chunked_prefill_workspace_size",
-    "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count", "EXPORTED_SYMBOLS",
+    "pa_chunked_prefill", "pa_get_device_error", "pa_last_launch_count",
+    "pa_testing_wait_fault", "EXPORTED_SYMBOLS",
     "PA_DEVERR",
 ]
 
@@ -50,11 +51,12 @@ _SIGS = [
                                         _i32, _i32, _vp]),
     ("pa_decode_fp8", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
                              _f, _i32, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
-    ("pa_block_pool_init", _i32, [_vp, _vp, _i32, _vp]),
-    ("pa_block_allocate", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _vp, _vp,
-                                 _vp]),
-    ("pa_block_free", _i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
-    ("pa_decode_shared_prefix_workspace_size", _sz, [_i32, _i32, _i32, _i32]),
+    ("pa_block_pool_init", _i32, [_vp, _vp, _vp, _i32, _vp]),
+    ("pa_block_allocate", _i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _vp,
+                                 _vp, _vp]),
+    ("pa_block_free", _i32, [_vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _vp]),
+    ("pa_block_share", _i32, [_vp, _i32, _vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _vp]),
+    ("pa_decode_shared_prefix_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_attention_varlen_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32]),
     ("pa_attention_varlen", _i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32,
                                    _i32, _i32, _i32, _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32,
@@ -70,6 +72,7 @@ _SIGS = [
                                   _i32, _f, _i32, _i32, _i32, _vp, _sz, _i32, _vp]),
     ("pa_get_device_error", _i32, [_vp, ctypes.POINTER(ctypes.c_int32)]),
     ("pa_last_launch_count", _i32, []),
+    ("pa_testing_wait_fault", _i32, [_i32, ctypes.c_longlong]),
 ]
 EXPORTED_SYMBOLS = [n for n, _, _ in _SIGS]
 
@@ -230,17 +233,29 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, seq_
            "pa_decode_fp8")
 
 
-def pa_block_pool_init(ring, state, stream=None):
-    """Fill the device ring (int32 [N]) with 0..N-1 and state (int32 [2]) with {0, N}."""
+def pa_block_pool_init(ring, state, block_refs=None, stream=None):
+    """Fill the device ring (int32 [N]) with 0..N-1, state (int32 [2]) with {0, N} and
+    ``block_refs`` (int32 [N], optional) with zeros."""
     _check(lib().pa_block_pool_init(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                                    _opt_i32(block_refs, "block_refs", ring.numel()),
                                     ring.numel(), _stream(stream)), "pa_block_pool_init")
 
 
+def _opt_i32(t, what, n):
+    if t is None:
+        return None
+    if t.numel() != n:
+        raise ValueError("%s needs %d entries" % (what, n))
+    return _i32tensor(t, what)
+
+
 def pa_block_allocate(ring, state, block_tables, blocks_owned, seq_lens, q_lens, block_size,
-                      slot_mapping, granted, stream=None):
+                      slot_mapping, granted, block_refs=None, stream=None):
     """One step of appends on the device pool: grows ``block_tables``/``blocks_owned`` in
-    place and writes ``slot_mapping`` (int32 [sum q_lens]) and ``granted`` (int32 [B])."""
+    place and writes ``slot_mapping`` (int32 [sum q_lens]) and ``granted`` (int32 [B]);
+    every block handed out gets one reference in ``block_refs`` (optional)."""
     _check(lib().pa_block_allocate(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                                   _opt_i32(block_refs, "block_refs", ring.numel()),
                                    ring.numel(), _i32tensor(block_tables, "block_tables"),
                                    block_tables.shape[1], _i32tensor(blocks_owned, "blocks_owned"),
                                    _i32tensor(seq_lens, "seq_lens"), _i32tensor(q_lens, "q_lens"),
@@ -250,10 +265,13 @@ def pa_block_allocate(ring, state, block_tables, blocks_owned, seq_lens, q_lens,
            "pa_block_allocate")
 
 
-def pa_block_free(ring, state, block_tables, blocks_owned, finished, stream=None):
-    """Return the blocks of every sequence with ``finished[s] != 0`` (int32 [B]) to the
-    back of the device ring."""
+def pa_block_free(ring, state, block_tables, blocks_owned, finished, block_refs=None,
+                  stream=None):
+    """Release the blocks of every sequence with ``finished[s] != 0`` (int32 [B]): each
+    goes to the back of the device ring, or, with ``block_refs``, when its last reference
+    is released."""
     _check(lib().pa_block_free(_i32tensor(ring, "ring"), _i32tensor(state, "state"),
+                               _opt_i32(block_refs, "block_refs", ring.numel()),
                                ring.numel(), _i32tensor(block_tables, "block_tables"),
                                block_tables.shape[1], _i32tensor(blocks_owned, "blocks_owned"),
                                _i32tensor(finished, "finished"), finished.numel(),
@@ -261,9 +279,25 @@ def pa_block_free(ring, state, block_tables, blocks_owned, finished, stream=None
            "pa_block_free")
 
 
-def pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len):
-    return int(lib().pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim,
-                                                            max_seq_len))
+def pa_block_share(block_refs, block_tables, blocks_owned, src_seqs, dst_seqs, num_shared,
+                   stream=None):
+    """Sequence ``dst_seqs[i]`` (owning no block) takes the first ``num_shared[i]`` blocks
+    of sequence ``src_seqs[i]``'s table, one more reference each (int32 [pairs] arrays)."""
+    n = src_seqs.numel()
+    if dst_seqs.numel() != n or num_shared.numel() != n:
+        raise ValueError("src_seqs, dst_seqs and num_shared need one entry per pair")
+    _check(lib().pa_block_share(_i32tensor(block_refs, "block_refs"), block_refs.numel(),
+                                _i32tensor(block_tables, "block_tables"), block_tables.shape[1],
+                                _i32tensor(blocks_owned, "blocks_owned"), blocks_owned.numel(),
+                                _i32tensor(src_seqs, "src_seqs"), _i32tensor(dst_seqs, "dst_seqs"),
+                                _i32tensor(num_shared, "num_shared"), n, _stream(stream)),
+           "pa_block_share")
+
+
+def pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                           max_seq_len):
+    return int(lib().pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                            head_dim, max_seq_len))
 
 
 def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, group_starts,
@@ -324,7 +358,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, m
     """pa_decode for callers that cannot allocate device memory: the split-K
     partials live in a fixed array inside the library
     (:func:`pa_decode_noalloc_scratch_bytes` per device, held until exit), as do
-    the merge records of the split-K pass.
+    the merge tickets of the split-K pass.
     Calls on one device share that array, so calls that overlap on the GPU
     race; make the first call on a device before any stream capture."""
     N, bs, Hkv, D = k_cache.shape
@@ -375,3 +409,11 @@ def pa_get_device_error(stream=None) -> int:
 
 def pa_last_launch_count() -> int:
     return int(lib().pa_last_launch_count())
+
+
+def pa_testing_wait_fault(kernel, wait_limit_cycles=0):
+    """Testing hook: the calling thread's next launch of ``kernel`` ("decode" or
+    "prefill"; None clears) withholds one pipeline arrival and gives every wait
+    ``wait_limit_cycles`` SM cycles, so the bounded-wait path runs (PA_DEVERR_TIMEOUT)."""
+    code = {None: 0, "decode": 1, "prefill": 2}[kernel]
+    _check(lib().pa_testing_wait_fault(code, int(wait_limit_cycles)), "pa_testing_wait_fault")

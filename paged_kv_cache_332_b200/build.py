@@ -54,14 +54,22 @@ def build(force=False, verbose=False, ptxas_verbose=False):
     if not force and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         cmd = [nvcc()] + ARCH + NVFLAGS + extra + ["-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, r
+
+    # the translation units are independent: compile them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(compile_one, sources()))
+    objs = []
+    for src, obj, r in results:
         if r.returncode != 0 or (ptxas_verbose and r.stderr):
             sys.stderr.write(r.stderr)
         if r.returncode != 0:

@@ -22,7 +22,8 @@
 //    a sequence is split only where a share boundary falls inside it.  The piece of a
 //    sequence that a CTA sees is a segment: a sequence held by one CTA is written to
 //    `out` directly; the others leave normalised partials (o, m, l) in the caller's
-//    workspace at slot c + group, merged by a log-sum-exp pass (lse_reduce_kernel).
+//    workspace at slot c + group; the last of them to finish (counted by a per-group
+//    ticket) merges them by log-sum-exp in the same launch.
 //    An explicit partition size caps the share, so no segment is longer.
 //  * One consumer warp per kv-head of the group handles all G q-heads of that kv-head,
 //    so no two warps share an output.  q.k: 8 lanes split a token's 128 dims (16 each,
@@ -40,9 +41,12 @@
 //    walks the tiles in order and issues the two boxes of each as soon as a slot of the
 //    shared ring frees (blocking waits take no issue slots from the consumers).
 // Two more modes share the kernel:
-//  * shared prefixes (pa_decode_shared_prefix): a sequence whose first tokens are shared
-//    with its group reads only its tiles after the prefix; the prefix pass (prefill.cu)
-//    left the attention over the prefix as partials, and the merge folds them in;
+//  * shared prefixes (pa_decode_shared_prefix; page "KV Cache管理优化：大模型推理显存瓶颈
+//    突破" 4.1, blocks shared by reference): a sequence whose first tokens are shared with
+//    its group reads only its tiles after the prefix; the group's members are cut into
+//    chunks of 16 q-rows per kv-head (16/G members), and each chunk is one more sequence of
+//    the schedule over the prefix, whose consumer warps run its rows as two tensor-core n8
+//    tiles; the tickets merge each member's own pieces with its chunk's;
 //  * varlen rows (pa_attention_varlen): only sequences with one query row are served,
 //    q and out rows come from query_start_loc, and CTA 0 lists the other sequences for
 //    the prefill kernel that follows.
@@ -61,11 +65,16 @@ namespace pa {
 
 struct DecodeArgs {
   void* out;
+  const void* q;   // [rows, Hq, 128] (read directly only by the shared-prefix chunk rows)
   const int32_t* block_tables;
   const int32_t* seq_lens;
   float* part_o;   // [slots, HB*G, 128]   normalised partial outputs
   float* part_ml;  // [slots, HB*G, 2]     (max in log2 units, sum)
-  int2* meta;      // [B * NHP]            (first slot, slot count) of each group
+  // merge tickets, [B * Hkv]: one per (sequence, kv-head), zeroed by the launch before
+  // this one (zero_tickets_kernel).  Every piece of a split (sequence, kv-head) adds to it:
+  // its first piece the balance kTicketTotal - (pieces - 1), the others 1; the warp whose
+  // addition completes kTicketTotal merges that kv-head's q-heads
+  unsigned* tickets;
   // append in the same launch (k_new != nullptr): the step's new token of each sequence,
   // [B, Hkv, 128], written into its cache slot at position seq_len-1 before it is read
   const void* k_new;
@@ -76,15 +85,18 @@ struct DecodeArgs {
   const float* k_scale;
   const float* v_scale;
   // shared-prefix decode (num_groups > 0): sequences [group_starts[g], group_starts[g+1])
-  // share their first prefix_lens[g] tokens.  The prefix pass left the attention of every
-  // member's q-heads over those tokens in pre_o / pre_ml ([pre_chunks][B * Hq rows],
-  // normalised rows and (max in log2 units, sum)); this launch reads only the keys after
-  // a sequence's prefix and the merge folds both parts together.
+  // share their first prefix_lens[g] tokens (whole blocks).  A sequence reads only its keys
+  // after the prefix.  The members of a group with a prefix are cut into chunks of `mc`
+  // members (16 rows per kv-head: mc * G); each chunk is a virtual sequence appended to the
+  // batch (indices num_seqs ..): prefix_lens[g] tokens read through the table row of the
+  // group's first member, its queries the chunk's members' q-heads, its normalised
+  // partial rows in vpart_o / vpart_ml ([slots, HB*16, 128] / [slots, HB*16, 2]).
   const int32_t* group_starts;
   const int32_t* prefix_lens;
-  const float* pre_o;
-  const float* pre_ml;
-  int num_groups, pre_chunks;
+  float* vpart_o;
+  float* vpart_ml;
+  int num_groups, mc, vcap;  // groups, members per chunk, bound on the chunks
+  int max_prefix;            // host bound on prefix_lens (a longer prefix is flagged)
   // varlen batch (qsl != nullptr): only sequences with one query row (qsl[s+1]-qsl[s] == 1)
   // are served here, reading q and writing out at row qsl[s] of num_q_rows
   const int32_t* qsl;
@@ -98,6 +110,8 @@ struct DecodeArgs {
   int seq_cap;
   int ring_off, nslots;  // shared-memory offset of the tile ring and its slot count
   float qscale;          // scale * log2(e)
+  long long wait_limit;  // SM cycles any pipeline wait may take before the CTA gives up
+  int test_withhold;     // testing hook: CTA 0's producer withholds its first tile
 };
 
 constexpr int kD = 128;
@@ -111,13 +125,23 @@ constexpr int kMaxGrid = 256;          // persistent grid: min(SMs, this)
 constexpr int kFirst = 1;   // first unit of a segment: load q, reset the softmax state
 constexpr int kLast = 2;    // last unit of a segment: write the result
 constexpr int kDirect = 4;  // the segment is the whole group: write `out`
+constexpr int kVirtual = 8;  // a chunk of a group's members over their shared prefix
+// a staged unit: [0] sequence (-1: no more work; >= num_seqs: a chunk), [1] head group,
+// [2..3] tiles [t0, t1), [4] flags, [5] partial slot of this segment, [6] append, [7] q /
+// out row (a chunk: its first member), [8] first slot of the group's segments, [9] segment
+// count, [10] members of a chunk
+constexpr int kUnitInts = 16;
+constexpr int kChunkRows = 16;           // q rows of a chunk per kv-head (members x G)
+constexpr unsigned kTicketTotal = 1u << 30;  // a merge ticket's count when every piece is in
 
-template <int G_, int HB_, bool F8_>
+template <int G_, int HB_, bool F8_, bool SP_ = false>
 struct DecodeCfg {
   static constexpr int G = G_;
   static constexpr int HB = HB_;                  // kv-heads per group = consumer warps
   static constexpr bool F8 = F8_;                 // e4m3 cache (else fp16/bf16)
-  static constexpr bool MMA = F8 || G == 8;       // tensor-core consumers
+  // tensor-core consumers: G = 8, an FP8 cache, and beside the chunk consumer of shared
+  // prefixes (which leaves no registers for the CUDA-core path's q in registers)
+  static constexpr bool MMA = F8 || G == 8 || SP_;
   static constexpr int KROW = kD * (F8 ? 1 : 2);  // one token of one kv-head in the cache
   static constexpr int GW = G;                    // q-heads per consumer warp
   static constexpr int WARP_PROD = 0;
@@ -137,8 +161,8 @@ struct DecodeCfg {
   static constexpr int OFF_TFULL = OFF_QEMPTY + kQSlots * 8;
   static constexpr int OFF_TEMPTY = OFF_TFULL + kQSlots * 8;
   static constexpr int OFF_ADONE = OFF_TEMPTY + kQSlots * 8;    // append of a unit written
-  static constexpr int OFF_UNIT = OFF_ADONE + kQSlots * 8;      // 8 ints per staged unit
-  static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 32;
+  static constexpr int OFF_UNIT = OFF_ADONE + kQSlots * 8;      // 16 ints per staged unit
+  static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 64;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
   static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerUnit * 4;
   // p pairs and alpha per warp (CUDA-core path only; the G = 8 path keeps them in
@@ -152,26 +176,44 @@ struct DecodeCfg {
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
 
-// merge records: (first slot, slot count | kHasPrefix when prefix partials join the merge)
-constexpr int kHasPrefix = 1 << 30;
 
-// Shared-prefix length of sequence s: prefix_lens[g] of the group holding s (the last g
-// with group_starts[g] <= s, if s < group_starts[g+1]), else 0.
-__device__ __forceinline__ int shared_prefix_of(const DecodeArgs& a, int s) {
-  if (a.num_groups <= 0 || s < __ldg(a.group_starts)) return 0;
+// Group holding sequence s: the last g with group_starts[g] <= s, if s < group_starts[g+1];
+// else -1.
+__device__ __forceinline__ int group_of(const DecodeArgs& a, int s) {
+  if (a.num_groups <= 0 || s < __ldg(a.group_starts)) return -1;
   int lo = 0, hi = a.num_groups - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (__ldg(a.group_starts + mid) <= s) lo = mid; else hi = mid - 1;
   }
-  return s < __ldg(a.group_starts + lo + 1) ? __ldg(a.prefix_lens + lo) : 0;
+  return s < __ldg(a.group_starts + lo + 1) ? lo : -1;
 }
 
-// Bounded wait that turns into a no-op once any warp of the CTA gave up.
+// Bounded wait that turns into a no-op once any warp of the CTA gave up (and stops
+// waiting as soon as one does).  After a wait that may have been skipped, a warp makes no
+// further arrival on a barrier that counts transaction bytes: its previous phase may still
+// be pending.
 __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag, int* err) {
-  if (*abort_flag) return;
-  if (!mbar_wait(bar, parity, err)) *abort_flag = 1;
+                                              volatile int* abort_flag, int* err,
+                                              long long limit) {
+  if (*abort_flag || mbar_try_wait(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return;
+    if (clock64() - t0 > limit) {
+      flag_error(err, PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+  }
+}
+
+// After an abort: wait (bounded, ignoring the abort flag) for the phase of `bar` that the
+// calling thread's last copy into a buffer completes, so that no bulk copy is still
+// writing the CTA's shared memory when it exits.
+__device__ __forceinline__ void drain_copy(uint64_t* bar, uint32_t parity, int* err,
+                                           long long limit) {
+  (void)mbar_wait(bar, parity, err, limit);
 }
 
 // Sum per-lane partial dot products over each 8-lane token group for GW heads at
@@ -285,12 +327,191 @@ __device__ __forceinline__ int cta_of(int pos, int T, int grid) {
   return (int)((((long long)pos + 1) * grid - 1) / T);
 }
 
-template <typename T, int G, int HB, bool F8>
-__global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
+// The schedule every CTA computes in its prologue: the sequences (the batch, then the
+// chunks of shared prefixes) with their tiles laid end to end; the first tile of each, its
+// clamped length, its first tile after a shared prefix (-1: not served), the chunk
+// numbering of the groups, and the grid that shares the tiles out.
+struct Sched {
+  const int* sstart;
+  const int* slen;
+  const int* sfirst;
+  const int* cstart;
+  int B, V, NHP, Ttot, grid;
+};
+
+// Segments of sequence s's head group hp (its keys after any prefix): first slot, count.
+__device__ __forceinline__ void own_pieces(const Sched& sc, int s, int hp, int& so0, int& no) {
+  so0 = no = 0;
+  const int cnt = sc.sfirst[s] < 0 ? 0 : cdiv(sc.slen[s], kTileTok) - sc.sfirst[s];
+  if (cnt <= 0) return;
+  const int gs = sc.sstart[s] + hp * cnt;
+  const int c0 = cta_of(gs, sc.Ttot, sc.grid), c1 = cta_of(gs + cnt - 1, sc.Ttot, sc.grid);
+  so0 = c0 + s * sc.NHP + hp;
+  no = c1 - c0 + 1;
+}
+
+// Segments of the chunk that holds member s, over its group's prefix (head group hp):
+// first slot, count, and the member's first row within the chunk's rows of a kv-head
+// (nv = 0 when s shares no prefix).
+template <int G>
+__device__ __forceinline__ void chunk_pieces(const DecodeArgs& a, const Sched& sc, int s, int hp,
+                                             int& sv0, int& nv, int& vrow) {
+  sv0 = nv = vrow = 0;
+  const int g = group_of(a, s);
+  if (g < 0 || __ldg(a.prefix_lens + g) <= 0) return;
+  const int off = s - __ldg(a.group_starts + g);
+  const int vs = sc.cstart[g] + off / a.mc;
+  if (vs >= sc.V) return;
+  const int vi = sc.B + vs;
+  const int cnt = cdiv(sc.slen[vi], kTileTok);
+  if (cnt <= 0) return;
+  const int gs = sc.sstart[vi] + hp * cnt;
+  const int c0 = cta_of(gs, sc.Ttot, sc.grid), c1 = cta_of(gs + cnt - 1, sc.Ttot, sc.grid);
+  sv0 = c0 + vs * sc.NHP + hp;
+  nv = c1 - c0 + 1;
+  vrow = (off % a.mc) * G;
+}
+
+// Log-sum-exp merge of one kv-head's G q-heads of one sequence over its pieces: its own
+// segments (partial rows in slots so0 .. so0+no-1) and the segments of the chunk that
+// holds it over a shared prefix (slots sv0 .. sv0+nv-1, rows vrow + j of the kv-head's 16).
+// o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the largest m_i.  One warp:
+// 32/G lanes per q-head, 4*G dims per lane; the rows are folded in rounds whose loads are
+// all in flight together, with a running maximum.  Reads go to L2 (other SMs wrote them).
+template <typename T, int G, int HB, bool SP>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs& a, int orow, int kvh, int so0,
+                                             int no, int sv0, int nv, int vrow, int lane) {
+  constexpr int HBG = HB * G;
+  constexpr int VROWS = HB * kChunkRows;  // rows of a chunk slot
+  constexpr int LPH = 32 / G;             // lanes per q-head
+  constexpr int NV = G;                   // float4 per lane and row
+  // rows per round: 8 float4 loads in flight; one row beside the chunk consumer, whose
+  // registers leave no room for more
+  constexpr int R = SP ? 1 : (G >= 2 ? 8 / G : 8);
+  const int jj = lane / LPH;
+  const int d0 = (lane % LPH) * 4 * G;
+  const int qh = kvh * G + jj;            // q-head
+  const int j = qh % HBG;                 // its row within a slot of the sequence
+  const int jv = (kvh % HB) * kChunkRows + vrow + jj;  // its row within a chunk slot
+  float M = -INFINITY, den = 0.f;
+  float4 num[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) num[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int total = no + nv;
+  for (int i0 = 0; i0 < total; i0 += R) {
+    float2 ml[R];
+    float4 ov[R][NV];
+    float Mr = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      const int i = i0 + u;
+      if (i < total) {
+        const bool own = i < no;
+        const long long row =
+            own ? (long long)(so0 + i) * HBG + j : (long long)(sv0 + i - no) * VROWS + jv;
+        const float* po = (own ? a.part_o : a.vpart_o) + row * kD + d0;
+        ml[u] = __ldcg(reinterpret_cast<const float2*>((own ? a.part_ml : a.vpart_ml) + row * 2));
+#pragma unroll
+        for (int v = 0; v < NV; ++v) ov[u][v] = __ldcg(reinterpret_cast<const float4*>(po) + v);
+        Mr = fmaxf(Mr, ml[u].x);
+      }
+    }
+    const float Mn = fmaxf(M, Mr);
+    if (Mn == -INFINITY) continue;  // only empty pieces so far
+    const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
+    den *= sc;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      num[v].x *= sc; num[v].y *= sc; num[v].z *= sc; num[v].w *= sc;
+    }
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      if (i0 + u < total) {
+        const float f = ml[u].x == -INFINITY ? 0.f : fast_exp2(ml[u].x - Mn) * ml[u].y;
+        den += f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          num[v].x += f * ov[u][v].x; num[v].y += f * ov[u][v].y;
+          num[v].z += f * ov[u][v].z; num[v].w += f * ov[u][v].w;
+        }
+      }
+    }
+    M = Mn;
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  T* ob = static_cast<T*>(a.out) + ((long long)orow * a.num_q_heads + qh) * kD + d0;
+#pragma unroll
+  for (int v = 0; v < NV; ++v)
+    reinterpret_cast<uint2*>(ob)[v] = make_uint2(Elem<T>::pack2(num[v].x * inv, num[v].y * inv),
+                                                 Elem<T>::pack2(num[v].z * inv, num[v].w * inv));
+}
+
+// End of one of sequence s's own segments that is not the whole (sequence, head group):
+// this warp's partial rows (kv-head kvh) are written.  Its ticket counts the pieces that are
+// done; the warp whose addition completes kTicketTotal merges.  No warp waits for another
+// CTA.  With a shared prefix, the chunk's first segment adds the balance (finish_chunk).
+template <typename T, int G, int HB, bool SP>
+__device__ __forceinline__ void finish_own(const DecodeArgs& a, const Sched& sc, int s, int orow,
+                                           int hp, int kvh, int pslot, int slot0, int nseg,
+                                           int lane) {
+  __threadfence();  // this lane's partial rows are visible GPU-wide before the ticket
+  __syncwarp();
+  griddep_wait();   // the tickets were zeroed by the launch before this one
+  int sv0 = 0, nv = 0, vrow = 0;
+  if constexpr (SP) chunk_pieces<G>(a, sc, s, hp, sv0, nv, vrow);
+  const unsigned add = (nv == 0 && pslot == slot0) ? kTicketTotal - (unsigned)(nseg - 1) : 1u;
+  unsigned old = 0;
+  if (lane == 0) old = atomic_add_acq_rel_gpu(a.tickets + (long long)s * a.num_kv_heads + kvh, add);
+  if (__shfl_sync(0xffffffffu, old, 0) + add != kTicketTotal) return;
+  __threadfence();
+  merge_pieces<T, G, HB, SP>(a, orow, kvh, slot0, nseg, sv0, nv, vrow, lane);
+}
+
+// End of a chunk segment (members m0 .. m0+nm-1 over their shared prefix, kv-head kvh):
+// one ticket arrival per member (lane i for member m0+i), the chunk's first segment adding
+// each member's balance; the members whose count completes are merged one after another.
+template <typename T, int G, int HB>
+__device__ __forceinline__ void finish_chunk(const DecodeArgs& a, const Sched& sc, int m0, int nm,
+                                             int hp, int kvh, int pslot, int slot0, int nseg,
+                                             int lane) {
+  __threadfence();
+  __syncwarp();
+  griddep_wait();
+  bool last = false;
+  if (lane < nm) {
+    const int sm = m0 + lane;
+    int so0, no;
+    own_pieces(sc, sm, hp, so0, no);
+    const unsigned add = pslot == slot0 ? kTicketTotal - (unsigned)(no + nseg - 1) : 1u;
+    const unsigned old =
+        atomic_add_acq_rel_gpu(a.tickets + (long long)sm * a.num_kv_heads + kvh, add);
+    last = old + add == kTicketTotal;
+  }
+  unsigned mask = __ballot_sync(0xffffffffu, last);
+  if (mask) __threadfence();
+  while (mask) {
+    const int i = __ffs(mask) - 1;
+    mask &= mask - 1;
+    int so0, no;
+    own_pieces(sc, m0 + i, hp, so0, no);
+    merge_pieces<T, G, HB, true>(a, m0 + i, kvh, so0, no, slot0, nseg, i * G, lane);
+  }
+}
+
+// Zero the merge tickets of a decode launch; that launch follows as a programmatic
+// dependent and waits for this grid before its first ticket.
+__global__ void __launch_bounds__(256) zero_tickets_kernel(unsigned* tickets, int n) {
+  griddep_launch_dependents();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    tickets[i] = 0;
+}
+
+template <typename T, int G, int HB, bool F8, bool SP>
+__global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
-  using C = DecodeCfg<G, HB, F8>;
+  using C = DecodeCfg<G, HB, F8, SP>;
   constexpr int GW = C::GW;
   constexpr int HBG = HB * G;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -308,43 +529,90 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
   float* abuf = reinterpret_cast<float*>(smem + C::OFF_A);
   const int B = a.num_seqs;
-  int* sstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);  // [B+1] first tile of each sequence
-  int* slen = sstart + B + 1;                                // [B]   clamped lengths
-  int* sfirst = slen + B;  // [B] first tile after the shared prefix (0 without one)
+  const int VC = SP ? a.vcap : 0;  // room for chunk sequences after the batch
+  int* sstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);  // [B+VC+1] first tile of each sequence
+  int* slen = sstart + B + VC + 1;                           // [B+VC] clamped lengths
+  int* sfirst = slen + B + VC;  // [B+VC] first tile after a shared prefix (0 without; -1 not served)
+  int* cstart = sfirst + B + VC;  // [groups+1] first chunk of each group
+  volatile int* nchunks = abort_flag + 1;  // chunks in the schedule (<= VC)
   uint8_t* ring = smem + a.ring_off;
   const int nslots = a.nslots;
   const int NHP = a.num_kv_heads / HB;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // the merge pass may be scheduled now; it waits for this grid's results itself
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- clamped lengths and the prefix of tiles over (sequence, head group)
   if (warp == 0) {
-    const int per = (B + 31) / 32;
-    const int lo = min(B, lane * per), hi = min(B, lo + per);
+    int V = 0;
+    if constexpr (SP) {
+      // the members of a group with a shared prefix, cut into chunks of a.mc: the chunk
+      // count of each group and their exclusive prefix sum
+      const int ng = a.num_groups;
+      const int gper = (ng + 31) / 32;
+      const int glo = min(ng, lane * gper), ghi = min(ng, glo + gper);
+      auto chunks_of = [&](int g) {
+        const int n = __ldg(a.group_starts + g + 1) - __ldg(a.group_starts + g);
+        return (n > 0 && __ldg(a.prefix_lens + g) > 0) ? cdiv(n, a.mc) : 0;
+      };
+      int csum = 0;
+      for (int g = glo; g < ghi; ++g) csum += chunks_of(g);
+      int cincl = csum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, cincl, o);
+        if (lane >= o) cincl += t;
+      }
+      int crun = cincl - csum;
+      for (int g = glo; g < ghi; ++g) {
+        cstart[g] = crun;
+        crun += chunks_of(g);
+      }
+      const int total = __shfl_sync(0xffffffffu, cincl, 31);
+      if (lane == 0) {
+        cstart[ng] = total;
+        if (total > VC && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_PREFIX);
+      }
+      V = min(total, VC);
+      __syncwarp();
+    }
+    const int NS = B + V;  // the batch, then the chunks
+    const int per = (NS + 31) / 32;
+    const int lo = min(NS, lane * per), hi = min(NS, lo + per);
     int sum = 0;
     for (int s = lo; s < hi; ++s) {
-      const int raw = a.seq_lens[s];
-      const int L = clamp_len(raw, a.seq_cap);
-      if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
-      slen[s] = L;
-      int first = 0;
-      if (a.qsl != nullptr) {  // varlen: decode rows only; the others are prefill chunks
-        const int q0 = __ldg(a.qsl + s), nq = __ldg(a.qsl + s + 1) - q0;
-        if (nq != 1) first = -1;
-        else if (q0 < 0 || q0 >= a.num_q_rows) {
-          if (blockIdx.x == 0) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
-          first = -1;
+      int L, first = 0;
+      if (SP && s >= B) {
+        // chunk s-B: its group's prefix, read through the group's first member's table row
+        const int vs = s - B;
+        int glo2 = 0, ghi2 = a.num_groups - 1;  // the last g with cstart[g] <= vs
+        while (glo2 < ghi2) {
+          const int mid = (glo2 + ghi2 + 1) >> 1;
+          if (cstart[mid] <= vs) glo2 = mid; else ghi2 = mid - 1;
+        }
+        L = clamp_len(__ldg(a.prefix_lens + glo2), min(a.seq_cap, a.max_prefix));
+      } else {
+        const int raw = a.seq_lens[s];
+        L = clamp_len(raw, a.seq_cap);
+        if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
+        if (a.qsl != nullptr) {  // varlen: decode rows only; the others are prefill chunks
+          const int q0 = __ldg(a.qsl + s), nq = __ldg(a.qsl + s + 1) - q0;
+          if (nq != 1) first = -1;
+          else if (q0 < 0 || q0 >= a.num_q_rows) {
+            if (blockIdx.x == 0) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
+            first = -1;
+          }
+        }
+        if (SP && first == 0) {
+          const int g = group_of(a, s);
+          const int p = g < 0 ? 0 : __ldg(a.prefix_lens + g);
+          if ((p < 0 || p > L || p > a.max_prefix || (p & ((1 << a.log2_bs) - 1))) &&
+              blockIdx.x == 0)
+            flag_error(a.err, PA_DEVERR_PREFIX);
+          first = clamp_len(p, L) / kTileTok;
         }
       }
-      if (first == 0 && a.num_groups > 0) {
-        const int p = shared_prefix_of(a, s);
-        if ((p < 0 || p > L || (p & ((1 << a.log2_bs) - 1))) && blockIdx.x == 0)
-          flag_error(a.err, PA_DEVERR_PREFIX);
-        first = clamp_len(p, L) / kTileTok;
-      }
+      slen[s] = L;
       sfirst[s] = first;
       sum += first < 0 ? 0 : NHP * (cdiv(L, kTileTok) - first);
     }
@@ -359,7 +627,10 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       sstart[s] = run;
       run += sfirst[s] < 0 ? 0 : NHP * (cdiv(slen[s], kTileTok) - sfirst[s]);
     }
-    if (lane == 31) sstart[B] = incl;
+    if (lane == 31) {
+      sstart[NS] = incl;
+      *nchunks = V;
+    }
     if (a.chunk_ids != nullptr && blockIdx.x == 0) {
       int c = 0;
       for (int s = lo; s < hi; ++s) c += (__ldg(a.qsl + s + 1) - __ldg(a.qsl + s)) > 1;
@@ -397,7 +668,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  const int Ttot = sstart[B];
+  const int V = *nchunks;
+  const int NS = B + V;
+  const int Ttot = sstart[NS];
   // The launch sizes the grid for the longest possible batch; when the batch holds
   // fewer tiles than CTAs, only the first Ttot CTAs take a share, so every share is
   // non-empty and the segments of a group sit in consecutive CTAs (and slots).
@@ -405,21 +678,28 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
   const int cta = blockIdx.x;
   const int r0 = cta < grid ? (int)(((long long)cta * Ttot) / grid) : Ttot;
   const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
+  // the schedule, rebuilt from shared memory where a segment end needs it (so that it
+  // holds no registers through the tile loops)
+  auto sched = [&]() -> Sched {
+    const volatile int* nc = nchunks;
+    const int v = SP ? *nc : 0;
+    const int tt = sstart[B + v];
+    return Sched{sstart, slen, sfirst, cstart, B, v, NHP, tt, min((int)gridDim.x, max(tt, 1))};
+  };
 
   if (warp < C::WARP_C0) {
     if (warp == C::WARP_FILL) {
-      // ===== empty sequences: no CTA visits them; zero their output and merge record =====
+      // ===== sequences without keys of their own: no CTA's share visits them =====
       for (int s = cta; s < B; s += gridDim.x) {
-        if (sfirst[s] < 0) {  // not served by this kernel: no merge, no output
-          for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
-          continue;
-        }
+        if (sfirst[s] < 0) continue;  // not served by this kernel
         if (cdiv(slen[s], kTileTok) != sfirst[s]) continue;
-        // no keys of its own: a sequence with a shared prefix takes the prefix part alone
-        const int pre = sfirst[s] > 0 ? kHasPrefix : 0;
-        for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, pre);
-        if (pre) continue;
         const int orow = a.qsl ? __ldg(a.qsl + s) : s;
+        if constexpr (SP) {
+          // all its keys are shared: its chunk's segments merge its output
+          int sv0, nv, vrow;
+          chunk_pieces<G>(a, sched(), s, 0, sv0, nv, vrow);
+          if (nv > 0) continue;
+        }
         T* ob = static_cast<T*>(a.out) + (long long)orow * a.num_q_heads * kD;
         for (int i = lane; i < a.num_q_heads * kD / 8; i += 32)
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -432,25 +712,37 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
       int pos = r0;
       int s = 0;
       if (pos < r1) {  // sequence holding pos: the last s with sstart[s] <= pos
-        int lo = 0, hi = B - 1;
+        int lo = 0, hi = NS - 1;
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
           if (sstart[mid] <= pos) lo = mid; else hi = mid - 1;
         }
         s = lo;
       }
+      uint32_t q_issued = 0;  // bit i: unit k-1-i copied q rows (as the producer's mask)
       for (int k = 0;; ++k) {
         const int qs = k % kQSlots;
         const uint32_t par = ((k / kQSlots) & 1) ^ 1;
-        wait_or_abort(&qempty[qs], par, abort_flag, a.err);  // consumers read unit k-2's q
-        wait_or_abort(&tempty[qs], par, abort_flag, a.err);  // its tiles were issued
-        volatile int* u = unit + qs * 8;
-        if (pos >= r1 || *abort_flag) {  // tell the other warps there is no more work
-          if (lane == 0) {
-            u[0] = -1;
-            mbar_arrive_expect_tx(&qfull[qs], 0);
-            mbar_arrive(&tfull[qs]);
-          }
+        wait_or_abort(&qempty[qs], par, abort_flag, a.err, a.wait_limit);  // consumers read unit k-2's q
+        wait_or_abort(&tempty[qs], par, abort_flag, a.err, a.wait_limit);  // its tiles were issued
+        volatile int* u = unit + qs * kUnitInts;
+        // after an abort a wait may have been skipped: no more arrivals
+        const bool stop = warp_flag(abort_flag);
+        if (!stop && pos >= r1 && lane == 0) {  // tell the other warps there is no more work
+          u[0] = -1;
+          mbar_arrive_expect_tx(&qfull[qs], 0);
+          mbar_arrive(&tfull[qs]);
+        }
+        if (stop || pos >= r1) {
+          // no q copy may still be landing when the CTA exits (a no-op unless the consumers
+          // abort): units k-1 and k-2 after an abort; only k-1 after the arrival above,
+          // which completed the phase after unit k-2's in the same slot
+          if (lane == 0)
+            for (int i = 0; i < (stop ? kQSlots : 1) && i < k; ++i)
+              if (q_issued & (1u << i)) {
+                const int c = k - 1 - i;
+                drain_copy(&qfull[c % kQSlots], (c / kQSlots) & 1, a.err, a.wait_limit);
+              }
           break;
         }
         const int nt = cdiv(slen[s], kTileTok);
@@ -460,21 +752,38 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
         const int hp = off / cnt;
         const int t0 = ts + off - hp * cnt;
         const int t1 = min(nt, t0 + min(r1 - pos, kMaxTilesPerUnit));
-        const int grp = s * NHP + hp;
         const int gs = sstart[s] + hp * cnt;  // the group's first and one-past-last tile
         const int ge = gs + cnt;
-        int flags = 0;
+        // a chunk (s >= B): members m0 .. m0+nm-1 of group g over its prefix, read through
+        // the table row of the group's first member; its slots are numbered apart
+        const bool virt = SP && s >= B;
+        int m0 = 0, nm = 0, trow_seq = s;
+        if (virt) {
+          const int vs = s - B;
+          int glo = 0, ghi = a.num_groups - 1;  // the last g with cstart[g] <= vs
+          while (glo < ghi) {
+            const int mid = (glo + ghi + 1) >> 1;
+            if (cstart[mid] <= vs) glo = mid; else ghi = mid - 1;
+          }
+          trow_seq = __ldg(a.group_starts + glo);
+          m0 = trow_seq + (vs - cstart[glo]) * a.mc;
+          nm = min(a.mc, __ldg(a.group_starts + glo + 1) - m0);
+        }
+        const int grp = (virt ? s - B : s) * NHP + hp;
+        int flags = virt ? kVirtual : 0;
         if (t0 == ts || pos == r0) flags |= kFirst;
         if (t1 == nt || pos + (t1 - t0) == r1) flags |= kLast;
-        if (gs >= r0 && ge <= r1 && ts == 0) flags |= kDirect;
-        const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
+        if (gs >= r0 && ge <= r1 && ts == 0 && !virt) flags |= kDirect;
+        // the group's segments sit in CTAs c0..c1, their partials in slots c0+grp..c1+grp
+        const int c0 = cta_of(gs, Ttot, grid), c1 = cta_of(ge - 1, Ttot, grid);
+        const int32_t* trow = a.block_tables + (long long)trow_seq * a.max_blocks;
         int ids[kMaxTilesPerUnit / 32];
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < kMaxTilesPerUnit / 32; ++j) {
           const int t = t0 + j * 32 + lane;
           ids[j] = t < t1 ? __ldg(trow + ((t * kTileTok) >> a.log2_bs)) : -1;
         }
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < kMaxTilesPerUnit / 32; ++j) {
           const int i = j * 32 + lane;
           if (t0 + i < t1) {
@@ -496,7 +805,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
         uint4* kd = nullptr;
         uint4* vd = nullptr;
         bool append = false;
-        if (a.k_new != nullptr && t1 == nt) {
+        if (a.k_new != nullptr && t1 == nt && !virt) {
           const int raw = __ldg(a.seq_lens + s);
           const int bid = tbl[qs * kMaxTilesPerUnit + (t1 - 1 - t0)];
           if (raw == slen[s] && bid >= 0) {
@@ -517,9 +826,6 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           }
         }
         if (lane == 0) {
-          if (t0 == ts)
-            a.meta[grp] = make_int2(cta + grp, (cta_of(ge - 1, Ttot, grid) - cta + 1) |
-                                                   (ts > 0 ? kHasPrefix : 0));
           u[0] = s;
           u[1] = hp;
           u[2] = t0;
@@ -527,10 +833,15 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           u[4] = flags;
           u[5] = cta + grp;
           u[6] = append ? 1 : 0;
-          u[7] = a.qsl ? __ldg(a.qsl + s) : s;  // q / out row
-          if (flags & kFirst) {
+          u[7] = virt ? m0 : (a.qsl ? __ldg(a.qsl + s) : s);  // q / out row
+          u[8] = c0 + grp;
+          u[9] = c1 - c0 + 1;
+          u[10] = nm;
+          q_issued <<= 1;
+          if ((flags & kFirst) && !virt) {  // a chunk's rows are read by its consumers
             mbar_arrive_expect_tx(&qfull[qs], C::QBYTES);
             tma_load_3d(qbuf + qs * C::QBYTES, &tmQ, 0, hp * HBG, u[7], &qfull[qs]);
+            q_issued |= 1u;
           } else {
             mbar_arrive_expect_tx(&qfull[qs], 0);
           }
@@ -550,7 +861,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&adone[qs]);  // every unit, so phases stay one per unit
         pos += t1 - t0;
-        while (s + 1 < B && sstart[s + 1] <= pos) ++s;
+        while (s + 1 < NS && sstart[s + 1] <= pos) ++s;
       }
       return;
     }
@@ -561,40 +872,218 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
         const int bs_mask = (1 << a.log2_bs) - 1;
+        // bit i: tile cnt-1-i was copied.  Each ring slot is reused only after its previous
+        // copy was consumed, so only the last nslots tiles can still be landing.
+        uint32_t issued = 0;
         int cnt = 0;
         for (int k = 0;; ++k) {
           const int qs = k % kQSlots;
-          wait_or_abort(&tfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-          const volatile int* u = unit + qs * 8;
+          wait_or_abort(&tfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+          const volatile int* u = unit + qs * kUnitInts;
           const int s = u[0];
-          if (s < 0 || *abort_flag) break;
+          if (s < 0 || *abort_flag) break;  // (one thread: a plain read)
           const int hp = u[1], t0 = u[2], t1 = u[3], append = u[6];
           for (int t = t0; t < t1; ++t, ++cnt) {
             const int slot = cnt % nslots;
             // the new token's row is in the last tile: its stores must have landed
             if (append && t == t1 - 1)
-              wait_or_abort(&adone[qs], (k / kQSlots) & 1, abort_flag, a.err);
-            wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err);
-            const int bid = *abort_flag ? -1 : tbl[qs * kMaxTilesPerUnit + (t - t0)];
+              wait_or_abort(&adone[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+            wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err, a.wait_limit);
+            if (*abort_flag) break;  // a wait may have been skipped: no more arrivals
+            issued <<= 1;
+            if (a.test_withhold && blockIdx.x == 0 && cnt == 0) continue;  // testing hook
+            const int bid = tbl[qs * kMaxTilesPerUnit + (t - t0)];
             mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
             if (bid >= 0) {
               const int row = (t * kTileTok) & bs_mask;
               uint8_t* dst = ring + slot * C::SLOT_BYTES;
               tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
               tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
+              issued |= 1u;
             }
           }
+          if (*abort_flag) break;
           mbar_arrive(&tempty[qs]);
         }
+        // no copy may still be landing in the ring when the CTA exits (the consumers have
+        // waited for all of them unless the CTA aborted)
+        for (int i = 0; i < nslots && i < cnt; ++i)
+          if (issued & (1u << i)) {
+            const int c = cnt - 1 - i;
+            drain_copy(&full[c % nslots], (c / nslots) & 1, a.err, a.wait_limit);
+          }
       }
       return;
     }
-
     return;  // warp 3 idles
   }
 
   // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
   const int w = warp - C::WARP_C0;
+
+  // A chunk segment (shared prefix): the 16 rows r = mloc*G + jj of kv-head hp*HB + w (member
+  // m0+mloc, q-head jj; rows past nm*G are zero queries, not written), as two mma.sync n8
+  // tiles that share every K and V^T fragment.  Per 16-token tile: S^T = K Q^T (M = 16
+  // tokens, N = 2 x 8 rows, K = 128 dims: 16 MMAs), the online softmax of each row, and
+  // O^T += V^T P^T (M = 128 dims in 8 tiles, K = 16 tokens: 16 MMAs).  Lane (g, tq) holds
+  // the logits of tokens g and g+8 for rows nt*8 + 2tq, +1 and their outputs for dims
+  // [16g, 16g+16); dims are paired as in the G = 8 consumer.  The rows' q is read from
+  // global memory once per segment.  Returns false when the CTA aborted.
+  auto chunk_segment = [&](int& k, int& cnt, int qs, const volatile int* u) -> bool {
+    const int s = u[0], hp = u[1], pslot = u[5], m0 = u[7], slot0 = u[8], nseg = u[9];
+    const int nm = u[10];
+    int t0 = u[2], t1 = u[3], flags = u[4];
+    constexpr int RS = HB * kRowBytes;  // bytes between consecutive tokens of a tile
+    const int g = lane >> 2, tq = lane & 3;
+    const int kvh = hp * HB + w;
+    uint32_t qf[2][8][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int r = nt * 8 + g, ml = r / G, jj = r % G;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          static_cast<const T*>(a.q) + ((long long)(m0 + ml) * a.num_q_heads + kvh * G + jj) * kD);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 v = ml < nm ? __ldg(src + tq + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
+        qf[nt][2 * j][0] = v.x;
+        qf[nt][2 * j][1] = v.y;
+        qf[nt][2 * j + 1][0] = v.z;
+        qf[nt][2 * j + 1][1] = v.w;
+      }
+    }
+    float oacc[2][8][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) oacc[nt][mt][0] = oacc[nt][mt][1] = oacc[nt][mt][2] = oacc[nt][mt][3] = 0.f;
+    float mh[2][2] = {{-INFINITY, -INFINITY}, {-INFINITY, -INFINITY}};
+    float lh[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    const int L = slen[s];
+    for (;;) {  // the segment's units
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qempty[qs]);
+      for (int t = t0; t < t1; ++t, ++cnt) {
+        const int slot = cnt % nslots;
+        wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
+        const int nvalid = min(kTileTok, L - t * kTileTok);
+        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+        const uint8_t* Vs = Ks + C::TILE_BYTES;
+        float sc4[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
+          const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            Mma<T>::run(sc4[nt], ka.x, kb.x, ka.y, kb.y, qf[nt][2 * j][0], qf[nt][2 * j][1]);
+            Mma<T>::run(sc4[nt], ka.z, kb.z, ka.w, kb.w, qf[nt][2 * j + 1][0], qf[nt][2 * j + 1][1]);
+          }
+        }
+        const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
+        uint32_t pb[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const float x0 = v0 ? sc4[nt][0] * a.qscale : -INFINITY;  // token g,   row 2tq
+          const float x1 = v0 ? sc4[nt][1] * a.qscale : -INFINITY;  // token g,   row 2tq+1
+          const float x2 = v8 ? sc4[nt][2] * a.qscale : -INFINITY;  // token g+8, row 2tq
+          const float x3 = v8 ? sc4[nt][3] * a.qscale : -INFINITY;  // token g+8, row 2tq+1
+          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          const float mn0 = fmaxf(mh[nt][0], mx0), mn1 = fmaxf(mh[nt][1], mx1);
+          const float al0 = fast_exp2(mh[nt][0] - mn0), al1 = fast_exp2(mh[nt][1] - mn1);
+          mh[nt][0] = mn0;
+          mh[nt][1] = mn1;
+          const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
+          const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+          lh[nt][0] = lh[nt][0] * al0 + (p0 + p2);
+          lh[nt][1] = lh[nt][1] * al1 + (p1 + p3);
+          if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+            const float2 al = make_float2(al0, al1);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              const float2 lo = __fmul2_rn(make_float2(oacc[nt][mt][0], oacc[nt][mt][1]), al);
+              const float2 hi = __fmul2_rn(make_float2(oacc[nt][mt][2], oacc[nt][mt][3]), al);
+              oacc[nt][mt][0] = lo.x;
+              oacc[nt][mt][1] = lo.y;
+              oacc[nt][mt][2] = hi.x;
+              oacc[nt][mt][3] = hi.y;
+            }
+          }
+          pb[nt][0] = transpose8x8(Mma<T>::pack(p0, p1));
+          pb[nt][1] = transpose8x8(Mma<T>::pack(p2, p3));
+        }
+        // V^T fragments, two m-tiles at a time: word r (dims 16g+2r, +1) and word 4+r
+        // (dims 16g+8+2r, +1) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (zero past the end)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          uint32_t lo[4], hi[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+            const bool ok = tk < nvalid;
+            const uint8_t* vr = Vs + tk * RS + g * 32 + r * 4;
+            lo[i] = ok ? *reinterpret_cast<const uint32_t*>(vr) : 0u;
+            hi[i] = ok ? *reinterpret_cast<const uint32_t*>(vr + 16) : 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const uint32_t sel = e ? 0x7632u : 0x5410u;
+            const uint32_t a0 = __byte_perm(lo[0], lo[1], sel), a1 = __byte_perm(hi[0], hi[1], sel);
+            const uint32_t a2 = __byte_perm(lo[2], lo[3], sel), a3 = __byte_perm(hi[2], hi[3], sel);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+              Mma<T>::run(oacc[nt][2 * r + e], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      ++k;
+      if (flags & kLast) break;
+      qs = k % kQSlots;
+      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+      u = unit + qs * kUnitInts;
+      if (u[0] < 0 || warp_flag(abort_flag)) return false;
+      t0 = u[2];
+      t1 = u[3];
+      flags = u[4];
+    }
+    // ---- end of segment: normalised partial rows of the chunk's slot, and (max, sum)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float lt0 = lh[nt][0], lt1 = lh[nt][1];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
+        lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = nt * 8 + 2 * tq + e;
+        if (r / G >= nm) continue;  // past the chunk's members
+        const float lt = e ? lt1 : lt0;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const long long row = (long long)pslot * (HB * kChunkRows) + w * kChunkRows + r;
+        float4* po = reinterpret_cast<float4*>(a.vpart_o + row * kD + 16 * g);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          po[i] = make_float4(oacc[nt][4 * i][e] * inv, oacc[nt][4 * i + 1][e] * inv,
+                              oacc[nt][4 * i + 2][e] * inv, oacc[nt][4 * i + 3][e] * inv);
+          po[2 + i] = make_float4(oacc[nt][4 * i][2 + e] * inv, oacc[nt][4 * i + 1][2 + e] * inv,
+                                  oacc[nt][4 * i + 2][2 + e] * inv, oacc[nt][4 * i + 3][2 + e] * inv);
+        }
+        if (g == 0)
+          *reinterpret_cast<float2*>(a.vpart_ml + row * 2) = make_float2(mh[nt][e], lt);
+      }
+    }
+    finish_chunk<T, G, HB>(a, sched(), m0, nm, hp, kvh, pslot, slot0, nseg, lane);
+    (void)s;
+    return true;
+  };
   if constexpr (C::MMA) {
     // Tensor-core consumer (G = 8, and every G on an FP8 cache).  Per 16-token tile: S^T = K Q^T (M = 16 tokens, N = 8
     // q-heads, K = 128 dims: 8 MMAs) and O^T += V^T P^T (M = 128 dims in 8 tiles, N = 8
@@ -610,18 +1099,27 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     using MT = typename std::conditional<F8, __half, T>::type;  // MMA operand type
     constexpr int RS = HB * C::KROW;  // bytes between consecutive tokens of a tile
     const int g = lane >> 2, tq = lane & 3;
-    uint32_t qf[8][2];  // Q^T fragments of the 8 k-steps
-    float oacc[8][4];   // O^T: [m-tile mt] dims 16g+mt / 16g+8+mt x heads 2tq, 2tq+1
-    float mh0 = -INFINITY, mh1 = -INFINITY, lh0 = 0.f, lh1 = 0.f;  // heads 2tq, 2tq+1
     int cnt = 0;
-    for (int k = 0;; ++k) {
-      const int qs = k % kQSlots;
-      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-      const volatile int* u = unit + qs * 8;
+    // one segment per iteration: its first unit (kFirst) loads q, its last (kLast) writes
+    // the result; the segment's state is dead once it is written
+    for (int k = 0;;) {
+      int qs = k % kQSlots;
+      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+      const volatile int* u = unit + qs * kUnitInts;
       const int s = u[0];
-      if (s < 0 || *abort_flag) break;
-      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5], orow = u[7];
-      if (flags & kFirst) {
+      if (s < 0 || warp_flag(abort_flag)) break;
+      if constexpr (SP) {
+        if (u[4] & kVirtual) {
+          if (!chunk_segment(k, cnt, qs, u)) break;
+          continue;
+        }
+      }
+      const int hp = u[1], pslot = u[5], orow = u[7], slot0 = u[8], nseg = u[9];
+      int t0 = u[2], t1 = u[3], flags = u[4];
+      uint32_t qf[8][2];  // Q^T fragments of the 8 k-steps
+      float oacc[8][4];   // O^T: [m-tile mt] dims 16g+mt / 16g+8+mt x heads 2tq, 2tq+1
+      float mh0 = -INFINITY, mh1 = -INFINITY, lh0 = 0.f, lh1 = 0.f;  // heads 2tq, 2tq+1
+      {
         const uint8_t* qrow = qbuf + qs * C::QBYTES + (w * G + g) * kRowBytes;
         if constexpr (F8) {
           // k-step 4c+i takes dims 4i..4i+3 of the 16-dim chunk tq + 4c (one 32-bit
@@ -645,134 +1143,147 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16);
+          for (int j = 0; j < 4; ++j) {  // q-heads past G (rows of the next warp): zero
+            const uint4 v = g < G ? *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16)
+                                  : make_uint4(0u, 0u, 0u, 0u);
             qf[2 * j][0] = v.x;
             qf[2 * j][1] = v.y;
             qf[2 * j + 1][0] = v.z;
             qf[2 * j + 1][1] = v.w;
           }
         }
-        mh0 = mh1 = -INFINITY;
-        lh0 = lh1 = 0.f;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[qs]);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
       const int L = slen[s];
       const int kvh = hp * HB + w;
       const float lsc = F8 ? a.qscale * __ldg(a.k_scale + kvh) : a.qscale;
+      bool stop = false;
+      for (;;) {  // the segment's units
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[qs]);
+        for (int t = t0; t < t1; ++t, ++cnt) {
+          const int slot = cnt % nslots;
+          wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
+          const int nvalid = min(kTileTok, L - t * kTileTok);
+          // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
+          const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * C::KROW;
+          const uint8_t* Vs = Ks + C::TILE_BYTES;
 
-      for (int t = t0; t < t1; ++t, ++cnt) {
-        const int slot = cnt % nslots;
-        wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
-        const int nvalid = min(kTileTok, L - t * kTileTok);
-        // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * C::KROW;
-        const uint8_t* Vs = Ks + C::TILE_BYTES;
-
-        // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (F8) {
+          // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
+          float sc[4] = {0.f, 0.f, 0.f, 0.f};
+          if constexpr (F8) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * c) * 16);
-            const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * c) * 16);
-            const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
+            for (int c = 0; c < 2; ++c) {
+              const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * c) * 16);
+              const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * c) * 16);
+              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              Mma<__half>::run(sc, e4m3x2_to_f16x2(wa[i]), e4m3x2_to_f16x2(wb[i]),
-                               e4m3x2_to_f16x2(wa[i] >> 16), e4m3x2_to_f16x2(wb[i] >> 16),
-                               qf[4 * c + i][0], qf[4 * c + i][1]);
+              for (int i = 0; i < 4; ++i)
+                Mma<__half>::run(sc, e4m3x2_to_f16x2(wa[i]), e4m3x2_to_f16x2(wb[i]),
+                                 e4m3x2_to_f16x2(wa[i] >> 16), e4m3x2_to_f16x2(wb[i] >> 16),
+                                 qf[4 * c + i][0], qf[4 * c + i][1]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
+              const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+              Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
+              Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+            }
           }
-        } else {
+          // ---- online softmax over the tile (log2 domain), per head
+          const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
+          const float x0 = v0 ? sc[0] * lsc : -INFINITY;  // token g,   head 2tq
+          const float x1 = v0 ? sc[1] * lsc : -INFINITY;  // token g,   head 2tq+1
+          const float x2 = v8 ? sc[2] * lsc : -INFINITY;  // token g+8, head 2tq
+          const float x3 = v8 ? sc[3] * lsc : -INFINITY;  // token g+8, head 2tq+1
+          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
-            const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
-            Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
-            Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
           }
-        }
-        // ---- online softmax over the tile (log2 domain), per head
-        const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
-        const float x0 = v0 ? sc[0] * lsc : -INFINITY;  // token g,   head 2tq
-        const float x1 = v0 ? sc[1] * lsc : -INFINITY;  // token g,   head 2tq+1
-        const float x2 = v8 ? sc[2] * lsc : -INFINITY;  // token g+8, head 2tq
-        const float x3 = v8 ? sc[3] * lsc : -INFINITY;  // token g+8, head 2tq+1
-        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+          const float mn0 = fmaxf(mh0, mx0), mn1 = fmaxf(mh1, mx1);
+          const float al0 = fast_exp2(mh0 - mn0), al1 = fast_exp2(mh1 - mn1);  // -inf -> 0
+          mh0 = mn0;
+          mh1 = mn1;
+          const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
+          const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+          lh0 = lh0 * al0 + (p0 + p2);
+          lh1 = lh1 * al1 + (p1 + p3);
+          if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+            const float2 al = make_float2(al0, al1);
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        const float mn0 = fmaxf(mh0, mx0), mn1 = fmaxf(mh1, mx1);
-        const float al0 = fast_exp2(mh0 - mn0), al1 = fast_exp2(mh1 - mn1);  // -inf -> 0
-        mh0 = mn0;
-        mh1 = mn1;
-        const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
-        const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
-        lh0 = lh0 * al0 + (p0 + p2);
-        lh1 = lh1 * al1 + (p1 + p3);
-        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-          const float2 al = make_float2(al0, al1);
+            for (int mt = 0; mt < 8; ++mt) {
+              const float2 lo = __fmul2_rn(make_float2(oacc[mt][0], oacc[mt][1]), al);
+              const float2 hi = __fmul2_rn(make_float2(oacc[mt][2], oacc[mt][3]), al);
+              oacc[mt][0] = lo.x;
+              oacc[mt][1] = lo.y;
+              oacc[mt][2] = hi.x;
+              oacc[mt][3] = hi.y;
+            }
+          }
+          // ---- P^T fragments: [tokens 2tq, 2tq+1 | 8+2tq, 9+2tq] x head g
+          const uint32_t pb0 = transpose8x8(Mma<MT>::pack(p0, p1));
+          const uint32_t pb1 = transpose8x8(Mma<MT>::pack(p2, p3));
+          // ---- V^T fragments: dims [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9,
+          // paired along tokens; rows past the sequence end are zeroed (p is 0 there, but
+          // the block's unused rows may hold anything)
+          uint32_t vw[4][8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+            uint4 lo, hi;
+            if constexpr (F8) {  // 16 e4m3 codes -> 8 f16 pairs
+              const uint4 c8 = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 16);
+              lo = make_uint4(e4m3x2_to_f16x2(c8.x), e4m3x2_to_f16x2(c8.x >> 16),
+                              e4m3x2_to_f16x2(c8.y), e4m3x2_to_f16x2(c8.y >> 16));
+              hi = make_uint4(e4m3x2_to_f16x2(c8.z), e4m3x2_to_f16x2(c8.z >> 16),
+                              e4m3x2_to_f16x2(c8.w), e4m3x2_to_f16x2(c8.w >> 16));
+            } else {
+              lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
+              hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
+            }
+            const bool ok = tk < nvalid;
+            vw[i][0] = ok ? lo.x : 0u;
+            vw[i][1] = ok ? lo.y : 0u;
+            vw[i][2] = ok ? lo.z : 0u;
+            vw[i][3] = ok ? lo.w : 0u;
+            vw[i][4] = ok ? hi.x : 0u;
+            vw[i][5] = ok ? hi.y : 0u;
+            vw[i][6] = ok ? hi.z : 0u;
+            vw[i][7] = ok ? hi.w : 0u;
+          }
+          // ---- O^T += V^T P^T, m-tile mt: rows dims 16g+mt (g) and 16g+8+mt (g+8)
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
-            const float2 lo = __fmul2_rn(make_float2(oacc[mt][0], oacc[mt][1]), al);
-            const float2 hi = __fmul2_rn(make_float2(oacc[mt][2], oacc[mt][3]), al);
-            oacc[mt][0] = lo.x;
-            oacc[mt][1] = lo.y;
-            oacc[mt][2] = hi.x;
-            oacc[mt][3] = hi.y;
+            const int r = mt >> 1;
+            const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
+            const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], sel);
+            const uint32_t a1 = __byte_perm(vw[0][4 + r], vw[1][4 + r], sel);
+            const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], sel);
+            const uint32_t a3 = __byte_perm(vw[2][4 + r], vw[3][4 + r], sel);
+            Mma<MT>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        // ---- P^T fragments: [tokens 2tq, 2tq+1 | 8+2tq, 9+2tq] x head g
-        const uint32_t pb0 = transpose8x8(Mma<MT>::pack(p0, p1));
-        const uint32_t pb1 = transpose8x8(Mma<MT>::pack(p2, p3));
-        // ---- V^T fragments: dims [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9,
-        // paired along tokens; rows past the sequence end are zeroed (p is 0 there, but
-        // the block's unused rows may hold anything)
-        uint32_t vw[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-          uint4 lo, hi;
-          if constexpr (F8) {  // 16 e4m3 codes -> 8 f16 pairs
-            const uint4 c8 = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 16);
-            lo = make_uint4(e4m3x2_to_f16x2(c8.x), e4m3x2_to_f16x2(c8.x >> 16),
-                            e4m3x2_to_f16x2(c8.y), e4m3x2_to_f16x2(c8.y >> 16));
-            hi = make_uint4(e4m3x2_to_f16x2(c8.z), e4m3x2_to_f16x2(c8.z >> 16),
-                            e4m3x2_to_f16x2(c8.w), e4m3x2_to_f16x2(c8.w >> 16));
-          } else {
-            lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
-            hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
-          }
-          const bool ok = tk < nvalid;
-          vw[i][0] = ok ? lo.x : 0u;
-          vw[i][1] = ok ? lo.y : 0u;
-          vw[i][2] = ok ? lo.z : 0u;
-          vw[i][3] = ok ? lo.w : 0u;
-          vw[i][4] = ok ? hi.x : 0u;
-          vw[i][5] = ok ? hi.y : 0u;
-          vw[i][6] = ok ? hi.z : 0u;
-          vw[i][7] = ok ? hi.w : 0u;
+        ++k;
+        if (flags & kLast) break;
+        qs = k % kQSlots;
+        wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+        u = unit + qs * kUnitInts;
+        if (u[0] < 0 || warp_flag(abort_flag)) {
+          stop = true;
+          break;
         }
-        // ---- O^T += V^T P^T, m-tile mt: rows dims 16g+mt (g) and 16g+8+mt (g+8)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          const int r = mt >> 1;
-          const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
-          const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], sel);
-          const uint32_t a1 = __byte_perm(vw[0][4 + r], vw[1][4 + r], sel);
-          const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], sel);
-          const uint32_t a3 = __byte_perm(vw[2][4 + r], vw[3][4 + r], sel);
-          Mma<MT>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
+        t0 = u[2];
+        t1 = u[3];
+        flags = u[4];
       }
-      if (!(flags & kLast)) continue;
+      if (stop) break;
 
       // ---- end of segment: sums over the 8 token rows g, then heads 2tq and 2tq+1
       float lt0 = lh0, lt1 = lh1;
@@ -815,6 +1326,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
                 make_float2(e ? mh1 : mh0, e ? lt1 : lt0);
         }
       }
+      if (!(flags & kDirect))
+        finish_own<T, G, HB, SP>(a, sched(), s, orow, hp, kvh, pslot, slot0, nseg, lane);
     }
     return;
   } else {
@@ -824,18 +1337,25 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
     const bool writer = (lane & C::DUPMASK) == 0;
     float2* pw = pbuf + w * kTileTok * GW;
     int cnt = 0;
-    float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
-    float m = -INFINITY, l = 0.f;
-    float2 acc[GW][2];
-
-    for (int k = 0;; ++k) {
-      const int qs = k % kQSlots;
-      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err);
-      const volatile int* u = unit + qs * 8;
+    // one segment per iteration, as in the tensor-core consumer
+    for (int k = 0;;) {
+      int qs = k % kQSlots;
+      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+      const volatile int* u = unit + qs * kUnitInts;
       const int s = u[0];
-      if (s < 0 || *abort_flag) break;
-      const int hp = u[1], t0 = u[2], t1 = u[3], flags = u[4], pslot = u[5], orow = u[7];
-      if (flags & kFirst) {
+      if (s < 0 || warp_flag(abort_flag)) break;
+      if constexpr (SP) {
+        if (u[4] & kVirtual) {
+          if (!chunk_segment(k, cnt, qs, u)) break;
+          continue;
+        }
+      }
+      const int hp = u[1], pslot = u[5], orow = u[7], slot0 = u[8], nseg = u[9];
+      int t0 = u[2], t1 = u[3], flags = u[4];
+      float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
+      float m = -INFINITY, l = 0.f;
+      float2 acc[GW][2];
+      {
         // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
         const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
 #pragma unroll
@@ -849,93 +1369,105 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
             q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
           }
         }
-        m = -INFINITY;
-        l = 0.f;
-#pragma unroll
-        for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qempty[qs]);
+#pragma unroll
+      for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
       const int L = slen[s];
-
-      for (int t = t0; t < t1; ++t, ++cnt) {
-        const int slot = cnt % nslots;
-        wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err);
-        const int nvalid = min(kTileTok, L - t * kTileTok);
-        // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
-        const uint8_t* Vs = Ks + C::TILE_BYTES;
-
-        // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
-        float x[4];
-#pragma unroll
-        for (int ps = 0; ps < 4; ++ps) {
-          const int rr = ps * 4 + tp;
-          const uint8_t* kr = Ks + rr * (HB * kRowBytes);
-          const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
-          const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
-          const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          float2 kf[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
-          float d[GW];
-#pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            float2 e = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
-            d[jj] = e.x + e.y;
-          }
-          const float xv = reduce_heads<GW>(d, lane);
-          x[ps] = rr < nvalid ? xv : -INFINITY;
-        }
-        // ---- online softmax over the tile, per head hh
-        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m, mx);
-        const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
-        m = m_new;
-        float psum = 0.f;
-#pragma unroll
-        for (int ps = 0; ps < 4; ++ps) {
-          const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
-          psum += pv;
-          if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
-        }
-        l = l * alpha + psum;
-        if (writer && tp == 0) abuf[w * GW + hh] = alpha;
+      bool stop = false;
+      for (;;) {  // the segment's units
         __syncwarp();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        if (lane == 0) mbar_arrive(&qempty[qs]);
+        for (int t = t0; t < t1; ++t, ++cnt) {
+          const int slot = cnt % nslots;
+          wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
+          const int nvalid = min(kTileTok, L - t * kTileTok);
+          // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
+          const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+          const uint8_t* Vs = Ks + C::TILE_BYTES;
+
+          // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
+          float x[4];
 #pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            const float al = abuf[w * GW + jj];
-            const float2 a2 = make_float2(al, al);
-            acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
-            acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
+          for (int ps = 0; ps < 4; ++ps) {
+            const int rr = ps * 4 + tp;
+            const uint8_t* kr = Ks + rr * (HB * kRowBytes);
+            const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
+            const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
+            const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            float2 kf[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
+            float d[GW];
+#pragma unroll
+            for (int jj = 0; jj < GW; ++jj) {
+              float2 e = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
+              d[jj] = e.x + e.y;
+            }
+            const float xv = reduce_heads<GW>(d, lane);
+            x[ps] = rr < nvalid ? xv : -INFINITY;
           }
-        }
-        // ---- p.V: lane owns dims [4*lane, 4*lane+4)
-        auto pv_row = [&](int tt) {
-          const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
-          const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
+          // ---- online softmax over the tile, per head hh
+          float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m, mx);
+          const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
+          m = m_new;
+          float psum = 0.f;
 #pragma unroll
-          for (int jj = 0; jj < GW; ++jj) {
-            const float2 pp = pw[tt * GW + jj];
-            acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
-            acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
+          for (int ps = 0; ps < 4; ++ps) {
+            const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
+            psum += pv;
+            if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
           }
-        };
-        if (nvalid == kTileTok) {
+          l = l * alpha + psum;
+          if (writer && tp == 0) abuf[w * GW + hh] = alpha;
+          __syncwarp();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
-        } else {
-          for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
+            for (int jj = 0; jj < GW; ++jj) {
+              const float al = abuf[w * GW + jj];
+              const float2 a2 = make_float2(al, al);
+              acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
+              acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
+            }
+          }
+          // ---- p.V: lane owns dims [4*lane, 4*lane+4)
+          auto pv_row = [&](int tt) {
+            const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
+            const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
+#pragma unroll
+            for (int jj = 0; jj < GW; ++jj) {
+              const float2 pp = pw[tt * GW + jj];
+              acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
+              acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
+            }
+          };
+          if (nvalid == kTileTok) {
+#pragma unroll
+            for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
+          } else {
+            for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
+        ++k;
+        if (flags & kLast) break;
+        qs = k % kQSlots;
+        wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
+        u = unit + qs * kUnitInts;
+        if (u[0] < 0 || warp_flag(abort_flag)) {
+          stop = true;
+          break;
+        }
+        t0 = u[2];
+        t1 = u[3];
+        flags = u[4];
       }
-      if (!(flags & kLast)) continue;
+      if (stop) break;
 
       // ---- end of segment: l summed over the 4 token groups; m and l of every head
       float lt = l + __shfl_xor_sync(0xffffffffu, l, 8);
@@ -958,95 +1490,15 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8>::THREADS, 1)
           if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
         }
       }
+      if (!(flags & kDirect))
+        finish_own<T, G, HB, SP>(a, sched(), s, orow, hp, hp * HB + w, pslot, slot0, nseg, lane);
     }
   }  // G < 8
 }
 
-// Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes
-// over head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the
-// largest m_i, over the segments i of the (sequence, head group), which sit in
-// consecutive slots, and the sequence's shared-prefix partials.
-//
-// Fold the segments of one output row into (M, den, num): the n slots of this launch
-// (rows row0 + i * hbg) and, with PRE, the npre shared-prefix partials (row gw of each).
-// One pass with a running maximum: up to eight segments per round, all loads of a round
-// in flight together (most groups span fewer than eight CTAs: one round).
-template <bool PRE>
-__device__ __forceinline__ void fold_segments(const DecodeArgs& a, long long row0, int hbg,
-                                              int n, int npre, int gw, int lane, float& M,
-                                              float& den, float4& num) {
-  const int total = n + (PRE ? npre : 0);
-  const long long prow_stride = (long long)a.num_seqs * a.num_q_heads;
-  for (int i0 = 0; i0 < total; i0 += 8) {
-    float2 mlv[8];
-    float4 ov[8];
-    float Mr = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u;
-      if (i < total) {
-        if (!PRE || i < n) {
-          const long long row = row0 + (long long)i * hbg;
-          mlv[u] = *reinterpret_cast<const float2*>(a.part_ml + row * 2);
-          ov[u] = *reinterpret_cast<const float4*>(a.part_o + row * kD + lane * 4);
-        } else {
-          const long long row = (long long)(i - n) * prow_stride + gw;
-          mlv[u] = *reinterpret_cast<const float2*>(a.pre_ml + row * 2);
-          ov[u] = *reinterpret_cast<const float4*>(a.pre_o + row * kD + lane * 4);
-        }
-        Mr = fmaxf(Mr, mlv[u].x);
-      }
-    }
-    const float Mn = fmaxf(M, Mr);
-    if (Mn == -INFINITY) continue;  // only empty segments so far
-    const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
-    den *= sc;
-    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (i0 + u < total) {
-        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
-        den += f;
-        num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
-      }
-    }
-    M = Mn;
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a, int hbg) {
-  // launched as a programmatic dependent of the decode kernel: its CTAs may start while
-  // the decode grid drains; this waits until that grid has finished and its writes are
-  // visible (a no-op when launched without the dependency)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= a.num_seqs * a.num_q_heads) return;
-  const int s = gw / a.num_q_heads;
-  const int qh = gw - s * a.num_q_heads;
-  const int nhp = a.num_q_heads / hbg;
-  const int j = qh % hbg;
-  const int2 mt = a.meta[s * nhp + qh / hbg];
-  const int n = mt.y & (kHasPrefix - 1);                 // segments of this launch
-  const int npre = (mt.y & kHasPrefix) ? a.pre_chunks : 0;  // shared-prefix partials
-  if (n <= 1 && npre == 0) return;  // written by the decode kernel
-  const long long row0 = (long long)mt.x * hbg + j;
-  float M = -INFINITY, den = 0.f;
-  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (npre == 0)
-    fold_segments<false>(a, row0, hbg, n, 0, gw, lane, M, den, num);
-  else
-    fold_segments<true>(a, row0, hbg, n, npre, gw, lane, M, den, num);
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  const long long orow = a.qsl ? __ldg(a.qsl + s) : s;
-  T* ob = static_cast<T*>(a.out) + (orow * a.num_q_heads + qh) * kD + lane * 4;
-  *reinterpret_cast<uint2*>(ob) =
-      make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
-}
-
 constexpr int kMaxPartition = kMaxTilesPerUnit * kTileTok;
 constexpr int kMaxSeqs = 4096;
+constexpr int kMaxSeqsShared = 2048;  // batch + chunks in the schedule arrays
 constexpr int kMaxSmem = 227 * 1024;
 
 // kv-heads per group: all of them up to eight (whole 2 KB rows for 8 heads of 128)
@@ -1058,77 +1510,86 @@ inline int heads_per_item(int num_kv_heads) {
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace of one launch: merge records, then partial outputs, then (m, l) pairs.
+// Workspace of one launch: merge tickets (one int per sequence and kv-head), then partial
+// outputs, then (m, l) pairs.
 struct WsLayout {
-  size_t meta, part_o, part_ml, total;
+  size_t tickets, part_o, part_ml, total;
 };
-inline WsLayout ws_layout(long long groups, long long slots, int hbg, int head_dim) {
+inline WsLayout ws_layout(long long tickets, long long slots, int hbg, int head_dim) {
   WsLayout w;
-  w.meta = 0;
-  w.part_o = align256((size_t)groups * sizeof(int2));
+  w.tickets = 0;
+  w.part_o = align256((size_t)tickets * sizeof(int));
   w.part_ml = w.part_o + (size_t)slots * hbg * head_dim * sizeof(float);
   w.total = w.part_ml + (size_t)slots * hbg * 2 * sizeof(float);
   return w;
 }
 
-template <typename T, int G, int HB, bool F8>
+template <typename T, int G, int HB, bool F8, bool SP>
 pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmQ,
                         DecodeArgs a, int grid, cudaStream_t stream) {
-  using C = DecodeCfg<G, HB, F8>;
-  const size_t ring_off = ((C::OFF_SEQ + (size_t)(3 * a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
+  using C = DecodeCfg<G, HB, F8, SP>;
+  // schedule arrays: 3 ints per sequence (batch and chunks) + 1, and the groups' chunk starts
+  const long long seq_ints = 3LL * (a.num_seqs + (SP ? a.vcap : 0)) + 1 + (SP ? a.num_groups + 1 : 0);
+  const size_t ring_off = ((C::OFF_SEQ + (size_t)seq_ints * 4 + 1023) / 1024) * 1024;
   const long long room = (long long)kMaxSmem - (long long)ring_off;
   const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
   if (nslots < 2) return PA_ERR_UNSUPPORTED;
   a.ring_off = (int)ring_off;
   a.nslots = nslots;
   const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
-  auto kern = paged_decode_kernel<T, G, HB, F8>;
+  auto kern = paged_decode_kernel<T, G, HB, F8, SP>;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
-  kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
-  if (check_launch() != PA_OK) return PA_ERR_CUDA;
+  // Split groups merge inside the launch through tickets that must start at zero: a small
+  // kernel zeroes them first, and the decode grid starts as its programmatic dependent
+  // (its prologue and first tiles overlap the zeroing; it waits before its first ticket).
+  const bool split = grid > 1 || a.num_groups > 0;
   int launches = 1;
-  if (grid > 1 || a.num_groups > 0) {
-    const int warps = a.num_seqs * a.num_q_heads;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, lse_reduce_kernel<T>, a, HB * G) != cudaSuccess)
-      return PA_ERR_CUDA;
+  if (split) {
+    const int n = a.num_seqs * a.num_kv_heads;
+    zero_tickets_kernel<<<std::min(32, (n + 4095) / 4096), 256, 0, stream>>>(a.tickets, n);
     if (check_launch() != PA_OK) return PA_ERR_CUDA;
     ++launches;
   }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = split ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, tmK, tmV, tmQ, a) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
   set_launch_count(launches);
   return PA_OK;
 }
 
-template <typename T, int G, bool F8>
+template <typename T, int G, bool F8, bool SP>
 pa_status dispatch_hb(int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                       const CUtensorMap& tmQ, const DecodeArgs& a, int grid, cudaStream_t stream) {
   switch (HB) {
-    case 1: return launch_decode<T, G, 1, F8>(tmK, tmV, tmQ, a, grid, stream);
-    case 2: return launch_decode<T, G, 2, F8>(tmK, tmV, tmQ, a, grid, stream);
-    case 4: return launch_decode<T, G, 4, F8>(tmK, tmV, tmQ, a, grid, stream);
-    case 8: return launch_decode<T, G, 8, F8>(tmK, tmV, tmQ, a, grid, stream);
+    case 1: return launch_decode<T, G, 1, F8, SP>(tmK, tmV, tmQ, a, grid, stream);
+    case 2: return launch_decode<T, G, 2, F8, SP>(tmK, tmV, tmQ, a, grid, stream);
+    case 4: return launch_decode<T, G, 4, F8, SP>(tmK, tmV, tmQ, a, grid, stream);
+    case 8: return launch_decode<T, G, 8, F8, SP>(tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
 
-template <typename T, bool F8>
+template <typename T, bool F8, bool SP = false>
 pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const CUtensorMap& tmQ, const DecodeArgs& a, int grid,
                          cudaStream_t stream) {
   switch (G) {
-    case 1: return dispatch_hb<T, 1, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 2: return dispatch_hb<T, 2, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 4: return dispatch_hb<T, 4, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
-    case 8: return dispatch_hb<T, 8, F8>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 1: return dispatch_hb<T, 1, F8, SP>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 2: return dispatch_hb<T, 2, F8, SP>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 4: return dispatch_hb<T, 4, F8, SP>(HB, tmK, tmV, tmQ, a, grid, stream);
+    case 8: return dispatch_hb<T, 8, F8, SP>(HB, tmK, tmV, tmQ, a, grid, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -1201,7 +1662,19 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   const long long cap_tbl = (long long)max_blocks_per_seq * block_size;
   const int seq_cap = (int)std::min<long long>(cap_tbl, max_seq_len);
   const long long nt_max = (seq_cap + pa::kTileTok - 1) / pa::kTileTok;
-  const long long tiles_max = (long long)num_seqs * NHP * nt_max;
+  // shared prefixes: the chunks of each group's members over the group's prefix join the
+  // schedule after the batch (at most one chunk per member)
+  int mc = 0, vcap = 0;
+  long long vtiles = 0;
+  if (sp) {
+    if (num_seqs > pa::kMaxSeqsShared) return PA_ERR_UNSUPPORTED;
+    mc = pa::kChunkRows / G;
+    vcap = (int)std::min<long long>(
+        num_seqs, (long long)sp->num_groups * ((sp->max_group_size + mc - 1) / mc));
+    vtiles = (long long)vcap * NHP *
+             ((std::min<long long>(sp->max_prefix_len, seq_cap) + pa::kTileTok - 1) / pa::kTileTok);
+  }
+  const long long tiles_max = (long long)num_seqs * NHP * nt_max + vtiles;
   if (tiles_max > INT_MAX / 2) return PA_ERR_UNSUPPORTED;
   // persistent grid of one CTA per SM; an explicit partition caps each CTA's share
   long long grid = std::min<long long>(std::max(1, pa::num_sms()), pa::kMaxGrid);
@@ -1209,19 +1682,20 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   if (partition_size > 0)
     grid = std::max<long long>(grid, (tiles_max + partition_size / 16 - 1) / (partition_size / 16));
   const long long groups = (long long)num_seqs * NHP;
-  const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
-  // shared prefix: the prefix pass's partial rows follow the decode workspace
-  pa::SharedPrefixPlan plan = {};
-  size_t pre_off = 0, need = lay.total;
+  const pa::WsLayout lay =
+      pa::ws_layout((long long)num_seqs * num_kv_heads, grid + groups, HBG, head_dim);
+  // shared prefixes: the chunks' partial rows follow, (grid + chunks x head groups) slots of
+  // HB x 16 rows
+  const long long vslots = sp ? grid + (long long)vcap * NHP : 0;
+  const long long vrows = vslots * HB * pa::kChunkRows;
+  size_t voff = 0, need = lay.total;
   if (sp) {
-    plan = pa::plan_shared_prefix(sp->num_groups, num_kv_heads, G, sp->max_group_size,
-                                  sp->max_prefix_len);
-    pre_off = pa::align256(lay.total);
-    need = pre_off + (size_t)plan.slots * num_seqs * num_q_heads * (head_dim + 2) * sizeof(float);
+    voff = pa::align256(lay.total);
+    need = voff + (size_t)vrows * (head_dim + 2) * sizeof(float);
   }
   if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
-  int* err = pa::device_error_flag();
+  int* err = pa::launch_prologue();
   if (!err) return PA_ERR_CUDA;
 
   CUtensorMap tmK, tmV, tmQ;
@@ -1247,7 +1721,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.out = out;
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
-  a.meta = reinterpret_cast<int2*>(ws + lay.meta);
+  a.q = q;
+  a.tickets = reinterpret_cast<unsigned*>(ws + lay.tickets);
   a.k_new = k_new;
   a.v_new = v_new;
   a.k_cache = const_cast<void*>(k_cache);
@@ -1267,37 +1742,30 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.ring_off = 0;
   a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
+  a.wait_limit = pa::take_wait_limit(pa::kTestDecode, &a.test_withhold);
   a.group_starts = a.prefix_lens = nullptr;
-  a.pre_o = a.pre_ml = nullptr;
-  a.num_groups = a.pre_chunks = 0;
+  a.vpart_o = a.vpart_ml = nullptr;
+  a.num_groups = a.mc = a.vcap = a.max_prefix = 0;
   a.qsl = qsl;
   a.num_q_rows = qsl ? num_q_rows : num_seqs;
   a.chunk_ids = chunk_ids;
   a.chunk_cap = chunk_cap;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (sp) {
-    // pass 1: every group's prefix, once for all its members (tensor cores); pass 2 (the
-    // decode kernel below) reads each sequence's own keys; the merge combines them
-    float* pre_o = reinterpret_cast<float*>(ws + pre_off);
-    float* pre_ml = pre_o + (size_t)plan.slots * num_seqs * num_q_heads * head_dim;
-    const pa_status ps = pa::shared_prefix_pass(
-        q, k_cache, v_cache, block_tables, max_blocks_per_seq, sp->group_starts,
-        sp->prefix_lens, sp->num_groups, sp->max_group_size, sp->max_prefix_len, num_seqs,
-        num_q_heads, num_kv_heads, scale, block_size, num_blocks, plan, pre_o, pre_ml, dtype,
-        err, st);
-    if (ps != PA_OK) return ps;
+    // one launch: every sequence's own keys, and each chunk of every group's members over
+    // the group's prefix (the prefix read once per chunk), merged through the tickets
     a.group_starts = sp->group_starts;
     a.prefix_lens = sp->prefix_lens;
     a.num_groups = sp->num_groups;
-    a.pre_o = pre_o;
-    a.pre_ml = pre_ml;
-    a.pre_chunks = plan.slots;
-    const pa_status ds =
-        dtype == PA_F16
-            ? pa::dispatch_group<__half, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
-            : pa::dispatch_group<__nv_bfloat16, false>(G, HB, tmK, tmV, tmQ, a, (int)grid, st);
-    if (ds == PA_OK) pa::set_launch_count(pa::launch_count() + 1);
-    return ds;
+    a.mc = mc;
+    a.vcap = vcap;
+    a.max_prefix = sp->max_prefix_len;
+    a.vpart_o = reinterpret_cast<float*>(ws + voff);
+    a.vpart_ml = a.vpart_o + (size_t)vrows * head_dim;
+    return dtype == PA_F16
+               ? pa::dispatch_group<__half, false, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
+               : pa::dispatch_group<__nv_bfloat16, false, true>(G, HB, tmK, tmV, tmQ, a,
+                                                                 (int)grid, st);
   }
   if (f8)
     return dtype == PA_F16
@@ -1358,7 +1826,7 @@ extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache
 // serving loop whose memory is entirely owned by an engine's pre-allocated pool (the
 // pool hands out KV blocks, not scratch buffers), plugins whose host framework forbids
 // raw cudaMalloc, and latency-critical paths where an allocation could synchronise the
-// device.  For them this entry point keeps its workspace (the merge records and the
+// device.  For them this entry point keeps its workspace (the merge tickets and the
 // split-K partials) in a fixed array that
 // lives in this file (kNoAllocScratchBytes on every GPU that loads the library, held
 // until the process exits) and otherwise runs exactly pa_decode.
@@ -1371,14 +1839,18 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[64] = {};
 
 // Device address of this device's scratch array (looked up once per device, with that
-// device current).  nullptr if the lookup failed.
+// device current, and kept for the life of the process: a cudaDeviceReset invalidates
+// it).  nullptr if the lookup failed.
 void* scratch_for_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();  // the failed lookup is reported here, not by a later launch
+      return nullptr;
+    }
     g_scratch_ptr[dev] = p;
   }
   return g_scratch_ptr[dev];
@@ -1407,11 +1879,14 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
 extern "C" size_t pa_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 extern "C" size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads,
-                                                         int head_dim, int max_seq_len) {
+                                                         int num_kv_heads, int head_dim,
+                                                         int max_seq_len) {
   const size_t base = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
-  if (base == 0) return 0;
-  return pa::align256(base) + (size_t)pa::kMaxPrefixChunks * num_seqs * num_q_heads *
-                                  (head_dim + 2) * sizeof(float);
+  if (base == 0 || num_kv_heads <= 0) return 0;
+  // the chunks' partial rows: (grid + chunks x head groups) slots of (kv-heads per group x 16)
+  // rows, at most (256 + num_seqs) x num_kv_heads x 16 rows of head_dim + 2 fp32
+  return pa::align256(base) + ((size_t)pa::kMaxGrid + num_seqs) * num_kv_heads *
+                                  pa::kChunkRows * (head_dim + 2) * sizeof(float);
 }
 
 extern "C" pa_status pa_decode_shared_prefix(

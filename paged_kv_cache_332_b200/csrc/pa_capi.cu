@@ -17,6 +17,8 @@ std::mutex g_mu;
 int* g_err_ptr[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 thread_local int g_last_launches = 0;
+thread_local int g_test_kind = 0;            // pa_testing_wait_fault: kernel kind, one-shot
+thread_local long long g_test_limit = 0;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -37,10 +39,18 @@ int* device_error_flag() {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_err_ptr[d]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_pa_device_error) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_pa_device_error) != cudaSuccess) {
+      (void)cudaGetLastError();  // reported by this call's status, not a later launch check
+      return nullptr;
+    }
     g_err_ptr[d] = static_cast<int*>(p);
   }
   return g_err_ptr[d];
+}
+
+int* launch_prologue() {
+  (void)cudaGetLastError();
+  return device_error_flag();
 }
 
 int num_sms() {
@@ -119,6 +129,15 @@ bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int 
   return encode_tmap_16bit(out, cache, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+long long take_wait_limit(int kind, int* withhold) {
+  *withhold = 0;
+  if (g_test_kind != kind) return kWaitLimitCycles;
+  *withhold = 1;
+  const long long lim = g_test_limit;
+  g_test_kind = 0;
+  return lim;
+}
+
 void set_launch_count(int n) { g_last_launches = n; }
 int launch_count() { return g_last_launches; }
 
@@ -154,5 +173,13 @@ pa_status pa_get_device_error(void* stream, int32_t* code) {
 }
 
 int pa_last_launch_count(void) { return pa::g_last_launches; }
+
+pa_status pa_testing_wait_fault(int kernel, long long wait_limit_cycles) {
+  if (kernel < 0 || kernel > 2 || (kernel != 0 && wait_limit_cycles <= 0))
+    return PA_ERR_INVALID_ARG;
+  pa::g_test_kind = kernel;
+  pa::g_test_limit = wait_limit_cycles;
+  return PA_OK;
+}
 
 }  // extern "C"

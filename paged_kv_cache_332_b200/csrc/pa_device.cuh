@@ -18,10 +18,6 @@
 
 namespace pa {
 
-// Longest any single pipeline wait may take before the kernel gives up, in SM clock
-// cycles (the per-SM counter is cheap to read; ~2 s at B200 clocks).
-constexpr long long kWaitLimitCycles = 4000000000ll;
-
 __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }
@@ -82,17 +78,43 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and flags PA_DEVERR_TIMEOUT) if that takes longer than kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// (and flags PA_DEVERR_TIMEOUT) if that takes longer than `limit` SM cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       flag_error(err, PA_DEVERR_TIMEOUT);
       return false;
     }
   }
+}
+
+// A CTA flag read by a whole warp with one answer for every lane, so that a decision on
+// it never splits the warp before a warp-collective instruction.
+__device__ __forceinline__ bool warp_flag(volatile int* f) {
+  return __any_sync(0xffffffffu, *f != 0);
+}
+
+// Grid dependency control (programmatic dependent launch): let the next grid of the
+// stream start launching, and wait until every prerequisite grid has completed with its
+// memory visible (both are no-ops without the launch attribute).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Atomic add at GPU scope with acquire-release order: releases this thread's earlier
+// writes with the increment and acquires the writes released by earlier increments.
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -12,6 +12,11 @@ namespace pa {
 // Device address of the calling device's PA_DEVERR_* flag (nullptr on failure).
 int* device_error_flag();
 
+// Start of every launching entry point, after its host-side checks: clears a non-sticky
+// CUDA error left pending on this thread by earlier, unrelated work (so that the launch
+// checks below report this call's launches only) and returns the device error flag.
+int* launch_prologue();
+
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 
@@ -37,21 +42,22 @@ bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint6
                        const uint64_t* strides_bytes, const uint32_t* box,
                        CUtensorMapSwizzle swizzle);
 
+// Longest any single pipeline wait may take before a kernel gives up, in SM clock cycles
+// (the per-SM counter is cheap to read; ~2 s at B200 clocks).  Kernels take the limit as
+// an argument: always this value, except under the testing hook that shortens it.
+constexpr long long kWaitLimitCycles = 4000000000ll;
+
+// Testing hook (pa_testing_wait_fault): the wait limit for the next launch of `kind` on
+// this thread, and whether that launch withholds one pipeline arrival.  One-shot: the
+// hook is cleared when taken; without it the limit is kWaitLimitCycles.
+constexpr int kTestDecode = 1;
+constexpr int kTestPrefill = 2;
+long long take_wait_limit(int kind, int* withhold);
+
 // Launch accounting for pa_last_launch_count().
 void set_launch_count(int n);
 int launch_count();
 
-// Shared-prefix decode, first pass (prefill.cu): the attention of every member's q-heads
-// over its group's shared prefix, on the tcgen05 prefill kernel (the members' queries of
-// one kv-head form the rows of one M-tile), as `chunks` pieces of normalised partial rows
-// in pre_o [slots][q_rows * num_q_heads][128] and (max, sum) in pre_ml.
-constexpr int kMaxPrefixChunks = 8;  // partial slots at most
-struct SharedPrefixPlan {
-  int ksplit;   // groups fit one M-tile: the two M-tiles take alternate key tiles
-  int qblocks;  // query blocks per (group, kv-head)
-  int pieces;   // key pieces per (group, kv-head, query block)
-  int slots;    // partial rows per output row: pieces (x 2 with ksplit)
-};
 // pa_chunked_prefill; with skip_single, sequences of one query row are left out (the
 // varlen call serves them with the decode kernel); with chunk_ids (a device list of the
 // sequences with more than one query row, its length at chunk_ids[chunk_cap]) the grid
@@ -64,16 +70,6 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
                                int max_seq_len, void* workspace, size_t workspace_bytes,
                                pa_dtype dtype, void* stream, bool skip_single,
                                const int32_t* chunk_ids, int chunk_cap);
-
-SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
-                                    int max_prefix_len);
-pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
-                             const int32_t* block_tables, int max_blocks_per_seq,
-                             const int32_t* group_starts, const int32_t* prefix_lens,
-                             int num_groups, int max_group_size, int max_prefix_len, int q_rows,
-                             int num_q_heads, int num_kv_heads, float scale, int block_size,
-                             int num_blocks, const SharedPrefixPlan& plan, float* pre_o,
-                             float* pre_ml, pa_dtype dtype, int* err, cudaStream_t stream);
 
 inline pa_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -31,10 +31,6 @@
 //  * Keys at or past L in the last tile: K is masked in the softmax; V rows are
 //    zero-filled (TMA out-of-range fill for whole runs, a shared-memory clear for the
 //    tail of a partial block) so that 0 * (stale value) never reaches the sum.
-// The same kernel is the first pass of the shared-prefix decode: the "sequence" is a
-// group, its queries the members' decode rows, its keys the shared prefix with no causal
-// mask, and its output normalised partial rows; when the group fits one M-tile the two
-// M-tiles take alternate key tiles as two independent softmax chains.
 // Every wait is bounded; on a timeout the CTA flags PA_DEVERR_TIMEOUT, runs to its end
 // without further waits and frees its TMEM.
 #include <algorithm>
@@ -71,24 +67,14 @@ struct Args {
   float* part_o;
   float* part_ml;
   int* rowmap;
-  // shared-prefix pass of the decode (prefix_chunks > 0): item "sequence" s is group s,
-  // whose queries are the decode rows qsl[s] .. qsl[s+1]-1 (one per member, q_rows rows
-  // in all) and whose keys are the first seq_lens[s] tokens, read through the table row
-  // of member qsl[s] and visible to every row (no causal mask).  The keys are cut into
-  // prefix_chunks pieces of whole tiles; each piece writes normalised partial rows and
-  // (max in log2 units, sum) to pre_o / pre_ml [piece][q_rows * num_q_heads].
-  // With ksplit (shared-prefix pass, every group within one M-tile of rows) the two
-  // M-tiles hold the same rows and take alternate key tiles, two independent softmax
-  // chains per CTA; each writes its own partial (piece 2 * piece + M-tile).
-  int prefix_chunks, q_rows, ksplit;
-  float* pre_o;
-  float* pre_ml;
   // varlen call: sequences with a single query row are left to the decode kernel.  With
   // chunk_ids, item "sequence" r is the r-th sequence with more than one query row,
   // chunk_ids[r] (chunk_ids[chunk_cap] holds how many; num_seqs = chunk_cap)
   int skip_single;
   const int32_t* chunk_ids;
   int chunk_cap;
+  long long wait_limit;  // SM cycles any pipeline wait may take before the CTA gives up
+  int test_withhold;     // testing hook: CTA 0's producer withholds its first K tile
 };
 
 // shared memory carve-up
@@ -96,8 +82,9 @@ constexpr int OFF_Q = 0;                               // 2 M-tiles x 32 KB
 constexpr int OFF_K = OFF_Q + 2 * kTileBytes;          // 2 stages x 32 KB
 constexpr int OFF_V = OFF_K + 2 * kTileBytes;          // 2 stages x 32 KB
 constexpr int OFF_BAR = OFF_V + 2 * kTileBytes;
-// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_full[2]
-constexpr int NBAR = 1 + 2 * 7;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2],
+// o_full[2], drain (the MMA issuer's last commit after an abort)
+constexpr int NBAR = 1 + 2 * 7 + 1;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TMEM + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;  // + alignment slack
@@ -221,11 +208,22 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Wait that stops waiting once the CTA has given up.
+// Wait that stops waiting once the CTA has given up (at once, or as soon as another warp
+// does).  After a wait that may have been skipped, a thread makes no further arrival on a
+// barrier that counts transaction bytes (its previous phase may still be pending).
 __device__ __forceinline__ void wait_or_abort(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag, int* err) {
-  if (*abort_flag) return;
-  if (!mbar_wait(bar, parity, err)) *abort_flag = 1;
+                                              volatile int* abort_flag, int* err,
+                                              long long limit) {
+  if (*abort_flag || mbar_try_wait(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return;
+    if (clock64() - t0 > limit) {
+      flag_error(err, PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+      return;
+    }
+  }
 }
 
 template <typename T>
@@ -250,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bar + 9;
   uint64_t* p_full = bar + 11;
   uint64_t* o_full = bar + 13;
+  uint64_t* drain = bar + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
 
@@ -261,12 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- which (sequence, kv-head, query block), and which part of its keys
   int item = blockIdx.x, part = -1;  // part -1: all keys; 0 / 1: first / second half
-  const bool pmode = a.prefix_chunks > 0;
-  int piece = 0;
-  if (pmode) {
-    piece = item % a.prefix_chunks;
-    item /= a.prefix_chunks;
-  } else if (a.split_items > 0 && (int)blockIdx.x >= a.whole_items) {
+  if (a.split_items > 0 && (int)blockIdx.x >= a.whole_items) {
     const int j = blockIdx.x - a.whole_items;
     item = a.whole_items + (j >> 1);
     part = j & 1;
@@ -290,16 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = a.qsl[s + 1] - q_begin;
   const int Lraw = a.seq_lens[s];
   const int L = Lraw < 0 ? 0 : (Lraw > a.seq_cap ? a.seq_cap : Lraw);
-  const bool ksplit = pmode && a.ksplit;
-  const int q0 = qb * (ksplit ? MQ : 2 * MQ);
-  if (pmode) {
-    // a group: members qsl[s] .. qsl[s+1]-1, prefix a multiple of the block size
-    const bool layout_bad = n < 0 || n > a.max_query_len || q_begin < 0 || q_begin + n > a.q_rows;
-    const bool prefix_bad = Lraw != L || (L & ((1 << a.log2_bs) - 1));
-    if ((layout_bad || prefix_bad) && threadIdx.x == 0 && qb == 0 && h == 0 && piece == 0)
-      flag_error(a.err, layout_bad ? PA_DEVERR_QUERY_LAYOUT : PA_DEVERR_PREFIX);
-    if (layout_bad) return;
-  } else if (n < 0 || n > L || n > a.max_query_len || Lraw != L) {
+  const int q0 = qb * 2 * MQ;
+  if (n < 0 || n > L || n > a.max_query_len || Lraw != L) {
     if (threadIdx.x == 0 && qb == 0 && h == 0)
       flag_error(a.err, (n < 0 || n > L || n > a.max_query_len) ? PA_DEVERR_QUERY_LAYOUT
                                                                : PA_DEVERR_SEQ_TOO_LONG);
@@ -313,12 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   // keys any row of this CTA can see: [0, kv_end); this CTA takes tiles [kt_lo, kt_hi)
-  const int kv_end = pmode ? L : min(L, L - n + min(n, q0 + 2 * MQ));
+  const int kv_end = min(L, L - n + min(n, q0 + 2 * MQ));
   const int n_kt_all = (kv_end + kBN - 1) / kBN;
-  const int kt_lo = pmode ? (int)((long long)piece * n_kt_all / a.prefix_chunks)
-                          : (part == 1 ? n_kt_all / 2 : 0);
-  const int kt_hi = pmode ? (int)((long long)(piece + 1) * n_kt_all / a.prefix_chunks)
-                          : (part == 0 ? n_kt_all / 2 : n_kt_all);
+  const int kt_lo = part == 1 ? n_kt_all / 2 : 0;
+  const int kt_hi = part == 0 ? n_kt_all / 2 : n_kt_all;
   const int n_kt = kt_hi - kt_lo;  // tiles here; loops below count them from 0
 
   if (threadIdx.x == 0) {
@@ -332,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 4);
       mbar_init(&o_full[i], 1);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -353,10 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int mt = (warp - 4) >> 2;
     const int wq = warp & 3;              // TMEM lane quarter
     const int r = wq * 32 + lane;         // row of the M-tile
-    const int qi = q0 + (ksplit ? 0 : mt * MQ) + r / G;  // query index within the chunk
+    const int qi = q0 + mt * MQ + r / G;  // query index within the chunk
     const bool row_valid = qi < n;
-    // last visible key (inclusive): causal, or the whole prefix for the shared-prefix pass
-    const int limit = pmode ? L - 1 : L - n + min(qi, n - 1);
+    // last visible key (inclusive), causal
+    const int limit = L - n + min(qi, n - 1);
     const uint32_t t_s = tmem + ((uint32_t)(wq * 32) << 16) + mt * 128;
     const uint32_t t_o = tmem + ((uint32_t)(wq * 32) << 16) + 256 + mt * 128;
     // lowest limit in the warp decides whether a tile needs the causal mask
@@ -380,10 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(q_full);
     }
     float m_ref = -INFINITY, l = 0.f;
-    // tiles kt of this M-tile (all of them; with ksplit, those with kt % 2 == mt), and
-    // j counts them
-    for (int kt = ksplit ? mt : 0, j = 0; kt < n_kt; kt += ksplit ? 2 : 1, ++j) {
-      wait_or_abort(&s_full[mt], j & 1, abort_flag, a.err);
+    for (int kt = 0, j = 0; kt < n_kt; ++kt, ++j) {
+      wait_or_abort(&s_full[mt], j & 1, abort_flag, a.err, a.wait_limit);
       tc_fence_after();
       const int key0 = (kt_lo + kt) * kBN;
       // the whole S row (128 keys) in registers: one pass over TMEM
@@ -442,8 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * alpha + sum;
       // keys past the sequence end in the last tile: clear their V rows
-      if ((ksplit || mt == 0) && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
-        wait_or_abort(&v_full[kt & 1], (kt >> 1) & 1, abort_flag, a.err);
+      if (mt == 0 && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
+        wait_or_abort(&v_full[kt & 1], (kt >> 1) & 1, abort_flag, a.err, a.wait_limit);
         uint8_t* vt = smem + OFF_V + (kt & 1) * kTileBytes;
         const int first = L - key0;  // first row to clear
         for (int i = threadIdx.x & 127; i < (kBN - first) * 16; i += 128) {
@@ -459,32 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&p_full[mt]);
     }
     // ---- epilogue: O / l -> out
-    wait_or_abort(&o_full[mt], 0, abort_flag, a.err);
+    wait_or_abort(&o_full[mt], 0, abort_flag, a.err, a.wait_limit);
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (pmode) {
-      // one piece of a group's prefix: normalised partial row and (reference max, sum)
-      const bool any = n_kt > 0 && l > 0.f;
-      const long long prow = (long long)(ksplit ? 2 * piece + mt : piece) * a.q_rows * a.num_q_heads +
-                             (long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(t_o + c * 32, v);
-        if (row_valid) {
-          float* po = a.pre_o + prow * kD + c * 32;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(po + j * 4) =
-                any ? make_float4(v[4 * j] * inv, v[4 * j + 1] * inv, v[4 * j + 2] * inv,
-                                  v[4 * j + 3] * inv)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      if (row_valid)
-        *reinterpret_cast<float2*>(a.pre_ml + prow * 2) =
-            any ? make_float2(m_ref, l) : make_float2(-INFINITY, 0.f);
-    } else if (part < 0) {
+    if (part < 0) {
       T* orow = static_cast<T*>(a.out) +
                 ((long long)(q_begin + qi) * a.num_q_heads + h * G + (r % G)) * kD;
 #pragma unroll
@@ -534,8 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        // the shared-prefix pass reads a group's prefix through its first member's row
-        const int32_t* trow = a.block_tables + (long long)(pmode ? q_begin : s) * a.max_blocks;
+        const int32_t* trow = a.block_tables + (long long)s * a.max_blocks;
         const int bs_mask = (1 << a.log2_bs) - 1;
         // block-table entries of a tile's eight 16-token runs, read one tile ahead so
         // that their latency overlaps the previous tile's waits and copies
@@ -548,6 +508,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         int next_id[8];
         if (n_kt > 0) table_ids(0, next_id);
+        // K tiles (V tiles) handled so far, and bit i: the copy of the i-th last of them was
+        // issued.  A stage is reused only after its previous tile was consumed, so only the
+        // last two tiles of each ring can still be landing.
+        uint32_t k_issued = 0, v_issued = 0;
+        int nk = 0, nv = 0;
         for (int kt = 0; kt < n_kt; ++kt) {
           const int st = kt & 1;
           const uint32_t ph = ((kt >> 1) & 1) ^ 1;
@@ -565,15 +530,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (kt + 1 < n_kt) table_ids(kt + 1, next_id);
-          wait_or_abort(&k_empty[st], ph, abort_flag, a.err);
-          mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          wait_or_abort(&k_empty[st], ph, abort_flag, a.err, a.wait_limit);
+          if (*abort_flag) break;  // a wait may have been skipped: no more arrivals
+          k_issued <<= 1;
+          ++nk;
+          if (!(a.test_withhold && blockIdx.x == 0 && kt == 0)) {  // (testing hook)
+            mbar_arrive_expect_tx(&k_full[st], kTileBytes);
   #pragma unroll
-          for (int r = 0; r < 8; ++r)
+            for (int r = 0; r < 8; ++r)
   #pragma unroll
-            for (int kh = 0; kh < 2; ++kh)
-              tma_load_4d(smem + OFF_K + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmK,
-                          kh * 64, h, row[r], bid[r], &k_full[st]);
-          wait_or_abort(&v_empty[st], ph, abort_flag, a.err);
+              for (int kh = 0; kh < 2; ++kh)
+                tma_load_4d(smem + OFF_K + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmK,
+                            kh * 64, h, row[r], bid[r], &k_full[st]);
+            k_issued |= 1u;
+          }
+          wait_or_abort(&v_empty[st], ph, abort_flag, a.err, a.wait_limit);
+          if (*abort_flag) break;
+          v_issued <<= 1;
+          ++nv;
           mbar_arrive_expect_tx(&v_full[st], kTileBytes);
   #pragma unroll
           for (int r = 0; r < 8; ++r)
@@ -581,6 +555,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kh = 0; kh < 2; ++kh)
               tma_load_4d(smem + OFF_V + st * kTileBytes + kh * kHalfBytes + r * 16 * 128, &tmV,
                           kh * 64, h, row[r], bid[r], &v_full[st]);
+          v_issued |= 1u;
+        }
+        {  // no copy may still be landing in shared memory at the exit (a no-op unless the
+           // CTA aborted: the MMA issuer has waited for every copy otherwise)
+          for (int i = 0; i < 2; ++i) {
+            const int ck = nk - 1 - i, cv = nv - 1 - i;
+            if (ck >= 0 && (k_issued & (1u << i)))
+              (void)mbar_wait(&k_full[ck & 1], (ck >> 1) & 1, a.err, a.wait_limit);
+            if (cv >= 0 && (v_issued & (1u << i)))
+              (void)mbar_wait(&v_full[cv & 1], (cv >> 1) & 1, a.err, a.wait_limit);
+          }
         }
       }
     } else if (warp == 1) {
@@ -611,59 +596,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8, db, id_pv, (acc || kk > 0));
           }
         };
-        wait_or_abort(q_full, 0, abort_flag, a.err);
+        wait_or_abort(q_full, 0, abort_flag, a.err, a.wait_limit);
         tc_fence_after();
-        if (ksplit) {
-          // two chains: M-tile mt takes tiles mt, mt + 2, ... (stage mt of each ring)
-          for (int mt = 0; mt < 2 && mt < n_kt; ++mt) {
-            wait_or_abort(&k_full[mt], 0, abort_flag, a.err);
+        if (n_kt > 0) {
+          wait_or_abort(&k_full[0], 0, abort_flag, a.err, a.wait_limit);
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          mma_commit(&k_empty[0]);
+        }
+        for (int kt = 0; kt < n_kt; ++kt) {
+          const int st = kt & 1;
+          const bool more = kt + 1 < n_kt;
+          wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err, a.wait_limit);
+          if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err, a.wait_limit);
+          for (int mt = 0; mt < 2; ++mt) {
+            wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err, a.wait_limit);
             tc_fence_after();
-            issue_s(mt, mt);
-            mma_commit(&k_empty[mt]);
+            issue_pv(mt, kt, kt > 0);
+            if (more) issue_s(mt, kt + 1);
           }
-          for (int j = 0; 2 * j < n_kt; ++j) {
-            for (int mt = 0; mt < 2; ++mt) {
-              const int kt = 2 * j + mt;
-              if (kt >= n_kt) break;
-              wait_or_abort(&p_full[mt], j & 1, abort_flag, a.err);
-              wait_or_abort(&v_full[mt], j & 1, abort_flag, a.err);
-              tc_fence_after();
-              issue_pv(mt, kt, j > 0);
-              mma_commit(&v_empty[mt]);
-              if (kt + 2 < n_kt) {
-                wait_or_abort(&k_full[mt], (j + 1) & 1, abort_flag, a.err);
-                tc_fence_after();
-                issue_s(mt, kt + 2);
-                mma_commit(&k_empty[mt]);
-              }
-            }
-          }
-          mma_commit(&o_full[0]);
-          mma_commit(&o_full[1]);
-        } else {
-          if (n_kt > 0) {
-            wait_or_abort(&k_full[0], 0, abort_flag, a.err);
-            tc_fence_after();
-            issue_s(0, 0);
-            issue_s(1, 0);
-            mma_commit(&k_empty[0]);
-          }
-          for (int kt = 0; kt < n_kt; ++kt) {
-            const int st = kt & 1;
-            const bool more = kt + 1 < n_kt;
-            wait_or_abort(&v_full[st], (kt >> 1) & 1, abort_flag, a.err);
-            if (more) wait_or_abort(&k_full[(kt + 1) & 1], ((kt + 1) >> 1) & 1, abort_flag, a.err);
-            for (int mt = 0; mt < 2; ++mt) {
-              wait_or_abort(&p_full[mt], kt & 1, abort_flag, a.err);
-              tc_fence_after();
-              issue_pv(mt, kt, kt > 0);
-              if (more) issue_s(mt, kt + 1);
-            }
-            if (more) mma_commit(&k_empty[(kt + 1) & 1]);
-            mma_commit(&v_empty[st]);
-          }
-          mma_commit(&o_full[0]);
-          mma_commit(&o_full[1]);
+          if (more) mma_commit(&k_empty[(kt + 1) & 1]);
+          mma_commit(&v_empty[st]);
+        }
+        mma_commit(&o_full[0]);
+        mma_commit(&o_full[1]);
+        if (*abort_flag) {
+          // the softmax warps may not have waited for the last products: the MMAs issued so
+          // far must be complete before the TMEM they write is freed
+          mma_commit(drain);
+          (void)mbar_wait(drain, 0, a.err, a.wait_limit);
         }
       }
     }
@@ -772,96 +734,7 @@ pa_status dispatch(int G, const CUtensorMap& tk, const CUtensorMap& tv, const Ar
   }
 }
 
-template <typename T, int G>
-pa_status launch_prefix(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a,
-                        long long grid, cudaStream_t stream) {
-  auto kern = chunked_prefill_kernel<T, G>;
-  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES)) return PA_ERR_CUDA;
-  kern<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(tk, tv, a);
-  return check_launch();
-}
-
 }  // namespace prefill
-
-SharedPrefixPlan plan_shared_prefix(int num_groups, int num_kv_heads, int G, int max_group_size,
-                                    int max_prefix_len) {
-  SharedPrefixPlan p;
-  const int MQ = prefill::kM / G;
-  // groups that fit one M-tile of rows: both M-tiles take the same rows, alternate tiles
-  p.ksplit = max_group_size <= MQ ? 1 : 0;
-  p.qblocks = p.ksplit ? 1 : (max_group_size + 2 * MQ - 1) / (2 * MQ);
-  const long long items = std::max<long long>(1, (long long)num_groups * num_kv_heads * p.qblocks);
-  const long long tiles = (std::max(0, max_prefix_len) + prefill::kBN - 1) / prefill::kBN;
-  const long long fill = std::max<long long>(1, num_sms() / items);  // pieces that fill one wave
-  const long long per_piece = p.ksplit ? 2 : 1;                        // partials per piece
-  p.pieces = (int)std::max<long long>(
-      1, std::min<long long>({kMaxPrefixChunks / per_piece, fill,
-                              std::max<long long>(1, tiles / per_piece)}));
-  p.slots = p.pieces * (int)per_piece;
-  return p;
-}
-
-pa_status shared_prefix_pass(const void* q, const void* k_cache, const void* v_cache,
-                             const int32_t* block_tables, int max_blocks_per_seq,
-                             const int32_t* group_starts, const int32_t* prefix_lens,
-                             int num_groups, int max_group_size, int max_prefix_len, int q_rows,
-                             int num_q_heads, int num_kv_heads, float scale, int block_size,
-                             int num_blocks, const SharedPrefixPlan& plan, float* pre_o,
-                             float* pre_ml, pa_dtype dtype, int* err, cudaStream_t stream) {
-  const int G = num_q_heads / num_kv_heads;
-  CUtensorMap tk, tv;
-  const uint64_t row = (uint64_t)prefill::kD * 2;
-  const uint64_t cdims[4] = {(uint64_t)prefill::kD, (uint64_t)num_kv_heads, (uint64_t)block_size,
-                             (uint64_t)num_blocks};
-  const uint64_t cstr[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
-  const uint32_t cbox[4] = {64, 1, 16, 1};
-  if (!encode_tmap_16bit(&tk, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap_16bit(&tv, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B))
-    return PA_ERR_CUDA;
-  prefill::Args a = {};
-  a.out = nullptr;
-  a.q = q;
-  a.block_tables = block_tables;
-  a.seq_lens = prefix_lens;
-  a.qsl = group_starts;
-  a.err = err;
-  a.num_seqs = num_groups;
-  a.num_q_heads = num_q_heads;
-  a.num_kv_heads = num_kv_heads;
-  a.max_blocks = max_blocks_per_seq;
-  a.log2_bs = block_size == 16 ? 4 : 5;
-  a.num_blocks = num_blocks;
-  a.max_query_len = max_group_size;
-  a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_prefix_len);
-  a.qblocks = plan.qblocks;
-  a.qscale = scale * 1.4426950408889634f;
-  a.whole_items = 0;
-  a.split_items = 0;
-  a.part_o = a.part_ml = nullptr;
-  a.rowmap = nullptr;
-  a.prefix_chunks = plan.pieces;
-  a.ksplit = plan.ksplit;
-  a.q_rows = q_rows;
-  a.pre_o = pre_o;
-  a.pre_ml = pre_ml;
-  a.skip_single = 0;
-  a.chunk_ids = nullptr;
-  a.chunk_cap = 0;
-  const long long grid = (long long)num_groups * num_kv_heads * a.qblocks * plan.pieces;
-  if (grid <= 0) return PA_OK;
-  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-  auto go = [&](auto tag) -> pa_status {
-    using T = decltype(tag);
-    switch (G) {
-      case 1: return prefill::launch_prefix<T, 1>(tk, tv, a, grid, stream);
-      case 2: return prefill::launch_prefix<T, 2>(tk, tv, a, grid, stream);
-      case 4: return prefill::launch_prefix<T, 4>(tk, tv, a, grid, stream);
-      case 8: return prefill::launch_prefix<T, 8>(tk, tv, a, grid, stream);
-      default: return PA_ERR_UNSUPPORTED;
-    }
-  };
-  return dtype == PA_F16 ? go(__half{}) : go(__nv_bfloat16{});
-}
 
 }  // namespace pa
 
@@ -901,7 +774,7 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
     return PA_ERR_INVALID_ARG;
   if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15)
     return PA_ERR_INVALID_ARG;
-  int* err = pa::device_error_flag();
+  int* err = pa::launch_prologue();
   if (!err) return PA_ERR_CUDA;
   const int MQ = 128 / G;
   CUtensorMap tk, tv;
@@ -930,13 +803,10 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
   a.seq_cap = (int)std::min<long long>((long long)max_blocks_per_seq * block_size, max_seq_len);
   a.qblocks = (max_query_len + 2 * MQ - 1) / (2 * MQ);
   a.qscale = scale * 1.4426950408889634f;
-  a.prefix_chunks = 0;
-  a.ksplit = 0;
+  a.wait_limit = pa::take_wait_limit(pa::kTestPrefill, &a.test_withhold);
   a.skip_single = skip_single ? 1 : 0;
   a.chunk_ids = chunk_ids;
   a.chunk_cap = chunk_cap;
-  a.q_rows = 0;
-  a.pre_o = a.pre_ml = nullptr;
   // the split's row map stores output row numbers as int
   const long long rows = (long long)num_seqs * max_query_len * num_q_heads;
   if (rows > 0x7fffffffLL) workspace = nullptr;

@@ -106,7 +106,7 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* k, const void* v, void
     return PA_ERR_INVALID_ARG;
   const uintptr_t al = (uintptr_t)k | (uintptr_t)v | (uintptr_t)k_cache | (uintptr_t)v_cache;
   if (al & 15) return PA_ERR_INVALID_ARG;
-  int* err = pa::device_error_flag();
+  int* err = pa::launch_prologue();
   if (!err) return PA_ERR_CUDA;
   const int row_vecs = num_kv_heads * head_dim / 8;  // 8 elements per step
   const int threads = 256;
@@ -143,7 +143,7 @@ extern "C" pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_
   if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
   const uintptr_t al = (uintptr_t)k | (uintptr_t)v | (uintptr_t)k_cache | (uintptr_t)v_cache;
   if (al & 15) return PA_ERR_INVALID_ARG;  // 16-byte vector access
-  int* err = pa::device_error_flag();
+  int* err = pa::launch_prologue();
   if (!err) return PA_ERR_CUDA;
   const int row_vecs = num_kv_heads * head_dim * 2 / 16;
   const int threads = 256;

@@ -7,6 +7,8 @@ import re
 
 import pytest
 
+from tests._devmem import devmem
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pagedattn.h")
 
@@ -55,7 +57,7 @@ def test_status_strings(palib):
 
 
 def _ws_bound(B, Hq, L, P, D=128):
-    """The documented upper bound: merge records (8 B per sequence and q-head, padded
+    """The documented upper bound: merge tickets (at most 8 B per sequence and q-head, padded
     to 256 B) and partial rows of D+2 fp32: (256 + B) * Hq, plus, with an explicit
     partition, B * Hq * ceil(ceil(L/16) / (P/16)) + Hq."""
     rows = (256 + B) * Hq
@@ -96,8 +98,9 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, -1, 8, 128, 16, 16, 0, nul) == 1
     assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 4, 8, 128, 16, 16, 0, nul) == 1
     assert L.pa_reshape_and_cache(nul, nul, nul, nul, nul, 0, 8, 128, 16, 16, 0, nul) == 0
-    p = ctypes.c_void_p(4096)
-    args = dict(out=p, q=p, kc=p, vc=p, bt=p, mb=8, sl=p, B=2, Hq=8, Hkv=8, D=128, scale=0.1,
+    m = devmem()
+    args = dict(out=m.region(), q=m.region(), kc=m.region(), vc=m.region(), bt=m.region(), mb=8,
+                sl=m.region(), B=2, Hq=8, Hkv=8, D=128, scale=0.1,
                 bs=16, N=16, maxlen=100, P=0, ws=None, wsb=0, dt=0, st=None)
 
     def dec(**kw):
@@ -113,25 +116,28 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(P=24) == 1                    # partition not a multiple of 16
     assert dec(P=4096) == 2                  # partition above 2048 tokens
     assert dec(q=None) == 1                  # null pointer
-    assert dec(q=ctypes.c_void_p(4100)) == 1  # misaligned
+    assert dec(q=m.region(4)) == 1           # misaligned
     assert dec(dt=3) == 2
     assert dec(B=0) == 0                     # nothing to do
     assert dec(B=5000) == 2                  # more sequences than the schedule holds
-    assert dec(P=512) == 3                   # every call needs a workspace (merge records)
-    assert dec(maxlen=8000, P=512, ws=p, wsb=100) == 3
-    assert dec(maxlen=8000, P=512, ws=ctypes.c_void_p(4096 + 16), wsb=1 << 24) == 1  # alignment
+    assert dec(P=512) == 3                   # every call needs a workspace (merge tickets)
+    assert dec(maxlen=8000, P=512, ws=m.region(), wsb=100) == 3
+    assert dec(maxlen=8000, P=512, ws=m.region(16), wsb=1 << 24) == 1  # alignment
+    assert palib.pa_last_launch_count() == 0
 
 
 def test_append_decode_arguments_rejected_on_host(palib):
     L = _raw(palib)
-    p = ctypes.c_void_p(4096)
+    m = devmem()
+    o, q, kc, vc, bt, sl = (m.region() for _ in range(6))
+    kn0, vn0 = m.region(), m.region()
 
-    def app(kn=p, vn=p, B=2, D=128, ws=None, wsb=0):
-        return L.pa_decode_append(p, p, kn, vn, p, p, p, 8, p, B, 8, 8, D, 0.1, 16, 16, 100, 512,
-                                  ws, wsb, 0, None)
+    def app(kn=kn0, vn=vn0, B=2, D=128, ws=None, wsb=0):
+        return L.pa_decode_append(o, q, kn, vn, kc, vc, bt, 8, sl, B, 8, 8, D, 0.1, 16, 16, 100,
+                                  512, ws, wsb, 0, None)
     assert app(kn=None) == 1                     # new K missing
     assert app(vn=None) == 1                     # new V missing
-    assert app(kn=ctypes.c_void_p(4100)) == 1    # misaligned
+    assert app(kn=m.region(4)) == 1              # misaligned
     assert app(D=64) == 2                        # head_dim must be 128
     assert app(B=0) == 0                         # nothing to do
     assert app() == 3                            # needs a workspace
@@ -140,17 +146,19 @@ def test_append_decode_arguments_rejected_on_host(palib):
 
 def test_fp8_arguments_rejected_on_host(palib):
     L = _raw(palib)
-    p = ctypes.c_void_p(4096)
+    m = devmem()
+    k, v, kc, vc, sm, ks0, vs0 = (m.region() for _ in range(7))
     nul = None
     # scatter: missing scales, odd block size, bad source type
-    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, nul, p, 4, 8, 128, 16, 16, 0, nul) == 1
-    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 4, 8, 128, 16, 24, 0, nul) == 2
-    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 4, 8, 128, 16, 16, 7, nul) == 2
-    assert L.pa_reshape_and_cache_fp8(p, p, p, p, p, p, p, 0, 8, 128, 16, 16, 0, nul) == 0
+    assert L.pa_reshape_and_cache_fp8(k, v, kc, vc, sm, nul, vs0, 4, 8, 128, 16, 16, 0, nul) == 1
+    assert L.pa_reshape_and_cache_fp8(k, v, kc, vc, sm, ks0, vs0, 4, 8, 128, 16, 24, 0, nul) == 2
+    assert L.pa_reshape_and_cache_fp8(k, v, kc, vc, sm, ks0, vs0, 4, 8, 128, 16, 16, 7, nul) == 2
+    assert L.pa_reshape_and_cache_fp8(k, v, kc, vc, sm, ks0, vs0, 0, 8, 128, 16, 16, 0, nul) == 0
+    o, q, bt, sl = (m.region() for _ in range(4))
 
-    def dec(ks=p, vs=p, B=2, ws=None, wsb=0):
-        return L.pa_decode_fp8(p, p, p, p, ks, vs, p, 8, p, B, 8, 8, 128, 0.1, 16, 16, 100, 512,
-                               ws, wsb, 0, None)
+    def dec(ks=ks0, vs=vs0, B=2, ws=None, wsb=0):
+        return L.pa_decode_fp8(o, q, kc, vc, ks, vs, bt, 8, sl, B, 8, 8, 128, 0.1, 16, 16, 100,
+                               512, ws, wsb, 0, None)
     assert dec(ks=None) == 1 and dec(vs=None) == 1
     assert dec(B=0) == 0
     assert dec() == 3  # needs a workspace
@@ -159,31 +167,36 @@ def test_fp8_arguments_rejected_on_host(palib):
 
 def test_shared_prefix_arguments_rejected_on_host(palib):
     L = _raw(palib)
-    p = ctypes.c_void_p(4096)
+    m = devmem()
+    o, q, kc, vc, bt, sl, gs0, pl0 = (m.region() for _ in range(8))
     nul = None
 
-    def dec(B=8, gs=p, pl=p, ng=2, mg=4, mp=256, ws=None, wsb=0):
-        return L.pa_decode_shared_prefix(p, p, p, p, p, 32, p, B, gs, pl, ng, mg, mp, 32, 8, 128,
-                                         0.1, 16, 1000, 512, ws, wsb, 0, nul)
+    def dec(B=8, gs=gs0, pl=pl0, ng=2, mg=4, mp=256, ws=None, wsb=0):
+        return L.pa_decode_shared_prefix(o, q, kc, vc, bt, 32, sl, B, gs, pl, ng, mg, mp, 32, 8,
+                                         128, 0.1, 16, 1000, 512, ws, wsb, 0, nul)
     assert dec(ng=-1) == 1 and dec(mg=-1) == 1 and dec(mp=-1) == 1
     assert dec(ng=9) == 1 and dec(mg=9) == 1       # more groups / members than sequences
     assert dec(gs=nul) == 1 and dec(pl=nul) == 1
     assert dec(B=0, ng=0, mg=0) == 0               # nothing to do
     assert dec() == 3 and dec(mp=0) == 3            # needs a workspace (shared or plain)
     base = palib.pa_decode_workspace_size(8, 32, 128, 512, 0)
-    assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 128, 512) >= base + 8 * 8 * 32 * 130 * 4
-    assert palib.pa_decode_shared_prefix_workspace_size(0, 32, 128, 512) == 0
+    # chunk partials: (256 + num_seqs) x num_kv_heads x 16 rows of 130 fp32 after the base
+    assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 8, 128, 512) == \
+        -(-base // 256) * 256 + (256 + 8) * 8 * 16 * 130 * 4
+    assert palib.pa_decode_shared_prefix_workspace_size(0, 32, 8, 128, 512) == 0
+    assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 0, 128, 512) == 0
     assert palib.pa_last_launch_count() == 0
 
 
 def test_varlen_arguments_rejected_on_host(palib):
     L = _raw(palib)
-    p = ctypes.c_void_p(4096)
+    m = devmem()
+    o, q, kc, vc, bt, sl, qsl0 = (m.region() for _ in range(7))
     nul = None
 
-    def call(B=4, rows=10, mq=5, qsl=p, ws=None, wsb=0):
-        return L.pa_attention_varlen(p, p, p, p, p, 32, p, qsl, B, rows, mq, -1, 32, 8, 128, 0.1,
-                                     16, 1000, 512, ws, wsb, 0, nul)
+    def call(B=4, rows=10, mq=5, qsl=qsl0, ws=None, wsb=0):
+        return L.pa_attention_varlen(o, q, kc, vc, bt, 32, sl, qsl, B, rows, mq, -1, 32, 8, 128,
+                                     0.1, 16, 1000, 512, ws, wsb, 0, nul)
     assert call(B=-1) == 1 and call(rows=-1) == 1 and call(mq=-1) == 1
     assert call(B=0) == 0 and call(rows=0) == 0 and call(mq=0) == 0   # nothing to do
     assert call(qsl=nul) == 1
@@ -196,22 +209,33 @@ def test_varlen_arguments_rejected_on_host(palib):
 
 def test_block_pool_arguments_rejected_on_host(palib):
     L = _raw(palib)
-    p = ctypes.c_void_p(4096)
+    m = devmem()
+    ring0, state, tables, owned, lens, qlens, slots0, granted, fin0 = (
+        m.region() for _ in range(9))
     nul = None
-    assert L.pa_block_pool_init(p, p, 0, nul) == 1          # empty pool
-    assert L.pa_block_pool_init(nul, p, 8, nul) == 1        # ring missing
+    refs = m.region()
+    assert L.pa_block_pool_init(ring0, state, refs, 0, nul) == 1  # empty pool
+    assert L.pa_block_pool_init(nul, state, refs, 8, nul) == 1    # ring missing
 
-    def alloc(ring=p, n=64, mb=8, B=4, bs=16, slots=p):
-        return L.pa_block_allocate(ring, p, n, p, mb, p, p, p, B, bs, slots, p, nul)
+    def alloc(ring=ring0, n=64, mb=8, B=4, bs=16, slots=slots0):
+        return L.pa_block_allocate(ring, state, refs, n, tables, mb, owned, lens, qlens, B, bs,
+                                   slots, granted, nul)
     assert alloc(n=0) == 1 and alloc(mb=0) == 1 and alloc(B=-1) == 1
     assert alloc(bs=8) == 2                                  # block size 16 or 32
     assert alloc(B=4097) == 2                                # one CTA's limit
     assert alloc(B=0) == 0                                   # nothing to do
     assert alloc(ring=nul) == 1 and alloc(slots=nul) == 1
 
-    def free(n=64, B=4, fin=p):
-        return L.pa_block_free(p, p, n, p, 8, p, fin, B, nul)
+    def free(n=64, B=4, fin=fin0):
+        return L.pa_block_free(ring0, state, refs, n, tables, 8, owned, fin, B, nul)
     assert free(n=0) == 1 and free(B=4097) == 2 and free(B=0) == 0 and free(fin=nul) == 1
+    src, dst, k = m.region(), m.region(), m.region()
+
+    def share(rf=refs, n=64, B=4, pairs=2, s_=src):
+        return L.pa_block_share(rf, n, tables, 8, owned, B, s_, dst, k, pairs, nul)
+    assert share(rf=nul) == 1                                # shares need reference counts
+    assert share(n=0) == 1 and share(B=-1) == 1 and share(pairs=-1) == 1
+    assert share(pairs=0) == 0 and share(s_=nul) == 1
     assert palib.pa_last_launch_count() == 0
 
 

@@ -1,9 +1,11 @@
 """GPU parity for device-side block-table maintenance through the C ABI: after every
-step, pa_block_allocate / pa_block_free must leave the ring, its {head, count}, the
-block tables and the owned counts exactly as the oracle's FIFO pool does, and write the
-same slot mapping and grant flags — including steps where the pool runs dry (a
-sequence preempted, later ones still served), table rows too short, prefill-sized
-appends, the 4096-sequence limit, and a full loop of allocate → scatter → decode."""
+step, pa_block_allocate / pa_block_free / pa_block_share must leave the ring, its
+{head, count}, the block tables, the owned counts and the reference counts exactly as
+the oracle's FIFO pool does, and write the same slot mapping and grant flags —
+including steps where the pool runs dry (a sequence preempted, later ones still
+served), table rows too short, prefill-sized appends, the 4096-sequence limit, prompt
+blocks shared by a group and released together, and a full loop of allocate → scatter
+→ decode."""
 import numpy as np
 import pytest
 import torch
@@ -20,7 +22,7 @@ DEV = "cuda"
 class _Pair:
     """The same pool and tables on both sides."""
 
-    def __init__(self, n_blocks, B, max_blocks, bs):
+    def __init__(self, n_blocks, B, max_blocks, bs, refs=False):
         self.bs = bs
         self.pool = obp.BlockPool(n_blocks)
         self.tables = np.zeros((B, max_blocks), dtype=np.int64)
@@ -28,7 +30,8 @@ class _Pair:
         self.lens = np.zeros(B, dtype=np.int64)
         self.ring = torch.full((n_blocks,), -7, dtype=torch.int32, device=DEV)
         self.state = torch.full((2,), -7, dtype=torch.int32, device=DEV)
-        pa.pa_block_pool_init(self.ring, self.state)
+        self.refs = torch.full((n_blocks,), -7, dtype=torch.int32, device=DEV) if refs else None
+        pa.pa_block_pool_init(self.ring, self.state, self.refs)
         self.d_tables = torch.zeros((B, max_blocks), dtype=torch.int32, device=DEV)
         self.d_owned = torch.zeros(B, dtype=torch.int32, device=DEV)
 
@@ -39,7 +42,7 @@ class _Pair:
         d_slots = torch.full((max(int(q.sum()), 1),), -9, dtype=torch.int32, device=DEV)
         d_granted = torch.full((len(q),), -9, dtype=torch.int32, device=DEV)
         pa.pa_block_allocate(self.ring, self.state, self.d_tables, self.d_owned, d_lens, d_q,
-                             self.bs, d_slots, d_granted)
+                             self.bs, d_slots, d_granted, block_refs=self.refs)
         slots, granted = obp.allocate_step(self.pool, self.tables, self.owned, self.lens, q,
                                            self.bs)
         self.lens += np.where(granted, q, 0)
@@ -53,14 +56,26 @@ class _Pair:
         fin = np.zeros(len(self.owned), dtype=bool)
         fin[list(seqs)] = True
         pa.pa_block_free(self.ring, self.state, self.d_tables, self.d_owned,
-                         torch.tensor(fin.astype(np.int32), device=DEV))
+                         torch.tensor(fin.astype(np.int32), device=DEV), block_refs=self.refs)
         obp.free_sequences(self.pool, self.tables, self.owned, fin)
         self.lens[fin] = 0
         self.check()
 
-    def check(self):
+    def share(self, pairs, expect_error=False):
+        src, dst, k = (np.asarray([p[i] for p in pairs], dtype=np.int64) for i in range(3))
+        dev = [torch.tensor(x, dtype=torch.int32, device=DEV) for x in (src, dst, k)]
+        pa.pa_block_share(self.refs, self.d_tables, self.d_owned, *dev)
+        done = obp.share_blocks(self.pool, self.tables, self.owned, src, dst, k)
+        self.lens[dst[done]] = k[done] * self.bs
+        self.check(expect_error=expect_error)
+        return done
+
+    def check(self, expect_error=False):
         torch.cuda.synchronize()
-        assert pa.pa_get_device_error() == 0
+        err = pa.pa_get_device_error()
+        assert err == (pa.PA_DEVERR["POOL"] if expect_error else 0), err
+        if self.refs is not None:
+            assert np.array_equal(self.refs.cpu().numpy(), self.pool.refs), "refs"
         st = self.state.cpu().numpy()
         assert (int(st[0]), int(st[1])) == (self.pool.head, self.pool.count), "head/count"
         assert np.array_equal(self.ring.cpu().numpy(), self.pool.ring), "ring"
@@ -79,6 +94,80 @@ def _run(seed, B, steps, n_blocks, bs, max_blocks, q_choices, free_every=4, n_fr
             _, granted = pair.alloc(rng.choice(q_choices, size=B))
             n_preempted += int((~granted).sum())
     return pair, n_preempted
+
+
+def test_shared_prompt_blocks_match_oracle():
+    # parallel sampling: the first sequence of each group of four prefills a prompt, the
+    # other three take its whole blocks, every member decodes, and members finish at
+    # different steps (whole groups together at the end)
+    rng = np.random.default_rng(21)
+    B, G = 16, 4
+    pair = _Pair(300, B, 40, 16, refs=True)
+    prompt = [0] * B
+    for g in range(B // G):
+        prompt[g * G] = int(rng.integers(20, 120))
+    pair.alloc(prompt)
+    pairs = [(g * G, g * G + m, int(pair.owned[g * G]) - (1 if prompt[g * G] % 16 else 0))
+             for g in range(B // G) for m in range(1, G)]
+    assert pair.share(pairs).all()
+    for t in range(12):
+        pair.alloc([1] * B)
+        if t == 5:
+            pair.free([1, 6, 11])
+        if t == 8:
+            pair.free([0, 4, 9, 14])
+    pair.free(range(B))  # the rest, shared blocks returning once each
+    assert pair.pool.count == 300 and (pair.pool.refs == 0).all()
+
+
+@pytest.mark.parametrize("seed", [31, 32, 33])
+def test_random_sharing_matches_oracle(seed):
+    rng = np.random.default_rng(seed)
+    B = 24
+    pair = _Pair(160, B, 24, 16, refs=True)
+    for t in range(30):
+        if t % 5 == 4:
+            pair.free(sorted(set(rng.integers(0, B, 4).tolist())))
+        elif t % 5 == 2:
+            empty = [s for s in range(B) if pair.owned[s] == 0]
+            holders = [s for s in range(B) if pair.owned[s] > 0]
+            rng.shuffle(empty)
+            pairs = []
+            for d in empty[:4]:
+                if not holders:
+                    break
+                src = int(rng.choice([h for h in holders if h not in empty[:4]] or [d]))
+                if src == d:
+                    continue
+                pairs.append((src, d, int(rng.integers(0, int(pair.owned[src]) + 1))))
+            if pairs:
+                pair.share(pairs)
+        else:
+            pair.alloc(rng.choice([0, 1, 1, 17, 40], size=B))
+
+
+def test_invalid_share_is_flagged_and_skipped():
+    pair = _Pair(40, 4, 8, 16, refs=True)
+    pair.alloc([20, 5, 0, 0])
+    done = pair.share([(0, 1, 1), (0, 2, 3), (0, 3, 2)], expect_error=True)
+    # dst 1 owns a block, and 3 blocks are more than seq 0 owns: only the last pair applies
+    assert done.tolist() == [False, False, True]
+
+
+def test_release_below_zero_is_flagged():
+    # a count cleared behind the pool's back: the block is released once more than it was
+    # held; the pool flags it and keeps the block out of the ring
+    pair = _Pair(8, 2, 4, 16, refs=True)
+    pair.alloc([20, 0])
+    blk = int(pair.tables[0, 1])
+    pair.refs[blk] = 0
+    pa.pa_block_free(pair.ring, pair.state, pair.d_tables, pair.d_owned,
+                     torch.tensor([1, 0], dtype=torch.int32, device=DEV), block_refs=pair.refs)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error() == pa.PA_DEVERR["POOL"]
+    head, count = pair.state.cpu().tolist()
+    free = [int(pair.ring[(head + i) % 8]) for i in range(count)]
+    assert blk not in free and int(pair.tables[0, 0]) in free and count == 7
 
 
 def test_init_fills_ring_in_order():

@@ -23,7 +23,8 @@ def _gpu_shared(b, group_starts=None, prefix_lens=None, max_prefix=None):
     gs = b.group_starts if group_starts is None else group_starts
     pl = b.prefix_lens if prefix_lens is None else prefix_lens
     B, Hq, D = b.q.shape
-    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_size(B, Hq, D, b.max_seq_len),
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_size(B, Hq, b.num_kv_heads, D,
+                                                               b.max_seq_len),
                      dtype=torch.uint8, device=DEV)
     out = torch.full_like(b.q, float("nan"))
     sizes = (gs[1:] - gs[:-1]).cpu()
@@ -62,7 +63,7 @@ def _grouped_batch(name, lens, groups, prefix, G, dtype, bs=16, Hkv=4, seed=0):
 def test_shared_prompt_workloads(bs):
     bc = workloads.shared_prefix(block_size=bs, scale=1 / 8)[0]
     _, launches = _vs_oracle(bc, "shared prefix bs%d" % bs)
-    assert launches == 3  # prefix pass, decode of the own keys, merge
+    assert launches == 2  # ticket zeroing, then one decode grid over own keys and chunks
 
 
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
@@ -85,8 +86,8 @@ def test_groups_with_nothing_shared_and_gaps():
 
 
 def test_many_members_long_prefix_several_pieces():
-    # 40 members of one group at G = 8: two query blocks of the prefix pass; a 1040-token
-    # prefix (9 key tiles, the last partial) cut into up to 8 pieces
+    # 40 members of one group at G = 8: twenty chunks of two members over a 1040-token
+    # prefix (65 tiles), spread over many CTAs
     lens = [1040 + 1 + (7 * i) % 90 for i in range(40)]
     bc = _grouped_batch("many", lens, [list(range(40))], 1040, 8, torch.bfloat16, Hkv=2, seed=5)
     _vs_oracle(bc, "40 members, prefix 1040")

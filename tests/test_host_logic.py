@@ -82,7 +82,7 @@ def test_bench_routes_each_batch_to_its_call():
     assert st.group_bounds[id(shared)] == (8, 256)
     # every batch got a workspace of the size its call asks for
     assert st.ws[id(shared)].numel() == pa.pa_decode_shared_prefix_workspace_size(
-        64, 32, 128, shared.max_seq_len)
+        64, 32, 8, 128, shared.max_seq_len)
     assert st.ws[id(varlen)].numel() == pa.pa_attention_varlen_workspace_size(
         36, 32, 64, 128, varlen.max_seq_len)
 
