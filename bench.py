@@ -343,10 +343,8 @@ def rooflines(step, dec_ms, pre_ms, peaks):
         kname = ("pa_decode_fp8" if dec.k_scale is not None else
                  "pa_decode_shared_prefix" if shared else
                  "pa_decode_append" if step.fused[id(dec)] else "pa_decode")
-        kparts = (" (chunked_prefill_kernel prefix pass + zero_tickets_kernel + paged_decode_kernel,"
-                  " merge inside the decode launch)"
-                  if shared else " (zero_tickets_kernel + paged_decode_kernel, merge inside the "
-                                 "decode launch)")
+        kparts = (" (paged_decode_kernel over own keys and prefix chunks + merge_kernel)"
+                  if shared else " (paged_decode_kernel + merge_kernel)")
         out["roofline"] = {"kernel": kname + kparts,
                            "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                            "peak_source": peaks["source"], "unit": "GB/s",
@@ -372,7 +370,7 @@ def rooflines(step, dec_ms, pre_ms, peaks):
             sum(int(L) - int(n) + i + 1 for i in range(int(n))) for L, n in zip(lens, ql) if n > 1)
         pmean = statistics.mean(pre_ms)
         ideal_ms = (dec_bytes / (peaks["hbm_gbs"] * 1e9) + fl / (peaks["bf16_tflops"] * 1e12)) * 1e3
-        out["roofline"] = {"kernel": "pa_attention_varlen (zero_tickets_kernel + paged_decode_kernel"
+        out["roofline"] = {"kernel": "pa_attention_varlen (paged_decode_kernel + merge_kernel"
                                      " + chunked_prefill_kernel)",
                            "bound": "hbm (decode rows) then tensor (chunks)",
                            "achieved": round(ideal_ms / pmean, 4), "peak": 1.0,

@@ -106,8 +106,7 @@ PA_API pa_status pa_reshape_and_cache(const void* k, const void* v, void* k_cach
 
 /*
  * Bytes of scratch `pa_decode` needs, as an upper bound valid for every kv-head count
- * and GPU: merge tickets (bounded by 8 bytes per sequence and q-head, padded to 256
- * bytes), then
+ * and GPU: merge records (8 bytes per sequence and q-head, padded to 256 bytes), then
  * split-K partial rows of head_dim+2 fp32 (normalised partial output, running max and
  * sum): (256 + num_seqs) * num_q_heads rows, plus, when partition_size > 0,
  * num_seqs * num_q_heads * ceil(ceil(max_seq_len/16) / (partition_size/16)) +
@@ -132,16 +131,13 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *   partition_size  0 = balanced split-K: the 16-token tiles of every (sequence, group of
  *                 up to 8 kv-heads) are laid end to end and a persistent grid of one CTA
  *                 per SM takes equal shares; a sequence held by one CTA is written
- *                 directly; the pieces of the others leave normalised partials, and the
- *                 last piece of each (sequence, kv-head) to finish, found by an atomic
- *                 ticket, merges them by log-sum-exp inside the same launch.  > 0 (a
+ *                 directly; the pieces of the others leave normalised partials that a
+ *                 second, dependent launch merges by log-sum-exp.  > 0 (a
  *                 multiple of 16, at most 2048) also caps every share at that many
  *                 tokens, using more CTAs.
  *   workspace     device scratch, 256-byte aligned, of at least
- *                 pa_decode_workspace_size(...) bytes; contents need no initialisation
- *                 (a small kernel launched first zeroes the tickets; the decode kernel
- *                 starts as its programmatic dependent).  Calls that overlap on the GPU
- *                 must not share a workspace.
+ *                 pa_decode_workspace_size(...) bytes; contents need no initialisation.
+ *                 Calls that overlap on the GPU must not share a workspace.
  * Limits: head_dim 128, block_size 16 or 32, G = num_q_heads/num_kv_heads in
  * {1, 2, 4, 8}, num_seqs <= 4096 (else PA_ERR_UNSUPPORTED).
  */
@@ -233,14 +229,14 @@ PA_API pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, co
  *                 the same K/V (normally the same physical blocks); they are read through
  *                 the table row of the group's first member
  *   max_group_size, max_prefix_len  host bounds (grid sizing)
- * Two launches: the ticket zeroing, then one decode grid over a schedule that holds
+ * Two launches: one decode grid over a schedule that holds
  * every sequence's keys after its prefix and, appended to the batch, the "chunks": each
  * group's members cut into runs of 16 / G, whose q-heads make 16 rows per kv-head, over the
  * group's prefix (read through the table row of its first member).  A chunk's tiles are
  * whole blocks, as for any sequence; its consumer warps run the 16 rows as two tensor-core
  * tiles, so the prefix is read once per chunk (two chunks of one group are scheduled side
- * by side, and the second read is served by L2).  The last piece of each (member, kv-head)
- * to finish, own keys or chunk, merges both parts by log-sum-exp.  Workspace: at least
+ * by side, and the second read is served by L2); then the merge pass folds each member's
+ * own pieces with its chunk's by log-sum-exp.  Workspace: at least
  * pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
  * max_seq_len) bytes, 256-byte aligned.  An invalid prefix sets PA_DEVERR_PREFIX (outputs
  * of its group unspecified).  fp16/bf16 caches, num_seqs <= 2048 (else
@@ -377,7 +373,7 @@ PA_API pa_status pa_block_share(int32_t* block_refs, int num_blocks, int32_t* bl
  * is owned by someone else (an engine's pre-allocated KV pool, a host framework that
  * forbids raw cudaMalloc) or who must not risk the device-wide synchronisation an
  * allocation can cause.  Arguments and results are those of pa_decode without the
- * workspace: the merge tickets and split-K partials go to a fixed array inside the library,
+ * workspace: the merge records and split-K partials go to a fixed array inside the library,
  * pa_decode_noalloc_scratch_bytes() long (32 MiB), which every GPU that loads the
  * library holds until the process exits.
  *  - Sizes whose partials need more than that (pa_decode_workspace_size(...) >
@@ -388,9 +384,8 @@ PA_API pa_status pa_block_share(int32_t* block_refs, int num_blocks, int32_t* bl
  *    the life of the process: after cudaDeviceReset, or anything else that destroys the
  *    device's primary context, do not call this function again in that process.
  *  - Every call on a device shares the one array and leaves its last contents there;
- *    each call zeroes the part that must start at zero (the merge tickets) itself.
- *    Calls that overlap on the GPU (different streams, no ordering between them) race
- *    on the array: order them.
+ *    nothing in it needs to start at zero.  Calls that overlap on the GPU (different
+ *    streams, no ordering between them) race on the array: order them.
  *  - The call itself allocates no memory.
  */
 PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,

@@ -358,7 +358,7 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, m
     """pa_decode for callers that cannot allocate device memory: the split-K
     partials live in a fixed array inside the library
     (:func:`pa_decode_noalloc_scratch_bytes` per device, held until exit), as do
-    the merge tickets of the split-K pass.
+    the merge records of the split-K pass.
     Calls on one device share that array, so calls that overlap on the GPU
     race; make the first call on a device before any stream capture."""
     N, bs, Hkv, D = k_cache.shape

@@ -22,8 +22,8 @@
 //    a sequence is split only where a share boundary falls inside it.  The piece of a
 //    sequence that a CTA sees is a segment: a sequence held by one CTA is written to
 //    `out` directly; the others leave normalised partials (o, m, l) in the caller's
-//    workspace at slot c + group; the last of them to finish (counted by a per-group
-//    ticket) merges them by log-sum-exp in the same launch.
+//    workspace at slot c + group, merged by a log-sum-exp pass (merge_kernel, a
+//    programmatic dependent of this launch).
 //    An explicit partition size caps the share, so no segment is longer.
 //  * One consumer warp per kv-head of the group handles all G q-heads of that kv-head,
 //    so no two warps share an output.  q.k: 8 lanes split a token's 128 dims (16 each,
@@ -46,7 +46,7 @@
 //    its group reads only its tiles after the prefix; the group's members are cut into
 //    chunks of 16 q-rows per kv-head (16/G members), and each chunk is one more sequence of
 //    the schedule over the prefix, whose consumer warps run its rows as two tensor-core n8
-//    tiles; the tickets merge each member's own pieces with its chunk's;
+//    tiles; the merge pass folds each member's own pieces with its chunk's;
 //  * varlen rows (pa_attention_varlen): only sequences with one query row are served,
 //    q and out rows come from query_start_loc, and CTA 0 lists the other sequences for
 //    the prefill kernel that follows.
@@ -70,11 +70,13 @@ struct DecodeArgs {
   const int32_t* seq_lens;
   float* part_o;   // [slots, HB*G, 128]   normalised partial outputs
   float* part_ml;  // [slots, HB*G, 2]     (max in log2 units, sum)
-  // merge tickets, [B * Hkv]: one per (sequence, kv-head), zeroed by the launch before
-  // this one (zero_tickets_kernel).  Every piece of a split (sequence, kv-head) adds to it:
-  // its first piece the balance kTicketTotal - (pieces - 1), the others 1; the warp whose
-  // addition completes kTicketTotal merges that kv-head's q-heads
-  unsigned* tickets;
+  // merge records for the log-sum-exp pass: (first slot, segment count) of each (sequence,
+  // head group) [B * NHP] and of each (chunk, head group) [vcap * NHP]; count 0 when
+  // nothing is left to merge (written directly, or no keys); and the chunk numbering of
+  // the groups [num_groups + 1] as CTA 0 computed it
+  int2* meta;
+  int2* vmeta;
+  int* cstart_out;
   // append in the same launch (k_new != nullptr): the step's new token of each sequence,
   // [B, Hkv, 128], written into its cache slot at position seq_len-1 before it is read
   const void* k_new;
@@ -132,7 +134,6 @@ constexpr int kVirtual = 8;  // a chunk of a group's members over their shared p
 // count, [10] members of a chunk
 constexpr int kUnitInts = 16;
 constexpr int kChunkRows = 16;           // q rows of a chunk per kv-head (members x G)
-constexpr unsigned kTicketTotal = 1u << 30;  // a merge ticket's count when every piece is in
 
 template <int G_, int HB_, bool F8_, bool SP_ = false>
 struct DecodeCfg {
@@ -327,183 +328,78 @@ __device__ __forceinline__ int cta_of(int pos, int T, int grid) {
   return (int)((((long long)pos + 1) * grid - 1) / T);
 }
 
-// The schedule every CTA computes in its prologue: the sequences (the batch, then the
-// chunks of shared prefixes) with their tiles laid end to end; the first tile of each, its
-// clamped length, its first tile after a shared prefix (-1: not served), the chunk
-// numbering of the groups, and the grid that shares the tiles out.
-struct Sched {
-  const int* sstart;
-  const int* slen;
-  const int* sfirst;
-  const int* cstart;
-  int B, V, NHP, Ttot, grid;
-};
-
-// Segments of sequence s's head group hp (its keys after any prefix): first slot, count.
-__device__ __forceinline__ void own_pieces(const Sched& sc, int s, int hp, int& so0, int& no) {
-  so0 = no = 0;
-  const int cnt = sc.sfirst[s] < 0 ? 0 : cdiv(sc.slen[s], kTileTok) - sc.sfirst[s];
-  if (cnt <= 0) return;
-  const int gs = sc.sstart[s] + hp * cnt;
-  const int c0 = cta_of(gs, sc.Ttot, sc.grid), c1 = cta_of(gs + cnt - 1, sc.Ttot, sc.grid);
-  so0 = c0 + s * sc.NHP + hp;
-  no = c1 - c0 + 1;
-}
-
-// Segments of the chunk that holds member s, over its group's prefix (head group hp):
-// first slot, count, and the member's first row within the chunk's rows of a kv-head
-// (nv = 0 when s shares no prefix).
-template <int G>
-__device__ __forceinline__ void chunk_pieces(const DecodeArgs& a, const Sched& sc, int s, int hp,
-                                             int& sv0, int& nv, int& vrow) {
-  sv0 = nv = vrow = 0;
-  const int g = group_of(a, s);
-  if (g < 0 || __ldg(a.prefix_lens + g) <= 0) return;
-  const int off = s - __ldg(a.group_starts + g);
-  const int vs = sc.cstart[g] + off / a.mc;
-  if (vs >= sc.V) return;
-  const int vi = sc.B + vs;
-  const int cnt = cdiv(sc.slen[vi], kTileTok);
-  if (cnt <= 0) return;
-  const int gs = sc.sstart[vi] + hp * cnt;
-  const int c0 = cta_of(gs, sc.Ttot, sc.grid), c1 = cta_of(gs + cnt - 1, sc.Ttot, sc.grid);
-  sv0 = c0 + vs * sc.NHP + hp;
-  nv = c1 - c0 + 1;
-  vrow = (off % a.mc) * G;
-}
-
-// Log-sum-exp merge of one kv-head's G q-heads of one sequence over its pieces: its own
-// segments (partial rows in slots so0 .. so0+no-1) and the segments of the chunk that
-// holds it over a shared prefix (slots sv0 .. sv0+nv-1, rows vrow + j of the kv-head's 16).
-// o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the largest m_i.  One warp:
-// 32/G lanes per q-head, 4*G dims per lane; the rows are folded in rounds whose loads are
-// all in flight together, with a running maximum.  Reads go to L2 (other SMs wrote them).
-template <typename T, int G, int HB, bool SP>
-__device__ __forceinline__ void merge_pieces(const DecodeArgs& a, int orow, int kvh, int so0,
-                                             int no, int sv0, int nv, int vrow, int lane) {
-  constexpr int HBG = HB * G;
-  constexpr int VROWS = HB * kChunkRows;  // rows of a chunk slot
-  constexpr int LPH = 32 / G;             // lanes per q-head
-  constexpr int NV = G;                   // float4 per lane and row
-  // rows per round: 8 float4 loads in flight; one row beside the chunk consumer, whose
-  // registers leave no room for more
-  constexpr int R = SP ? 1 : (G >= 2 ? 8 / G : 8);
-  const int jj = lane / LPH;
-  const int d0 = (lane % LPH) * 4 * G;
-  const int qh = kvh * G + jj;            // q-head
-  const int j = qh % HBG;                 // its row within a slot of the sequence
-  const int jv = (kvh % HB) * kChunkRows + vrow + jj;  // its row within a chunk slot
-  float M = -INFINITY, den = 0.f;
-  float4 num[NV];
-#pragma unroll
-  for (int v = 0; v < NV; ++v) num[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+// Log-sum-exp merge of the split-K partials: one warp per (sequence, q-head), lanes over
+// head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the largest m_i,
+// over the sequence's own segments (consecutive slots of its head group's record) and, with
+// a shared prefix, the segments of the chunk that holds it (rows of its chunk slots).  One
+// pass with a running maximum, up to eight rows per round with all their loads in flight.
+// Launched as a programmatic dependent of the decode kernel.
+template <typename T, int G, bool SP>
+__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) {
+  griddep_wait();  // the decode grid has finished and its writes are visible
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= a.num_seqs * a.num_q_heads) return;
+  const int s = gw / a.num_q_heads;
+  const int qh = gw - s * a.num_q_heads;
+  const int hbg = HB * G, NHP = a.num_kv_heads / HB;
+  const int hp = qh / hbg, j = qh - hp * hbg;
+  const int2 mo = a.meta[s * NHP + hp];
+  const int so0 = mo.x, no = mo.y;
+  int sv0 = 0, nv = 0, vrow = 0;
+  if constexpr (SP) {
+    const int g = group_of(a, s);
+    if (g >= 0 && __ldg(a.prefix_lens + g) > 0) {
+      const int off = s - __ldg(a.group_starts + g);
+      const int vs = a.cstart_out[g] + off / a.mc;
+      if (vs < min(a.cstart_out[a.num_groups], a.vcap)) {
+        const int2 mv = a.vmeta[vs * NHP + hp];
+        sv0 = mv.x;
+        nv = mv.y;
+        vrow = (j / G) * kChunkRows + (off % a.mc) * G + (qh % G);
+      }
+    }
+  }
   const int total = no + nv;
-  for (int i0 = 0; i0 < total; i0 += R) {
-    float2 ml[R];
-    float4 ov[R][NV];
+  if (total == 0) return;  // written by the decode kernel (or nothing to write)
+  float M = -INFINITY, den = 0.f;
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < total; i0 += 8) {
+    float2 mlv[8];
+    float4 ov[8];
     float Mr = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < R; ++u) {
+    for (int u = 0; u < 8; ++u) {
       const int i = i0 + u;
       if (i < total) {
         const bool own = i < no;
-        const long long row =
-            own ? (long long)(so0 + i) * HBG + j : (long long)(sv0 + i - no) * VROWS + jv;
-        const float* po = (own ? a.part_o : a.vpart_o) + row * kD + d0;
-        ml[u] = __ldcg(reinterpret_cast<const float2*>((own ? a.part_ml : a.vpart_ml) + row * 2));
-#pragma unroll
-        for (int v = 0; v < NV; ++v) ov[u][v] = __ldcg(reinterpret_cast<const float4*>(po) + v);
-        Mr = fmaxf(Mr, ml[u].x);
+        const long long row = own ? (long long)(so0 + i) * hbg + j
+                                  : (long long)(sv0 + i - no) * (HB * kChunkRows) + vrow;
+        mlv[u] = *reinterpret_cast<const float2*>((own ? a.part_ml : a.vpart_ml) + row * 2);
+        ov[u] = *reinterpret_cast<const float4*>((own ? a.part_o : a.vpart_o) + row * kD + lane * 4);
+        Mr = fmaxf(Mr, mlv[u].x);
       }
     }
     const float Mn = fmaxf(M, Mr);
-    if (Mn == -INFINITY) continue;  // only empty pieces so far
+    if (Mn == -INFINITY) continue;  // only empty segments so far
     const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
     den *= sc;
+    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      num[v].x *= sc; num[v].y *= sc; num[v].z *= sc; num[v].w *= sc;
-    }
-#pragma unroll
-    for (int u = 0; u < R; ++u) {
+    for (int u = 0; u < 8; ++u) {
       if (i0 + u < total) {
-        const float f = ml[u].x == -INFINITY ? 0.f : fast_exp2(ml[u].x - Mn) * ml[u].y;
+        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
         den += f;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          num[v].x += f * ov[u][v].x; num[v].y += f * ov[u][v].y;
-          num[v].z += f * ov[u][v].z; num[v].w += f * ov[u][v].w;
-        }
+        num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
       }
     }
     M = Mn;
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  T* ob = static_cast<T*>(a.out) + ((long long)orow * a.num_q_heads + qh) * kD + d0;
-#pragma unroll
-  for (int v = 0; v < NV; ++v)
-    reinterpret_cast<uint2*>(ob)[v] = make_uint2(Elem<T>::pack2(num[v].x * inv, num[v].y * inv),
-                                                 Elem<T>::pack2(num[v].z * inv, num[v].w * inv));
-}
-
-// End of one of sequence s's own segments that is not the whole (sequence, head group):
-// this warp's partial rows (kv-head kvh) are written.  Its ticket counts the pieces that are
-// done; the warp whose addition completes kTicketTotal merges.  No warp waits for another
-// CTA.  With a shared prefix, the chunk's first segment adds the balance (finish_chunk).
-template <typename T, int G, int HB, bool SP>
-__device__ __forceinline__ void finish_own(const DecodeArgs& a, const Sched& sc, int s, int orow,
-                                           int hp, int kvh, int pslot, int slot0, int nseg,
-                                           int lane) {
-  __threadfence();  // this lane's partial rows are visible GPU-wide before the ticket
-  __syncwarp();
-  griddep_wait();   // the tickets were zeroed by the launch before this one
-  int sv0 = 0, nv = 0, vrow = 0;
-  if constexpr (SP) chunk_pieces<G>(a, sc, s, hp, sv0, nv, vrow);
-  const unsigned add = (nv == 0 && pslot == slot0) ? kTicketTotal - (unsigned)(nseg - 1) : 1u;
-  unsigned old = 0;
-  if (lane == 0) old = atomic_add_acq_rel_gpu(a.tickets + (long long)s * a.num_kv_heads + kvh, add);
-  if (__shfl_sync(0xffffffffu, old, 0) + add != kTicketTotal) return;
-  __threadfence();
-  merge_pieces<T, G, HB, SP>(a, orow, kvh, slot0, nseg, sv0, nv, vrow, lane);
-}
-
-// End of a chunk segment (members m0 .. m0+nm-1 over their shared prefix, kv-head kvh):
-// one ticket arrival per member (lane i for member m0+i), the chunk's first segment adding
-// each member's balance; the members whose count completes are merged one after another.
-template <typename T, int G, int HB>
-__device__ __forceinline__ void finish_chunk(const DecodeArgs& a, const Sched& sc, int m0, int nm,
-                                             int hp, int kvh, int pslot, int slot0, int nseg,
-                                             int lane) {
-  __threadfence();
-  __syncwarp();
-  griddep_wait();
-  bool last = false;
-  if (lane < nm) {
-    const int sm = m0 + lane;
-    int so0, no;
-    own_pieces(sc, sm, hp, so0, no);
-    const unsigned add = pslot == slot0 ? kTicketTotal - (unsigned)(no + nseg - 1) : 1u;
-    const unsigned old =
-        atomic_add_acq_rel_gpu(a.tickets + (long long)sm * a.num_kv_heads + kvh, add);
-    last = old + add == kTicketTotal;
-  }
-  unsigned mask = __ballot_sync(0xffffffffu, last);
-  if (mask) __threadfence();
-  while (mask) {
-    const int i = __ffs(mask) - 1;
-    mask &= mask - 1;
-    int so0, no;
-    own_pieces(sc, m0 + i, hp, so0, no);
-    merge_pieces<T, G, HB, true>(a, m0 + i, kvh, so0, no, slot0, nseg, i * G, lane);
-  }
-}
-
-// Zero the merge tickets of a decode launch; that launch follows as a programmatic
-// dependent and waits for this grid before its first ticket.
-__global__ void __launch_bounds__(256) zero_tickets_kernel(unsigned* tickets, int n) {
-  griddep_launch_dependents();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
-    tickets[i] = 0;
+  const long long orow = a.qsl ? __ldg(a.qsl + s) : s;
+  T* ob = static_cast<T*>(a.out) + (orow * a.num_q_heads + qh) * kD + lane * 4;
+  *reinterpret_cast<uint2*>(ob) =
+      make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
 }
 
 template <typename T, int G, int HB, bool F8, bool SP>
@@ -541,6 +437,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the merge pass may be scheduled now; it waits for this grid's results itself
+  griddep_launch_dependents();
 
   // ---- clamped lengths and the prefix of tiles over (sequence, head group)
   if (warp == 0) {
@@ -678,31 +576,33 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
   const int cta = blockIdx.x;
   const int r0 = cta < grid ? (int)(((long long)cta * Ttot) / grid) : Ttot;
   const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
-  // the schedule, rebuilt from shared memory where a segment end needs it (so that it
-  // holds no registers through the tile loops)
-  auto sched = [&]() -> Sched {
-    const volatile int* nc = nchunks;
-    const int v = SP ? *nc : 0;
-    const int tt = sstart[B + v];
-    return Sched{sstart, slen, sfirst, cstart, B, v, NHP, tt, min((int)gridDim.x, max(tt, 1))};
-  };
 
   if (warp < C::WARP_C0) {
     if (warp == C::WARP_FILL) {
-      // ===== sequences without keys of their own: no CTA's share visits them =====
+      // ===== sequences without keys of their own: no CTA's share visits them; their merge
+      // records say "nothing to merge" and their outputs are zeros (all keys shared: the
+      // merge pass takes its chunk's pieces alone) =====
       for (int s = cta; s < B; s += gridDim.x) {
+        if (sfirst[s] >= 0 && cdiv(slen[s], kTileTok) != sfirst[s]) continue;
+        for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
         if (sfirst[s] < 0) continue;  // not served by this kernel
-        if (cdiv(slen[s], kTileTok) != sfirst[s]) continue;
-        const int orow = a.qsl ? __ldg(a.qsl + s) : s;
         if constexpr (SP) {
-          // all its keys are shared: its chunk's segments merge its output
-          int sv0, nv, vrow;
-          chunk_pieces<G>(a, sched(), s, 0, sv0, nv, vrow);
-          if (nv > 0) continue;
+          const int g = group_of(a, s);
+          if (g >= 0 && __ldg(a.prefix_lens + g) > 0 &&
+              cstart[g] + (s - __ldg(a.group_starts + g)) / a.mc < V)
+            continue;
         }
+        const int orow = a.qsl ? __ldg(a.qsl + s) : s;
         T* ob = static_cast<T*>(a.out) + (long long)orow * a.num_q_heads * kD;
         for (int i = lane; i < a.num_q_heads * kD / 8; i += 32)
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if constexpr (SP) {
+        for (int v = cta; v < V; v += gridDim.x)  // chunks without tiles
+          if (slen[B + v] == 0)
+            for (int h = lane; h < NHP; h += 32) a.vmeta[v * NHP + h] = make_int2(0, 0);
+        if (cta == 0)  // the chunk numbering, for the merge pass
+          for (int g = lane; g <= a.num_groups; g += 32) a.cstart_out[g] = cstart[g];
       }
       return;
     }
@@ -826,6 +726,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
           }
         }
         if (lane == 0) {
+          if (t0 == ts)  // the group's first unit: its merge record
+            (virt ? a.vmeta : a.meta)[grp] =
+                make_int2(c0 + grp, (flags & kDirect) ? 0 : c1 - c0 + 1);
           u[0] = s;
           u[1] = hp;
           u[2] = t0;
@@ -1080,8 +983,9 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
           *reinterpret_cast<float2*>(a.vpart_ml + row * 2) = make_float2(mh[nt][e], lt);
       }
     }
-    finish_chunk<T, G, HB>(a, sched(), m0, nm, hp, kvh, pslot, slot0, nseg, lane);
     (void)s;
+    (void)slot0;
+    (void)nseg;
     return true;
   };
   if constexpr (C::MMA) {
@@ -1326,8 +1230,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
                 make_float2(e ? mh1 : mh0, e ? lt1 : lt0);
         }
       }
-      if (!(flags & kDirect))
-        finish_own<T, G, HB, SP>(a, sched(), s, orow, hp, kvh, pslot, slot0, nseg, lane);
+      (void)slot0;
+      (void)nseg;
     }
     return;
   } else {
@@ -1490,8 +1394,8 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
           if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
         }
       }
-      if (!(flags & kDirect))
-        finish_own<T, G, HB, SP>(a, sched(), s, orow, hp, hp * HB + w, pslot, slot0, nseg, lane);
+      (void)slot0;
+      (void)nseg;
     }
   }  // G < 8
 }
@@ -1510,15 +1414,15 @@ inline int heads_per_item(int num_kv_heads) {
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace of one launch: merge tickets (one int per sequence and kv-head), then partial
-// outputs, then (m, l) pairs.
+// Workspace of one launch: merge records (first slot, count) of each (sequence, head
+// group), then partial outputs, then (m, l) pairs.
 struct WsLayout {
-  size_t tickets, part_o, part_ml, total;
+  size_t meta, part_o, part_ml, total;
 };
-inline WsLayout ws_layout(long long tickets, long long slots, int hbg, int head_dim) {
+inline WsLayout ws_layout(long long groups, long long slots, int hbg, int head_dim) {
   WsLayout w;
-  w.tickets = 0;
-  w.part_o = align256((size_t)tickets * sizeof(int));
+  w.meta = 0;
+  w.part_o = align256((size_t)groups * sizeof(int2));
   w.part_ml = w.part_o + (size_t)slots * hbg * head_dim * sizeof(float);
   w.total = w.part_ml + (size_t)slots * hbg * 2 * sizeof(float);
   return w;
@@ -1539,32 +1443,30 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
   auto kern = paged_decode_kernel<T, G, HB, F8, SP>;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
-  // Split groups merge inside the launch through tickets that must start at zero: a small
-  // kernel zeroes them first, and the decode grid starts as its programmatic dependent
-  // (its prologue and first tiles overlap the zeroing; it waits before its first ticket).
-  const bool split = grid > 1 || a.num_groups > 0;
+  kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
-  if (split) {
-    const int n = a.num_seqs * a.num_kv_heads;
-    zero_tickets_kernel<<<std::min(32, (n + 4095) / 4096), 256, 0, stream>>>(a.tickets, n);
+  if (grid > 1 || SP) {
+    // the merge of split groups, as a programmatic dependent: its CTAs may start while the
+    // decode grid drains and wait for it inside
+    const int warps = a.num_seqs * a.num_q_heads;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((warps + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, merge_kernel<T, G, SP>, a, HB) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
     if (check_launch() != PA_OK) return PA_ERR_CUDA;
     ++launches;
   }
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = split ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, kern, tmK, tmV, tmQ, a) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return PA_ERR_CUDA;
-  }
-  if (check_launch() != PA_OK) return PA_ERR_CUDA;
   set_launch_count(launches);
   return PA_OK;
 }
@@ -1682,16 +1584,17 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   if (partition_size > 0)
     grid = std::max<long long>(grid, (tiles_max + partition_size / 16 - 1) / (partition_size / 16));
   const long long groups = (long long)num_seqs * NHP;
-  const pa::WsLayout lay =
-      pa::ws_layout((long long)num_seqs * num_kv_heads, grid + groups, HBG, head_dim);
+  const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
   // shared prefixes: the chunks' partial rows follow, (grid + chunks x head groups) slots of
-  // HB x 16 rows
+  // HB x 16 rows, then the chunks' merge records and the groups' chunk numbering
   const long long vslots = sp ? grid + (long long)vcap * NHP : 0;
   const long long vrows = vslots * HB * pa::kChunkRows;
-  size_t voff = 0, need = lay.total;
+  size_t voff = 0, vmeta_off = 0, cstart_off = 0, need = lay.total;
   if (sp) {
     voff = pa::align256(lay.total);
-    need = voff + (size_t)vrows * (head_dim + 2) * sizeof(float);
+    vmeta_off = pa::align256(voff + (size_t)vrows * (head_dim + 2) * sizeof(float));
+    cstart_off = pa::align256(vmeta_off + (size_t)vcap * NHP * sizeof(int2));
+    need = cstart_off + (size_t)(sp->num_groups + 1) * sizeof(int);
   }
   if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
@@ -1722,7 +1625,9 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.block_tables = block_tables;
   a.seq_lens = seq_lens;
   a.q = q;
-  a.tickets = reinterpret_cast<unsigned*>(ws + lay.tickets);
+  a.meta = reinterpret_cast<int2*>(ws + lay.meta);
+  a.vmeta = nullptr;
+  a.cstart_out = nullptr;
   a.k_new = k_new;
   a.v_new = v_new;
   a.k_cache = const_cast<void*>(k_cache);
@@ -1752,8 +1657,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.chunk_cap = chunk_cap;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (sp) {
-    // one launch: every sequence's own keys, and each chunk of every group's members over
-    // the group's prefix (the prefix read once per chunk), merged through the tickets
+    // one decode grid: every sequence's own keys, and each chunk of every group's members
+    // over the group's prefix (the prefix read once per chunk); the merge pass folds both
     a.group_starts = sp->group_starts;
     a.prefix_lens = sp->prefix_lens;
     a.num_groups = sp->num_groups;
@@ -1762,6 +1667,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     a.max_prefix = sp->max_prefix_len;
     a.vpart_o = reinterpret_cast<float*>(ws + voff);
     a.vpart_ml = a.vpart_o + (size_t)vrows * head_dim;
+    a.vmeta = reinterpret_cast<int2*>(ws + vmeta_off);
+    a.cstart_out = reinterpret_cast<int*>(ws + cstart_off);
     return dtype == PA_F16
                ? pa::dispatch_group<__half, false, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
                : pa::dispatch_group<__nv_bfloat16, false, true>(G, HB, tmK, tmV, tmQ, a,
@@ -1826,7 +1733,7 @@ extern "C" pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache
 // serving loop whose memory is entirely owned by an engine's pre-allocated pool (the
 // pool hands out KV blocks, not scratch buffers), plugins whose host framework forbids
 // raw cudaMalloc, and latency-critical paths where an allocation could synchronise the
-// device.  For them this entry point keeps its workspace (the merge tickets and the
+// device.  For them this entry point keeps its workspace (the merge records and the
 // split-K partials) in a fixed array that
 // lives in this file (kNoAllocScratchBytes on every GPU that loads the library, held
 // until the process exits) and otherwise runs exactly pa_decode.
@@ -1884,9 +1791,13 @@ extern "C" size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q
   const size_t base = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
   if (base == 0 || num_kv_heads <= 0) return 0;
   // the chunks' partial rows: (grid + chunks x head groups) slots of (kv-heads per group x 16)
-  // rows, at most (256 + num_seqs) x num_kv_heads x 16 rows of head_dim + 2 fp32
-  return pa::align256(base) + ((size_t)pa::kMaxGrid + num_seqs) * num_kv_heads *
-                                  pa::kChunkRows * (head_dim + 2) * sizeof(float);
+  // rows, at most (256 + num_seqs) x num_kv_heads x 16 rows of head_dim + 2 fp32; their merge
+  // records (at most num_seqs x num_kv_heads) and the chunk numbering (num_seqs + 1 ints)
+  return pa::align256(pa::align256(pa::align256(base) + ((size_t)pa::kMaxGrid + num_seqs) *
+                                                            num_kv_heads * pa::kChunkRows *
+                                                            (head_dim + 2) * sizeof(float)) +
+                      (size_t)num_seqs * num_kv_heads * sizeof(int2)) +
+         (size_t)(num_seqs + 1) * sizeof(int);
 }
 
 extern "C" pa_status pa_decode_shared_prefix(

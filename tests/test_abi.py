@@ -57,7 +57,7 @@ def test_status_strings(palib):
 
 
 def _ws_bound(B, Hq, L, P, D=128):
-    """The documented upper bound: merge tickets (at most 8 B per sequence and q-head, padded
+    """The documented upper bound: merge records (8 B per sequence and q-head, padded
     to 256 B) and partial rows of D+2 fp32: (256 + B) * Hq, plus, with an explicit
     partition, B * Hq * ceil(ceil(L/16) / (P/16)) + Hq."""
     rows = (256 + B) * Hq
@@ -120,7 +120,7 @@ def test_invalid_arguments_rejected_on_host(palib):
     assert dec(dt=3) == 2
     assert dec(B=0) == 0                     # nothing to do
     assert dec(B=5000) == 2                  # more sequences than the schedule holds
-    assert dec(P=512) == 3                   # every call needs a workspace (merge tickets)
+    assert dec(P=512) == 3                   # every call needs a workspace (merge records)
     assert dec(maxlen=8000, P=512, ws=m.region(), wsb=100) == 3
     assert dec(maxlen=8000, P=512, ws=m.region(16), wsb=1 << 24) == 1  # alignment
     assert palib.pa_last_launch_count() == 0
@@ -180,9 +180,11 @@ def test_shared_prefix_arguments_rejected_on_host(palib):
     assert dec(B=0, ng=0, mg=0) == 0               # nothing to do
     assert dec() == 3 and dec(mp=0) == 3            # needs a workspace (shared or plain)
     base = palib.pa_decode_workspace_size(8, 32, 128, 512, 0)
-    # chunk partials: (256 + num_seqs) x num_kv_heads x 16 rows of 130 fp32 after the base
+    # chunk partials: (256 + num_seqs) x num_kv_heads x 16 rows of 130 fp32 after the base,
+    # then the chunks' merge records (num_seqs x num_kv_heads int2) and the chunk numbering
+    up = lambda n: -(-n // 256) * 256  # noqa: E731
     assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 8, 128, 512) == \
-        -(-base // 256) * 256 + (256 + 8) * 8 * 16 * 130 * 4
+        up(up(up(base) + (256 + 8) * 8 * 16 * 130 * 4) + 8 * 8 * 8) + 9 * 4
     assert palib.pa_decode_shared_prefix_workspace_size(0, 32, 8, 128, 512) == 0
     assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 0, 128, 512) == 0
     assert palib.pa_last_launch_count() == 0

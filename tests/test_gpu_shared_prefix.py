@@ -63,7 +63,7 @@ def _grouped_batch(name, lens, groups, prefix, G, dtype, bs=16, Hkv=4, seed=0):
 def test_shared_prompt_workloads(bs):
     bc = workloads.shared_prefix(block_size=bs, scale=1 / 8)[0]
     _, launches = _vs_oracle(bc, "shared prefix bs%d" % bs)
-    assert launches == 2  # ticket zeroing, then one decode grid over own keys and chunks
+    assert launches == 2  # one decode grid over own keys and chunks, then the merge
 
 
 @pytest.mark.parametrize("G", [1, 2, 4, 8])

@@ -4,7 +4,7 @@ Some callers of this library never call cudaMalloc themselves: their device memo
 belongs to an engine's pre-allocated KV pool or to a host framework that forbids raw
 allocations, or they run in a latency-critical loop where an allocation could
 synchronise the device.  pa_decode_noalloc serves them by keeping its workspace (the
-merge tickets and the split-K partials) in a fixed array inside the library.
+merge records and the split-K partials) in a fixed array inside the library.
 These checks run through the C ABI on a GPU: two calls in a row must reproduce
 pa_decode with a caller-provided workspace (within the parity tolerance), and sizes
 whose partials do not fit the array must be refused before anything is launched.  The file sorts last so a fail-fast run has already run
@@ -65,7 +65,7 @@ def _fresh_workspace_decode(b, partition_size):
 
 
 def test_noalloc_smaller_batch_after_larger():
-    # a large batch leaves merge tickets and partial rows in the shared array; the next,
+    # a large batch leaves merge records and partial rows in the shared array; the next,
     # smaller call (explicit 512-token partitions, some sequences empty or short) must not
     # pick up any of them
     big = workloads.mixed_lengths(scale=1 / 4, device="cuda")[0]
