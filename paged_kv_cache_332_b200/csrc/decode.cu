@@ -60,6 +60,7 @@
 
 #include "pa_device.cuh"
 #include "pa_host.h"
+#include "prefill_body.cuh"
 
 namespace pa {
 
@@ -402,15 +403,16 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) 
       make_uint2(Elem<T>::pack2(num.x * inv, num.y * inv), Elem<T>::pack2(num.z * inv, num.w * inv));
 }
 
+// The decode CTA `cta` of `ncta` (the persistent grid's share of the tiles), with its
+// dynamic shared memory at `smem` (1024-byte aligned).  The CTA may hold more threads than
+// the configuration's; the extra warps leave after the prologue.
 template <typename T, int G, int HB, bool F8, bool SP>
-__global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
-    paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
+__device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                            const CUtensorMap& tmQ, const DecodeArgs& a,
+                                            uint8_t* smem, const int cta, const int ncta) {
   using C = DecodeCfg<G, HB, F8, SP>;
   constexpr int GW = C::GW;
   constexpr int HBG = HB * G;
-  extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + C::OFF_QFULL);
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
       const int total = __shfl_sync(0xffffffffu, cincl, 31);
       if (lane == 0) {
         cstart[ng] = total;
-        if (total > VC && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_PREFIX);
+        if (total > VC && cta == 0) flag_error(a.err, PA_DEVERR_PREFIX);
       }
       V = min(total, VC);
       __syncwarp();
@@ -492,12 +494,12 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
       } else {
         const int raw = a.seq_lens[s];
         L = clamp_len(raw, a.seq_cap);
-        if (raw != L && blockIdx.x == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
+        if (raw != L && cta == 0) flag_error(a.err, PA_DEVERR_SEQ_TOO_LONG);
         if (a.qsl != nullptr) {  // varlen: decode rows only; the others are prefill chunks
           const int q0 = __ldg(a.qsl + s), nq = __ldg(a.qsl + s + 1) - q0;
           if (nq != 1) first = -1;
           else if (q0 < 0 || q0 >= a.num_q_rows) {
-            if (blockIdx.x == 0) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
+            if (cta == 0) flag_error(a.err, PA_DEVERR_QUERY_LAYOUT);
             first = -1;
           }
         }
@@ -505,7 +507,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
           const int g = group_of(a, s);
           const int p = g < 0 ? 0 : __ldg(a.prefix_lens + g);
           if ((p < 0 || p > L || p > a.max_prefix || (p & ((1 << a.log2_bs) - 1))) &&
-              blockIdx.x == 0)
+              cta == 0)
             flag_error(a.err, PA_DEVERR_PREFIX);
           first = clamp_len(p, L) / kTileTok;
         }
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
       sstart[NS] = incl;
       *nchunks = V;
     }
-    if (a.chunk_ids != nullptr && blockIdx.x == 0) {
+    if (a.chunk_ids != nullptr && cta == 0) {
       int c = 0;
       for (int s = lo; s < hi; ++s) c += (__ldg(a.qsl + s + 1) - __ldg(a.qsl + s)) > 1;
       int ci = c;
@@ -572,8 +574,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
   // The launch sizes the grid for the longest possible batch; when the batch holds
   // fewer tiles than CTAs, only the first Ttot CTAs take a share, so every share is
   // non-empty and the segments of a group sit in consecutive CTAs (and slots).
-  const int grid = min((int)gridDim.x, max(Ttot, 1));
-  const int cta = blockIdx.x;
+  const int grid = min(ncta, max(Ttot, 1));
   const int r0 = cta < grid ? (int)(((long long)cta * Ttot) / grid) : Ttot;
   const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
 
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
       // ===== sequences without keys of their own: no CTA's share visits them; their merge
       // records say "nothing to merge" and their outputs are zeros (all keys shared: the
       // merge pass takes its chunk's pieces alone) =====
-      for (int s = cta; s < B; s += gridDim.x) {
+      for (int s = cta; s < B; s += ncta) {
         if (sfirst[s] >= 0 && cdiv(slen[s], kTileTok) != sfirst[s]) continue;
         for (int h = lane; h < NHP; h += 32) a.meta[s * NHP + h] = make_int2(0, 0);
         if (sfirst[s] < 0) continue;  // not served by this kernel
@@ -598,7 +599,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
       }
       if constexpr (SP) {
-        for (int v = cta; v < V; v += gridDim.x)  // chunks without tiles
+        for (int v = cta; v < V; v += ncta)  // chunks without tiles
           if (slen[B + v] == 0)
             for (int h = lane; h < NHP; h += 32) a.vmeta[v * NHP + h] = make_int2(0, 0);
         if (cta == 0)  // the chunk numbering, for the merge pass
@@ -794,7 +795,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
             wait_or_abort(&empty[slot], ((cnt / nslots) & 1) ^ 1, abort_flag, a.err, a.wait_limit);
             if (*abort_flag) break;  // a wait may have been skipped: no more arrivals
             issued <<= 1;
-            if (a.test_withhold && blockIdx.x == 0 && cnt == 0) continue;  // testing hook
+            if (a.test_withhold && cta == 0 && cnt == 0) continue;  // testing hook
             const int bid = tbl[qs * kMaxTilesPerUnit + (t - t0)];
             mbar_arrive_expect_tx(&full[slot], bid >= 0 ? C::SLOT_BYTES : 0);
             if (bid >= 0) {
@@ -823,6 +824,7 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
 
   // ===================== consumer warps: warp w <-> kv-head hp*HB + w =====================
   const int w = warp - C::WARP_C0;
+  if (w >= HB) return;  // a CTA shared with other work may hold more threads
 
   // A chunk segment (shared prefix): the 16 rows r = mloc*G + jj of kv-head hp*HB + w (member
   // m0+mloc, q-head jj; rows past nm*G are zero queries, not written), as two mma.sync n8
@@ -1400,6 +1402,79 @@ __global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
   }  // G < 8
 }
 
+template <typename T, int G, int HB, bool F8, bool SP>
+__global__ void __launch_bounds__(DecodeCfg<G, HB, F8, SP>::THREADS, 1)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  decode_body<T, G, HB, F8, SP>(tmK, tmV, tmQ, a, smem, blockIdx.x, gridDim.x);
+}
+
+// A mixed step in one grid (pa_attention_varlen): CTAs [0, D) are the persistent decode grid
+// over the sequences of one query row; the rest are chunked-prefill items over the listed
+// chunk sequences, which take the SMs left free and then those the decode CTAs leave, so the
+// chunks' tensor-core work runs beside the decode rows' HBM stream instead of after it.
+template <typename T, int G, int HB>
+__global__ void __launch_bounds__(prefill::kThreads, 1)
+    varlen_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tpK,
+                  const __grid_constant__ CUtensorMap tpV, const DecodeArgs a,
+                  const prefill::Args p, int D) {
+  static_assert(DecodeCfg<G, HB, false>::THREADS <= prefill::kThreads, "CTA size");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((int)blockIdx.x < D)
+    decode_body<T, G, HB, false, false>(tmK, tmV, tmQ, a, smem, blockIdx.x, D);
+  else
+    prefill::prefill_body<T, G>(tpK, tpV, p, smem, blockIdx.x - D);
+}
+
+// The sequences of a mixed step with more than one query row (the chunks), in index order:
+// chunk_ids[0..n), n = chunk_ids[cap] <= cap; more of them than cap is flagged.  The
+// mixed-step kernel starts as its programmatic dependent and its prefill CTAs wait for it.
+__global__ void __launch_bounds__(1024) varlen_list_kernel(const int32_t* __restrict__ qsl, int B,
+                                                           int32_t* __restrict__ chunk_ids,
+                                                           int cap, int* err) {
+  griddep_launch_dependents();
+  __shared__ int wsum[33];
+  const int per = (B + 1023) / 1024;
+  const int lo = min(B, (int)threadIdx.x * per), hi = min(B, lo + per);
+  int c = 0;
+  for (int s = lo; s < hi; ++s) c += (__ldg(qsl + s + 1) - __ldg(qsl + s)) > 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int wv = wsum[lane];
+    int wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    wsum[lane] = wi - wv;
+    if (lane == 31) wsum[32] = wi;
+  }
+  __syncthreads();
+  int run = wsum[warp] + incl - c;
+  for (int s = lo; s < hi; ++s)
+    if (__ldg(qsl + s + 1) - __ldg(qsl + s) > 1) {
+      if (run < cap) chunk_ids[run] = s;
+      ++run;
+    }
+  if (threadIdx.x == 0) {
+    chunk_ids[cap] = min(wsum[32], cap);
+    if (wsum[32] > cap) flag_error(err, PA_DEVERR_QUERY_LAYOUT);
+  }
+}
+
 constexpr int kMaxPartition = kMaxTilesPerUnit * kTileTok;
 constexpr int kMaxSeqs = 4096;
 constexpr int kMaxSeqsShared = 2048;  // batch + chunks in the schedule arrays
@@ -1483,6 +1558,14 @@ pa_status dispatch_hb(int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
   }
 }
 
+// A decode launch's arguments, prepared by decode_impl for a caller that launches them in
+// a kernel of its own (the mixed-step kernel of pa_attention_varlen).
+struct PreparedDecode {
+  DecodeArgs a;
+  CUtensorMap tmK, tmV, tmQ;
+  int grid, G, HB;
+};
+
 template <typename T, bool F8, bool SP = false>
 pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const CUtensorMap& tmQ, const DecodeArgs& a, int grid,
@@ -1495,6 +1578,81 @@ pa_status dispatch_group(int G, int HB, const CUtensorMap& tmK, const CUtensorMa
     default: return PA_ERR_UNSUPPORTED;
   }
 }
+
+// The mixed step: the chunk list, the mixed-step grid (D decode CTAs + P prefill items, a
+// programmatic dependent of the list) and the merge of the decode rows' split groups.
+template <typename T, int G, int HB>
+pa_status launch_varlen(PreparedDecode& d, const prefill::Args& p, const CUtensorMap& tpK,
+                        const CUtensorMap& tpV, int D, int P, const int32_t* qsl, int B,
+                        int32_t* chunk_ids, int cap, cudaStream_t stream) {
+  using C = DecodeCfg<G, HB, false>;
+  const size_t ring_off =
+      ((C::OFF_SEQ + (size_t)(3LL * d.a.num_seqs + 1) * 4 + 1023) / 1024) * 1024;
+  const long long room = (long long)kMaxSmem - (long long)ring_off;
+  const int nslots = (int)std::min<long long>(kMaxSlots, room / C::SLOT_BYTES);
+  if (nslots < 2) return PA_ERR_UNSUPPORTED;
+  d.a.ring_off = (int)ring_off;
+  d.a.nslots = nslots;
+  const size_t smem =
+      std::max(ring_off + (size_t)nslots * C::SLOT_BYTES, (size_t)prefill::SMEM_BYTES);
+  auto kern = varlen_kernel<T, G, HB>;
+  if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
+  varlen_list_kernel<<<1, 1024, 0, stream>>>(qsl, B, chunk_ids, cap, d.a.err);
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(D + P));
+  cfg.blockDim = dim3(prefill::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, d.tmK, d.tmV, d.tmQ, tpK, tpV, d.a, p, D) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
+  const int warps = d.a.num_seqs * d.a.num_q_heads;
+  cudaLaunchConfig_t mcfg = cfg;
+  mcfg.gridDim = dim3((unsigned)((warps + 7) / 8));
+  mcfg.blockDim = dim3(256);
+  mcfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&mcfg, merge_kernel<T, G, false>, d.a, HB) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  if (check_launch() != PA_OK) return PA_ERR_CUDA;
+  set_launch_count(3);
+  return PA_OK;
+}
+
+template <typename T>
+pa_status dispatch_varlen(PreparedDecode& d, const prefill::Args& p, const CUtensorMap& tpK,
+                          const CUtensorMap& tpV, int D, int P, const int32_t* qsl, int B,
+                          int32_t* chunk_ids, int cap, cudaStream_t stream) {
+#define PA_VARLEN_HB(GG)                                                                 \
+  switch (d.HB) {                                                                        \
+    case 1: return launch_varlen<T, GG, 1>(d, p, tpK, tpV, D, P, qsl, B, chunk_ids, cap, stream); \
+    case 2: return launch_varlen<T, GG, 2>(d, p, tpK, tpV, D, P, qsl, B, chunk_ids, cap, stream); \
+    case 4: return launch_varlen<T, GG, 4>(d, p, tpK, tpV, D, P, qsl, B, chunk_ids, cap, stream); \
+    case 8: return launch_varlen<T, GG, 8>(d, p, tpK, tpV, D, P, qsl, B, chunk_ids, cap, stream); \
+    default: return PA_ERR_UNSUPPORTED;                                                  \
+  }
+  switch (d.G) {
+    case 1: PA_VARLEN_HB(1)
+    case 2: PA_VARLEN_HB(2)
+    case 4: PA_VARLEN_HB(4)
+    case 8: PA_VARLEN_HB(8)
+    default: return PA_ERR_UNSUPPORTED;
+  }
+#undef PA_VARLEN_HB
+}
+
+// Share of the SMs the decode rows of a mixed step take; the chunks' items run on the
+// others and then on those the decode CTAs leave.
+constexpr int kVarlenDecodeShareNum = 2, kVarlenDecodeShareDen = 3;
 
 }  // namespace pa
 
@@ -1535,7 +1693,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
                       int block_size, int num_blocks, int max_seq_len, int partition_size,
                       void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream,
                       const SharedPrefixArgs* sp = nullptr, const int32_t* qsl = nullptr,
-                      int num_q_rows = 0, int32_t* chunk_ids = nullptr, int chunk_cap = 0) {
+                      int num_q_rows = 0, int32_t* chunk_ids = nullptr, int chunk_cap = 0,
+                      pa::PreparedDecode* prep = nullptr) {
   pa::set_launch_count(0);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0 ||
@@ -1656,6 +1815,16 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.chunk_ids = chunk_ids;
   a.chunk_cap = chunk_cap;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (prep) {  // the caller launches (the mixed-step kernel)
+    prep->a = a;
+    prep->tmK = tmK;
+    prep->tmV = tmV;
+    prep->tmQ = tmQ;
+    prep->grid = (int)grid;
+    prep->G = G;
+    prep->HB = HB;
+    return PA_OK;
+  }
   if (sp) {
     // one decode grid: every sequence's own keys, and each chunk of every group's members
     // over the group's prefix (the prefix read once per chunk); the merge pass folds both
@@ -1861,25 +2030,36 @@ extern "C" pa_status pa_attention_varlen(
   int32_t* chunk_ids = max_query_len > 1
                            ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + dws)
                            : nullptr;
-  // the rows of one query: the decode kernel (it skips the others, and lists the chunks)
+  if (cap == 0)  // rows of one query only: the decode kernel (it lists stray chunks)
+    return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
+                       block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len, 0,
+                       workspace, dws, dtype, stream, nullptr, query_start_loc, num_q_rows,
+                       chunk_ids, 0);
+  // one grid for both: the decode rows' arguments and the chunks' items, prepared
+  pa::PreparedDecode d;
   pa_status st = decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr,
                              block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_q_heads,
                              num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len,
                              0, workspace, dws, dtype, stream, nullptr, query_start_loc,
-                             num_q_rows, chunk_ids, cap);
+                             num_q_rows, nullptr, 0, &d);
   if (st != PA_OK) return st;
-  int launches = pa::launch_count();
-  if (cap > 0) {
-    // the chunks: the prefill kernel over the listed sequences
-    const size_t rest = workspace_bytes - dws - lws;
-    st = pa::chunked_prefill_impl(
-        out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens, query_start_loc,
-        num_seqs, max_query_len, num_q_heads, num_kv_heads, head_dim, scale, block_size,
-        num_blocks, max_seq_len, rest ? static_cast<uint8_t*>(workspace) + dws + lws : nullptr,
-        rest, dtype, stream, true, chunk_ids, cap);
-    if (st != PA_OK) return st;
-    launches += pa::launch_count();
-  }
-  pa::set_launch_count(launches);
-  return PA_OK;
+  pa::prefill::Args p;
+  CUtensorMap tpK, tpV;
+  st = pa::chunked_prefill_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                seq_lens, query_start_loc, num_seqs, max_query_len, num_q_heads,
+                                num_kv_heads, head_dim, scale, block_size, num_blocks, max_seq_len,
+                                nullptr, 0, dtype, stream, true, chunk_ids, cap, &p, &tpK, &tpV);
+  if (st != PA_OK) return st;
+  p.wait_list = 1;
+  const int D = std::max(
+      1, std::min(d.grid, (pa::num_sms() * pa::kVarlenDecodeShareNum + pa::kVarlenDecodeShareDen - 1) /
+                              pa::kVarlenDecodeShareDen));
+  if ((long long)D + p.whole_items > INT_MAX) return PA_ERR_UNSUPPORTED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return dtype == PA_F16 ? pa::dispatch_varlen<__half>(d, p, tpK, tpV, D, p.whole_items,
+                                                       query_start_loc, num_seqs, chunk_ids, cap, cs)
+                         : pa::dispatch_varlen<__nv_bfloat16>(d, p, tpK, tpV, D, p.whole_items,
+                                                              query_start_loc, num_seqs, chunk_ids,
+                                                              cap, cs);
 }

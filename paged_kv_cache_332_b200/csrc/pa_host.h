@@ -62,6 +62,8 @@ int launch_count();
 // varlen call serves them with the decode kernel); with chunk_ids (a device list of the
 // sequences with more than one query row, its length at chunk_ids[chunk_cap]) the grid
 // covers chunk_cap sequences of that list instead of all num_seqs.
+// With `prep_args` (a prefill::Args) and the two tensor maps, nothing is launched: the
+// prepared arguments are returned for a kernel of the caller's.
 pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* block_tables, int max_blocks_per_seq,
                                const int32_t* seq_lens, const int32_t* query_start_loc,
@@ -69,7 +71,8 @@ pa_status chunked_prefill_impl(void* out, const void* q, const void* k_cache, co
                                int head_dim, float scale, int block_size, int num_blocks,
                                int max_seq_len, void* workspace, size_t workspace_bytes,
                                pa_dtype dtype, void* stream, bool skip_single,
-                               const int32_t* chunk_ids, int chunk_cap);
+                               const int32_t* chunk_ids, int chunk_cap, void* prep_args = nullptr,
+                               CUtensorMap* prep_tk = nullptr, CUtensorMap* prep_tv = nullptr);
 
 inline pa_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

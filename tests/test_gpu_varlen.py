@@ -2,7 +2,7 @@
 ABI: a varlen batch of decode rows and prefill chunks ([P1] "工程边界与架构取舍", chunked
 prefill mixed with decode steps) must match the oracle's chunked prefill row by row;
 a batch of decode rows only must equal pa_decode bit for bit, a batch of chunks only
-pa_chunked_prefill; sequences without rows are left alone and a decode row outside q is
+the oracle and pa_chunked_prefill (to the rounding of its wave-tail merge); sequences without rows are left alone and a decode row outside q is
 flagged, not read."""
 import dataclasses
 
@@ -90,7 +90,9 @@ def test_decode_rows_only_equal_pa_decode_bitwise():
     assert torch.equal(got.view(torch.int16), want.view(torch.int16))
 
 
-def test_chunks_only_equal_pa_chunked_prefill_bitwise():
+def test_chunks_only_match_oracle_and_pa_chunked_prefill():
+    # pa_chunked_prefill may run the items of its last wave as two halves merged after;
+    # the mixed-step grid runs every item whole, so the two agree to the merge's rounding
     bc = workloads.prefill_plus_decode(scale=1 / 16)[0]
     b = bc.to(DEV)
     P.gpu_append(b)
@@ -101,10 +103,14 @@ def test_chunks_only_equal_pa_chunked_prefill_bitwise():
     want = torch.empty_like(b.q)
     pa.pa_chunked_prefill(want, b.q, b.k_cache, b.v_cache, b.block_tables, b.seq_lens,
                           b.query_start_loc, b.scale, b.max_query_len, b.max_seq_len, ws)
-    got = _varlen(b)  # the same prefill workspace share: the same wave-tail split
+    got = _varlen(b)
     torch.cuda.synchronize()
     assert pa.pa_get_device_error() == 0
-    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    ref = P.oracle_prefill(bc)
+    P.compare(got, ref, bc.dtype, "varlen, chunks only")
+    P.compare(want, ref, bc.dtype, "pa_chunked_prefill")
+    diff = (got.float() - want.float()).abs().max().item()
+    assert diff <= 2 * torch.finfo(bc.dtype).eps * max(1.0, want.float().abs().max().item())
 
 
 def test_decode_row_outside_q_flagged():
