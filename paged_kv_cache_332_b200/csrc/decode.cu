@@ -154,6 +154,11 @@ struct DecodeCfg {
   static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);  // CUDA-core path (G <= 4)
   static constexpr int TILE_BYTES = kTileTok * HB * KROW;       // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
+  // A K (V) tile is copied as 128-byte-wide column slabs of its rows (two slabs of 64 dims
+  // for 16-bit elements, one of 128 e4m3 codes), each laid out [kv-head][token][128 B] with
+  // the 128-byte swizzle: see swz().
+  static constexpr int SLABS = KROW / 128;
+  static constexpr int SLAB_BYTES = TILE_BYTES / SLABS;
   static constexpr int QBYTES = HB * G * kRowBytes;             // q rows of a group
   // shared-memory carve-up (bytes); the sequence arrays and then the ring follow
   static constexpr int OFF_FULL = 0;
@@ -177,6 +182,15 @@ struct DecodeCfg {
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+// Byte offset, inside one column slab of a ring tile, of 16-byte chunk c (0..7) of token t of
+// kv-head w.  The slab holds 128-byte rows ordered [kv-head][token]; the copy's 128-byte
+// swizzle stores chunk c of row r at chunk position c ^ (r & 7) (the slab starts on a
+// 1024-byte boundary, so r & 7 = t & 7).  Rows of consecutive tokens then start in different
+// banks, which the consumers' fragment reads rely on to be free of bank conflicts.
+__device__ __forceinline__ int swz(int w, int t, int c) {
+  return ((w * kTileTok + t) << 7) | ((c ^ (t & 7)) << 4);
+}
 
 
 // Group holding sequence s: the last g with group_starts[g] <= s, if s < group_starts[g+1];
@@ -321,6 +335,103 @@ __device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
   return d;
+}
+
+// Tensor-core consumers, S^T = K Q^T over a 16-bit tile: k-steps 2j and 2j+1 of lane quad tq
+// take the eight dims of 16-byte chunk kchunk(tq, j) (of 16; chunks 0..7 in slab 0).  The
+// contraction may visit dims in any order as long as K and Q agree; this one puts the lanes
+// of tokens g and g^1 (one shared-memory phase) on chunks of opposite parity, so that under
+// the slab swizzle the eight 16-byte reads of a phase hit eight different bank groups.
+__device__ __forceinline__ int kchunk(int tq, int j) { return 8 * (j >> 1) + 2 * tq + (j & 1); }
+
+// O^T += V^T P^T for one 16-token tile of kv-head w (tensor-core consumers).  Lane (g, tq)
+// reads one 16-byte chunk per token for tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (zero past nvalid):
+// chunk g of each slab (16-bit: dims [8g, 8g+8) and [64+8g, 64+8g+8)) or, for e4m3, the 16
+// codes [16g, 16g+16).  Word r of a lane's chunk h makes m-tile 4h+r, its row g the chunk's
+// dim 2r and its row g+8 dim 2r+1, with tokens paired along k as the P^T fragments pb0
+// (tokens 2tq, 2tq+1) and pb1 (2tq+8, 2tq+9) expect.  Under the swizzle the reads of a
+// phase (tokens 2tq+b of chunks g, g^1) fall in eight different bank groups.  NT column
+// tiles of 8 share every V fragment; SLAB is the tile's slab size in bytes.
+template <bool F8, typename MT, int NT, int SLAB>
+__device__ __forceinline__ void pv_tile(float (&oacc)[NT][8][4], const uint8_t* Vs, int w, int g,
+                                        int tq, int nvalid, const uint32_t (&pb)[NT][2]) {
+  // token 2tq+b+8c sits 8 rows (1 KB) after token 2tq+b, with the same swizzle
+  const int vofs0 = swz(w, 2 * tq, g), vofs1 = swz(w, 2 * tq + 1, g);
+  auto vofs = [&](int i) { return ((i & 1) ? vofs1 : vofs0) + (i >> 1) * 1024; };
+  uint4 v8[4];
+  if constexpr (F8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+      v8[i] = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + vofs(i))
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t vw[4][4];  // [token i][word r]
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if constexpr (F8) {
+        const uint32_t c0 = h ? v8[i].z : v8[i].x, c1 = h ? v8[i].w : v8[i].y;
+        vw[i][0] = e4m3x2_to_f16x2(c0);
+        vw[i][1] = e4m3x2_to_f16x2(c0 >> 16);
+        vw[i][2] = e4m3x2_to_f16x2(c1);
+        vw[i][3] = e4m3x2_to_f16x2(c1 >> 16);
+      } else {
+        const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+        const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        vw[i][0] = c.x;
+        vw[i][1] = c.y;
+        vw[i][2] = c.z;
+        vw[i][3] = c.w;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], 0x5410);
+      const uint32_t a1 = __byte_perm(vw[0][r], vw[1][r], 0x7632);
+      const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], 0x5410);
+      const uint32_t a3 = __byte_perm(vw[2][r], vw[3][r], 0x7632);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        Mma<MT>::run(oacc[nt][4 * h + r], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+    }
+  }
+}
+
+// The output dims pv_tile leaves in a lane (g, tq): for column e of its tiles, dims d0 + 2i
+// and d0 + 2i + 1 in acc[i][e] and acc[i][2+e] (i < 4) and dims d1 + 2i, +1 in acc[4+i][..],
+// with (d0, d1) = (8g, 64+8g) for 16-bit tiles and (16g, 16g+8) for e4m3 ones.  These write
+// them, times inv, as two runs of 8: to a 16-bit row, or to an fp32 row.
+template <bool F8>
+__device__ __forceinline__ int pv_dim(int g, int h) {
+  return F8 ? 16 * g + 8 * h : 8 * g + 64 * h;
+}
+template <typename T, bool F8>
+__device__ __forceinline__ void store_pv_row(T* row, const float (&acc)[8][4], int e, float inv,
+                                             int g) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float(*c)[4] = acc + 4 * h;
+    *reinterpret_cast<uint4*>(row + pv_dim<F8>(g, h)) =
+        make_uint4(Elem<T>::pack2(c[0][e] * inv, c[0][2 + e] * inv),
+                   Elem<T>::pack2(c[1][e] * inv, c[1][2 + e] * inv),
+                   Elem<T>::pack2(c[2][e] * inv, c[2][2 + e] * inv),
+                   Elem<T>::pack2(c[3][e] * inv, c[3][2 + e] * inv));
+  }
+}
+template <bool F8>
+__device__ __forceinline__ void store_pv_row_f32(float* row, const float (&acc)[8][4], int e,
+                                                 float inv, int g) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float(*c)[4] = acc + 4 * h;
+    float4* d = reinterpret_cast<float4*>(row + pv_dim<F8>(g, h));
+    d[0] = make_float4(c[0][e] * inv, c[0][2 + e] * inv, c[1][e] * inv, c[1][2 + e] * inv);
+    d[1] = make_float4(c[2][e] * inv, c[2][2 + e] * inv, c[3][e] * inv, c[3][2 + e] * inv);
+  }
 }
 
 // CTA holding global tile `pos` when T tiles are shared out over `grid` CTAs
@@ -801,8 +912,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
             if (bid >= 0) {
               const int row = (t * kTileTok) & bs_mask;
               uint8_t* dst = ring + slot * C::SLOT_BYTES;
-              tma_load_4d(dst, &tmK, 0, hp * HB, row, bid, &full[slot]);
-              tma_load_4d(dst + C::TILE_BYTES, &tmV, 0, hp * HB, row, bid, &full[slot]);
+#pragma unroll
+              for (int h = 0; h < C::SLABS; ++h) {  // map coordinates: dim, token, kv-head, block
+                tma_load_4d(dst + h * C::SLAB_BYTES, &tmK, h * 64, row, hp * HB, bid, &full[slot]);
+                tma_load_4d(dst + C::TILE_BYTES + h * C::SLAB_BYTES, &tmV, h * 64, row, hp * HB,
+                            bid, &full[slot]);
+              }
               issued |= 1u;
             }
           }
@@ -831,16 +946,17 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
   // tiles that share every K and V^T fragment.  Per 16-token tile: S^T = K Q^T (M = 16
   // tokens, N = 2 x 8 rows, K = 128 dims: 16 MMAs), the online softmax of each row, and
   // O^T += V^T P^T (M = 128 dims in 8 tiles, K = 16 tokens: 16 MMAs).  Lane (g, tq) holds
-  // the logits of tokens g and g+8 for rows nt*8 + 2tq, +1 and their outputs for dims
-  // [16g, 16g+16); dims are paired as in the G = 8 consumer.  The rows' q is read from
-  // global memory once per segment.  Returns false when the CTA aborted.
+  // the logits of tokens g and g+8 for rows nt*8 + 2tq, +1 and their outputs for the dims
+  // pv_tile gives it; K and q dims go in kchunk order.  The rows' q is read from global
+  // memory once per segment.  Returns false when the CTA aborted.
   auto chunk_segment = [&](int& k, int& cnt, int qs, const volatile int* u) -> bool {
     const int s = u[0], hp = u[1], pslot = u[5], m0 = u[7], slot0 = u[8], nseg = u[9];
     const int nm = u[10];
     int t0 = u[2], t1 = u[3], flags = u[4];
-    constexpr int RS = HB * kRowBytes;  // bytes between consecutive tokens of a tile
     const int g = lane >> 2, tq = lane & 3;
     const int kvh = hp * HB + w;
+    // K chunks 2tq (k-steps j even) and 2tq+1 (j odd) of token g; kchunk adds the slab
+    const int kofs0 = swz(w, g, 2 * tq), kofs1 = swz(w, g, 2 * tq + 1);
     uint32_t qf[2][8][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -849,7 +965,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           static_cast<const T*>(a.q) + ((long long)(m0 + ml) * a.num_q_heads + kvh * G + jj) * kD);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 v = ml < nm ? __ldg(src + tq + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v = ml < nm ? __ldg(src + kchunk(tq, j)) : make_uint4(0u, 0u, 0u, 0u);
         qf[nt][2 * j][0] = v.x;
         qf[nt][2 * j][1] = v.y;
         qf[nt][2 * j + 1][0] = v.z;
@@ -871,13 +987,14 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
         const int slot = cnt % nslots;
         wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
         const int nvalid = min(kTileTok, L - t * kTileTok);
-        const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+        const uint8_t* Ks = ring + slot * C::SLOT_BYTES;
         const uint8_t* Vs = Ks + C::TILE_BYTES;
         float sc4[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
-          const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+          const uint8_t* kj = Ks + (j >> 1) * C::SLAB_BYTES + ((j & 1) ? kofs1 : kofs0);
+          const uint4 ka = *reinterpret_cast<const uint4*>(kj);
+          const uint4 kb = *reinterpret_cast<const uint4*>(kj + 1024);  // token g+8
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             Mma<T>::run(sc4[nt], ka.x, kb.x, ka.y, kb.y, qf[nt][2 * j][0], qf[nt][2 * j][1]);
@@ -921,29 +1038,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           pb[nt][0] = transpose8x8(Mma<T>::pack(p0, p1));
           pb[nt][1] = transpose8x8(Mma<T>::pack(p2, p3));
         }
-        // V^T fragments, two m-tiles at a time: word r (dims 16g+2r, +1) and word 4+r
-        // (dims 16g+8+2r, +1) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (zero past the end)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          uint32_t lo[4], hi[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-            const bool ok = tk < nvalid;
-            const uint8_t* vr = Vs + tk * RS + g * 32 + r * 4;
-            lo[i] = ok ? *reinterpret_cast<const uint32_t*>(vr) : 0u;
-            hi[i] = ok ? *reinterpret_cast<const uint32_t*>(vr + 16) : 0u;
-          }
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const uint32_t sel = e ? 0x7632u : 0x5410u;
-            const uint32_t a0 = __byte_perm(lo[0], lo[1], sel), a1 = __byte_perm(hi[0], hi[1], sel);
-            const uint32_t a2 = __byte_perm(lo[2], lo[3], sel), a3 = __byte_perm(hi[2], hi[3], sel);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-              Mma<T>::run(oacc[nt][2 * r + e], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-          }
-        }
+        pv_tile<false, T, 2, C::SLAB_BYTES>(oacc, Vs, w, g, tq, nvalid, pb);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
       }
@@ -973,14 +1068,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
         const float lt = e ? lt1 : lt0;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
         const long long row = (long long)pslot * (HB * kChunkRows) + w * kChunkRows + r;
-        float4* po = reinterpret_cast<float4*>(a.vpart_o + row * kD + 16 * g);
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          po[i] = make_float4(oacc[nt][4 * i][e] * inv, oacc[nt][4 * i + 1][e] * inv,
-                              oacc[nt][4 * i + 2][e] * inv, oacc[nt][4 * i + 3][e] * inv);
-          po[2 + i] = make_float4(oacc[nt][4 * i][2 + e] * inv, oacc[nt][4 * i + 1][2 + e] * inv,
-                                  oacc[nt][4 * i + 2][2 + e] * inv, oacc[nt][4 * i + 3][2 + e] * inv);
-        }
+        store_pv_row_f32<false>(a.vpart_o + row * kD, oacc[nt], e, inv, g);
         if (g == 0)
           *reinterpret_cast<float2*>(a.vpart_ml + row * 2) = make_float2(mh[nt][e], lt);
       }
@@ -1003,8 +1091,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
     // K scale folded into the logit scale and the V scale into the final normalisation;
     // with G < 8 the q-heads past G are zero columns of the MMAs and are not written.
     using MT = typename std::conditional<F8, __half, T>::type;  // MMA operand type
-    constexpr int RS = HB * C::KROW;  // bytes between consecutive tokens of a tile
     const int g = lane >> 2, tq = lane & 3;
+    // K chunks 2tq and 2tq+1 of token g (16-bit: k-steps of even / odd j, slab j/2; e4m3:
+    // c = 0 / 1)
+    const int kofs0 = swz(w, g, 2 * tq), kofs1 = swz(w, g, 2 * tq + 1);
     int cnt = 0;
     // one segment per iteration: its first unit (kFirst) loads q, its last (kLast) writes
     // the result; the segment's state is dead once it is written
@@ -1022,17 +1112,18 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
       }
       const int hp = u[1], pslot = u[5], orow = u[7], slot0 = u[8], nseg = u[9];
       int t0 = u[2], t1 = u[3], flags = u[4];
-      uint32_t qf[8][2];  // Q^T fragments of the 8 k-steps
-      float oacc[8][4];   // O^T: [m-tile mt] dims 16g+mt / 16g+8+mt x heads 2tq, 2tq+1
+      uint32_t qf[8][2];    // Q^T fragments of the 8 k-steps
+      float oaccs[1][8][4];  // O^T: [m-tile] x heads 2tq, 2tq+1 (dims: pv_tile)
+      float(&oacc)[8][4] = oaccs[0];
       float mh0 = -INFINITY, mh1 = -INFINITY, lh0 = 0.f, lh1 = 0.f;  // heads 2tq, 2tq+1
       {
         const uint8_t* qrow = qbuf + qs * C::QBYTES + (w * G + g) * kRowBytes;
         if constexpr (F8) {
-          // k-step 4c+i takes dims 4i..4i+3 of the 16-dim chunk tq + 4c (one 32-bit
+          // k-step 4c+i takes dims 4i..4i+3 of the 16-dim chunk 2tq + c (one 32-bit
           // word of e4m3 codes); Q takes the same dims, as f16 pairs
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            const uint8_t* src = qrow + (tq + 4 * c) * 32;
+            const uint8_t* src = qrow + (2 * tq + c) * 32;
             uint32_t wq[8];
             *reinterpret_cast<uint4*>(wq) = *reinterpret_cast<const uint4*>(src);
             *reinterpret_cast<uint4*>(wq + 4) = *reinterpret_cast<const uint4*>(src + 16);
@@ -1050,7 +1141,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
         } else {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // q-heads past G (rows of the next warp): zero
-            const uint4 v = g < G ? *reinterpret_cast<const uint4*>(qrow + (tq + 4 * j) * 16)
+            const uint4 v = g < G ? *reinterpret_cast<const uint4*>(qrow + kchunk(tq, j) * 16)
                                   : make_uint4(0u, 0u, 0u, 0u);
             qf[2 * j][0] = v.x;
             qf[2 * j][1] = v.y;
@@ -1072,8 +1163,8 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           const int slot = cnt % nslots;
           wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
           const int nvalid = min(kTileTok, L - t * kTileTok);
-          // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-          const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * C::KROW;
+          // tile layout: column slabs of [HB kv-heads][16 tokens][128 B] (swz)
+          const uint8_t* Ks = ring + slot * C::SLOT_BYTES;
           const uint8_t* Vs = Ks + C::TILE_BYTES;
 
           // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
@@ -1081,8 +1172,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           if constexpr (F8) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * c) * 16);
-              const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * c) * 16);
+              const uint8_t* kc = Ks + (c ? kofs1 : kofs0);
+              const uint4 ka = *reinterpret_cast<const uint4*>(kc);
+              const uint4 kb = *reinterpret_cast<const uint4*>(kc + 1024);  // token g+8
               const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i)
@@ -1093,8 +1185,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint4 ka = *reinterpret_cast<const uint4*>(Ks + g * RS + (tq + 4 * j) * 16);
-              const uint4 kb = *reinterpret_cast<const uint4*>(Ks + (g + 8) * RS + (tq + 4 * j) * 16);
+              const uint8_t* kj = Ks + (j >> 1) * C::SLAB_BYTES + ((j & 1) ? kofs1 : kofs0);
+              const uint4 ka = *reinterpret_cast<const uint4*>(kj);
+              const uint4 kb = *reinterpret_cast<const uint4*>(kj + 1024);  // token g+8
               Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
               Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
             }
@@ -1134,45 +1227,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           // ---- P^T fragments: [tokens 2tq, 2tq+1 | 8+2tq, 9+2tq] x head g
           const uint32_t pb0 = transpose8x8(Mma<MT>::pack(p0, p1));
           const uint32_t pb1 = transpose8x8(Mma<MT>::pack(p2, p3));
-          // ---- V^T fragments: dims [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9,
-          // paired along tokens; rows past the sequence end are zeroed (p is 0 there, but
-          // the block's unused rows may hold anything)
-          uint32_t vw[4][8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-            uint4 lo, hi;
-            if constexpr (F8) {  // 16 e4m3 codes -> 8 f16 pairs
-              const uint4 c8 = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 16);
-              lo = make_uint4(e4m3x2_to_f16x2(c8.x), e4m3x2_to_f16x2(c8.x >> 16),
-                              e4m3x2_to_f16x2(c8.y), e4m3x2_to_f16x2(c8.y >> 16));
-              hi = make_uint4(e4m3x2_to_f16x2(c8.z), e4m3x2_to_f16x2(c8.z >> 16),
-                              e4m3x2_to_f16x2(c8.w), e4m3x2_to_f16x2(c8.w >> 16));
-            } else {
-              lo = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32);
-              hi = *reinterpret_cast<const uint4*>(Vs + tk * RS + g * 32 + 16);
-            }
-            const bool ok = tk < nvalid;
-            vw[i][0] = ok ? lo.x : 0u;
-            vw[i][1] = ok ? lo.y : 0u;
-            vw[i][2] = ok ? lo.z : 0u;
-            vw[i][3] = ok ? lo.w : 0u;
-            vw[i][4] = ok ? hi.x : 0u;
-            vw[i][5] = ok ? hi.y : 0u;
-            vw[i][6] = ok ? hi.z : 0u;
-            vw[i][7] = ok ? hi.w : 0u;
-          }
-          // ---- O^T += V^T P^T, m-tile mt: rows dims 16g+mt (g) and 16g+8+mt (g+8)
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const int r = mt >> 1;
-            const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
-            const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], sel);
-            const uint32_t a1 = __byte_perm(vw[0][4 + r], vw[1][4 + r], sel);
-            const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], sel);
-            const uint32_t a3 = __byte_perm(vw[2][4 + r], vw[3][4 + r], sel);
-            Mma<MT>::run(oacc[mt], a0, a1, a2, a3, pb0, pb1);
-          }
+          // ---- O^T += V^T P^T (rows past the sequence end are zeroed: p is 0 there, but the
+          // block's unused rows may hold anything)
+          const uint32_t pb[1][2] = {{pb0, pb1}};
+          pv_tile<F8, MT, 1, C::SLAB_BYTES>(oaccs, Vs, w, g, tq, nvalid, pb);
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);
         }
@@ -1207,26 +1265,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
         if (2 * tq + e >= G) continue;  // a zero column (G < 8)
         const float inv = e ? inv1 : inv0;
         if (flags & kDirect) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            pk[i] = Elem<T>::pack2(oacc[2 * i][e] * inv, oacc[2 * i + 1][e] * inv);
-            pk[4 + i] = Elem<T>::pack2(oacc[2 * i][2 + e] * inv, oacc[2 * i + 1][2 + e] * inv);
-          }
-          T* ob = static_cast<T*>(a.out) +
-                  ((long long)orow * a.num_q_heads + hp * HBG + j0 + e) * kD + 16 * g;
-          reinterpret_cast<uint4*>(ob)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          reinterpret_cast<uint4*>(ob)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          store_pv_row<T, F8>(static_cast<T*>(a.out) +
+                                  ((long long)orow * a.num_q_heads + hp * HBG + j0 + e) * kD,
+                              oacc, e, inv, g);
         } else {
           const long long row = (long long)pslot * HBG + j0 + e;
-          float4* po = reinterpret_cast<float4*>(a.part_o + row * kD + 16 * g);
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            po[i] = make_float4(oacc[4 * i][e] * inv, oacc[4 * i + 1][e] * inv,
-                                oacc[4 * i + 2][e] * inv, oacc[4 * i + 3][e] * inv);
-            po[2 + i] = make_float4(oacc[4 * i][2 + e] * inv, oacc[4 * i + 1][2 + e] * inv,
-                                    oacc[4 * i + 2][2 + e] * inv, oacc[4 * i + 3][2 + e] * inv);
-          }
+          store_pv_row_f32<F8>(a.part_o + row * kD, oacc, e, inv, g);
           if (g == 0)
             *reinterpret_cast<float2*>(a.part_ml + row * 2) =
                 make_float2(e ? mh1 : mh0, e ? lt1 : lt0);
@@ -1287,8 +1331,8 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           const int slot = cnt % nslots;
           wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
           const int nvalid = min(kTileTok, L - t * kTileTok);
-          // tile layout (TMA box): [16 tokens][HB kv-heads][128 dims]
-          const uint8_t* Ks = ring + slot * C::SLOT_BYTES + w * kRowBytes;
+          // tile layout: two slabs (dims 0..63, 64..127) of [HB kv-heads][16 tokens][128 B]
+          const uint8_t* Ks = ring + slot * C::SLOT_BYTES;
           const uint8_t* Vs = Ks + C::TILE_BYTES;
 
           // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
@@ -1296,9 +1340,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
 #pragma unroll
           for (int ps = 0; ps < 4; ++ps) {
             const int rr = ps * 4 + tp;
-            const uint8_t* kr = Ks + rr * (HB * kRowBytes);
-            const uint4 w0 = *reinterpret_cast<const uint4*>(kr + sub * 16);
-            const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 128 + sub * 16);
+            const uint8_t* kr = Ks + swz(w, rr, sub);  // dims 8sub.. of slab 0, then of slab 1
+            const uint4 w0 = *reinterpret_cast<const uint4*>(kr);
+            const uint4 w1 = *reinterpret_cast<const uint4*>(kr + C::SLAB_BYTES);
             const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
             float2 kf[8];
 #pragma unroll
@@ -1340,9 +1384,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
               acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
             }
           }
-          // ---- p.V: lane owns dims [4*lane, 4*lane+4)
+          // ---- p.V: lane owns dims [4*lane, 4*lane+4): slab lane/16, chunk (lane%16)/2
+          const uint8_t* Vl = Vs + (lane >> 4) * C::SLAB_BYTES + (lane & 1) * 8;
           auto pv_row = [&](int tt) {
-            const uint2 vw = *reinterpret_cast<const uint2*>(Vs + tt * (HB * kRowBytes) + lane * 8);
+            const uint2 vw = *reinterpret_cast<const uint2*>(Vl + swz(w, tt, (lane & 15) >> 1));
             const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
 #pragma unroll
             for (int jj = 0; jj < GW; ++jj) {
@@ -1763,18 +1808,21 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   CUtensorMap tmK, tmV, tmQ;
   const uint64_t row = (uint64_t)head_dim * 2;
   const uint64_t crow = (uint64_t)head_dim * (f8 ? 1 : 2);  // one kv-head of one token
-  const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
+  // the cache viewed as [block][token][kv-head][dim] with token and kv-head swapped in the
+  // map: a box of 16 tokens x HB kv-heads x one 128-byte column slab lands as
+  // [kv-head][token][128 B], swizzled (the kernel's swz)
+  const uint64_t cdims[4] = {(uint64_t)head_dim, (uint64_t)block_size, (uint64_t)num_kv_heads,
                              (uint64_t)num_blocks};
-  const uint64_t cstr[3] = {crow, crow * num_kv_heads, crow * num_kv_heads * block_size};
-  const uint32_t cbox[4] = {(uint32_t)head_dim, (uint32_t)HB, 16, 1};
+  const uint64_t cstr[3] = {crow * num_kv_heads, crow, crow * num_kv_heads * block_size};
+  const uint32_t cbox[4] = {f8 ? 128u : 64u, 16, (uint32_t)HB, 1};
   const uint64_t qdims[3] = {(uint64_t)head_dim, (uint64_t)num_q_heads,
                              (uint64_t)(qsl ? num_q_rows : num_seqs)};
   const uint64_t qstr[2] = {row, row * num_q_heads};
   const uint32_t qbox[3] = {(uint32_t)head_dim, (uint32_t)HBG, 1};
   const CUtensorMapDataType ct =
       f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-  if (!pa::encode_tmap(&tmK, ct, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !pa::encode_tmap(&tmV, ct, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  if (!pa::encode_tmap(&tmK, ct, k_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !pa::encode_tmap(&tmV, ct, v_cache, 4, cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !pa::encode_tmap_16bit(&tmQ, q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_SWIZZLE_NONE))
     return PA_ERR_CUDA;
 

@@ -118,16 +118,6 @@ bool encode_tmap_16bit(CUtensorMap* out, const void* base, int rank, const uint6
                      swizzle);
 }
 
-bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,
-                       int num_kv_heads, int head_dim, int box_rows) {
-  // innermost first: head_dim, kv-head, token-in-block, block
-  const uint64_t dims[4] = {(uint64_t)head_dim, (uint64_t)num_kv_heads, (uint64_t)block_size,
-                            (uint64_t)num_blocks};
-  const uint64_t row = (uint64_t)head_dim * 2;
-  const uint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
-  const uint32_t box[4] = {(uint32_t)head_dim, 1, (uint32_t)box_rows, 1};
-  return encode_tmap_16bit(out, cache, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
 
 long long take_wait_limit(int kind, int* withhold) {
   *withhold = 0;

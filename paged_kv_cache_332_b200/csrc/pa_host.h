@@ -25,16 +25,9 @@ int num_sms();
 // calls cost a map lookup instead of a driver call.
 bool ensure_dynamic_smem(const void* func, int bytes);
 
-// Encode a 4-D tiled TMA descriptor over a KV cache
-// [num_blocks, block_size, num_kv_heads, head_dim] of 16-bit elements whose box is
-// `box_rows` consecutive tokens x head_dim of one kv-head of one block.
-bool encode_cache_tmap(CUtensorMap* out, const void* cache, int num_blocks, int block_size,
-                       int num_kv_heads, int head_dim, int box_rows);
-
-// Encode a tiled TMA descriptor over a row-major tensor of 16-bit elements.
-// dims/box innermost first; strides_bytes[i] is the stride of dimension i+1.
 // Encode a tiled TMA descriptor of `type` elements (rank <= 5, dims innermost first,
-// strides in bytes for dims 1.., element strides 1, no interleave, L2 promotion 256 B).
+// strides in bytes for dims 1.., element strides 1, no interleave, L2 promotion 256 B);
+// the _16bit form takes 16-bit elements.
 bool encode_tmap(CUtensorMap* out, CUtensorMapDataType type, const void* base, int rank,
                  const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                  CUtensorMapSwizzle swizzle);

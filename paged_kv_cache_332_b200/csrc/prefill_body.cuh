@@ -336,8 +336,8 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
       if (lane == 0) mbar_arrive(q_full);
     }
     float m_ref = -INFINITY, l = 0.f;
-    for (int kt = 0, j = 0; kt < n_kt; ++kt, ++j) {
-      wait_or_abort(&s_full[mt], j & 1, abort_flag, a.err, a.wait_limit);
+    for (int kt = 0; kt < n_kt; ++kt) {
+      wait_or_abort(&s_full[mt], kt & 1, abort_flag, a.err, a.wait_limit);
       tc_fence_after();
       const int key0 = (kt_lo + kt) * kBN;
       // the whole S row (128 keys) in registers: one pass over TMEM
@@ -366,7 +366,7 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
         alpha = fast_exp2(m_ref - mx);  // m_ref = -inf -> 0
         m_ref = mx;
       }
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float o[32];
