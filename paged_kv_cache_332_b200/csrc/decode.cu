@@ -71,13 +71,12 @@ struct DecodeArgs {
   const int32_t* seq_lens;
   float* part_o;   // [slots, HB*G, 128]   normalised partial outputs
   float* part_ml;  // [slots, HB*G, 2]     (max in log2 units, sum)
-  // merge records for the log-sum-exp pass: (first slot, segment count) of each (sequence,
-  // head group) [B * NHP] and of each (chunk, head group) [vcap * NHP]; count 0 when
-  // nothing is left to merge (written directly, or no keys); and the chunk numbering of
-  // the groups [num_groups + 1] as CTA 0 computed it
+  // merge records for the log-sum-exp pass, per (sequence, head group) [B * NHP]: its own
+  // segments (first slot, segment count; count 0 when nothing is left to merge: written
+  // directly, or no keys), and with shared prefixes its chunk's segments (first chunk slot,
+  // count, the member's first row in the chunk's rows of a kv-head, 0)
   int2* meta;
-  int2* vmeta;
-  int* cstart_out;
+  int4* cmeta;
   // append in the same launch (k_new != nullptr): the step's new token of each sequence,
   // [B, Hkv, 128], written into its cache slot at position seq_len-1 before it is read
   const void* k_new;
@@ -447,7 +446,7 @@ __device__ __forceinline__ int cta_of(int pos, int T, int grid) {
 // pass with a running maximum, up to eight rows per round with all their loads in flight.
 // Launched as a programmatic dependent of the decode kernel.
 template <typename T, int G, bool SP>
-__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) {
+__global__ void __launch_bounds__(256, 2) merge_kernel(const DecodeArgs a, int HB) {
   griddep_wait();  // the decode grid has finished and its writes are visible
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -459,29 +458,23 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) 
   const int2 mo = a.meta[s * NHP + hp];
   const int so0 = mo.x, no = mo.y;
   int sv0 = 0, nv = 0, vrow = 0;
-  if constexpr (SP) {
-    const int g = group_of(a, s);
-    if (g >= 0 && __ldg(a.prefix_lens + g) > 0) {
-      const int off = s - __ldg(a.group_starts + g);
-      const int vs = a.cstart_out[g] + off / a.mc;
-      if (vs < min(a.cstart_out[a.num_groups], a.vcap)) {
-        const int2 mv = a.vmeta[vs * NHP + hp];
-        sv0 = mv.x;
-        nv = mv.y;
-        vrow = (j / G) * kChunkRows + (off % a.mc) * G + (qh % G);
-      }
-    }
+  if constexpr (SP) {  // loaded beside the own record: one round trip for both
+    const int4 cm = a.cmeta[s * NHP + hp];
+    sv0 = cm.x;
+    nv = cm.y;
+    vrow = (j / G) * kChunkRows + cm.z + (qh % G);
   }
   const int total = no + nv;
   if (total == 0) return;  // written by the decode kernel (or nothing to write)
   float M = -INFINITY, den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < total; i0 += 8) {
-    float2 mlv[8];
-    float4 ov[8];
+  constexpr int R = 16;  // pieces per round, all their loads in flight
+  for (int i0 = 0; i0 < total; i0 += R) {
+    float2 mlv[R];
+    float4 ov[R];
     float Mr = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < R; ++u) {
       const int i = i0 + u;
       if (i < total) {
         const bool own = i < no;
@@ -498,7 +491,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) 
     den *= sc;
     num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < R; ++u) {
       if (i0 + u < total) {
         const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
         den += f;
@@ -710,11 +703,30 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           reinterpret_cast<uint4*>(ob)[i] = make_uint4(0u, 0u, 0u, 0u);
       }
       if constexpr (SP) {
-        for (int v = cta; v < V; v += ncta)  // chunks without tiles
-          if (slen[B + v] == 0)
-            for (int h = lane; h < NHP; h += 32) a.vmeta[v * NHP + h] = make_int2(0, 0);
-        if (cta == 0)  // the chunk numbering, for the merge pass
-          for (int g = lane; g <= a.num_groups; g += 32) a.cstart_out[g] = cstart[g];
+        // each member's chunk record for the merge pass: the chunk's segments over its
+        // prefix (as the staging warps cut them: first slot, count) and the member's rows
+        for (int s = cta; s < B; s += ncta) {
+          int vs = -1, voff = 0;
+          const int g = group_of(a, s);
+          if (g >= 0 && __ldg(a.prefix_lens + g) > 0) {
+            const int off = s - __ldg(a.group_starts + g);
+            const int v = cstart[g] + off / a.mc;
+            if (v < V) {
+              vs = v;
+              voff = (off % a.mc) * G;
+            }
+          }
+          const int cntv = vs >= 0 ? cdiv(slen[B + vs], kTileTok) : 0;
+          for (int h = lane; h < NHP; h += 32) {
+            int4 r = make_int4(0, 0, 0, 0);
+            if (cntv > 0) {
+              const int gs = sstart[B + vs] + h * cntv;
+              const int c0 = cta_of(gs, Ttot, grid), c1 = cta_of(gs + cntv - 1, Ttot, grid);
+              r = make_int4(c0 + vs * NHP + h, c1 - c0 + 1, voff, 0);
+            }
+            a.cmeta[s * NHP + h] = r;
+          }
+        }
       }
       return;
     }
@@ -838,9 +850,8 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           }
         }
         if (lane == 0) {
-          if (t0 == ts)  // the group's first unit: its merge record
-            (virt ? a.vmeta : a.meta)[grp] =
-                make_int2(c0 + grp, (flags & kDirect) ? 0 : c1 - c0 + 1);
+          if (t0 == ts && !virt)  // the group's first unit: its merge record
+            a.meta[grp] = make_int2(c0 + grp, (flags & kDirect) ? 0 : c1 - c0 + 1);
           u[0] = s;
           u[1] = hp;
           u[2] = t0;
@@ -886,6 +897,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
       if (lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
+        const uint64_t pol_stream = l2_policy_evict_first(), pol_keep = l2_policy_evict_normal();
         const int bs_mask = (1 << a.log2_bs) - 1;
         // bit i: tile cnt-1-i was copied.  Each ring slot is reused only after its previous
         // copy was consumed, so only the last nslots tiles can still be landing.
@@ -898,6 +910,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           const int s = u[0];
           if (s < 0 || *abort_flag) break;  // (one thread: a plain read)
           const int hp = u[1], t0 = u[2], t1 = u[3], append = u[6];
+          // a sequence's own keys are read once: evict them first from L2, so the stream
+          // displaces itself rather than other lines; a shared prefix is read again by the
+          // group's other chunks
+          const uint64_t pol = (u[4] & kVirtual) ? pol_keep : pol_stream;
           for (int t = t0; t < t1; ++t, ++cnt) {
             const int slot = cnt % nslots;
             // the new token's row is in the last tile: its stores must have landed
@@ -914,9 +930,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
               uint8_t* dst = ring + slot * C::SLOT_BYTES;
 #pragma unroll
               for (int h = 0; h < C::SLABS; ++h) {  // map coordinates: dim, token, kv-head, block
-                tma_load_4d(dst + h * C::SLAB_BYTES, &tmK, h * 64, row, hp * HB, bid, &full[slot]);
-                tma_load_4d(dst + C::TILE_BYTES + h * C::SLAB_BYTES, &tmV, h * 64, row, hp * HB,
-                            bid, &full[slot]);
+                tma_load_4d_hint(dst + h * C::SLAB_BYTES, &tmK, h * 64, row, hp * HB, bid,
+                                 &full[slot], pol);
+                tma_load_4d_hint(dst + C::TILE_BYTES + h * C::SLAB_BYTES, &tmV, h * 64, row,
+                                 hp * HB, bid, &full[slot], pol);
               }
               issued |= 1u;
             }
@@ -1790,15 +1807,14 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   const long long groups = (long long)num_seqs * NHP;
   const pa::WsLayout lay = pa::ws_layout(groups, grid + groups, HBG, head_dim);
   // shared prefixes: the chunks' partial rows follow, (grid + chunks x head groups) slots of
-  // HB x 16 rows, then the chunks' merge records and the groups' chunk numbering
+  // HB x 16 rows, then the members' chunk records (one per sequence and head group)
   const long long vslots = sp ? grid + (long long)vcap * NHP : 0;
   const long long vrows = vslots * HB * pa::kChunkRows;
-  size_t voff = 0, vmeta_off = 0, cstart_off = 0, need = lay.total;
+  size_t voff = 0, cmeta_off = 0, need = lay.total;
   if (sp) {
     voff = pa::align256(lay.total);
-    vmeta_off = pa::align256(voff + (size_t)vrows * (head_dim + 2) * sizeof(float));
-    cstart_off = pa::align256(vmeta_off + (size_t)vcap * NHP * sizeof(int2));
-    need = cstart_off + (size_t)(sp->num_groups + 1) * sizeof(int);
+    cmeta_off = pa::align256(voff + (size_t)vrows * (head_dim + 2) * sizeof(float));
+    need = cmeta_off + (size_t)num_seqs * NHP * sizeof(int4);
   }
   if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE_TOO_SMALL;
   if ((uintptr_t)workspace & 255) return PA_ERR_INVALID_ARG;
@@ -1833,8 +1849,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.seq_lens = seq_lens;
   a.q = q;
   a.meta = reinterpret_cast<int2*>(ws + lay.meta);
-  a.vmeta = nullptr;
-  a.cstart_out = nullptr;
+  a.cmeta = nullptr;
   a.k_new = k_new;
   a.v_new = v_new;
   a.k_cache = const_cast<void*>(k_cache);
@@ -1884,8 +1899,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
     a.max_prefix = sp->max_prefix_len;
     a.vpart_o = reinterpret_cast<float*>(ws + voff);
     a.vpart_ml = a.vpart_o + (size_t)vrows * head_dim;
-    a.vmeta = reinterpret_cast<int2*>(ws + vmeta_off);
-    a.cstart_out = reinterpret_cast<int*>(ws + cstart_off);
+    a.cmeta = reinterpret_cast<int4*>(ws + cmeta_off);
     return dtype == PA_F16
                ? pa::dispatch_group<__half, false, true>(G, HB, tmK, tmV, tmQ, a, (int)grid, st)
                : pa::dispatch_group<__nv_bfloat16, false, true>(G, HB, tmK, tmV, tmQ, a,
@@ -2008,13 +2022,11 @@ extern "C" size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q
   const size_t base = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_seq_len, 0);
   if (base == 0 || num_kv_heads <= 0) return 0;
   // the chunks' partial rows: (grid + chunks x head groups) slots of (kv-heads per group x 16)
-  // rows, at most (256 + num_seqs) x num_kv_heads x 16 rows of head_dim + 2 fp32; their merge
-  // records (at most num_seqs x num_kv_heads) and the chunk numbering (num_seqs + 1 ints)
-  return pa::align256(pa::align256(pa::align256(base) + ((size_t)pa::kMaxGrid + num_seqs) *
-                                                            num_kv_heads * pa::kChunkRows *
-                                                            (head_dim + 2) * sizeof(float)) +
-                      (size_t)num_seqs * num_kv_heads * sizeof(int2)) +
-         (size_t)(num_seqs + 1) * sizeof(int);
+  // rows, at most (256 + num_seqs) x num_kv_heads x 16 rows of head_dim + 2 fp32; then the
+  // members' chunk records (at most num_seqs x num_kv_heads int4)
+  return pa::align256(pa::align256(base) + ((size_t)pa::kMaxGrid + num_seqs) * num_kv_heads *
+                                               pa::kChunkRows * (head_dim + 2) * sizeof(float)) +
+         (size_t)num_seqs * num_kv_heads * 4 * sizeof(int);
 }
 
 extern "C" pa_status pa_decode_shared_prefix(

@@ -124,6 +124,30 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, int
       : "memory");
 }
 
+// L2 cache policies for bulk copies: data read once (evict first, so that it displaces
+// itself rather than other lines), and data other CTAs read again soon (normal priority).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 4-D tiled bulk tensor load global -> shared with an L2 cache policy (no multicast).
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* m, int c0, int c1,
+                                                 int c2, int c3, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)),
+      "l"(policy)
+      : "memory");
+}
+
 // 3-D tiled bulk tensor load global -> shared (no multicast).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, int c0, int c1, int c2,
                                             uint64_t* bar) {

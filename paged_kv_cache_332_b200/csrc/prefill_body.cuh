@@ -59,6 +59,13 @@ constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TMEM + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;  // + alignment slack
 
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes,
                                                uint32_t sbo_bytes) {
   return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)(lbo_bytes >> 4) << 16) |
@@ -143,6 +150,45 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 128 consecutive columns of this thread's TMEM lane in one load, waited for inside the
+// same asm statement (one wait per row of S instead of two).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t r[128];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]),
+        "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]),
+        "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]),
+        "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]),
+        "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]),
+        "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]),
+        "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]),
+        "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]),
+        "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]),
+        "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+        "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]),
+        "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]),
+        "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -303,8 +349,8 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 4) {
-    // softmax warpgroups: 208 registers each thread (one S row of 128 fp32 in registers)
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+    // softmax warpgroups: 192 registers each thread (one S row of 128 fp32 in registers)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ======================== softmax warpgroups ========================
     const int mt = (warp - 4) >> 2;
     const int wq = warp & 3;              // TMEM lane quarter
@@ -342,23 +388,24 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
       const int key0 = (kt_lo + kt) * kBN;
       // the whole S row (128 keys) in registers: one pass over TMEM
       float v[kBN];
-      tmem_ld64(t_s, v);
-      tmem_ld64(t_s + 64, v + 64);
+      tmem_ld128(t_s, v);
       if (key0 + kBN - 1 > wlim) {  // causal diagonal or sequence end in this tile
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (key0 + i > limit) v[i] = -INFINITY;
       }
-      // row max as a tree of independent maxima (no 128-long dependency chain)
+      // row max: eight independent chains of three-input maxima (the softmax warps are
+      // bound by instruction issue, so every instruction here counts)
       float mx8[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(v[j], v[j + 8]);
+      for (int j = 0; j < 8; ++j) {
+        mx8[j] = v[j];
 #pragma unroll
-      for (int i = 16; i < kBN; i += 8)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(mx8[j], v[i + j]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+        for (int i = 8; i < kBN - 8; i += 16) mx8[j] = fmax3(mx8[j], v[i + j], v[i + 8 + j]);
+        mx8[j] = fmaxf(mx8[j], v[kBN - 8 + j]);
+      }
+      const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7])) *
                        a.qscale;
       // lazy reference max: move it only when this tile exceeds it by more than 8
       float alpha = 1.f;
@@ -372,28 +419,35 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
           float o[32];
           tmem_ld32(t_o + c * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = __fmul2_rn(make_float2(o[i], o[i + 1]), make_float2(alpha, alpha));
+            o[i] = r.x;
+            o[i + 1] = r.y;
+          }
           tmem_st32(t_o + c * 32, o);
         }
       }
       // p = 2^(x*qscale - m_ref); masked keys hold -inf and give 0 (the offset is kept
-      // finite while every key so far was masked)
+      // finite while every key so far was masked); pairs of logits scaled and summed as
+      // f32x2 (one instruction per pair)
       const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float2 qs2 = make_float2(a.qscale, a.qscale), nm2 = make_float2(nm, nm);
+      float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = fast_exp2(fmaf(v[c * 32 + i], a.qscale, nm));
-          const float p1 = fast_exp2(fmaf(v[c * 32 + i + 1], a.qscale, nm));
-          sum8[(i >> 1) & 7] += p0 + p1;
-          w[i >> 1] = pack16<T>(p0, p1);
+          const float2 x = __ffma2_rn(make_float2(v[c * 32 + i], v[c * 32 + i + 1]), qs2, nm2);
+          const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          sum4[(i >> 1) & 3] = __fadd2_rn(sum4[(i >> 1) & 3], p);
+          w[i >> 1] = pack16<T>(p.x, p.y);
         }
         tmem_st16(t_s + c * 16, w);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
-                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      const float sum = ((sum4[0].x + sum4[0].y) + (sum4[1].x + sum4[1].y)) +
+                        ((sum4[2].x + sum4[2].y) + (sum4[3].x + sum4[3].y));
       l = l * alpha + sum;
       // keys past the sequence end in the last tile: clear their V rows
       if (mt == 0 && kt_lo + kt == n_kt_all - 1 && L < key0 + kBN) {
@@ -458,9 +512,10 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& tmK, const CUten
                 : -1;
     }
   } else {
-    // producer / MMA issuer / two idle warps: 88 registers each thread
-    // (128 x 88 + 256 x 208 = 384 x 168, the registers the CTA is launched with)
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    // producer / MMA issuer / two idle warps: 120 registers each thread (fewer spill the
+    // producer's block-id runs); 128 x 120 + 256 x 192 = 384 x 168, the registers the CTA
+    // is launched with
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 120;\n" ::: "memory");
     if (warp == 0) {
       // ======================== TMA producer ========================
       if (lane == 0) {

@@ -181,10 +181,10 @@ def test_shared_prefix_arguments_rejected_on_host(palib):
     assert dec() == 3 and dec(mp=0) == 3            # needs a workspace (shared or plain)
     base = palib.pa_decode_workspace_size(8, 32, 128, 512, 0)
     # chunk partials: (256 + num_seqs) x num_kv_heads x 16 rows of 130 fp32 after the base,
-    # then the chunks' merge records (num_seqs x num_kv_heads int2) and the chunk numbering
+    # then the members' chunk records (num_seqs x num_kv_heads int4)
     up = lambda n: -(-n // 256) * 256  # noqa: E731
     assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 8, 128, 512) == \
-        up(up(up(base) + (256 + 8) * 8 * 16 * 130 * 4) + 8 * 8 * 8) + 9 * 4
+        up(up(base) + (256 + 8) * 8 * 16 * 130 * 4) + 8 * 8 * 16
     assert palib.pa_decode_shared_prefix_workspace_size(0, 32, 8, 128, 512) == 0
     assert palib.pa_decode_shared_prefix_workspace_size(8, 32, 0, 128, 512) == 0
     assert palib.pa_last_launch_count() == 0
