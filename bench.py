@@ -370,9 +370,9 @@ def rooflines(step, dec_ms, pre_ms, peaks):
             sum(int(L) - int(n) + i + 1 for i in range(int(n))) for L, n in zip(lens, ql) if n > 1)
         pmean = statistics.mean(pre_ms)
         ideal_ms = (dec_bytes / (peaks["hbm_gbs"] * 1e9) + fl / (peaks["bf16_tflops"] * 1e12)) * 1e3
-        out["roofline"] = {"kernel": "pa_attention_varlen (paged_decode_kernel + merge_kernel"
-                                     " + chunked_prefill_kernel)",
-                           "bound": "hbm (decode rows) then tensor (chunks)",
+        out["roofline"] = {"kernel": "pa_attention_varlen (varlen_list_kernel + varlen_kernel:"
+                                     " decode CTAs beside chunked-prefill CTAs + merge_kernel)",
+                           "bound": "hbm (decode rows) beside tensor (chunks)",
                            "achieved": round(ideal_ms / pmean, 4), "peak": 1.0,
                            "unit": "fraction of the serial speed of light",
                            "frac": round(ideal_ms / pmean, 4), "ms_per_launch": round(pmean, 5),

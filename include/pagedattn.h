@@ -33,8 +33,8 @@
  *    calling thread's last call launched.
  *  - Return value: PA_OK once the kernels are launched, or an error found on the host
  *    before any launch (nothing is launched then).  PA_ERR_CUDA reports a failed launch
- *    or tensor-map encoding; a call of two kernels may have queued the first when the
- *    second fails to launch.  A launching call first clears a non-sticky CUDA error left
+ *    or tensor-map encoding; a call of several kernels may have queued the earlier ones
+ *    when a later one fails to launch.  A launching call first clears a non-sticky CUDA error left
  *    pending on the calling thread by earlier work (cudaGetLastError), so its status
  *    reports its own launches only.
  *  - Errors that depend on device data (a slot or block id outside the cache, a
@@ -262,14 +262,17 @@ PA_API pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k
  * sequences and prefill chunks ([P1] "工程边界与架构取舍": long prompts are prefilled in
  * chunks with decode steps in between).  Layout as pa_chunked_prefill: sequence s has
  * n = query_start_loc[s+1] - query_start_loc[s] query rows (its last n tokens, already
- * cached), q / out [num_q_rows, num_q_heads, 128].  Sequences with n == 1 run on the
- * decode kernel (reading q and writing out at row query_start_loc[s]), those with n > 1
- * on the tcgen05 prefill kernel; the result of each row is that of pa_chunked_prefill.
- * The call launches both kernels (and their merges) on `stream`.  The decode kernel
- * also lists the sequences with more than one
- * query row, and the prefill grid covers max_chunk_seqs of them (a host bound on their
- * number, like max_query_len; negative = num_seqs; more chunks than the bound set
- * PA_DEVERR_QUERY_LAYOUT and the extra ones are not computed).  Workspace: at least
+ * cached), q / out [num_q_rows, num_q_heads, 128].  Sequences with n == 1 are served as
+ * by pa_decode (reading q and writing out at row query_start_loc[s]), those with n > 1
+ * as by pa_chunked_prefill on the tcgen05 tensor cores; the result of each row is that
+ * of pa_chunked_prefill (a chunk item always runs whole, without the wave-tail split).
+ * Launches on `stream`: a small kernel lists the sequences with more than one query row;
+ * one persistent grid, whose first CTAs run the split-K decode over the one-row
+ * sequences and whose other CTAs run the chunks' prefill items (max_chunk_seqs of them:
+ * a host bound on their number, like max_query_len; negative = num_seqs; more chunks
+ * than the bound set PA_DEVERR_QUERY_LAYOUT and the extra ones are not computed); then
+ * the merge of the decode rows' split segments.  With max_query_len <= 1 (or a bound of
+ * 0) it is the decode launch and its merge only.  Workspace: at least
  * pa_attention_varlen_workspace_size(...) bytes, 256-byte aligned.  Limits as pa_decode
  * and pa_chunked_prefill; a decode row outside [0, num_q_rows) sets
  * PA_DEVERR_QUERY_LAYOUT and is skipped.
