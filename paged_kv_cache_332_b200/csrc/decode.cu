@@ -114,6 +114,7 @@ struct DecodeArgs {
   float qscale;          // scale * log2(e)
   long long wait_limit;  // SM cycles any pipeline wait may take before the CTA gives up
   int test_withhold;     // testing hook: CTA 0's producer withholds its first tile
+  int wait_prior;        // launched as a programmatic dependent: wait before reading inputs
 };
 
 constexpr int kD = 128;
@@ -545,6 +546,18 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
   const int lane = threadIdx.x & 31;
   // the merge pass may be scheduled now; it waits for this grid's results itself
   griddep_launch_dependents();
+  // This CTA's slice of the block tables into L2 (a hint: the lines are read later, after
+  // the lengths, by the staging warp), then, when this grid was launched as a dependent of
+  // the previous kernel of the stream, wait for it before any input is read.
+  if (threadIdx.x == 0 && ((uintptr_t)a.block_tables & 15) == 0) {
+    const long long tb = ((long long)B * a.max_blocks * 4) & ~15LL;
+    const long long per = (((tb + ncta - 1) / ncta) + 15) & ~15LL;
+    const long long off = per * cta;
+    if (off < tb)
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(a.block_tables) + off,
+                       (uint32_t)min(per, tb - off));
+  }
+  if (a.wait_prior) griddep_wait();
 
   // ---- clamped lengths and the prefix of tiles over (sequence, head group)
   if (warp == 0) {
@@ -1580,7 +1593,25 @@ pa_status launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const CU
   const size_t smem = ring_off + (size_t)nslots * C::SLOT_BYTES;
   auto kern = paged_decode_kernel<T, G, HB, F8, SP>;
   if (!ensure_dynamic_smem(reinterpret_cast<const void*>(kern), (int)smem)) return PA_ERR_CUDA;
-  kern<<<grid, C::THREADS, smem, stream>>>(tmK, tmV, tmQ, a);
+  // a programmatic dependent of the stream's previous kernel: the grid's launch and setup
+  // overlap that kernel's end; the CTAs wait for it before reading any input
+  a.wait_prior = 1;
+  {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tmK, tmV, tmQ, a) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return PA_ERR_CUDA;
+    }
+  }
   if (check_launch() != PA_OK) return PA_ERR_CUDA;
   int launches = 1;
   if (grid > 1 || SP) {
@@ -1870,6 +1901,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_new, const void* v
   a.nslots = 0;
   a.qscale = scale * 1.4426950408889634f;
   a.wait_limit = pa::take_wait_limit(pa::kTestDecode, &a.test_withhold);
+  a.wait_prior = 0;  // set by the launch that makes the grid a programmatic dependent
   a.group_starts = a.prefix_lens = nullptr;
   a.vpart_o = a.vpart_ml = nullptr;
   a.num_groups = a.mc = a.vcap = a.max_prefix = 0;

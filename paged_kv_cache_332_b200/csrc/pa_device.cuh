@@ -124,6 +124,11 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, int
       : "memory");
 }
 
+// Prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // L2 cache policies for bulk copies: data read once (evict first, so that it displaces
 // itself rather than other lines), and data other CTAs read again soon (normal priority).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
