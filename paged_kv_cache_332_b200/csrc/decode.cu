@@ -26,15 +26,13 @@
 //    programmatic dependent of this launch).
 //    An explicit partition size caps the share, so no segment is longer.
 //  * One consumer warp per kv-head of the group handles all G q-heads of that kv-head,
-//    so no two warps share an output.  q.k: 8 lanes split a token's 128 dims (16 each,
-//    two 16-byte shared-memory reads), packed f32x2 FMAs, then a warp-shuffle halving
-//    exchange that sums all G heads at once.  Online softmax (running max m, sum l) in
-//    the log2 domain (q pre-scaled by scale*log2 e: one ex2 per logit); p.V with lanes
-//    over head_dim.
-//  * G = 8 (LLaMA-70B-style GQA) is the exception: its two contractions cost 4 FMAs per
-//    byte of KV, more than the FP32 pipe sustains at HBM rate, so q.k and p.V of a tile
-//    run as mma.sync m16n8k16 tensor-core fragments (fp32 accumulate); the online
-//    softmax, masking and the split-K bookkeeping are the same.
+//    so no two warps share an output.  q.k and p.V of a tile run as mma.sync m16n8k16
+//    tensor-core fragments (fp32 accumulate; q-heads past G are zero columns): S^T = K Q^T
+//    (M = 16 tokens, N = 8 heads), online softmax (running max m, sum l) in the log2
+//    domain on the accumulator fragment (q pre-scaled by scale*log2 e: one ex2 per logit),
+//    O^T += V^T P^T.  At G = 8 the two contractions cost 4 FMAs per byte of KV, more than
+//    the FP32 pipe sustains at HBM rate; warp-shuffle dot products on CUDA cores, kept for
+//    G <= 4 at first, were also measured slower there (mixed batch 88.1 -> 84.0 us).
 //  * A staging warp cuts the CTA's share into units of at most 128 tiles and, up to two
 //    units ahead, copies their block-table entries into shared memory (one coalesced
 //    read per 32 entries) and starts the TMA copy of their q rows.  A producer thread
@@ -141,17 +139,12 @@ struct DecodeCfg {
   static constexpr int G = G_;
   static constexpr int HB = HB_;                  // kv-heads per group = consumer warps
   static constexpr bool F8 = F8_;                 // e4m3 cache (else fp16/bf16)
-  // tensor-core consumers: G = 8, an FP8 cache, and beside the chunk consumer of shared
-  // prefixes (which leaves no registers for the CUDA-core path's q in registers)
-  static constexpr bool MMA = F8 || G == 8 || SP_;
   static constexpr int KROW = kD * (F8 ? 1 : 2);  // one token of one kv-head in the cache
-  static constexpr int GW = G;                    // q-heads per consumer warp
   static constexpr int WARP_PROD = 0;
   static constexpr int WARP_STAGE = 1;
   static constexpr int WARP_FILL = 2;             // zero-fills empty sequences
   static constexpr int WARP_C0 = 4;               // first consumer warp
   static constexpr int THREADS = 128 + HB * 32;
-  static constexpr int DUPMASK = GW == 4 ? 1 : (GW == 2 ? 3 : 7);  // CUDA-core path (G <= 4)
   static constexpr int TILE_BYTES = kTileTok * HB * KROW;       // K (or V) of a tile
   static constexpr int SLOT_BYTES = 2 * TILE_BYTES;
   // A K (V) tile is copied as 128-byte-wide column slabs of its rows (two slabs of 64 dims
@@ -172,12 +165,8 @@ struct DecodeCfg {
   static constexpr int OFF_ABORT = OFF_UNIT + kQSlots * 64;
   static constexpr int OFF_TBL = ((OFF_ABORT + 16 + 127) / 128) * 128;
   static constexpr int OFF_Q = OFF_TBL + kQSlots * kMaxTilesPerUnit * 4;
-  // p pairs and alpha per warp (CUDA-core path only; the G = 8 path keeps them in
-  // registers, which leaves room for a third 64 KB ring slot)
-  static constexpr int OFF_P = OFF_Q + kQSlots * QBYTES;
-  static constexpr int OFF_A = OFF_P + (MMA ? 0 : HB * kTileTok * GW * 8);
-  static constexpr int OFF_SEQ = ((OFF_A + (MMA ? 0 : HB * GW * 4) + 15) / 16) * 16;  // 3B+1 ints
-  static_assert(OFF_Q % 128 == 0 && OFF_P % 16 == 0, "alignment");
+  static constexpr int OFF_SEQ = OFF_Q + kQSlots * QBYTES;  // the schedule arrays
+  static_assert(OFF_Q % 128 == 0 && OFF_SEQ % 16 == 0, "alignment");
 };
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -231,60 +220,6 @@ __device__ __forceinline__ void drain_copy(uint64_t* bar, uint32_t parity, int* 
                                            long long limit) {
   (void)mbar_wait(bar, parity, err, limit);
 }
-
-// Sum per-lane partial dot products over each 8-lane token group for GW heads at
-// once (halving exchange).  Returns the sum for head hh(lane):
-//   GW=4: hh = 2*bit2 + bit1;  GW=2: hh = bit2;
-//   GW=1: hh = 0.
-template <int GW>
-__device__ __forceinline__ float reduce_heads(const float (&d)[GW], int lane);
-
-template <>
-__device__ __forceinline__ float reduce_heads<4>(const float (&d)[4], int lane) {
-  const bool b2 = lane & 4;
-  float k0 = b2 ? d[2] : d[0], k1 = b2 ? d[3] : d[1];
-  const float s0 = b2 ? d[0] : d[2], s1 = b2 ? d[1] : d[3];
-  k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
-  k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
-  const bool b1 = lane & 2;
-  float k = b1 ? k1 : k0;
-  const float s = b1 ? k0 : k1;
-  k += __shfl_xor_sync(0xffffffffu, s, 2);
-  k += __shfl_xor_sync(0xffffffffu, k, 1);
-  return k;
-}
-
-template <>
-__device__ __forceinline__ float reduce_heads<2>(const float (&d)[2], int lane) {
-  const bool b2 = lane & 4;
-  float k = b2 ? d[1] : d[0];
-  const float s = b2 ? d[0] : d[1];
-  k += __shfl_xor_sync(0xffffffffu, s, 4);
-  k += __shfl_xor_sync(0xffffffffu, k, 2);
-  k += __shfl_xor_sync(0xffffffffu, k, 1);
-  return k;
-}
-
-template <>
-__device__ __forceinline__ float reduce_heads<1>(const float (&d)[1], int lane) {
-  float k = d[0];
-  k += __shfl_xor_sync(0xffffffffu, k, 4);
-  k += __shfl_xor_sync(0xffffffffu, k, 2);
-  k += __shfl_xor_sync(0xffffffffu, k, 1);
-  return k;
-}
-
-template <int GW>
-__device__ __forceinline__ int head_of_lane(int lane) {
-  return GW == 4 ? (((lane >> 2) & 1) * 2 + ((lane >> 1) & 1)) : (GW == 2 ? ((lane >> 2) & 1) : 0);
-}
-
-// A lane that holds head jj's value after reduce_heads (with tp = 0).
-template <int GW>
-__device__ __forceinline__ int lane_of_head(int jj) {
-  return GW == 4 ? (((jj >> 1) << 2) | ((jj & 1) << 1)) : (GW == 2 ? jj * 4 : 0);
-}
-
 
 // mma.sync m16n8k16 with fp32 accumulate, A row-major / B column-major fragments, and
 // the packing of two fp32 values into one register of the element type.
@@ -516,7 +451,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
                                             const CUtensorMap& tmQ, const DecodeArgs& a,
                                             uint8_t* smem, const int cta, const int ncta) {
   using C = DecodeCfg<G, HB, F8, SP>;
-  constexpr int GW = C::GW;
   constexpr int HBG = HB * G;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_FULL);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + C::OFF_EMPTY);
@@ -529,8 +463,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
   int* tbl = reinterpret_cast<int*>(smem + C::OFF_TBL);
   uint8_t* qbuf = smem + C::OFF_Q;
-  float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
-  float* abuf = reinterpret_cast<float*>(smem + C::OFF_A);
   const int B = a.num_seqs;
   const int VC = SP ? a.vcap : 0;  // room for chunk sequences after the batch
   int* sstart = reinterpret_cast<int*>(smem + C::OFF_SEQ);  // [B+VC+1] first tile of each sequence
@@ -1108,7 +1040,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
     (void)nseg;
     return true;
   };
-  if constexpr (C::MMA) {
+  {
     // Tensor-core consumer (G = 8, and every G on an FP8 cache).  Per 16-token tile: S^T = K Q^T (M = 16 tokens, N = 8
     // q-heads, K = 128 dims: 8 MMAs) and O^T += V^T P^T (M = 128 dims in 8 tiles, N = 8
     // q-heads, K = 16 tokens: 8 MMAs).  Lane (g, tq) = (lane/4, lane%4) holds the logits
@@ -1309,172 +1241,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
       (void)slot0;
       (void)nseg;
     }
-    return;
-  } else {
-    const int sub = lane & 7;
-    const int tp = lane >> 3;
-    const int hh = head_of_lane<GW>(lane);
-    const bool writer = (lane & C::DUPMASK) == 0;
-    float2* pw = pbuf + w * kTileTok * GW;
-    int cnt = 0;
-    // one segment per iteration, as in the tensor-core consumer
-    for (int k = 0;;) {
-      int qs = k % kQSlots;
-      wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
-      const volatile int* u = unit + qs * kUnitInts;
-      const int s = u[0];
-      if (s < 0 || warp_flag(abort_flag)) break;
-      if constexpr (SP) {
-        if (u[4] & kVirtual) {
-          if (!chunk_segment(k, cnt, qs, u)) break;
-          continue;
-        }
-      }
-      const int hp = u[1], pslot = u[5], orow = u[7], slot0 = u[8], nseg = u[9];
-      int t0 = u[2], t1 = u[3], flags = u[4];
-      float2 q2[GW][8];  // q of this warp's G heads (dims of lane `sub`), log2-domain scaled
-      float m = -INFINITY, l = 0.f;
-      float2 acc[GW][2];
-      {
-        // dims [8*sub, 8*sub+8) and [64+8*sub, 64+8*sub+8) as (even, odd) pairs
-        const uint8_t* qb = qbuf + qs * C::QBYTES + w * G * kRowBytes;
-#pragma unroll
-        for (int j = 0; j < GW; ++j) {
-          const uint4 w0 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + sub * 16);
-          const uint4 w1 = *reinterpret_cast<const uint4*>(qb + j * kRowBytes + 128 + sub * 16);
-          const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 f = Elem<T>::unpack2(wd[i]);
-            q2[j][i] = make_float2(f.x * a.qscale, f.y * a.qscale);
-          }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < GW; ++j) acc[j][0] = acc[j][1] = make_float2(0.f, 0.f);
-      const int L = slen[s];
-      bool stop = false;
-      for (;;) {  // the segment's units
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&qempty[qs]);
-        for (int t = t0; t < t1; ++t, ++cnt) {
-          const int slot = cnt % nslots;
-          wait_or_abort(&full[slot], (cnt / nslots) & 1, abort_flag, a.err, a.wait_limit);
-          const int nvalid = min(kTileTok, L - t * kTileTok);
-          // tile layout: two slabs (dims 0..63, 64..127) of [HB kv-heads][16 tokens][128 B]
-          const uint8_t* Ks = ring + slot * C::SLOT_BYTES;
-          const uint8_t* Vs = Ks + C::TILE_BYTES;
-
-          // ---- logits of the tile's 16 tokens (4 passes of 4 tokens)
-          float x[4];
-#pragma unroll
-          for (int ps = 0; ps < 4; ++ps) {
-            const int rr = ps * 4 + tp;
-            const uint8_t* kr = Ks + swz(w, rr, sub);  // dims 8sub.. of slab 0, then of slab 1
-            const uint4 w0 = *reinterpret_cast<const uint4*>(kr);
-            const uint4 w1 = *reinterpret_cast<const uint4*>(kr + C::SLAB_BYTES);
-            const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            float2 kf[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) kf[i] = Elem<T>::unpack2(wd[i]);
-            float d[GW];
-#pragma unroll
-            for (int jj = 0; jj < GW; ++jj) {
-              float2 e = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) e = __ffma2_rn(q2[jj][i], kf[i], e);
-              d[jj] = e.x + e.y;
-            }
-            const float xv = reduce_heads<GW>(d, lane);
-            x[ps] = rr < nvalid ? xv : -INFINITY;
-          }
-          // ---- online softmax over the tile, per head hh
-          float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float m_new = fmaxf(m, mx);
-          const float alpha = fast_exp2(m - m_new);  // m = -inf -> 0
-          m = m_new;
-          float psum = 0.f;
-#pragma unroll
-          for (int ps = 0; ps < 4; ++ps) {
-            const float pv = fast_exp2(x[ps] - m_new);  // masked -> 0
-            psum += pv;
-            if (writer) pw[(ps * 4 + tp) * GW + hh] = make_float2(pv, pv);
-          }
-          l = l * alpha + psum;
-          if (writer && tp == 0) abuf[w * GW + hh] = alpha;
-          __syncwarp();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-            for (int jj = 0; jj < GW; ++jj) {
-              const float al = abuf[w * GW + jj];
-              const float2 a2 = make_float2(al, al);
-              acc[jj][0] = __fmul2_rn(acc[jj][0], a2);
-              acc[jj][1] = __fmul2_rn(acc[jj][1], a2);
-            }
-          }
-          // ---- p.V: lane owns dims [4*lane, 4*lane+4): slab lane/16, chunk (lane%16)/2
-          const uint8_t* Vl = Vs + (lane >> 4) * C::SLAB_BYTES + (lane & 1) * 8;
-          auto pv_row = [&](int tt) {
-            const uint2 vw = *reinterpret_cast<const uint2*>(Vl + swz(w, tt, (lane & 15) >> 1));
-            const float2 v01 = Elem<T>::unpack2(vw.x), v23 = Elem<T>::unpack2(vw.y);
-#pragma unroll
-            for (int jj = 0; jj < GW; ++jj) {
-              const float2 pp = pw[tt * GW + jj];
-              acc[jj][0] = __ffma2_rn(pp, v01, acc[jj][0]);
-              acc[jj][1] = __ffma2_rn(pp, v23, acc[jj][1]);
-            }
-          };
-          if (nvalid == kTileTok) {
-#pragma unroll
-            for (int tt = 0; tt < kTileTok; ++tt) pv_row(tt);
-          } else {
-            for (int tt = 0; tt < nvalid; ++tt) pv_row(tt);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[slot]);
-        }
-        ++k;
-        if (flags & kLast) break;
-        qs = k % kQSlots;
-        wait_or_abort(&qfull[qs], (k / kQSlots) & 1, abort_flag, a.err, a.wait_limit);
-        u = unit + qs * kUnitInts;
-        if (u[0] < 0 || warp_flag(abort_flag)) {
-          stop = true;
-          break;
-        }
-        t0 = u[2];
-        t1 = u[3];
-        flags = u[4];
-      }
-      if (stop) break;
-
-      // ---- end of segment: l summed over the 4 token groups; m and l of every head
-      float lt = l + __shfl_xor_sync(0xffffffffu, l, 8);
-      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
-#pragma unroll
-      for (int jj = 0; jj < GW; ++jj) {
-        const float lj = __shfl_sync(0xffffffffu, lt, lane_of_head<GW>(jj));
-        const float mj = __shfl_sync(0xffffffffu, m, lane_of_head<GW>(jj));
-        const float inv = lj > 0.f ? 1.f / lj : 0.f;
-        const int j = w * G + jj;  // q-head within the group
-        const float o0 = acc[jj][0].x * inv, o1 = acc[jj][0].y * inv;
-        const float o2 = acc[jj][1].x * inv, o3 = acc[jj][1].y * inv;
-        if (flags & kDirect) {
-          T* ob = static_cast<T*>(a.out) + ((long long)orow * a.num_q_heads + hp * HBG + j) * kD +
-                  lane * 4;
-          *reinterpret_cast<uint2*>(ob) = make_uint2(Elem<T>::pack2(o0, o1), Elem<T>::pack2(o2, o3));
-        } else {
-          const long long row = (long long)pslot * HBG + j;
-          *reinterpret_cast<float4*>(a.part_o + row * kD + lane * 4) = make_float4(o0, o1, o2, o3);
-          if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + row * 2) = make_float2(mj, lj);
-        }
-      }
-      (void)slot0;
-      (void)nseg;
-    }
-  }  // G < 8
+  }
 }
 
 template <typename T, int G, int HB, bool F8, bool SP>
