@@ -379,8 +379,8 @@ __device__ __forceinline__ int cta_of(int pos, int T, int grid) {
 // head_dim.  o = sum_i w_i o_i / sum_i w_i with w_i = l_i * 2^(m_i - M), M the largest m_i,
 // over the sequence's own segments (consecutive slots of its head group's record) and, with
 // a shared prefix, the segments of the chunk that holds it (rows of its chunk slots).  One
-// pass with a running maximum, up to eight rows per round with all their loads in flight.
-// Launched as a programmatic dependent of the decode kernel.
+// pass with a running maximum, in rounds of 4, 8 or 16 rows by the piece count, all their
+// loads in flight.  Launched as a programmatic dependent of the decode kernel.
 template <typename T, int G, bool SP>
 __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) {
   griddep_wait();  // the decode grid has finished and its writes are visible
@@ -404,38 +404,48 @@ __global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, int HB) 
   if (total == 0) return;  // written by the decode kernel (or nothing to write)
   float M = -INFINITY, den = 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  constexpr int R = 8;  // pieces per round, all their loads in flight (16 measured slower)
-  for (int i0 = 0; i0 < total; i0 += R) {
-    float2 mlv[R];
-    float4 ov[R];
-    float Mr = -INFINITY;
+  // Rounds of R pieces, R = 4, 8 or 16 by the piece count (uniform over the warp).  A
+  // round's loads are unconditional (past the last piece: its row again, ignored after) so
+  // that they are all in flight before the first is used; loads behind a branch each
+  // waited for the previous piece's use (measured: LLaMA-70B 57.1 -> 55.1 us per call).
+  auto rounds = [&](auto rc) {
+    constexpr int R = decltype(rc)::value;
+    for (int i0 = 0; i0 < total; i0 += R) {
+      float2 mlv[R];
+      float4 ov[R];
 #pragma unroll
-    for (int u = 0; u < R; ++u) {
-      const int i = i0 + u;
-      if (i < total) {
+      for (int u = 0; u < R; ++u) {
+        const int i = min(i0 + u, total - 1);
         const bool own = i < no;
         const long long row = own ? (long long)(so0 + i) * hbg + j
                                   : (long long)(sv0 + i - no) * (HB * kChunkRows) + vrow;
-        mlv[u] = *reinterpret_cast<const float2*>((own ? a.part_ml : a.vpart_ml) + row * 2);
-        ov[u] = *reinterpret_cast<const float4*>((own ? a.part_o : a.vpart_o) + row * kD + lane * 4);
-        Mr = fmaxf(Mr, mlv[u].x);
+        mlv[u] = __ldg(reinterpret_cast<const float2*>((own ? a.part_ml : a.vpart_ml) + row * 2));
+        ov[u] = __ldg(reinterpret_cast<const float4*>((own ? a.part_o : a.vpart_o) + row * kD) +
+                      lane);
       }
-    }
-    const float Mn = fmaxf(M, Mr);
-    if (Mn == -INFINITY) continue;  // only empty segments so far
-    const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
-    den *= sc;
-    num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+      float Mr = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < R; ++u) {
-      if (i0 + u < total) {
-        const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
-        den += f;
-        num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
+      for (int u = 0; u < R; ++u)
+        if (i0 + u < total) Mr = fmaxf(Mr, mlv[u].x);
+      const float Mn = fmaxf(M, Mr);
+      if (Mn == -INFINITY) continue;  // only empty segments so far
+      const float sc = fast_exp2(M - Mn);  // M = -inf -> 0
+      den *= sc;
+      num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+#pragma unroll
+      for (int u = 0; u < R; ++u) {
+        if (i0 + u < total) {
+          const float f = mlv[u].x == -INFINITY ? 0.f : fast_exp2(mlv[u].x - Mn) * mlv[u].y;
+          den += f;
+          num.x += f * ov[u].x; num.y += f * ov[u].y; num.z += f * ov[u].z; num.w += f * ov[u].w;
+        }
       }
+      M = Mn;
     }
-    M = Mn;
-  }
+  };
+  if (total <= 4) rounds(std::integral_constant<int, 4>{});
+  else if (total <= 8) rounds(std::integral_constant<int, 8>{});
+  else rounds(std::integral_constant<int, 16>{});
   const float inv = den > 0.f ? 1.f / den : 0.f;
   const long long orow = a.qsl ? __ldg(a.qsl + s) : s;
   T* ob = static_cast<T*>(a.out) + (orow * a.num_q_heads + qh) * kD + lane * 4;
