@@ -49,7 +49,6 @@
 //    q and out rows come from query_start_loc, and CTA 0 lists the other sequences for
 //    the prefill kernel that follows.
 // Every wait is bounded; bad table entries or lengths never fault (skipped, flagged).
-#include <cuda_fp8.h>
 
 #include <algorithm>
 #include <climits>
@@ -256,12 +255,15 @@ struct Mma<__half> {
   }
 };
 
-// Two e4m3 codes (low 16 bits of x; the lower code first) -> their f16 values as one
-// f16x2 register.  Exact: every e4m3 value is an f16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
-  const __half2_raw h =
-      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(x & 0xFFFFu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four e4m3 codes (byte 0 of x first) -> their f16 values as two f16x2 registers: lo holds
+// codes 0 and 1, hi codes 2 and 3, each with the lower byte's value in its low half.  One
+// conversion per pair, with the 16-bit halves of x as its operands (no shifts or masks).
+// Exact: every e4m3 value is an f16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // Transpose of an 8x8 matrix of 16-bit elements held as one fragment register per lane
@@ -302,26 +304,44 @@ __device__ __forceinline__ void pv_tile(float (&oacc)[NT][8][4], const uint8_t* 
                           : make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  if constexpr (F8) {
+    // the codes of tokens 2p and 2p+1 paired byte by byte before the conversion, so that
+    // each converted f16x2 is already the fragment register (token 2p in its low half)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t fr[4][4];  // [word r][a0..a3]
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const uint4& t0 = v8[2 * p];
+        const uint4& t1 = v8[2 * p + 1];
+        const uint32_t x0 = h ? t0.z : t0.x, y0 = h ? t1.z : t1.x;  // codes 0-3 of the chunk half
+        const uint32_t x1 = h ? t0.w : t0.y, y1 = h ? t1.w : t1.y;  // codes 4-7
+        e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x5140), fr[0][2 * p], fr[0][2 * p + 1]);
+        e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x7362), fr[1][2 * p], fr[1][2 * p + 1]);
+        e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x5140), fr[2][2 * p], fr[2][2 * p + 1]);
+        e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x7362), fr[3][2 * p], fr[3][2 * p + 1]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          Mma<MT>::run(oacc[nt][4 * h + r], fr[r][0], fr[r][1], fr[r][2], fr[r][3], pb[nt][0],
+                       pb[nt][1]);
+    }
+    return;
+  }
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t vw[4][4];  // [token i][word r]
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      if constexpr (F8) {
-        const uint32_t c0 = h ? v8[i].z : v8[i].x, c1 = h ? v8[i].w : v8[i].y;
-        vw[i][0] = e4m3x2_to_f16x2(c0);
-        vw[i][1] = e4m3x2_to_f16x2(c0 >> 16);
-        vw[i][2] = e4m3x2_to_f16x2(c1);
-        vw[i][3] = e4m3x2_to_f16x2(c1 >> 16);
-      } else {
-        const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-        const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
-                                    : make_uint4(0u, 0u, 0u, 0u);
-        vw[i][0] = c.x;
-        vw[i][1] = c.y;
-        vw[i][2] = c.z;
-        vw[i][3] = c.w;
-      }
+      const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+      const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+      vw[i][0] = c.x;
+      vw[i][1] = c.y;
+      vw[i][2] = c.z;
+      vw[i][3] = c.w;
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -1149,10 +1169,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
               const uint4 kb = *reinterpret_cast<const uint4*>(kc + 1024);  // token g+8
               const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                Mma<__half>::run(sc, e4m3x2_to_f16x2(wa[i]), e4m3x2_to_f16x2(wb[i]),
-                                 e4m3x2_to_f16x2(wa[i] >> 16), e4m3x2_to_f16x2(wb[i] >> 16),
-                                 qf[4 * c + i][0], qf[4 * c + i][1]);
+              for (int i = 0; i < 4; ++i) {
+                uint32_t alo, ahi, blo, bhi;
+                e4m3x4_to_f16x2x2(wa[i], alo, ahi);
+                e4m3x4_to_f16x2x2(wb[i], blo, bhi);
+                Mma<__half>::run(sc, alo, blo, ahi, bhi, qf[4 * c + i][0], qf[4 * c + i][1]);
+              }
             }
           } else {
 #pragma unroll
