@@ -289,69 +289,84 @@ __device__ __forceinline__ int kchunk(int tq, int j) { return 8 * (j >> 1) + 2 *
 // (tokens 2tq, 2tq+1) and pb1 (2tq+8, 2tq+9) expect.  Under the swizzle the reads of a
 // phase (tokens 2tq+b of chunks g, g^1) fall in eight different bank groups.  NT column
 // tiles of 8 share every V fragment; SLAB is the tile's slab size in bytes.
+// e4m3 tiles: pv_tile's V^T fragments and its products as two steps, so that a consumer can
+// issue a tile's V reads and conversions before the tile's softmax.  Fragment [h][r][0..3]
+// is the A operand of m-tile 4h+r: the codes of tokens 2p and 2p+1 paired byte by byte
+// before the conversion, so that each converted f16x2 is already a fragment register
+// (token 2p in its low half).
+__device__ __forceinline__ void pv_frags_f8(const uint8_t* Vs, int w, int g, int tq, int nvalid,
+                                            uint32_t (&fr)[2][4][4]) {
+  // token 2tq+b+8c sits 8 rows (1 KB) after token 2tq+b, with the same swizzle
+  const int vofs0 = swz(w, 2 * tq, g), vofs1 = swz(w, 2 * tq + 1, g);
+  uint4 v8[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+    v8[i] = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + ((i & 1) ? vofs1 : vofs0) +
+                                                          (i >> 1) * 1024)
+                        : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const uint4& t0 = v8[2 * p];
+      const uint4& t1 = v8[2 * p + 1];
+      const uint32_t x0 = h ? t0.z : t0.x, y0 = h ? t1.z : t1.x;  // codes 0-3 of the chunk half
+      const uint32_t x1 = h ? t0.w : t0.y, y1 = h ? t1.w : t1.y;  // codes 4-7
+      e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x5140), fr[h][0][2 * p], fr[h][0][2 * p + 1]);
+      e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x7362), fr[h][1][2 * p], fr[h][1][2 * p + 1]);
+      e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x5140), fr[h][2][2 * p], fr[h][2][2 * p + 1]);
+      e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x7362), fr[h][3][2 * p], fr[h][3][2 * p + 1]);
+    }
+}
+template <int NT>
+__device__ __forceinline__ void pv_mma_f8(float (&oacc)[NT][8][4], const uint32_t (&fr)[2][4][4],
+                                          const uint32_t (&pb)[NT][2]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        Mma<__half>::run(oacc[nt][4 * h + r], fr[h][r][0], fr[h][r][1], fr[h][r][2], fr[h][r][3],
+                         pb[nt][0], pb[nt][1]);
+}
+
 template <bool F8, typename MT, int NT, int SLAB>
 __device__ __forceinline__ void pv_tile(float (&oacc)[NT][8][4], const uint8_t* Vs, int w, int g,
                                         int tq, int nvalid, const uint32_t (&pb)[NT][2]) {
   // token 2tq+b+8c sits 8 rows (1 KB) after token 2tq+b, with the same swizzle
   const int vofs0 = swz(w, 2 * tq, g), vofs1 = swz(w, 2 * tq + 1, g);
   auto vofs = [&](int i) { return ((i & 1) ? vofs1 : vofs0) + (i >> 1) * 1024; };
-  uint4 v8[4];
   if constexpr (F8) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-      v8[i] = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + vofs(i))
-                          : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  if constexpr (F8) {
-    // the codes of tokens 2p and 2p+1 paired byte by byte before the conversion, so that
-    // each converted f16x2 is already the fragment register (token 2p in its low half)
+    uint32_t fr[2][4][4];
+    pv_frags_f8(Vs, w, g, tq, nvalid, fr);
+    pv_mma_f8<NT>(oacc, fr, pb);
+  } else {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t fr[4][4];  // [word r][a0..a3]
+      uint32_t vw[4][4];  // [token i][word r]
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const uint4& t0 = v8[2 * p];
-        const uint4& t1 = v8[2 * p + 1];
-        const uint32_t x0 = h ? t0.z : t0.x, y0 = h ? t1.z : t1.x;  // codes 0-3 of the chunk half
-        const uint32_t x1 = h ? t0.w : t0.y, y1 = h ? t1.w : t1.y;  // codes 4-7
-        e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x5140), fr[0][2 * p], fr[0][2 * p + 1]);
-        e4m3x4_to_f16x2x2(__byte_perm(x0, y0, 0x7362), fr[1][2 * p], fr[1][2 * p + 1]);
-        e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x5140), fr[2][2 * p], fr[2][2 * p + 1]);
-        e4m3x4_to_f16x2x2(__byte_perm(x1, y1, 0x7362), fr[3][2 * p], fr[3][2 * p + 1]);
+      for (int i = 0; i < 4; ++i) {
+        const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+        const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        vw[i][0] = c.x;
+        vw[i][1] = c.y;
+        vw[i][2] = c.z;
+        vw[i][3] = c.w;
       }
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], 0x5410);
+        const uint32_t a1 = __byte_perm(vw[0][r], vw[1][r], 0x7632);
+        const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], 0x5410);
+        const uint32_t a3 = __byte_perm(vw[2][r], vw[3][r], 0x7632);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
-          Mma<MT>::run(oacc[nt][4 * h + r], fr[r][0], fr[r][1], fr[r][2], fr[r][3], pb[nt][0],
-                       pb[nt][1]);
-    }
-    return;
-  }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t vw[4][4];  // [token i][word r]
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-      const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
-                                  : make_uint4(0u, 0u, 0u, 0u);
-      vw[i][0] = c.x;
-      vw[i][1] = c.y;
-      vw[i][2] = c.z;
-      vw[i][3] = c.w;
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], 0x5410);
-      const uint32_t a1 = __byte_perm(vw[0][r], vw[1][r], 0x7632);
-      const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], 0x5410);
-      const uint32_t a3 = __byte_perm(vw[2][r], vw[3][r], 0x7632);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        Mma<MT>::run(oacc[nt][4 * h + r], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+          Mma<MT>::run(oacc[nt][4 * h + r], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
     }
   }
 }
@@ -1161,6 +1176,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
 
           // ---- S^T = K Q^T: rows tokens g, g+8; columns heads 2tq, 2tq+1
           float sc[4] = {0.f, 0.f, 0.f, 0.f};
+          // e4m3: the tile's V^T fragments first, so that their reads and conversions
+          // overlap the S products and the softmax
+          uint32_t vfr[2][4][4];
+          if constexpr (F8) pv_frags_f8(Vs, w, g, tq, nvalid, vfr);
           if constexpr (F8) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -1224,7 +1243,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           // ---- O^T += V^T P^T (rows past the sequence end are zeroed: p is 0 there, but the
           // block's unused rows may hold anything)
           const uint32_t pb[1][2] = {{pb0, pb1}};
-          pv_tile<F8, MT, 1, C::SLAB_BYTES>(oaccs, Vs, w, g, tq, nvalid, pb);
+          if constexpr (F8)
+            pv_mma_f8<1>(oaccs, vfr, pb);
+          else
+            pv_tile<F8, MT, 1, C::SLAB_BYTES>(oaccs, Vs, w, g, tq, nvalid, pb);
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);
         }
