@@ -1181,6 +1181,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           uint32_t vfr[2][4][4];
           if constexpr (F8) pv_frags_f8(Vs, w, g, tq, nvalid, vfr);
           if constexpr (F8) {
+            float sc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const uint8_t* kc = Ks + (c ? kofs1 : kofs0);
@@ -1192,9 +1193,13 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
                 uint32_t alo, ahi, blo, bhi;
                 e4m3x4_to_f16x2x2(wa[i], alo, ahi);
                 e4m3x4_to_f16x2x2(wb[i], blo, bhi);
-                Mma<__half>::run(sc, alo, blo, ahi, bhi, qf[4 * c + i][0], qf[4 * c + i][1]);
+                // two accumulators: two chains of four dependent products, not one of eight
+                Mma<__half>::run((i & 1) ? sc2 : sc, alo, blo, ahi, bhi, qf[4 * c + i][0],
+                                 qf[4 * c + i][1]);
               }
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[e] += sc2[e];
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
