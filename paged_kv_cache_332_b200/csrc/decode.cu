@@ -281,16 +281,50 @@ __device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
 // the slab swizzle the eight 16-byte reads of a phase hit eight different bank groups.
 __device__ __forceinline__ int kchunk(int tq, int j) { return 8 * (j >> 1) + 2 * tq + (j & 1); }
 
-// O^T += V^T P^T for one 16-token tile of kv-head w (tensor-core consumers).  Lane (g, tq)
-// reads one 16-byte chunk per token for tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (zero past nvalid):
-// chunk g of each slab (16-bit: dims [8g, 8g+8) and [64+8g, 64+8g+8)) or, for e4m3, the 16
-// codes [16g, 16g+16).  Word r of a lane's chunk h makes m-tile 4h+r, its row g the chunk's
-// dim 2r and its row g+8 dim 2r+1, with tokens paired along k as the P^T fragments pb0
-// (tokens 2tq, 2tq+1) and pb1 (2tq+8, 2tq+9) expect.  Under the swizzle the reads of a
-// phase (tokens 2tq+b of chunks g, g^1) fall in eight different bank groups.  NT column
-// tiles of 8 share every V fragment; SLAB is the tile's slab size in bytes.
-// e4m3 tiles: pv_tile's V^T fragments and its products as two steps, so that a consumer can
-// issue a tile's V reads and conversions before the tile's softmax.  Fragment [h][r][0..3]
+// O^T += V^T P^T for one 16-token tile of kv-head w (tensor-core consumers, 16-bit cache).
+// Lane (g, tq) reads one 16-byte chunk per token for tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (zero
+// past nvalid): chunk g of each slab, dims [8g, 8g+8) and [64+8g, 64+8g+8).  Word r of a
+// lane's chunk h makes m-tile 4h+r, its row g the chunk's dim 2r and its row g+8 dim 2r+1,
+// with tokens paired along k as the P^T fragments pb0 (tokens 2tq, 2tq+1) and pb1 (2tq+8,
+// 2tq+9) expect.  Under the swizzle the reads of a phase (tokens 2tq+b of chunks g, g^1) fall
+// in eight different bank groups.  NT column tiles of 8 share every V fragment; SLAB is the
+// tile's slab size in bytes.
+template <typename MT, int NT, int SLAB>
+__device__ __forceinline__ void pv_tile(float (&oacc)[NT][8][4], const uint8_t* Vs, int w, int g,
+                                        int tq, int nvalid, const uint32_t (&pb)[NT][2]) {
+  // token 2tq+b+8c sits 8 rows (1 KB) after token 2tq+b, with the same swizzle
+  const int vofs0 = swz(w, 2 * tq, g), vofs1 = swz(w, 2 * tq + 1, g);
+  auto vofs = [&](int i) { return ((i & 1) ? vofs1 : vofs0) + (i >> 1) * 1024; };
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t vw[4][4];  // [token i][word r]
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
+      const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+      vw[i][0] = c.x;
+      vw[i][1] = c.y;
+      vw[i][2] = c.z;
+      vw[i][3] = c.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], 0x5410);
+      const uint32_t a1 = __byte_perm(vw[0][r], vw[1][r], 0x7632);
+      const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], 0x5410);
+      const uint32_t a3 = __byte_perm(vw[2][r], vw[3][r], 0x7632);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        Mma<MT>::run(oacc[nt][4 * h + r], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+    }
+  }
+}
+
+// The same product over an e4m3 tile, as two steps, so that a consumer can issue a tile's V
+// reads and conversions before the tile's softmax.  Lane (g, tq) reads the 16 codes
+// [16g, 16g+16) of tokens 2tq, 2tq+1, 2tq+8, 2tq+9 (one 16-byte chunk each, zero past
+// nvalid).  Fragment [h][r][0..3]
 // is the A operand of m-tile 4h+r: the codes of tokens 2p and 2p+1 paired byte by byte
 // before the conversion, so that each converted f16x2 is already a fragment register
 // (token 2p in its low half).
@@ -331,44 +365,6 @@ __device__ __forceinline__ void pv_mma_f8(float (&oacc)[NT][8][4], const uint32_
       for (int nt = 0; nt < NT; ++nt)
         Mma<__half>::run(oacc[nt][4 * h + r], fr[h][r][0], fr[h][r][1], fr[h][r][2], fr[h][r][3],
                          pb[nt][0], pb[nt][1]);
-}
-
-template <bool F8, typename MT, int NT, int SLAB>
-__device__ __forceinline__ void pv_tile(float (&oacc)[NT][8][4], const uint8_t* Vs, int w, int g,
-                                        int tq, int nvalid, const uint32_t (&pb)[NT][2]) {
-  // token 2tq+b+8c sits 8 rows (1 KB) after token 2tq+b, with the same swizzle
-  const int vofs0 = swz(w, 2 * tq, g), vofs1 = swz(w, 2 * tq + 1, g);
-  auto vofs = [&](int i) { return ((i & 1) ? vofs1 : vofs0) + (i >> 1) * 1024; };
-  if constexpr (F8) {
-    uint32_t fr[2][4][4];
-    pv_frags_f8(Vs, w, g, tq, nvalid, fr);
-    pv_mma_f8<NT>(oacc, fr, pb);
-  } else {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t vw[4][4];  // [token i][word r]
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tk = 2 * tq + (i & 1) + (i >> 1) * 8;
-        const uint4 c = tk < nvalid ? *reinterpret_cast<const uint4*>(Vs + h * SLAB + vofs(i))
-                                    : make_uint4(0u, 0u, 0u, 0u);
-        vw[i][0] = c.x;
-        vw[i][1] = c.y;
-        vw[i][2] = c.z;
-        vw[i][3] = c.w;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint32_t a0 = __byte_perm(vw[0][r], vw[1][r], 0x5410);
-        const uint32_t a1 = __byte_perm(vw[0][r], vw[1][r], 0x7632);
-        const uint32_t a2 = __byte_perm(vw[2][r], vw[3][r], 0x5410);
-        const uint32_t a3 = __byte_perm(vw[2][r], vw[3][r], 0x7632);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          Mma<MT>::run(oacc[nt][4 * h + r], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-      }
-    }
-  }
 }
 
 // The output dims pv_tile leaves in a lane (g, tq): for column e of its tiles, dims d0 + 2i
@@ -1045,7 +1041,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           pb[nt][0] = transpose8x8(Mma<T>::pack(p0, p1));
           pb[nt][1] = transpose8x8(Mma<T>::pack(p2, p3));
         }
-        pv_tile<false, T, 2, C::SLAB_BYTES>(oacc, Vs, w, g, tq, nvalid, pb);
+        pv_tile<T, 2, C::SLAB_BYTES>(oacc, Vs, w, g, tq, nvalid, pb);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
       }
@@ -1251,7 +1247,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           if constexpr (F8)
             pv_mma_f8<1>(oaccs, vfr, pb);
           else
-            pv_tile<F8, MT, 1, C::SLAB_BYTES>(oaccs, Vs, w, g, tq, nvalid, pb);
+            pv_tile<MT, 1, C::SLAB_BYTES>(oaccs, Vs, w, g, tq, nvalid, pb);
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);
         }
