@@ -128,8 +128,7 @@ constexpr int kDirect = 4;  // the segment is the whole group: write `out`
 constexpr int kVirtual = 8;  // a chunk of a group's members over their shared prefix
 // a staged unit: [0] sequence (-1: no more work; >= num_seqs: a chunk), [1] head group,
 // [2..3] tiles [t0, t1), [4] flags, [5] partial slot of this segment, [6] append, [7] q /
-// out row (a chunk: its first member), [8] first slot of the group's segments, [9] segment
-// count, [10] members of a chunk
+// out row (a chunk: its first member), [10] members of a chunk
 constexpr int kUnitInts = 16;
 constexpr int kChunkRows = 16;           // q rows of a chunk per kv-head (members x G)
 
@@ -665,8 +664,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
   // fewer tiles than CTAs, only the first Ttot CTAs take a share, so every share is
   // non-empty and the segments of a group sit in consecutive CTAs (and slots).
   const int grid = min(ncta, max(Ttot, 1));
-  const int r0 = cta < grid ? (int)(((long long)cta * Ttot) / grid) : Ttot;
-  const int r1 = cta < grid ? (int)(((long long)(cta + 1) * Ttot) / grid) : Ttot;
+  // c*Ttot/grid in 32-bit arithmetic: c*(Ttot/grid) + c*(Ttot%grid)/grid, c*(Ttot%grid) < grid^2
+  const int tq = Ttot / grid, tr = Ttot % grid;
+  const int r0 = cta < grid ? cta * tq + (cta * tr) / grid : Ttot;
+  const int r1 = cta < grid ? (cta + 1) * tq + ((cta + 1) * tr) / grid : Ttot;
 
   if (warp < C::WARP_C0) {
     if (warp == C::WARP_FILL) {
@@ -733,8 +734,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
       for (int k = 0;; ++k) {
         const int qs = k % kQSlots;
         const uint32_t par = ((k / kQSlots) & 1) ^ 1;
-        wait_or_abort(&qempty[qs], par, abort_flag, a.err, a.wait_limit);  // consumers read unit k-2's q
-        wait_or_abort(&tempty[qs], par, abort_flag, a.err, a.wait_limit);  // its tiles were issued
+        if (k >= kQSlots) {  // the first units' slots were never used
+          wait_or_abort(&qempty[qs], par, abort_flag, a.err, a.wait_limit);  // consumers read unit k-2's q
+          wait_or_abort(&tempty[qs], par, abort_flag, a.err, a.wait_limit);  // its tiles were issued
+        }
         volatile int* u = unit + qs * kUnitInts;
         // after an abort a wait may have been skipped: no more arrivals
         const bool stop = warp_flag(abort_flag);
@@ -784,8 +787,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
         if (t0 == ts || pos == r0) flags |= kFirst;
         if (t1 == nt || pos + (t1 - t0) == r1) flags |= kLast;
         if (gs >= r0 && ge <= r1 && ts == 0 && !virt) flags |= kDirect;
-        // the group's segments sit in CTAs c0..c1, their partials in slots c0+grp..c1+grp
-        const int c0 = cta_of(gs, Ttot, grid), c1 = cta_of(ge - 1, Ttot, grid);
         const int32_t* trow = a.block_tables + (long long)trow_seq * a.max_blocks;
         int ids[kMaxTilesPerUnit / 32];
 #pragma unroll
@@ -836,8 +837,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           }
         }
         if (lane == 0) {
-          if (t0 == ts && !virt)  // the group's first unit: its merge record
-            a.meta[grp] = make_int2(c0 + grp, (flags & kDirect) ? 0 : c1 - c0 + 1);
           u[0] = s;
           u[1] = hp;
           u[2] = t0;
@@ -846,8 +845,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           u[5] = cta + grp;
           u[6] = append ? 1 : 0;
           u[7] = virt ? m0 : (a.qsl ? __ldg(a.qsl + s) : s);  // q / out row
-          u[8] = c0 + grp;
-          u[9] = c1 - c0 + 1;
           u[10] = nm;
           q_issued <<= 1;
           if ((flags & kFirst) && !virt) {  // a chunk's rows are read by its consumers
@@ -858,6 +855,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
             mbar_arrive_expect_tx(&qfull[qs], 0);
           }
           mbar_arrive(&tfull[qs]);
+          if (t0 == ts && !virt) {
+            // the group's first unit, once published: its merge record (the group's segments
+            // sit in CTAs c0..c1, their partials in slots c0+grp..c1+grp)
+            const int c0 = cta_of(gs, Ttot, grid), c1 = cta_of(ge - 1, Ttot, grid);
+            a.meta[grp] = make_int2(c0 + grp, (flags & kDirect) ? 0 : c1 - c0 + 1);
+          }
         }
         if (append) {
 #pragma unroll
@@ -953,7 +956,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
   // pv_tile gives it; K and q dims go in kchunk order.  The rows' q is read from global
   // memory once per segment.  Returns false when the CTA aborted.
   auto chunk_segment = [&](int& k, int& cnt, int qs, const volatile int* u) -> bool {
-    const int s = u[0], hp = u[1], pslot = u[5], m0 = u[7], slot0 = u[8], nseg = u[9];
+    const int s = u[0], hp = u[1], pslot = u[5], m0 = u[7];
     const int nm = u[10];
     int t0 = u[2], t1 = u[3], flags = u[4];
     const int g = lane >> 2, tq = lane & 3;
@@ -1077,8 +1080,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
       }
     }
     (void)s;
-    (void)slot0;
-    (void)nseg;
     return true;
   };
   {
@@ -1113,7 +1114,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
           continue;
         }
       }
-      const int hp = u[1], pslot = u[5], orow = u[7], slot0 = u[8], nseg = u[9];
+      const int hp = u[1], pslot = u[5], orow = u[7];
       int t0 = u[2], t1 = u[3], flags = u[4];
       uint32_t qf[8][2];    // Q^T fragments of the 8 k-steps
       float oaccs[1][8][4];  // O^T: [m-tile] x heads 2tq, 2tq+1 (dims: pv_tile)
@@ -1293,8 +1294,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
                 make_float2(e ? mh1 : mh0, e ? lt1 : lt0);
         }
       }
-      (void)slot0;
-      (void)nseg;
     }
   }
 }
