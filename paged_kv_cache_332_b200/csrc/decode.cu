@@ -1198,14 +1198,17 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmK, const CUtens
 #pragma unroll
             for (int e = 0; e < 4; ++e) sc[e] += sc2[e];
           } else {
+            float sc2[4] = {0.f, 0.f, 0.f, 0.f};  // odd k-steps: two chains of four products
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint8_t* kj = Ks + (j >> 1) * C::SLAB_BYTES + ((j & 1) ? kofs1 : kofs0);
               const uint4 ka = *reinterpret_cast<const uint4*>(kj);
               const uint4 kb = *reinterpret_cast<const uint4*>(kj + 1024);  // token g+8
               Mma<T>::run(sc, ka.x, kb.x, ka.y, kb.y, qf[2 * j][0], qf[2 * j][1]);
-              Mma<T>::run(sc, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
+              Mma<T>::run(sc2, ka.z, kb.z, ka.w, kb.w, qf[2 * j + 1][0], qf[2 * j + 1][1]);
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[e] += sc2[e];
           }
           // ---- online softmax over the tile (log2 domain), per head
           const bool v0 = g < nvalid, v8 = g + 8 < nvalid;
